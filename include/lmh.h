@@ -1,0 +1,215 @@
+/*
+ * lmh.h — C ABI of the deterministic chunked LM-head + loss for NVIDIA B200 (sm_100a).
+ *
+ * The operation (FlashInfer PR #8059 "feat(cake_lm_head_det_loss): det names for the
+ * chunked LM-head + loss backend", description): logits z = H W^T are computed chunk by
+ * chunk over rows and vocabulary, never stored as a full N x V matrix in HBM, and reduced
+ * to a per-row log-sum-exp, cross-entropy loss and target log-probability; the backward
+ * recomputes (or reuses) softmax minus one-hot and contracts it into dH and dW. The same
+ * description names the entries chunked_lm_head_det_{loss, logprob, support_logprob,
+ * support_kl} and states the determinism contract: for fixed inputs, hardware, chunk plan
+ * and initial accumulation buffers, forward and backward give bitwise-identical results run
+ * to run. This library keeps that contract: no floating-point atomics, every reduction in a
+ * fixed order, and no result depends on how many SMs the GPU has or which SM ran which tile.
+ *
+ * Conventions shared by every entry
+ * ---------------------------------
+ * - H [N, d] and W [V, d] are bf16, row-major and contiguous (row stride d elements);
+ *   lmh_bf16 is the raw 16-bit pattern. d must be a positive multiple of 64.
+ * - Every pointer argument is a DEVICE pointer unless marked "host", 16-byte aligned, and
+ *   owned by the caller. The library never allocates device memory, never frees it, and
+ *   never synchronises the host: each call only enqueues work on `stream` (a cudaStream_t;
+ *   NULL is the legacy default stream) and returns.
+ * - The workspace must hold at least lmh_workspace_size(shape, entry) bytes, be 256-byte
+ *   aligned, and must not be used by another call in flight at the same time.
+ * - Labels (miles-ext-kernels PR #14 "[Cake 13/13]", lm_head op commit, "Review items"):
+ *   every negative label marks an ignored row (LMH_IGNORE_INDEX = -100 is the customary
+ *   value). A label >= V is out of range: the row is treated as ignored and the device
+ *   error word gets LMH_DEVERR_LABEL_RANGE (no trap; read it with lmh_read_errors).
+ * - Rows are processed in chunks of shape->chunk_rows rows (0 selects 4096, the default of
+ *   the same commit's --cake-lm-head-chunk-size), in ascending order. The chunk plan only
+ *   changes the summation order of dW across chunks; every other output is independent
+ *   of it bit for bit.
+ * - Return value: LMH_OK, or an error found on the host before anything was enqueued
+ *   (invalid argument, misalignment, short workspace, unsupported device), or
+ *   LMH_ERR_CUDA when a launch failed. Errors found on the device go to the error word.
+ */
+#ifndef LMH_H_
+#define LMH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LMH_API __attribute__((visibility("default")))
+#else
+#define LMH_API
+#endif
+
+typedef uint16_t lmh_bf16;
+
+typedef enum lmh_status {
+  LMH_OK = 0,
+  LMH_ERR_INVALID_ARG = 1,
+  LMH_ERR_UNSUPPORTED_DEVICE = 2,
+  LMH_ERR_WORKSPACE_TOO_SMALL = 3,
+  LMH_ERR_ALIGNMENT = 4,
+  LMH_ERR_CUDA = 5
+} lmh_status;
+
+#define LMH_IGNORE_INDEX (-100)
+
+/* Bits of the device error word (first 4 bytes of the workspace). */
+#define LMH_DEVERR_LABEL_RANGE 0x1u /* a label or candidate id was >= V          */
+#define LMH_DEVERR_TIMEOUT 0x2u     /* a bounded wait inside a kernel gave up     */
+#define LMH_DEVERR_NONFINITE 0x4u   /* a row's log-sum-exp came out inf or NaN    */
+
+/* shape->flags */
+#define LMH_F_MEAN 0x1u         /* fused CE gradient is of the mean over valid rows    */
+#define LMH_F_FUSED_BWD 0x2u    /* sizing only: lmh_loss_fwd will also produce dH/dW   */
+#define LMH_F_DW_ACC_GIVEN 0x4u /* sizing only: the caller passes an fp32 dW_acc       */
+
+/* entries, for lmh_workspace_size */
+#define LMH_ENTRY_LOSS_FWD 0
+#define LMH_ENTRY_LOSS_BWD 1
+#define LMH_ENTRY_LOGPROB 2
+#define LMH_ENTRY_SUPPORT_LOGPROB 3
+#define LMH_ENTRY_SUPPORT_KL 4
+
+/* objectives of lmh_loss_bwd */
+#define LMH_BWD_CE 0              /* L = sum_i g_i loss_i                                */
+#define LMH_BWD_LOGPROB 1         /* L = sum_i g_i logprob_i                             */
+#define LMH_BWD_SUPPORT_LOGPROB 2 /* L = sum_ik g_ik lp_ik                               */
+#define LMH_BWD_SUPPORT_KL 3      /* L = sum_i g_i KL_i                                  */
+
+#define LMH_MAX_K 1024 /* largest candidate count per row of the support entries */
+
+typedef struct lmh_shape {
+  int64_t N;          /* rows (tokens), >= 0                                     */
+  int64_t d;          /* hidden size, multiple of 64                             */
+  int64_t V;          /* vocabulary size, 1 .. 2^31 - 1                          */
+  int64_t K;          /* candidates per row for the support entries, 1..LMH_MAX_K */
+  int64_t chunk_rows; /* rows per chunk; 0 selects 4096                          */
+  uint32_t flags;     /* LMH_F_*                                                 */
+  uint32_t reserved;  /* must be 0                                               */
+} lmh_shape;
+
+/*
+ * lmh_workspace_size — bytes of workspace the entry needs for `shape` (host, pure; no CUDA
+ * call). Memory budget (FlashInfer PR #8059, CodeRabbit summary: "memory-budgeted backend
+ * options ... workspace reporting"): the largest term is one chunk's bf16 softmax/gradient
+ * buffer, chunk_rows x round_up(V, 8) x 2 bytes, present for LMH_ENTRY_LOSS_BWD and for
+ * LMH_ENTRY_LOSS_FWD with LMH_F_FUSED_BWD; an fp32 [V, d] dW accumulator is added when the
+ * plan has more than one chunk, dW is produced, and LMH_F_DW_ACC_GIVEN is not set.
+ * Returns 0 for an invalid shape or entry.
+ */
+LMH_API size_t lmh_workspace_size(const lmh_shape* shape, int entry);
+
+/*
+ * lmh_loss_fwd — cross-entropy forward, optionally fused with its backward.
+ * Passage: FlashInfer PR #8059, description (chunked_lm_head_det_loss; "covers the CE and
+ * policy losses"); miles-ext-kernels PR #14, lm_head op commit (labels, FP32 dW accumulator
+ * cast to BF16 dW).
+ *   labels    [N] int32.
+ *   loss_rows [N] fp32 out (required): lse_i - z_i,y_i, 0 for ignored rows.
+ *   lse       [N] fp32 out (required): log sum_v exp z_iv, for every row.
+ *   logprob   [N] fp32 out, nullable: z_i,y_i - lse_i, 0 for ignored rows.
+ *   argmax    [N] int32 out, nullable: smallest v attaining max_v z_iv (fp32 logits).
+ *   loss_mean [1] fp32 out, nullable: sum of loss_rows over valid rows / n_valid (0 if none).
+ *   n_valid   [1] int32 out, nullable: rows with 0 <= label < V.
+ *   n_valid_given [1] int32 in, nullable: if given, the mean divides by this count instead.
+ *   dH [N, d] bf16 out, dW [V, d] bf16 out, dW_acc [V, d] fp32 in/out — all nullable. If dH
+ *     or dW is given the call also runs the backward of loss_mean (LMH_F_MEAN set) or of
+ *     sum_i loss_i (not set), reusing the forward's softmax instead of recomputing logits.
+ *     dW_acc, if given, is incremented by this call's dW in chunk order (zero it first for
+ *     a fresh gradient) and dW, if given, receives its round-to-nearest-even bf16 cast.
+ *     Without dW_acc and with one chunk, dW is the bf16 cast of the fp32 tile sums.
+ */
+LMH_API lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,
+                        const int32_t* labels, float* loss_rows, float* lse, float* logprob,
+                        int32_t* argmax, float* loss_mean, int32_t* n_valid,
+                        const int32_t* n_valid_given, lmh_bf16* dH, lmh_bf16* dW,
+                        float* dW_acc, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * lmh_loss_bwd — backward of any of the four row objectives, recomputing the logits chunk
+ * by chunk from H and W (FlashInfer PR #8059, CodeRabbit walkthrough: "memory-budget
+ * planning and recomputation"). With P = softmax(z) it forms
+ *   G_iv = alpha_i P_iv - sum_k beta_ik [v = t_ik]
+ * and returns dH = G W and dW = G^T H, where, by `mode`:
+ *   LMH_BWD_CE:              targets = labels [N];  grad [N] = dL/dloss_i;
+ *                            alpha_i = beta_i = g_i (valid rows; 0 for ignored rows).
+ *   LMH_BWD_LOGPROB:         targets = labels [N];  grad [N] = dL/dlogprob_i;
+ *                            alpha_i = beta_i = -g_i.
+ *   LMH_BWD_SUPPORT_LOGPROB: targets = ids [N, K]; grad [N, K] = dL/dlp_ik;
+ *                            alpha_i = -sum_k g_ik, beta_ik = -g_ik.
+ *   LMH_BWD_SUPPORT_KL:      targets = ids [N, K]; grad [N] = dL/dKL_i; ref_logp [N, K];
+ *                            alpha_i = g_i sum_k exp(r_ik), beta_ik = g_i exp(r_ik).
+ * Candidate ids < 0 are padding and are skipped. lse [N] is the forward's output.
+ * dH, dW, dW_acc: as in lmh_loss_fwd (nullable; dW_acc accumulates in chunk order).
+ */
+LMH_API lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,
+                        const lmh_bf16* W, const int32_t* targets, const float* lse,
+                        const float* grad, const float* ref_logp, lmh_bf16* dH, lmh_bf16* dW,
+                        float* dW_acc, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * lmh_logprob — per-row target log-probability (FlashInfer PR #8059, description:
+ * chunked_lm_head_det_logprob; miles-ext-kernels PR #14, lm_head op commit: log_probs).
+ *   logprob [N] fp32 out: z_i,y_i - lse_i, 0 for ignored rows.  lse [N] fp32 out (required).
+ */
+LMH_API lmh_status lmh_logprob(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,
+                       const int32_t* labels, float* logprob, float* lse, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
+ * lmh_support_logprob — "candidate-restricted log-probabilities" (FlashInfer PR #8059,
+ * CodeRabbit summary and walkthrough). Reading taken: the full-vocabulary log-probability
+ * evaluated at each candidate, lp_ik = z_i,c_ik - lse_i.
+ *   ids [N, K] int32 in (K = shape->K; ids < 0 are padding, lp = 0 there; ids >= V flag
+ *   LMH_DEVERR_LABEL_RANGE and are treated as padding). lp [N, K] fp32 out. lse [N] out.
+ */
+LMH_API lmh_status lmh_support_logprob(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,
+                               const int32_t* ids, float* lp, float* lse, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
+ * lmh_support_kl — forward KL over the candidate set (FlashInfer PR #8059, CodeRabbit
+ * walkthrough: "candidate-support log-probability and forward-KL APIs"). Reading taken:
+ * KL(ref || model) = sum_k exp(r_ik) (r_ik - lp_ik) over the valid candidates of row i,
+ * with r = ref_logp the given reference log-probs.
+ *   ids [N, K], ref_logp [N, K] fp32 in. kl_rows [N] fp32 out. kl_mean [1] fp32 out,
+ *   nullable (mean over all N rows). lp [N, K] fp32 out, nullable. lse [N] out (required).
+ */
+LMH_API lmh_status lmh_support_kl(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,
+                          const int32_t* ids, const float* ref_logp, float* kl_rows,
+                          float* kl_mean, float* lp, float* lse, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
+ * lmh_read_errors — synchronises `stream`, then copies the device error word of the last
+ * call that used `workspace` into *errors (host). Each entry clears the word when it starts.
+ */
+LMH_API lmh_status lmh_read_errors(const void* workspace, uint32_t* errors, void* stream);
+
+/*
+ * Measurement hook (not part of the method). lmh_profile_enable(1) makes every later call
+ * bracket each kernel it enqueues with a pair of CUDA events on the call's stream (host-side
+ * event objects only; process-wide; lmh_profile_enable(0) stops). lmh_profile_read
+ * synchronises the recorded events, writes up to max_records (kernel id, milliseconds)
+ * pairs to the host arrays, returns how many it wrote and forgets all records.
+ * lmh_kernel_name maps an id to a stable name ("gemm_dW", "row_finalize", ...).
+ */
+LMH_API lmh_status lmh_profile_enable(int on);
+LMH_API int lmh_profile_read(int max_records, int32_t* kernel_ids, float* ms);
+LMH_API const char* lmh_kernel_name(int kernel_id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LMH_H_ */

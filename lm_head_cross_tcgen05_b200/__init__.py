@@ -1,0 +1,227 @@
+"""Deterministic chunked LM-head + loss on B200 (sm_100a): Python binding of liblmh.so.
+
+The functions named ``lmh_*`` mirror the C ABI of ``include/lmh.h`` one to one: they take
+torch CUDA tensors, check dtype / contiguity / device, and pass raw pointers and the
+current stream through ctypes. Every step of the computation runs in the library's CUDA
+kernels; there is no fallback path, and importing this package fails if ``liblmh.so`` has
+not been built (``python -m lm_head_cross_tcgen05_b200.build``).
+
+The lower-case helpers (``loss_fwd``, ``loss_bwd``, ``logprob``, ``support_logprob``,
+``support_kl``) allocate the outputs and the workspace with torch and call the same entries.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEVERR_LABEL_RANGE,
+                   DEVERR_NONFINITE, DEVERR_TIMEOUT, ENTRY_LOGPROB, ENTRY_LOSS_BWD,
+                   ENTRY_LOSS_FWD, ENTRY_SUPPORT_KL, ENTRY_SUPPORT_LOGPROB, F_DW_ACC_GIVEN,
+                   F_FUSED_BWD, F_MEAN, IGNORE_INDEX, MAX_K, STATUS_NAMES, lib, lmh_shape)
+
+__all__ = [
+    "lmh_shape", "make_shape", "lmh_workspace_size", "lmh_loss_fwd", "lmh_loss_bwd",
+    "lmh_logprob", "lmh_support_logprob", "lmh_support_kl", "lmh_read_errors", "LmhError",
+    "loss_fwd", "loss_bwd", "logprob", "support_logprob", "support_kl", "workspace",
+    "IGNORE_INDEX", "BWD_CE", "BWD_LOGPROB", "BWD_SUPPORT_LOGPROB", "BWD_SUPPORT_KL",
+    "F_MEAN", "F_FUSED_BWD", "F_DW_ACC_GIVEN", "ENTRY_LOSS_FWD", "ENTRY_LOSS_BWD",
+    "ENTRY_LOGPROB", "ENTRY_SUPPORT_LOGPROB", "ENTRY_SUPPORT_KL", "DEVERR_LABEL_RANGE",
+    "DEVERR_TIMEOUT", "DEVERR_NONFINITE", "MAX_K",
+]
+
+lib()  # load now: a missing library is an import error, never a silent fallback
+
+
+class LmhError(RuntimeError):
+    def __init__(self, entry: str, status: int):
+        super().__init__(f"{entry}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+def make_shape(N: int, d: int, V: int, K: int = 0, chunk_rows: int = 0,
+               flags: int = 0) -> lmh_shape:
+    return lmh_shape(int(N), int(d), int(V), int(K), int(chunk_rows), int(flags), 0)
+
+
+def _p(t: Optional[torch.Tensor], dtype=None, what: str = "tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{what} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ok(name: str, status: int):
+    if status != 0:
+        raise LmhError(name, status)
+
+
+_bf, _f32, _i32, _u8 = torch.bfloat16, torch.float32, torch.int32, torch.uint8
+
+
+# ----------------------------------------------------------------------------- C ABI mirror
+
+def lmh_workspace_size(shape: lmh_shape, entry: int) -> int:
+    return int(lib().lmh_workspace_size(ctypes.byref(shape), int(entry)))
+
+
+def lmh_loss_fwd(shape, H, W, labels, loss_rows, lse, logprob=None, argmax=None, loss_mean=None,
+                 n_valid=None, n_valid_given=None, dH=None, dW=None, dW_acc=None, *, workspace,
+                 stream=None) -> None:
+    st = lib().lmh_loss_fwd(
+        ctypes.byref(shape), _p(H, _bf, "H"), _p(W, _bf, "W"), _p(labels, _i32, "labels"),
+        _p(loss_rows, _f32, "loss_rows"), _p(lse, _f32, "lse"), _p(logprob, _f32, "logprob"),
+        _p(argmax, _i32, "argmax"), _p(loss_mean, _f32, "loss_mean"),
+        _p(n_valid, _i32, "n_valid"), _p(n_valid_given, _i32, "n_valid_given"),
+        _p(dH, _bf, "dH"), _p(dW, _bf, "dW"), _p(dW_acc, _f32, "dW_acc"),
+        _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
+    _ok("lmh_loss_fwd", st)
+
+
+def lmh_loss_bwd(shape, mode, H, W, targets, lse, grad, ref_logp=None, dH=None, dW=None,
+                 dW_acc=None, *, workspace, stream=None) -> None:
+    st = lib().lmh_loss_bwd(
+        ctypes.byref(shape), int(mode), _p(H, _bf, "H"), _p(W, _bf, "W"),
+        _p(targets, _i32, "targets"), _p(lse, _f32, "lse"), _p(grad, _f32, "grad"),
+        _p(ref_logp, _f32, "ref_logp"), _p(dH, _bf, "dH"), _p(dW, _bf, "dW"),
+        _p(dW_acc, _f32, "dW_acc"), _p(workspace, _u8, "workspace"), workspace.numel(),
+        _s(stream))
+    _ok("lmh_loss_bwd", st)
+
+
+def lmh_logprob(shape, H, W, labels, logprob, lse, *, workspace, stream=None) -> None:
+    st = lib().lmh_logprob(ctypes.byref(shape), _p(H, _bf, "H"), _p(W, _bf, "W"),
+                           _p(labels, _i32, "labels"), _p(logprob, _f32, "logprob"),
+                           _p(lse, _f32, "lse"), _p(workspace, _u8, "workspace"),
+                           workspace.numel(), _s(stream))
+    _ok("lmh_logprob", st)
+
+
+def lmh_support_logprob(shape, H, W, ids, lp, lse, *, workspace, stream=None) -> None:
+    st = lib().lmh_support_logprob(ctypes.byref(shape), _p(H, _bf, "H"), _p(W, _bf, "W"),
+                                   _p(ids, _i32, "ids"), _p(lp, _f32, "lp"), _p(lse, _f32, "lse"),
+                                   _p(workspace, _u8, "workspace"), workspace.numel(),
+                                   _s(stream))
+    _ok("lmh_support_logprob", st)
+
+
+def lmh_support_kl(shape, H, W, ids, ref_logp, kl_rows, kl_mean=None, lp=None, lse=None, *,
+                   workspace, stream=None) -> None:
+    st = lib().lmh_support_kl(ctypes.byref(shape), _p(H, _bf, "H"), _p(W, _bf, "W"),
+                              _p(ids, _i32, "ids"), _p(ref_logp, _f32, "ref_logp"),
+                              _p(kl_rows, _f32, "kl_rows"), _p(kl_mean, _f32, "kl_mean"),
+                              _p(lp, _f32, "lp"), _p(lse, _f32, "lse"),
+                              _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
+    _ok("lmh_support_kl", st)
+
+
+def lmh_read_errors(workspace: torch.Tensor, stream=None) -> int:
+    out = ctypes.c_uint32(0)
+    _ok("lmh_read_errors", lib().lmh_read_errors(_p(workspace, _u8, "workspace"),
+                                                 ctypes.byref(out), _s(stream)))
+    return int(out.value)
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def workspace(shape: lmh_shape, entry: int, device) -> torch.Tensor:
+    n = lmh_workspace_size(shape, entry)
+    if n == 0:
+        raise ValueError("invalid shape for this entry")
+    return torch.empty(n, dtype=_u8, device=device)
+
+
+def loss_fwd(H, W, labels, *, chunk_rows: int = 0, mean: bool = True, grads: bool = False,
+             want_dH: bool = True, want_dW: bool = True, dW_acc=None, n_valid_given=None,
+             ws=None, stream=None) -> dict:
+    """CE forward (loss_rows, lse, logprob, argmax, loss_mean, n_valid); with grads=True also
+    dH / dW of the mean (or summed) loss, fused with the forward."""
+    N, d = H.shape
+    V = W.shape[0]
+    dev = H.device
+    flags = (F_MEAN if mean else 0) | (F_FUSED_BWD if grads else 0) | (
+        F_DW_ACC_GIVEN if dW_acc is not None else 0)
+    shape = make_shape(N, d, V, 0, chunk_rows, flags)
+    out = dict(loss_rows=torch.empty(N, dtype=_f32, device=dev),
+               lse=torch.empty(N, dtype=_f32, device=dev),
+               logprob=torch.empty(N, dtype=_f32, device=dev),
+               argmax=torch.empty(N, dtype=_i32, device=dev),
+               loss_mean=torch.empty(1, dtype=_f32, device=dev),
+               n_valid=torch.empty(1, dtype=_i32, device=dev))
+    if grads:
+        out["dH"] = torch.empty(N, d, dtype=_bf, device=dev) if want_dH else None
+        out["dW"] = torch.empty(V, d, dtype=_bf, device=dev) if want_dW else None
+    ws = workspace(shape, ENTRY_LOSS_FWD, dev) if ws is None else ws
+    lmh_loss_fwd(shape, H, W, labels, out["loss_rows"], out["lse"], out["logprob"],
+                 out["argmax"], out["loss_mean"], out["n_valid"], n_valid_given,
+                 out.get("dH"), out.get("dW"), dW_acc, workspace=ws, stream=stream)
+    out["workspace"] = ws
+    return out
+
+
+def loss_bwd(mode: int, H, W, targets, lse, grad, ref_logp=None, *, chunk_rows: int = 0,
+             want_dH: bool = True, want_dW: bool = True, dW_acc=None, ws=None,
+             stream=None) -> dict:
+    N, d = H.shape
+    V = W.shape[0]
+    K = targets.shape[1] if targets.dim() == 2 else 1
+    dev = H.device
+    shape = make_shape(N, d, V, K, chunk_rows, F_DW_ACC_GIVEN if dW_acc is not None else 0)
+    out = dict(dH=torch.empty(N, d, dtype=_bf, device=dev) if want_dH else None,
+               dW=torch.empty(V, d, dtype=_bf, device=dev) if want_dW else None)
+    ws = workspace(shape, ENTRY_LOSS_BWD, dev) if ws is None else ws
+    lmh_loss_bwd(shape, mode, H, W, targets, lse, grad, ref_logp, out["dH"], out["dW"], dW_acc,
+                 workspace=ws, stream=stream)
+    out["workspace"] = ws
+    return out
+
+
+def logprob(H, W, labels, *, chunk_rows: int = 0, ws=None, stream=None) -> dict:
+    N, d = H.shape
+    shape = make_shape(N, d, W.shape[0], 0, chunk_rows)
+    out = dict(logprob=torch.empty(N, dtype=_f32, device=H.device),
+               lse=torch.empty(N, dtype=_f32, device=H.device))
+    ws = workspace(shape, ENTRY_LOGPROB, H.device) if ws is None else ws
+    lmh_logprob(shape, H, W, labels, out["logprob"], out["lse"], workspace=ws, stream=stream)
+    out["workspace"] = ws
+    return out
+
+
+def support_logprob(H, W, ids, *, chunk_rows: int = 0, ws=None, stream=None) -> dict:
+    N, d = H.shape
+    K = ids.shape[1]
+    shape = make_shape(N, d, W.shape[0], K, chunk_rows)
+    out = dict(lp=torch.empty(N, K, dtype=_f32, device=H.device),
+               lse=torch.empty(N, dtype=_f32, device=H.device))
+    ws = workspace(shape, ENTRY_SUPPORT_LOGPROB, H.device) if ws is None else ws
+    lmh_support_logprob(shape, H, W, ids, out["lp"], out["lse"], workspace=ws, stream=stream)
+    out["workspace"] = ws
+    return out
+
+
+def support_kl(H, W, ids, ref_logp, *, chunk_rows: int = 0, ws=None, stream=None) -> dict:
+    N, d = H.shape
+    K = ids.shape[1]
+    shape = make_shape(N, d, W.shape[0], K, chunk_rows)
+    dev = H.device
+    out = dict(kl_rows=torch.empty(N, dtype=_f32, device=dev),
+               kl_mean=torch.empty(1, dtype=_f32, device=dev),
+               lp=torch.empty(N, K, dtype=_f32, device=dev),
+               lse=torch.empty(N, dtype=_f32, device=dev))
+    ws = workspace(shape, ENTRY_SUPPORT_KL, dev) if ws is None else ws
+    lmh_support_kl(shape, H, W, ids, ref_logp, out["kl_rows"], out["kl_mean"], out["lp"],
+                   out["lse"], workspace=ws, stream=stream)
+    out["workspace"] = ws
+    return out

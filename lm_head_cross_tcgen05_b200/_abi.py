@@ -1,0 +1,65 @@
+"""ctypes declarations of liblmh.so (include/lmh.h). Loading fails loudly if it is not built."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "liblmh.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "lmh.h")
+
+c_int64, c_uint32, c_int, c_size_t, c_void_p = (ctypes.c_int64, ctypes.c_uint32, ctypes.c_int,
+                                                ctypes.c_size_t, ctypes.c_void_p)
+
+LMH_OK = 0
+STATUS_NAMES = {0: "LMH_OK", 1: "LMH_ERR_INVALID_ARG", 2: "LMH_ERR_UNSUPPORTED_DEVICE",
+                3: "LMH_ERR_WORKSPACE_TOO_SMALL", 4: "LMH_ERR_ALIGNMENT", 5: "LMH_ERR_CUDA"}
+
+IGNORE_INDEX = -100
+DEVERR_LABEL_RANGE, DEVERR_TIMEOUT, DEVERR_NONFINITE = 0x1, 0x2, 0x4
+F_MEAN, F_FUSED_BWD, F_DW_ACC_GIVEN = 0x1, 0x2, 0x4
+ENTRY_LOSS_FWD, ENTRY_LOSS_BWD, ENTRY_LOGPROB, ENTRY_SUPPORT_LOGPROB, ENTRY_SUPPORT_KL = range(5)
+BWD_CE, BWD_LOGPROB, BWD_SUPPORT_LOGPROB, BWD_SUPPORT_KL = range(4)
+MAX_K = 1024
+
+
+class lmh_shape(ctypes.Structure):
+    _fields_ = [("N", c_int64), ("d", c_int64), ("V", c_int64), ("K", c_int64),
+                ("chunk_rows", c_int64), ("flags", c_uint32), ("reserved", c_uint32)]
+
+
+_P = c_void_p
+_SIGS = {
+    "lmh_workspace_size": (c_size_t, [ctypes.POINTER(lmh_shape), c_int]),
+    "lmh_loss_fwd": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 14 + [c_size_t, _P]),
+    "lmh_loss_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 10 + [c_size_t, _P]),
+    "lmh_logprob": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6 + [c_size_t, _P]),
+    "lmh_support_logprob": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6 + [c_size_t, _P]),
+    "lmh_support_kl": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 9 + [c_size_t, _P]),
+    "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),
+}
+
+
+def header_symbols(path: str = HEADER):
+    """Names of the functions include/lmh.h declares."""
+    src = open(path).read()
+    return re.findall(r"^LMH_API\s+\w+\s+(lmh_\w+)\s*\(", src, flags=re.M)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is not built; run `python -m lm_head_cross_tcgen05_b200.build` "
+                "(this package has no fallback path)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib

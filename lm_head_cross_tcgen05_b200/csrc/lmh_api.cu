@@ -1,0 +1,658 @@
+// lmh_api.cu — the C ABI of include/lmh.h: argument validation, the chunk plan and the
+// workspace carve-up, TMA descriptor encoding, and the stream-ordered sequence of kernels of
+// each entry. Nothing here allocates device memory or waits for the device (except
+// lmh_read_errors, whose job is to).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "../../include/lmh.h"
+#include "epilogues.cuh"
+#include "gemm.cuh"
+#include "rowops.cuh"
+
+using namespace lmh;
+
+namespace {
+
+constexpr int64_t kDefaultChunk = 4096;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------------------ plan
+// The row partition and the byte offsets of every workspace region.
+struct Plan {
+  int64_t N, d, V, K, Vp, T, c, nchunks;
+  bool cands;   // per-row candidate lists (support entries, candidate backward)
+  bool gbuf;    // chunk softmax / gradient buffer
+  bool acc;     // internal fp32 dW accumulator
+  size_t o_zt, o_sorted, o_nuniq, o_rank, o_pm, o_ps, o_pi, o_alpha, o_beta, o_gbuf, o_acc;
+  size_t total;
+};
+
+bool shape_ok(const lmh_shape* s) {
+  if (!s) return false;
+  if (s->N < 0 || s->d <= 0 || (s->d % 64) != 0 || s->V <= 0 || s->V > 0x7fffffffLL)
+    return false;
+  if (s->d > (1LL << 24) || s->chunk_rows < 0 || s->reserved != 0) return false;
+  return true;
+}
+
+// fused: the entry keeps a [c, Vp] bf16 buffer; need_acc: an fp32 [V, d] accumulator.
+Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
+  Plan p{};
+  p.N = s->N;
+  p.d = s->d;
+  p.V = s->V;
+  p.Vp = (s->V + 7) / 8 * 8;
+  p.T = cdiv(s->V, BN);
+  const int64_t c = s->chunk_rows > 0 ? s->chunk_rows : kDefaultChunk;
+  p.c = p.N > 0 ? (c < p.N ? c : p.N) : 0;
+  p.nchunks = p.N > 0 ? cdiv(p.N, p.c) : 0;
+  p.cands = (entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL ||
+             entry == LMH_ENTRY_LOSS_BWD);
+  p.K = p.cands ? (s->K > 0 ? s->K : 1) : 1;
+  p.gbuf = (entry == LMH_ENTRY_LOSS_BWD) || (entry == LMH_ENTRY_LOSS_FWD && fused);
+  p.acc = p.gbuf && dw_without_acc && p.nchunks > 1;
+  const bool stats = entry != LMH_ENTRY_LOSS_BWD;
+  size_t o = sizeof(WsHeader);
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  const size_t N = static_cast<size_t>(p.N);
+  p.o_zt = stats ? take(N * p.K * 4) : 0;
+  p.o_sorted = p.cands ? take(N * p.K * 4) : 0;
+  p.o_nuniq = p.cands ? take(N * 4) : 0;
+  p.o_rank = p.cands ? take(N * p.K * 4) : 0;
+  const size_t cT = static_cast<size_t>(p.c) * p.T;
+  p.o_pm = stats ? take(cT * 4) : 0;
+  p.o_ps = stats ? take(cT * 4) : 0;
+  p.o_pi = stats ? take(cT * 4) : 0;
+  p.o_alpha = (entry == LMH_ENTRY_LOSS_BWD) ? take(N * 4) : 0;
+  p.o_beta = (entry == LMH_ENTRY_LOSS_BWD) ? take(N * p.K * 4) : 0;
+  p.o_gbuf = p.gbuf ? take(static_cast<size_t>(p.c) * p.Vp * 2) : 0;
+  p.o_acc = p.acc ? take(static_cast<size_t>(p.V) * p.d * 4) : 0;
+  p.total = o;
+  return p;
+}
+
+// ------------------------------------------------------------------------ device state
+struct DevState {
+  bool init = false;
+  bool ok = false;
+  int sms = 0;
+};
+std::mutex g_mu;
+DevState g_dev[64];
+
+lmh_status current_device(int* dev_out, int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LMH_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevState& ds = g_dev[dev];
+  if (!ds.init) {
+    int major = 0, minor = 0, n = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return LMH_ERR_CUDA;
+    ds.ok = (major == 10 && minor == 0);
+    ds.sms = n;
+    ds.init = true;
+  }
+  if (!ds.ok) return LMH_ERR_UNSUPPORTED_DEVICE;
+  *dev_out = dev;
+  *sms = ds.sms;
+  return LMH_OK;
+}
+
+// ------------------------------------------------------------------------ stage timing
+// Measurement hook: while enabled, every kernel the library enqueues is bracketed by a pair
+// of CUDA events on its stream (host-side objects; no device memory is allocated).
+enum KernelId {
+  KID_COUNT_LABELS, KID_PREP_CANDS, KID_GEMM_LOGITS, KID_GEMM_LOGITS_P, KID_GEMM_GRAD,
+  KID_GEMM_DH, KID_GEMM_DW, KID_FINALIZE, KID_GBUILD, KID_FIX_LABELS, KID_MEAN,
+  KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_COUNT
+};
+const char* const kKernelNames[KID_COUNT] = {
+    "count_labels", "prep_cands", "gemm_logits_stats", "gemm_logits_stats_store",
+    "gemm_logits_grad", "gemm_dH", "gemm_dW", "row_finalize", "gbuild", "fix_labels",
+    "mean", "support_out", "bwd_coef", "cast_bf16"};
+
+struct ProfRec {
+  int id;
+  cudaEvent_t a, b;
+};
+std::atomic<bool> g_prof_on{false};
+std::mutex g_prof_mu;
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct ProfScope {
+  int id = -1;
+  cudaEvent_t a = nullptr;
+  cudaStream_t st;
+  ProfScope(int kid, cudaStream_t s) : st(s) {
+    if (!g_prof_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    a = prof_event();
+    if (a && cudaEventRecord(a, st) == cudaSuccess) id = kid;
+  }
+  ~ProfScope() {
+    if (id < 0) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    cudaEvent_t b = prof_event();
+    if (b && cudaEventRecord(b, st) == cudaSuccess) g_prof_recs.push_back({id, a, b});
+  }
+};
+
+// ------------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] with row stride `ld` elements; box {64, box_outer}, 128-byte
+// swizzle, zero fill out of bounds.
+bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+             uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------------ launches
+template <class Epi>
+lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap& b,
+                       int64_t M, int64_t Ncols, int64_t K, int n_fastest, uint32_t* err,
+                       const typename Epi::Params& ep, cudaStream_t st) {
+  static std::atomic<uint64_t> attr_done{0};
+  const uint64_t bit = 1ull << dev;
+  if (!(attr_done.load() & bit)) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GEMM_SMEM_BYTES) != cudaSuccess)
+      return LMH_ERR_CUDA;
+    attr_done.fetch_or(bit);
+  }
+  GemmGrid g;
+  g.m_tiles = static_cast<int>(cdiv(M, BM));
+  g.n_tiles = static_cast<int>(cdiv(Ncols, BN));
+  g.k_blocks = static_cast<int>(cdiv(K, BK));
+  g.n_fastest = n_fastest;
+  g.err = err;
+  const int64_t tiles = static_cast<int64_t>(g.m_tiles) * g.n_tiles;
+  if (tiles <= 0) return LMH_OK;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  ProfScope ps(Epi::kId, st);
+  gemm_tc_kernel<Epi><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(a, b, g, ep);
+  return cudaGetLastError() == cudaSuccess ? LMH_OK : LMH_ERR_CUDA;
+}
+
+#define LMH_TRY(x)                      \
+  do {                                  \
+    lmh_status _s = (x);                \
+    if (_s != LMH_OK) return _s;        \
+  } while (0)
+
+lmh_status last_launch() { return cudaGetLastError() == cudaSuccess ? LMH_OK : LMH_ERR_CUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Ws {
+  uint8_t* base;
+  WsHeader* h;
+  template <class T>
+  T* at(size_t off) const { return reinterpret_cast<T*>(base + off); }
+};
+
+lmh_status common_checks(const lmh_shape* s, const void* H, const void* W, void* ws,
+                         size_t ws_bytes, size_t need, int* dev, int* sms) {
+  if (!shape_ok(s)) return LMH_ERR_INVALID_ARG;
+  if (s->N > 0 && (!H || !W)) return LMH_ERR_INVALID_ARG;
+  if (!ws) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(H) || !aligned16(W)) return LMH_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return LMH_ERR_ALIGNMENT;
+  if (ws_bytes < need) return LMH_ERR_WORKSPACE_TOO_SMALL;
+  return current_device(dev, sms);
+}
+
+// Per-chunk logits statistics GEMM + row finalize.
+template <int TK, bool kStoreP>
+lmh_status run_stats(const Plan& P, int dev, int sms, const lmh_bf16* H, const lmh_bf16* W,
+                     const Targets& tg, int64_t r0, int rows, const Ws& ws, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, H + r0 * P.d, P.d, rows, P.d, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BN))
+    return LMH_ERR_CUDA;
+  typename EpiStats<TK, kStoreP>::Params ep;
+  ep.rows = rows;
+  ep.row0 = r0;
+  ep.V = static_cast<int>(P.V);
+  ep.T = static_cast<int>(P.T);
+  ep.ldp = P.Vp;
+  ep.tg = tg;
+  ep.zt = ws.at<float>(P.o_zt);
+  ep.part_m = ws.at<float>(P.o_pm);
+  ep.part_s = ws.at<float>(P.o_ps);
+  ep.part_i = ws.at<int32_t>(P.o_pi);
+  ep.P = kStoreP ? ws.at<__nv_bfloat16>(P.o_gbuf) : nullptr;
+  return launch_gemm<EpiStats<TK, kStoreP>>(dev, sms, ta, tb, rows, P.V, P.d, 0, &ws.h->err, ep,
+                                           st);
+}
+
+lmh_status run_finalize(const Plan& P, int kind, int64_t r0, int rows, const int32_t* labels,
+                        float* lse, float* loss, float* logprob, int32_t* argmax, int write_scale,
+                        int mean, const int32_t* n_given, const Ws& ws, cudaStream_t st) {
+  FinParams f;
+  f.rows = rows;
+  f.row0 = r0;
+  f.T = static_cast<int>(P.T);
+  f.V = static_cast<int>(P.V);
+  f.kind = kind;
+  f.part_m = ws.at<float>(P.o_pm);
+  f.part_s = ws.at<float>(P.o_ps);
+  f.part_i = ws.at<int32_t>(P.o_pi);
+  f.labels = labels;
+  f.zt = ws.at<float>(P.o_zt);
+  f.lse = lse;
+  f.loss = loss;
+  f.logprob = logprob;
+  f.argmax = argmax;
+  f.write_scale = write_scale;
+  f.mean = mean;
+  f.n_given = n_given;
+  f.h = ws.h;
+  const int warps = 8;
+  ProfScope ps(KID_FINALIZE, st);
+  finalize_rows_kernel<<<static_cast<unsigned>(cdiv(rows, warps)), 32 * warps, 0, st>>>(f);
+  return last_launch();
+}
+
+// dH = G W and dW (+)= G^T H_c for one chunk whose G sits in the workspace buffer.
+lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H,
+                              const lmh_bf16* W, int64_t r0, int rows, int chunk_idx,
+                              lmh_bf16* dH, lmh_bf16* dW, float* dW_acc, const Ws& ws,
+                              cudaStream_t st) {
+  const __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
+  if (dH) {
+    CUtensorMap ta, tb;
+    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, 64))
+      return LMH_ERR_CUDA;
+    EpiDH::Params ep;
+    ep.rows = rows;
+    ep.row0 = r0;
+    ep.d = static_cast<int>(P.d);
+    ep.dH = reinterpret_cast<__nv_bfloat16*>(dH);
+    LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, rows, P.d, P.V, 1, &ws.h->err, ep, st));
+  }
+  if (dW || dW_acc) {
+    CUtensorMap ta, tb;
+    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, 64) || !tmap_2d(&tb, H + r0 * P.d, P.d, rows, P.d, 64))
+      return LMH_ERR_CUDA;
+    EpiDW::Params ep;
+    ep.V = static_cast<int>(P.V);
+    ep.d = static_cast<int>(P.d);
+    const bool last = chunk_idx == P.nchunks - 1;
+    if (dW_acc) {
+      ep.acc = dW_acc;
+      ep.acc_mode = 2;
+    } else if (P.acc) {
+      ep.acc = ws.at<float>(P.o_acc);
+      ep.acc_mode = chunk_idx == 0 ? 1 : 2;
+    } else {
+      ep.acc = nullptr;
+      ep.acc_mode = 0;
+    }
+    ep.out = (dW && last) ? reinterpret_cast<__nv_bfloat16*>(dW) : nullptr;
+    LMH_TRY(launch_gemm<EpiDW>(dev, sms, ta, tb, P.V, P.d, rows, 1, &ws.h->err, ep, st));
+  }
+  return LMH_OK;
+}
+
+lmh_status clear_header(const Ws& ws, cudaStream_t st) {
+  return cudaMemsetAsync(ws.h, 0, sizeof(WsHeader), st) == cudaSuccess ? LMH_OK : LMH_ERR_CUDA;
+}
+
+lmh_status count_labels(const Plan& P, const int32_t* labels, const Ws& ws, cudaStream_t st) {
+  if (P.N == 0) return LMH_OK;
+  const int64_t blocks = cdiv(P.N, 256);
+  ProfScope ps(KID_COUNT_LABELS, st);
+  count_labels_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 256, 0, st>>>(
+      labels, P.N, static_cast<int>(P.V), ws.h);
+  return last_launch();
+}
+
+lmh_status prep_cands(const Plan& P, const int32_t* ids, const Ws& ws, cudaStream_t st) {
+  if (P.N == 0) return LMH_OK;
+  const int threads = static_cast<int>(cdiv(P.K, 32) * 32);
+  const int64_t blocks = P.N < 65535 ? P.N : 65535;
+  ProfScope ps(KID_PREP_CANDS, st);
+  prep_cands_kernel<<<static_cast<unsigned>(blocks), threads, 3 * P.K * sizeof(int32_t), st>>>(
+      ids, P.N, static_cast<int>(P.K), static_cast<int>(P.V), ws.at<int32_t>(P.o_sorted),
+      ws.at<int32_t>(P.o_nuniq), ws.at<int32_t>(P.o_rank), ws.h);
+  return last_launch();
+}
+
+// Outputs of a call without rows: zero counts / means, dW = cast of the given accumulator.
+lmh_status empty_call(const Plan& P, float* mean_out, int32_t* nvalid_out, lmh_bf16* dW,
+                      float* dW_acc, cudaStream_t st) {
+  if (mean_out && cudaMemsetAsync(mean_out, 0, 4, st) != cudaSuccess) return LMH_ERR_CUDA;
+  if (nvalid_out && cudaMemsetAsync(nvalid_out, 0, 4, st) != cudaSuccess) return LMH_ERR_CUDA;
+  if (dW) {
+    const int64_t n = P.V * P.d;
+    if (dW_acc) {
+      ProfScope ps(KID_CAST, st);
+      cast_bf16_kernel<<<1024, 256, 0, st>>>(dW_acc, n, reinterpret_cast<__nv_bfloat16*>(dW));
+      return last_launch();
+    }
+    if (cudaMemsetAsync(dW, 0, n * 2, st) != cudaSuccess) return LMH_ERR_CUDA;
+  }
+  return LMH_OK;
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+
+extern "C" size_t lmh_workspace_size(const lmh_shape* shape, int entry) {
+  if (!shape_ok(shape) || entry < LMH_ENTRY_LOSS_FWD || entry > LMH_ENTRY_SUPPORT_KL) return 0;
+  if ((entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL) &&
+      (shape->K < 1 || shape->K > LMH_MAX_K))
+    return 0;
+  const bool fused = entry == LMH_ENTRY_LOSS_FWD && (shape->flags & LMH_F_FUSED_BWD);
+  const bool want_acc = !(shape->flags & LMH_F_DW_ACC_GIVEN);
+  return make_plan(shape, entry, fused, want_acc).total;
+}
+
+extern "C" lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,
+                                   const int32_t* labels, float* loss_rows, float* lse,
+                                   float* logprob, int32_t* argmax, float* loss_mean,
+                                   int32_t* n_valid, const int32_t* n_valid_given, lmh_bf16* dH,
+                                   lmh_bf16* dW, float* dW_acc, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (!shape_ok(shape)) return LMH_ERR_INVALID_ARG;
+  const bool fused = dH || dW || dW_acc;
+  const Plan P = make_plan(shape, LMH_ENTRY_LOSS_FWD, fused, dW && !dW_acc);
+  int dev, sms;
+  LMH_TRY(common_checks(shape, H, W, workspace, workspace_bytes, P.total, &dev, &sms));
+  if (P.N > 0 && (!labels || !loss_rows || !lse)) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(dH) || !aligned16(dW) || !aligned16(dW_acc)) return LMH_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return empty_call(P, loss_mean, n_valid, dW, dW_acc, st);
+  LMH_TRY(count_labels(P, labels, ws, st));
+  const int mean = (shape->flags & LMH_F_MEAN) ? 1 : 0;
+  Targets tg{};
+  tg.labels = labels;
+  tg.K = 1;
+  for (int64_t ci = 0; ci < P.nchunks; ++ci) {
+    const int64_t r0 = ci * P.c;
+    const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
+    if (fused) {
+      LMH_TRY((run_stats<kLabel, true>(P, dev, sms, H, W, tg, r0, rows, ws, st)));
+    } else {
+      LMH_TRY((run_stats<kLabel, false>(P, dev, sms, H, W, tg, r0, rows, ws, st)));
+    }
+    LMH_TRY(run_finalize(P, 0, r0, rows, labels, lse, loss_rows, logprob, argmax, fused ? 1 : 0,
+                         mean, n_valid_given, ws, st));
+    if (fused) {
+      __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
+      const int64_t nv = P.Vp / 8;
+      const int64_t bx = cdiv(nv, 256);
+      dim3 grid(static_cast<unsigned>(bx < 64 ? bx : 64),
+                static_cast<unsigned>(rows < 65535 ? rows : 65535));
+      {
+        ProfScope ps(KID_GBUILD, st);
+        gbuild_kernel<<<grid, 256, 0, st>>>(rows, P.Vp, static_cast<int>(P.T),
+                                            ws.at<float>(P.o_ps), G);
+      }
+      LMH_TRY(last_launch());
+      {
+        ProfScope ps(KID_FIX_LABELS, st);
+        fix_labels_kernel<<<static_cast<unsigned>(cdiv(rows, 256)), 256, 0, st>>>(
+            rows, r0, static_cast<int>(P.V), P.Vp, labels, ws.at<float>(P.o_zt), lse, mean,
+            n_valid_given, ws.h, G);
+      }
+      LMH_TRY(last_launch());
+      LMH_TRY(run_backward_gemms(P, dev, sms, H, W, r0, rows, static_cast<int>(ci), dH, dW,
+                                 dW_acc, ws, st));
+    }
+  }
+  if (loss_mean) {
+    ProfScope ps(KID_MEAN, st);
+    mean_kernel<<<1, 1024, 0, st>>>(loss_rows, P.N, 1, n_valid_given, ws.h, loss_mean);
+    LMH_TRY(last_launch());
+  }
+  if (n_valid &&
+      cudaMemcpyAsync(n_valid, &ws.h->n_valid, 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return LMH_ERR_CUDA;
+  return LMH_OK;
+}
+
+extern "C" lmh_status lmh_logprob(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,
+                                  const int32_t* labels, float* logprob, float* lse,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!shape_ok(shape)) return LMH_ERR_INVALID_ARG;
+  const Plan P = make_plan(shape, LMH_ENTRY_LOGPROB, false, false);
+  int dev, sms;
+  LMH_TRY(common_checks(shape, H, W, workspace, workspace_bytes, P.total, &dev, &sms));
+  if (P.N > 0 && (!labels || !logprob || !lse)) return LMH_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return LMH_OK;
+  LMH_TRY(count_labels(P, labels, ws, st));
+  Targets tg{};
+  tg.labels = labels;
+  tg.K = 1;
+  for (int64_t ci = 0; ci < P.nchunks; ++ci) {
+    const int64_t r0 = ci * P.c;
+    const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
+    LMH_TRY((run_stats<kLabel, false>(P, dev, sms, H, W, tg, r0, rows, ws, st)));
+    LMH_TRY(run_finalize(P, 1, r0, rows, labels, lse, nullptr, logprob, nullptr, 0, 0, nullptr,
+                         ws, st));
+  }
+  return LMH_OK;
+}
+
+static lmh_status support_fwd(const lmh_shape* shape, int entry, const lmh_bf16* H,
+                              const lmh_bf16* W, const int32_t* ids, const float* ref,
+                              float* lp, float* kl_rows, float* kl_mean, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  if (!shape_ok(shape) || shape->K < 1 || shape->K > LMH_MAX_K) return LMH_ERR_INVALID_ARG;
+  const Plan P = make_plan(shape, entry, false, false);
+  int dev, sms;
+  LMH_TRY(common_checks(shape, H, W, workspace, workspace_bytes, P.total, &dev, &sms));
+  if (P.N > 0 && (!ids || !lse)) return LMH_ERR_INVALID_ARG;
+  if (entry == LMH_ENTRY_SUPPORT_LOGPROB && P.N > 0 && !lp) return LMH_ERR_INVALID_ARG;
+  if (entry == LMH_ENTRY_SUPPORT_KL && P.N > 0 && (!ref || !kl_rows)) return LMH_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) {
+    if (kl_mean && cudaMemsetAsync(kl_mean, 0, 4, st) != cudaSuccess) return LMH_ERR_CUDA;
+    return LMH_OK;
+  }
+  LMH_TRY(prep_cands(P, ids, ws, st));
+  Targets tg{};
+  tg.sorted = ws.at<int32_t>(P.o_sorted);
+  tg.nuniq = ws.at<int32_t>(P.o_nuniq);
+  tg.K = static_cast<int>(P.K);
+  for (int64_t ci = 0; ci < P.nchunks; ++ci) {
+    const int64_t r0 = ci * P.c;
+    const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
+    LMH_TRY((run_stats<kCands, false>(P, dev, sms, H, W, tg, r0, rows, ws, st)));
+    LMH_TRY(run_finalize(P, 2, r0, rows, nullptr, lse, nullptr, nullptr, nullptr, 0, 0, nullptr,
+                         ws, st));
+  }
+  {
+    ProfScope ps(KID_SUPPORT_OUT, st);
+    support_out_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
+      P.N, static_cast<int>(P.K), ws.at<int32_t>(P.o_rank), ws.at<float>(P.o_zt), lse,
+      entry == LMH_ENTRY_SUPPORT_KL ? ref : nullptr, lp,
+      entry == LMH_ENTRY_SUPPORT_KL ? kl_rows : nullptr);
+  }
+  LMH_TRY(last_launch());
+  if (entry == LMH_ENTRY_SUPPORT_KL && kl_mean) {
+    ProfScope ps(KID_MEAN, st);
+    mean_kernel<<<1, 1024, 0, st>>>(kl_rows, P.N, 0, nullptr, ws.h, kl_mean);
+    LMH_TRY(last_launch());
+  }
+  return LMH_OK;
+}
+
+extern "C" lmh_status lmh_support_logprob(const lmh_shape* shape, const lmh_bf16* H,
+                                          const lmh_bf16* W, const int32_t* ids, float* lp,
+                                          float* lse, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  return support_fwd(shape, LMH_ENTRY_SUPPORT_LOGPROB, H, W, ids, nullptr, lp, nullptr, nullptr,
+                     lse, workspace, workspace_bytes, stream);
+}
+
+extern "C" lmh_status lmh_support_kl(const lmh_shape* shape, const lmh_bf16* H,
+                                     const lmh_bf16* W, const int32_t* ids,
+                                     const float* ref_logp, float* kl_rows, float* kl_mean,
+                                     float* lp, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  return support_fwd(shape, LMH_ENTRY_SUPPORT_KL, H, W, ids, ref_logp, lp, kl_rows, kl_mean, lse,
+                     workspace, workspace_bytes, stream);
+}
+
+extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,
+                                   const lmh_bf16* W, const int32_t* targets, const float* lse,
+                                   const float* grad, const float* ref_logp, lmh_bf16* dH,
+                                   lmh_bf16* dW, float* dW_acc, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (!shape_ok(shape) || mode < LMH_BWD_CE || mode > LMH_BWD_SUPPORT_KL)
+    return LMH_ERR_INVALID_ARG;
+  const bool cands = mode >= LMH_BWD_SUPPORT_LOGPROB;
+  if (cands && (shape->K < 1 || shape->K > LMH_MAX_K)) return LMH_ERR_INVALID_ARG;
+  const Plan P = make_plan(shape, LMH_ENTRY_LOSS_BWD, true, dW && !dW_acc);
+  int dev, sms;
+  LMH_TRY(common_checks(shape, H, W, workspace, workspace_bytes, P.total, &dev, &sms));
+  if (P.N > 0 && (!targets || !lse || !grad)) return LMH_ERR_INVALID_ARG;
+  if (mode == LMH_BWD_SUPPORT_KL && P.N > 0 && !ref_logp) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(dH) || !aligned16(dW) || !aligned16(dW_acc)) return LMH_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return empty_call(P, nullptr, nullptr, dW, dW_acc, st);
+  if (!dH && !dW && !dW_acc) return LMH_OK;
+  Targets tg{};
+  if (cands) {
+    LMH_TRY(prep_cands(P, targets, ws, st));
+    tg.sorted = ws.at<int32_t>(P.o_sorted);
+    tg.nuniq = ws.at<int32_t>(P.o_nuniq);
+    tg.K = static_cast<int>(P.K);
+  } else {
+    LMH_TRY(count_labels(P, targets, ws, st));
+    tg.labels = targets;
+    tg.K = 1;
+  }
+  float* alpha = ws.at<float>(P.o_alpha);
+  float* beta = ws.at<float>(P.o_beta);
+  {
+    ProfScope ps(KID_BWD_COEF, st);
+    bwd_coef_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
+      mode, P.N, cands ? static_cast<int>(P.K) : 1, static_cast<int>(P.V), targets, grad,
+      ref_logp, cands ? ws.at<int32_t>(P.o_rank) : nullptr,
+      cands ? ws.at<int32_t>(P.o_nuniq) : nullptr, alpha, beta);
+  }
+  LMH_TRY(last_launch());
+  for (int64_t ci = 0; ci < P.nchunks; ++ci) {
+    const int64_t r0 = ci * P.c;
+    const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
+    CUtensorMap ta, tb;
+    if (!tmap_2d(&ta, H + r0 * P.d, P.d, rows, P.d, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BN))
+      return LMH_ERR_CUDA;
+    if (cands) {
+      EpiGrad<kCands>::Params ep{rows, r0, static_cast<int>(P.V), P.Vp, tg, lse, alpha, beta,
+                                 ws.at<__nv_bfloat16>(P.o_gbuf)};
+      LMH_TRY(launch_gemm<EpiGrad<kCands>>(dev, sms, ta, tb, rows, P.V, P.d, 0, &ws.h->err, ep,
+                                           st));
+    } else {
+      EpiGrad<kLabel>::Params ep{rows, r0, static_cast<int>(P.V), P.Vp, tg, lse, alpha, beta,
+                                 ws.at<__nv_bfloat16>(P.o_gbuf)};
+      LMH_TRY(launch_gemm<EpiGrad<kLabel>>(dev, sms, ta, tb, rows, P.V, P.d, 0, &ws.h->err, ep,
+                                           st));
+    }
+    LMH_TRY(run_backward_gemms(P, dev, sms, H, W, r0, rows, static_cast<int>(ci), dH, dW, dW_acc,
+                               ws, st));
+  }
+  return LMH_OK;
+}
+
+extern "C" lmh_status lmh_read_errors(const void* workspace, uint32_t* errors, void* stream) {
+  if (!workspace || !errors) return LMH_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LMH_ERR_CUDA;
+  if (cudaMemcpy(errors, workspace, 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LMH_ERR_CUDA;
+  return LMH_OK;
+}
+
+extern "C" lmh_status lmh_profile_enable(int on) {
+  g_prof_on.store(on != 0);
+  return LMH_OK;
+}
+
+extern "C" int lmh_profile_read(int max_records, int32_t* kernel_ids, float* ms) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  int n = 0;
+  for (const ProfRec& r : g_prof_recs) {
+    if (n < max_records && kernel_ids && ms) {
+      float t = -1.f;
+      if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+        t = -1.f;
+      kernel_ids[n] = r.id;
+      ms[n] = t;
+      ++n;
+    }
+    g_prof_pool.push_back(r.a);
+    g_prof_pool.push_back(r.b);
+  }
+  g_prof_recs.clear();
+  return n;
+}
+
+extern "C" const char* lmh_kernel_name(int kernel_id) {
+  return (kernel_id >= 0 && kernel_id < KID_COUNT) ? kKernelNames[kernel_id] : "";
+}

@@ -1,0 +1,221 @@
+"""GPU parity of every entry against the fp64 oracle, element by element, at sizes that span
+several tiles with ragged row, vocabulary and hidden tails. Calls go through the C ABI."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import lm_head_cross_tcgen05_b200 as L
+from tests.gpu_common import O, check_argmax, check_ce_fused, check_grad, check_rows, device_inputs, digest
+from tests.parity import rejects
+from workloads import WORKLOADS, ragged
+
+pytestmark = pytest.mark.gpu
+
+# (N, d, V, ignored rows): tiles of 128 rows x 256 words, K blocks of 64
+SHAPES = [
+    (64, 256, 2048, 8),     # the tiny workload's shape
+    (300, 192, 1000, 5),    # ragged rows (128+128+44), d not a multiple of 256, V tail of 232
+    (129, 64, 257, 3),      # one K block, V one past a tile, padded row stride
+    (200, 512, 4100, 20),   # V = 4100: row stride 4104, 17 vocabulary tiles
+    (1, 128, 300, 0),       # a single row
+    (130, 128, 100, 0),     # V smaller than one tile
+]
+
+
+def _wl(N, d, V, ign, **kw):
+    return ragged(N, d, V, n_ignored=ign, seed=1000 + N + d + V, **kw)
+
+
+@pytest.mark.parametrize("N,d,V,ign", SHAPES)
+@pytest.mark.parametrize("chunk", [0, 128, 100])
+def test_fused_ce(N, d, V, ign, chunk):
+    x, xc = device_inputs(_wl(N, d, V, ign))
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=chunk, grads=True)
+    torch.cuda.synchronize()
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
+    check_ce_fused(out, ref)
+
+
+def test_tiny_workload_and_gates_reject_scaled_output():
+    x, xc = device_inputs(WORKLOADS["tiny"])
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
+    check_ce_fused(out, ref)
+    assert int(out["n_valid"].item()) == 56
+    # the gates fail an output 2 % off
+    assert rejects(check_grad, out["dW"].float() * 1.02, ref["dW"])
+    assert rejects(check_grad, out["dH"].float() * 1.02, ref["dH"])
+    assert rejects(check_rows, out["loss_rows"] * 1.02, ref["loss_rows"])
+
+
+@pytest.mark.parametrize("N,d,V,ign", SHAPES[:4])
+def test_forward_only_matches_fused_bits(N, d, V, ign):
+    x, _ = device_inputs(_wl(N, d, V, ign))
+    a = L.loss_fwd(x["H"], x["W"], x["labels"], grads=False)
+    b = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    for k in ("loss_rows", "lse", "logprob", "argmax", "loss_mean", "n_valid"):
+        assert torch.equal(a[k], b[k]), k
+
+
+@pytest.mark.parametrize("N,d,V,ign", SHAPES[:4])
+def test_logprob_entry(N, d, V, ign):
+    x, xc = device_inputs(_wl(N, d, V, ign))
+    out = L.logprob(x["H"], x["W"], x["labels"], chunk_rows=100)
+    ref = O.logprob_forward(xc["H"], xc["W"], xc["labels"])
+    check_rows(out["logprob"], ref["logprob"], what="logprob")
+    check_rows(out["lse"], ref["lse"], what="lse")
+
+
+def _support_inputs(N, d, V, K, seed):
+    wl = ragged(N, d, V, K=K, seed=seed)
+    x, xc = device_inputs(wl)
+    ids = xc["ids"].clone()
+    if K >= 4:
+        # a repeated id and padding slots exercise de-duplication and skipping
+        ids[0, 1] = ids[0, 0]
+        ids[1, -1] = -1
+        ids[2, 3] = -7
+    x["ids"] = ids.cuda()
+    xc["ids"] = ids
+    return x, xc
+
+
+@pytest.mark.parametrize("N,d,V,K", [(200, 128, 3000, 16), (130, 64, 700, 64), (64, 256, 2048, 1)])
+def test_support_logprob_and_kl(N, d, V, K):
+    x, xc = _support_inputs(N, d, V, K, 77 + K)
+    ref = O.support_kl(xc["H"], xc["W"], xc["ids"], xc["ref_logp"])
+    a = L.support_logprob(x["H"], x["W"], x["ids"], chunk_rows=128)
+    check_rows(a["lp"], ref["lp"], what="lp")
+    check_rows(a["lse"], ref["lse"], what="lse")
+    b = L.support_kl(x["H"], x["W"], x["ids"], x["ref_logp"], chunk_rows=0)
+    check_rows(b["kl_rows"], ref["kl_rows"], what="kl_rows")
+    check_rows(b["kl_mean"], np.array([ref["kl_mean"]]), what="kl_mean")
+    check_rows(b["lp"], ref["lp"], what="lp(kl)")
+    assert torch.equal(a["lp"], b["lp"])
+
+
+@pytest.mark.parametrize("mode", [L.BWD_CE, L.BWD_LOGPROB, L.BWD_SUPPORT_LOGPROB, L.BWD_SUPPORT_KL])
+@pytest.mark.parametrize("chunk", [0, 96])
+def test_loss_bwd_modes(mode, chunk):
+    N, d, V, K = 260, 192, 1500, 12
+    x, xc = _support_inputs(N, d, V, K, 300 + mode)
+    g = torch.Generator().manual_seed(5 + mode)
+    if mode in (L.BWD_CE, L.BWD_LOGPROB):
+        targets, tc = x["labels"], xc["labels"]
+        grad = torch.randn(N, generator=g) / N
+        lse = L.logprob(x["H"], x["W"], x["labels"])["lse"]
+    else:
+        targets, tc = x["ids"], xc["ids"]
+        grad = (torch.randn(N, K, generator=g) / N) if mode == L.BWD_SUPPORT_LOGPROB else (
+            torch.rand(N, generator=g) / N)
+        lse = L.support_logprob(x["H"], x["W"], x["ids"])["lse"]
+    ref_lp = x["ref_logp"] if mode == L.BWD_SUPPORT_KL else None
+    out = L.loss_bwd(mode, x["H"], x["W"], targets, lse, grad.cuda(), ref_lp, chunk_rows=chunk)
+    ref = O.backward(mode, xc["H"], xc["W"], tc, grad,
+                     xc["ref_logp"] if mode == L.BWD_SUPPORT_KL else None)
+    check_grad(out["dH"], ref["dH"], "dH")
+    check_grad(out["dW"], ref["dW"], "dW")
+
+
+def test_fused_equals_standalone_backward_within_tolerance():
+    x, xc = device_inputs(_wl(300, 192, 1000, 5))
+    f = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    n = int(f["n_valid"].item())
+    grad = torch.full((300,), 1.0 / n, device="cuda")
+    b = L.loss_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], f["lse"], grad)
+    check_grad(b["dH"], f["dH"].float().cpu().double().numpy(), "dH")
+    check_grad(b["dW"], f["dW"].float().cpu().double().numpy(), "dW")
+
+
+def test_determinism_ten_runs():
+    x, _ = device_inputs(_wl(520, 256, 5000, 9))
+    ref = None
+    for _ in range(10):
+        o = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=200, grads=True)
+        h = digest(o["loss_rows"], o["lse"], o["logprob"], o["argmax"], o["loss_mean"], o["dH"],
+                   o["dW"])
+        ref = ref or h
+        assert h == ref
+
+
+def test_chunk_plan_changes_only_dW_bits():
+    x, xc = device_inputs(_wl(300, 128, 1000, 4))
+    base = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
+    for c in (128, 100, 37, 1):
+        o = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=c, grads=True)
+        for k in ("loss_rows", "lse", "logprob", "argmax", "dH"):
+            assert torch.equal(o[k], base[k]), (c, k)
+        check_grad(o["dW"], ref["dW"], f"dW chunk {c}")
+
+
+def test_dW_is_bf16_cast_of_fp32_accumulator():
+    x, xc = device_inputs(_wl(300, 128, 1000, 4))
+    acc = torch.zeros(1000, 128, dtype=torch.float32, device="cuda")
+    o = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=128, grads=True, dW_acc=acc)
+    assert torch.equal(o["dW"], acc.to(torch.bfloat16))
+    ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
+    check_grad(acc, ref["dW"], "dW_acc")
+    # a second call accumulates on top, in the same fixed order
+    acc2 = acc.clone()
+    o2 = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=128, grads=True, dW_acc=acc2)
+    check_grad(acc2, 2 * ref["dW"], "dW_acc twice")
+    assert torch.equal(o2["dW"], acc2.to(torch.bfloat16))
+    # internal accumulator (no dW_acc given) gives the same bits as a zeroed external one
+    o3 = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=128, grads=True)
+    assert torch.equal(o3["dW"], o["dW"])
+
+
+def test_no_valid_rows_and_empty_call():
+    x, xc = device_inputs(_wl(140, 64, 500, 0))
+    y = torch.full_like(x["labels"], -100)
+    y[3] = -1
+    o = L.loss_fwd(x["H"], x["W"], y, grads=True)
+    assert int(o["n_valid"].item()) == 0 and float(o["loss_mean"].item()) == 0.0
+    assert torch.count_nonzero(o["dH"]) == 0 and torch.count_nonzero(o["dW"]) == 0
+    assert torch.count_nonzero(o["loss_rows"]) == 0
+    ref = O.ce_forward(xc["H"], xc["W"], y.cpu())
+    check_rows(o["lse"], ref["lse"], what="lse")
+    e = L.loss_fwd(x["H"][:0], x["W"], y[:0], grads=True)
+    assert int(e["n_valid"].item()) == 0 and torch.count_nonzero(e["dW"]) == 0
+
+
+def test_label_out_of_range_sets_error_word():
+    x, xc = device_inputs(_wl(100, 64, 300, 0))
+    y = x["labels"].clone()
+    y[7] = 300
+    y[9] = 10 ** 6
+    o = L.loss_fwd(x["H"], x["W"], y, grads=True)
+    assert L.lmh_read_errors(o["workspace"]) & L.DEVERR_LABEL_RANGE
+    ref = O.ce_fused(xc["H"], xc["W"], y.cpu())
+    check_ce_fused(o, ref)
+    ok = L.loss_fwd(x["H"], x["W"], x["labels"], ws=o["workspace"])
+    assert L.lmh_read_errors(ok["workspace"]) == 0
+
+
+def test_side_stream_same_bits():
+    x, _ = device_inputs(_wl(300, 192, 1000, 5))
+    a = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        b = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True, stream=s)
+    s.synchronize()
+    assert digest(a["dW"], a["dH"], a["lse"]) == digest(b["dW"], b["dH"], b["lse"])
+
+
+def test_host_rejections():
+    x, _ = device_inputs(_wl(64, 64, 300, 0))
+    shape = L.make_shape(64, 64, 300)
+    ws = L.workspace(shape, L.ENTRY_LOSS_FWD, "cuda")
+    lr, lse = torch.empty(64, device="cuda"), torch.empty(64, device="cuda")
+    with pytest.raises(L.LmhError, match="WORKSPACE_TOO_SMALL"):
+        L.lmh_loss_fwd(shape, x["H"], x["W"], x["labels"], lr, lse, workspace=ws[:100])
+    bad = L.make_shape(64, 96, 300)
+    with pytest.raises(L.LmhError, match="INVALID_ARG"):
+        L.lmh_loss_fwd(bad, x["H"], x["W"], x["labels"], lr, lse, workspace=ws)
+    with pytest.raises(L.LmhError, match="ALIGNMENT"):
+        L.lmh_loss_fwd(shape, x["H"], x["W"], x["labels"], lr, lse, workspace=ws[8:])
