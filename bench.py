@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Throughput of the fused LM-head + cross-entropy forward+backward on B200.
+
+One step = one call of lmh_loss_fwd with dH and dW requested on the large-vocabulary
+workload (N = 8192 rows, d = 4096, V = 128256, Zipf(1.1) labels, 3 % ignored rows): the
+logits GEMM with its online-LSE epilogue, the row finalize, the softmax-gradient rescale, and
+the dH and dW GEMMs, over one chunk of all rows. TFLOP/s counts 6 N V d per step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With --gpus N > 1 (under torch.distributed.run, one process per GPU) every rank runs its
+own replica on its own seeded batch (weak scaling, no collective on the data path); the
+time is the maximum over ranks. --impl reference times the fp64 CPU oracle instead, on a
+bounded sample of the same workload, on the host cores. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LM-head+CE fwd+bwd TFLOP/s (6·N·V·d) and % of bf16 tensor peak, 1×B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["lm_head_cross_tcgen05_b200/csrc/gemm.cuh",
+                  "lm_head_cross_tcgen05_b200/csrc/epilogues.cuh",
+                  "lm_head_cross_tcgen05_b200/csrc/sm100.cuh",
+                  "lm_head_cross_tcgen05_b200/csrc/rowops.cuh",
+                  "lm_head_cross_tcgen05_b200/csrc/lmh_api.cu"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="large_vocab")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def workload_config(wl, chunk_rows, n_gpus):
+    return {"workload": f"{wl.name}: fused CE forward+backward, N={wl.N} d={wl.d} V={wl.V}, "
+                        f"{wl.labels} labels, {wl.num_ignored} ignored rows, bf16 H/W",
+            "N": wl.N, "d": wl.d, "V": wl.V, "chunk_rows": chunk_rows,
+            "rows_per_gpu": wl.N, "total_rows": wl.N * n_gpus,
+            "l2": "inputs larger than L2 (W alone is %.2f GB)" % (wl.V * wl.d * 2 / 1e9)}
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def replica_seed(wl, rank: int) -> int:
+    """Each rank's replica draws its own batch (weak scaling: rows per GPU are fixed)."""
+    return wl.seed + 1000 * rank
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Maximum of a per-rank value over all ranks (the job time is the slowest rank's)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's step time."""
+    return flops_per_rank_step * world / (ms_per_step / 1e3) / 1e12
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, f[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_id_for_smi(torch, dev) -> str:
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        return vis.split(",")[dev] if vis else str(dev)
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def oracle_sample(wl, target_s: float):
+    """Times the fp64 oracle's fused forward+backward on the first n rows of the workload
+    (full V and d), with n chosen so that the run takes about target_s seconds."""
+    import threadpoolctl
+
+    from oracle import lmh_oracle as O
+    from workloads import make_inputs
+    x = make_inputs(wl.scaled(N=min(wl.N, 4096)), device="cpu")
+
+    def run(n):
+        t = time.perf_counter()
+        O.ce_fused(x["H"][:n], x["W"], x["labels"][:n])
+        return time.perf_counter() - t
+
+    # t(n) = a + b n: a is the per-call fp64 widening of W, b the per-row work
+    t8, t40 = run(8), run(40)
+    b = max((t40 - t8) / 32.0, 1e-6)
+    a = max(t8 - 8 * b, 0.0)
+    n = int(max(8, min(1024, (target_s - a) / b)))
+    t = run(n)
+    info = threadpoolctl.threadpool_info()
+    cores = max([i.get("num_threads", 1) for i in info] + [1])
+    return n, t, cores
+
+
+def run_reference(args, wl, n_gpus):
+    """The oracle as it stands, on the host cores, steps of a bounded sample."""
+    import threadpoolctl
+
+    from oracle import lmh_oracle as O
+    from workloads import make_inputs
+    x = make_inputs(wl.scaled(N=min(wl.N, 4096)), device="cpu")
+    budget = 150.0 / max(1, args.steps + args.warmup)       # seconds per step
+
+    def run(n):
+        t = time.perf_counter()
+        O.ce_fused(x["H"][:n], x["W"], x["labels"][:n])
+        return time.perf_counter() - t
+
+    t4, t20 = run(4), run(20)
+    b = max((t20 - t4) / 16.0, 1e-6)
+    a = max(t4 - 4 * b, 0.0)
+    n = int(max(4, min(1024, (budget - a) / b)))
+    for _ in range(args.warmup):
+        O.ce_fused(x["H"][:n], x["W"], x["labels"][:n])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.ce_fused(x["H"][:n], x["W"], x["labels"][:n])
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    value = 6.0 * n * wl.V * wl.d / dt / 1e12
+    cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+    sample = (f"first {n} rows of {wl.name} (full V={wl.V}, d={wl.d}) per step, "
+              f"fp64 numpy oracle ce_fused (forward, dH, dW)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": n_gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl, wl.N, 1),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from workloads import WORKLOADS, make_inputs
+    wl = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, wl, world)
+        return
+
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import lm_head_cross_tcgen05_b200 as L
+    from lm_head_cross_tcgen05_b200._abi import lib
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        return reduce_max(v, world, dev)
+
+    x = make_inputs(wl, device=dev, seed=replica_seed(wl, rank))
+    H, W, y = x["H"], x["W"], x["labels"]
+    N, d, V = wl.N, wl.d, wl.V
+    chunk = wl.chunk_rows or N
+    shape = L.make_shape(N, d, V, 0, chunk, L.F_MEAN | L.F_FUSED_BWD)
+    ws = L.workspace(shape, L.ENTRY_LOSS_FWD, dev)
+    f32, i32, bf = torch.float32, torch.int32, torch.bfloat16
+    out = dict(loss_rows=torch.empty(N, dtype=f32, device=dev),
+               lse=torch.empty(N, dtype=f32, device=dev),
+               logprob=torch.empty(N, dtype=f32, device=dev),
+               argmax=torch.empty(N, dtype=i32, device=dev),
+               loss_mean=torch.empty(1, dtype=f32, device=dev),
+               n_valid=torch.empty(1, dtype=i32, device=dev),
+               dH=torch.empty(N, d, dtype=bf, device=dev),
+               dW=torch.empty(V, d, dtype=bf, device=dev))
+    stream = torch.cuda.current_stream()
+
+    def step(Hs=H, ys=y):
+        L.lmh_loss_fwd(shape, Hs, W, ys, out["loss_rows"], out["lse"], out["logprob"],
+                       out["argmax"], out["loss_mean"], out["n_valid"], None, out["dH"],
+                       out["dW"], None, workspace=ws, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    barrier()
+
+    sampler = ClockSampler(gpu_id_for_smi(torch, local))
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lib().lmh_profile_enable(1)
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    lib().lmh_profile_enable(0)
+    clocks = sampler.stop()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_step = ms_total / args.steps
+    flops_step = 6.0 * N * V * d
+    value = job_tflops(flops_step, world, ms_step)
+
+    # per-kernel device times of the timed region (event pairs on the launching stream)
+    import ctypes
+    cap = 64 * args.steps + 64
+    ids = (ctypes.c_int32 * cap)()
+    mss = (ctypes.c_float * cap)()
+    n_rec = lib().lmh_profile_read(cap, ids, mss)
+    per = {}
+    for i in range(n_rec):
+        name = lib().lmh_kernel_name(ids[i]).decode()
+        c, t = per.get(name, (0, 0.0))
+        per[name] = (c + 1, t + mss[i])
+    kernels = {k: {"launches": c, "total_ms": t, "avg_ms": t / c,
+                   "share": t / max(1e-9, sum(v[1] for v in per.values()))}
+               for k, (c, t) in sorted(per.items(), key=lambda kv: -kv[1][1])}
+    dom = next(iter(kernels)) if kernels else None
+    peaks, peak_src = load_peaks()
+    roofline = None
+    if dom:
+        gemm_flops = 2.0 * chunk * V * d      # one GEMM launch over one chunk
+        hbm_bytes = {"gbuild": 4.0 * chunk * ((V + 7) // 8 * 8)}
+        if dom.startswith("gemm"):
+            ach = gemm_flops / (kernels[dom]["avg_ms"] / 1e3) / 1e12
+            pk = peaks["bf16_tflops_sustained"]
+            roofline = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": pk,
+                        "unit": "TFLOP/s", "frac": ach / pk,
+                        "peak_kind": f"bf16 dense, sustained, of {peak_src}",
+                        "algorithmic_per_launch": gemm_flops}
+        else:
+            b = hbm_bytes.get(dom, 0.0)
+            ach = b / (kernels[dom]["avg_ms"] / 1e3) / 1e9
+            pk = peaks["hbm_gbs"]
+            roofline = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": pk,
+                        "unit": "GB/s", "frac": ach / pk, "peak_kind": f"copy, of {peak_src}",
+                        "algorithmic_per_launch": b}
+        roofline["traffic"] = None
+        tpath = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(tpath):
+            with open(tpath) as fh:
+                tr = json.load(fh)
+            ent = tr.get(dom)
+            if ent and ent.get("source_hash") == source_hash():
+                roofline["traffic"] = ent["bytes_per_launch"]
+
+    # end to end through the public API: pinned host batch in, loss out, every step
+    e2e = None
+    if not args.no_e2e:
+        Hh = H.cpu().pin_memory()
+        yh = y.cpu().pin_memory()
+        Hd, yd = torch.empty_like(H), torch.empty_like(y)
+        loss_h = torch.empty(1, dtype=f32).pin_memory()
+        nv_h = torch.empty(1, dtype=i32).pin_memory()
+
+        def e2e_step():
+            Hd.copy_(Hh, non_blocking=True)
+            yd.copy_(yh, non_blocking=True)
+            step(Hd, yd)
+            loss_h.copy_(out["loss_mean"], non_blocking=True)
+            nv_h.copy_(out["n_valid"], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+        e2e = {"value": job_tflops(flops_step, world, ms_e2e), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": Hh.numel() * 2 + yh.numel() * 4,
+               "d2h_bytes_per_step": 8, "ms_per_step": ms_e2e,
+               "note": "H and labels copied in from pinned host memory and the mean loss and "
+                       "valid count read back every step; W stays resident as model state"}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, t, cores = oracle_sample(wl, args.cpu_seconds)
+        cpu_baseline = {"value": 6.0 * n * V * d / t / 1e12, "unit": "TFLOP/s", "cores": cores,
+                        "kind": "oracle",
+                        "sample": f"first {n} rows of {wl.name} (full V={V}, d={d}): fp64 "
+                                  f"numpy oracle ce_fused (forward, dH, dW), {t:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": workload_config(wl, chunk, world),
+                "peak_frac": {"of_burst": value / world / peaks["bf16_tflops"],
+                              "of_sustained": value / world / peaks["bf16_tflops_sustained"],
+                              "peaks": peak_src},
+                "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
+                "gpu_launches": n_rec, "kernels": kernels, "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

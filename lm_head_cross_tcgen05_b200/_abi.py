@@ -38,13 +38,17 @@ _SIGS = {
     "lmh_support_logprob": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6 + [c_size_t, _P]),
     "lmh_support_kl": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 9 + [c_size_t, _P]),
     "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),
+    "lmh_profile_enable": (c_int, [c_int]),
+    "lmh_profile_read": (c_int, [c_int, ctypes.POINTER(ctypes.c_int32),
+                                 ctypes.POINTER(ctypes.c_float)]),
+    "lmh_kernel_name": (ctypes.c_char_p, [c_int]),
 }
 
 
 def header_symbols(path: str = HEADER):
     """Names of the functions include/lmh.h declares."""
     src = open(path).read()
-    return re.findall(r"^LMH_API\s+\w+\s+(lmh_\w+)\s*\(", src, flags=re.M)
+    return re.findall(r"^LMH_API\s+[\w\s\*]*?\b(lmh_\w+)\s*\(", src, flags=re.M)
 
 
 _lib = None

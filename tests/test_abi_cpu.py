@@ -1,0 +1,77 @@
+"""The C ABI without a GPU: every symbol include/lmh.h declares is exported by liblmh.so, the
+workspace planner follows its documented rules, and argument errors are reported on the host
+before any CUDA call."""
+import ctypes
+
+import pytest
+
+from lm_head_cross_tcgen05_b200 import _abi
+import lm_head_cross_tcgen05_b200 as L
+
+
+def test_header_symbols_exported():
+    names = _abi.header_symbols()
+    assert {"lmh_workspace_size", "lmh_loss_fwd", "lmh_loss_bwd", "lmh_logprob",
+            "lmh_support_logprob", "lmh_support_kl", "lmh_read_errors"} <= set(names)
+    lib = ctypes.CDLL(_abi.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def ws(N, d, V, K=0, chunk=0, flags=0, entry=L.ENTRY_LOSS_FWD):
+    return L.lmh_workspace_size(L.make_shape(N, d, V, K, chunk, flags), entry)
+
+
+def test_invalid_shapes_size_zero():
+    assert ws(10, 96, 100) == 0           # d not a multiple of 64
+    assert ws(-1, 64, 100) == 0
+    assert ws(10, 64, 0) == 0
+    assert ws(10, 64, 100, K=0, entry=L.ENTRY_SUPPORT_KL) == 0
+    assert ws(10, 64, 100, K=L.MAX_K + 1, entry=L.ENTRY_SUPPORT_LOGPROB) == 0
+    assert ws(10, 64, 100, entry=7) == 0
+
+
+def test_chunk_buffer_term():
+    N, d, V = 8192, 4096, 128256
+    base = ws(N, d, V, chunk=N)
+    fused = ws(N, d, V, chunk=N, flags=L.F_FUSED_BWD)
+    # the fused forward adds one chunk's bf16 softmax buffer [c, round_up(V, 8)]
+    assert fused - base == pytest.approx(N * 128256 * 2, abs=256)
+    # one chunk: no internal dW accumulator
+    assert ws(N, d, V, chunk=N, flags=L.F_FUSED_BWD | L.F_DW_ACC_GIVEN) == fused
+
+
+def test_budgeted_workload_fits_two_gigabytes():
+    N, d, V = 16384, 5120, 151936
+    b = ws(N, d, V, chunk=2048, flags=L.F_FUSED_BWD | L.F_MEAN | L.F_DW_ACC_GIVEN)
+    assert b <= 2 * 1024 ** 3
+    # without a caller accumulator the fp32 [V, d] one is added for the multi-chunk plan
+    b2 = ws(N, d, V, chunk=2048, flags=L.F_FUSED_BWD)
+    assert b2 - b == pytest.approx(V * d * 4, abs=512)
+
+
+def test_default_chunk_is_4096_rows():
+    N, d, V = 10000, 64, 1000
+    a = ws(N, d, V, chunk=0, flags=L.F_FUSED_BWD | L.F_DW_ACC_GIVEN)
+    b = ws(N, d, V, chunk=4096, flags=L.F_FUSED_BWD | L.F_DW_ACC_GIVEN)
+    assert a == b
+
+
+def test_backward_and_support_sizes():
+    assert ws(100, 64, 1000, K=8, entry=L.ENTRY_LOSS_BWD) > ws(100, 64, 1000, entry=L.ENTRY_LOGPROB)
+    assert ws(100, 64, 1000, K=8, entry=L.ENTRY_SUPPORT_KL) > 0
+    assert ws(0, 64, 1000, entry=L.ENTRY_LOSS_FWD) > 0   # header only
+
+
+def test_host_argument_errors_without_gpu():
+    lib = _abi.lib()
+    shape = L.make_shape(4, 64, 100)
+    # null H/W with N > 0: rejected on the host before any CUDA call
+    st = lib.lmh_loss_fwd(ctypes.byref(shape), *([None] * 13), ctypes.c_void_p(256), 1 << 20, None)
+    assert st == 1
+    bad = L.make_shape(4, 100, 100)
+    st = lib.lmh_logprob(ctypes.byref(bad), *([None] * 6), 0, None)
+    assert st == 1
+    st = lib.lmh_loss_bwd(ctypes.byref(shape), 9, *([None] * 10), 0, None)
+    assert st == 1
+    assert lib.lmh_read_errors(None, None, None) == 1

@@ -1,0 +1,185 @@
+"""Parity at the full sizes of the four large workloads, in the launch configuration bench.py
+uses (one chunk of all rows for large_vocab, 2048-row chunks for budgeted).
+
+Per-row outputs (loss, lse, logprob, argmax, dH rows, support lp / KL rows) are compared with
+the fp64 oracle on sampled rows, which it computes one by one. dW depends on every row's
+log-sum-exp, so at full N it is checked through properties that hold at any size (columns
+sum to zero, fused forward+backward == recompute backward, one chunk == many chunks within
+tolerance, bitwise repeats), and element by element against the oracle at full V and d on a
+128-row slice. ``LMH_FULL_ORACLE=1`` adds the complete fp64 dW of the large-vocab workload
+(row-blocked; minutes of CPU time)."""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import lm_head_cross_tcgen05_b200 as L
+from tests.gpu_common import O, check_argmax, check_grad, check_rows, digest, f64
+from workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def sample_rows(y: torch.Tensor, n: int = 12, seed: int = 0) -> np.ndarray:
+    """n rows spread over the batch, with at least one ignored row when there is one."""
+    N = y.shape[0]
+    g = np.random.default_rng(seed)
+    rows = set(g.choice(N, size=n, replace=False).tolist()) | {0, N - 1}
+    ign = torch.nonzero(y < 0).flatten().tolist()
+    if ign:
+        rows.add(ign[0])
+    return np.array(sorted(rows))
+
+
+def dev_inputs(name):
+    wl = WORKLOADS[name]
+    return wl, make_inputs(wl, device="cuda")
+
+
+def check_sampled_ce(out, x, rows, n_valid_total):
+    Hs, ys = x["H"][rows].cpu(), x["labels"][rows].cpu()
+    Wc = x["W"].cpu()
+    f = O.ce_forward(Hs, Wc, ys)
+    check_rows(out["loss_rows"][rows], f["loss_rows"], what="loss_rows")
+    check_rows(out["lse"][rows], f["lse"], what="lse")
+    check_rows(out["logprob"][rows], f["logprob"], what="logprob")
+    check_argmax(out["argmax"][rows], f["z"])
+    if out.get("dH") is not None:
+        valid = (ys.numpy() >= 0)
+        g = np.where(valid, 1.0 / n_valid_total, 0.0)
+        b = O.backward(O.BWD_CE, Hs, Wc, ys, g)
+        check_grad(out["dH"][rows], b["dH"], "dH rows")
+
+
+def check_dw_properties(dW: torch.Tensor):
+    s = dW.float().sum(0).double()                     # sum over the vocabulary
+    a = dW.float().abs().sum(0).double()
+    assert torch.all(s.abs() <= 2e-3 * a + 1e-6), float((s.abs() / (a + 1e-30)).max())
+    assert torch.isfinite(dW.float()).all()
+
+
+@pytest.fixture(scope="module")
+def large_vocab():
+    wl, x = dev_inputs("large_vocab")
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=wl.N, grads=True)
+    torch.cuda.synchronize()
+    return wl, x, out
+
+
+def test_large_vocab_sampled_rows(large_vocab):
+    wl, x, out = large_vocab
+    y = x["labels"]
+    n_valid = int(((y >= 0) & (y < wl.V)).sum())
+    assert int(out["n_valid"].item()) == n_valid == wl.N - wl.num_ignored
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    check_sampled_ce(out, x, sample_rows(y), n_valid)
+    # the mean is the fixed-order mean of the per-row losses over valid rows
+    lr = out["loss_rows"].double()
+    assert abs(float(out["loss_mean"]) - float(lr.sum() / n_valid)) < 1e-4
+
+
+def test_large_vocab_dw_properties_and_repeats(large_vocab):
+    wl, x, out = large_vocab
+    check_dw_properties(out["dW"])
+    h = digest(out["dW"], out["dH"], out["lse"], out["loss_rows"])
+    ws = out["workspace"]
+    for _ in range(9):
+        o = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=wl.N, grads=True, ws=ws)
+        assert digest(o["dW"], o["dH"], o["lse"], o["loss_rows"]) == h
+
+
+def test_large_vocab_fused_matches_recompute_and_chunking(large_vocab):
+    wl, x, out = large_vocab
+    n = int(out["n_valid"].item())
+    grad = torch.where(x["labels"] >= 0, 1.0 / n, 0.0).float()
+    b = L.loss_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], out["lse"], grad, chunk_rows=wl.N)
+    ref_dw = f64(out["dW"])
+    check_grad(b["dW"], ref_dw, "dW recompute vs fused")
+    check_grad(b["dH"], f64(out["dH"]), "dH recompute vs fused")
+    del b
+    c = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=3000, grads=True)
+    assert torch.equal(c["dH"], out["dH"]) and torch.equal(c["lse"], out["lse"])
+    check_grad(c["dW"], ref_dw, "dW 3 chunks vs 1")
+
+
+def test_full_vocab_and_hidden_dw_slice():
+    """dW element by element at V = 128256, d = 4096 on a 128-row slice."""
+    wl = WORKLOADS["large_vocab"].scaled(N=128)
+    x = make_inputs(wl, device="cuda")
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    ref = O.ce_fused(x["H"].cpu(), x["W"].cpu(), x["labels"].cpu())
+    check_grad(out["dW"], ref["dW"], "dW")
+    check_grad(out["dH"], ref["dH"], "dH")
+    check_rows(out["lse"], ref["lse"], what="lse")
+
+
+@pytest.mark.skipif(os.environ.get("LMH_FULL_ORACLE") != "1", reason="minutes of fp64 CPU work")
+def test_large_vocab_full_fp64_dw(large_vocab):
+    wl, x, out = large_vocab
+    Hc, Wc, yc = x["H"].cpu(), x["W"].cpu(), x["labels"].cpu()
+    n = int(((yc >= 0) & (yc < wl.V)).sum())
+    dW = np.zeros((wl.V, wl.d))
+    for r0 in range(0, wl.N, 512):
+        r1 = min(wl.N, r0 + 512)
+        z = O.logits(Hc[r0:r1], Wc)
+        lse = O.logsumexp_rows(z)
+        g = np.where(yc[r0:r1].numpy() >= 0, 1.0 / n, 0.0)
+        G = O.grad_logits(O.BWD_CE, z, lse, yc[r0:r1], g)
+        dW += G.T @ O.as_f64(Hc[r0:r1])
+    check_grad(out["dW"], dW, "dW full")
+
+
+def test_small_workload_full_oracle():
+    wl, x = dev_inputs("small")
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=wl.N, grads=True)
+    ref = O.ce_fused(x["H"].cpu(), x["W"].cpu(), x["labels"].cpu())
+    check_rows(out["loss_rows"], ref["loss_rows"], what="loss_rows")
+    check_rows(out["lse"], ref["lse"], what="lse")
+    check_rows(out["logprob"], ref["logprob"], what="logprob")
+    check_rows(out["loss_mean"], np.array([ref["loss_mean"]]), what="loss_mean")
+    assert int(out["n_valid"].item()) == ref["n_valid"]
+    check_argmax(out["argmax"], ref["z"])
+    check_grad(out["dH"], ref["dH"], "dH")
+    check_grad(out["dW"], ref["dW"], "dW")
+
+
+def test_budgeted_workload_chunked_with_caller_accumulator():
+    wl, x = dev_inputs("budgeted")
+    shape = L.make_shape(wl.N, wl.d, wl.V, 0, wl.chunk_rows,
+                         L.F_MEAN | L.F_FUSED_BWD | L.F_DW_ACC_GIVEN)
+    assert L.lmh_workspace_size(shape, L.ENTRY_LOSS_FWD) <= 2 * 1024 ** 3
+    acc = torch.zeros(wl.V, wl.d, dtype=torch.float32, device="cuda")
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=wl.chunk_rows, grads=True,
+                     dW_acc=acc)
+    assert torch.equal(out["dW"], acc.to(torch.bfloat16))
+    check_dw_properties(out["dW"])
+    y = x["labels"]
+    check_sampled_ce(out, x, sample_rows(y, seed=3), wl.N)
+    lp = L.logprob(x["H"], x["W"], y, chunk_rows=wl.chunk_rows)
+    assert torch.equal(lp["logprob"], out["logprob"]) and torch.equal(lp["lse"], out["lse"])
+
+
+def test_support_workload_sampled_rows():
+    wl, x = dev_inputs("support")
+    ids, ref = x["ids"], x["ref_logp"]
+    kl = L.support_kl(x["H"], x["W"], ids, ref, chunk_rows=wl.N)
+    lp = L.support_logprob(x["H"], x["W"], ids, chunk_rows=wl.N)
+    assert torch.equal(kl["lp"], lp["lp"])
+    rows = sample_rows(x["labels"], seed=5)
+    Hs, Wc = x["H"][rows].cpu(), x["W"].cpu()
+    r = O.support_kl(Hs, Wc, ids[rows].cpu(), ref[rows].cpu())
+    check_rows(kl["lp"][rows], r["lp"], what="lp")
+    check_rows(kl["kl_rows"][rows], r["kl_rows"], what="kl_rows")
+    check_rows(kl["lse"][rows], r["lse"], what="lse")
+    assert abs(float(kl["kl_mean"]) - float(kl["kl_rows"].double().mean())) < 1e-4
+    # backward of the mean KL
+    grad = torch.full((wl.N,), 1.0 / wl.N, device="cuda")
+    b = L.loss_bwd(L.BWD_SUPPORT_KL, x["H"], x["W"], ids, kl["lse"], grad, ref,
+                   chunk_rows=wl.N)
+    rb = O.backward(O.BWD_SUPPORT_KL, Hs, Wc, ids[rows].cpu(), np.full(len(rows), 1.0 / wl.N),
+                    ref[rows].cpu())
+    check_grad(b["dH"][rows], rb["dH"], "dH rows (KL)")
+    check_dw_properties(b["dW"])
