@@ -58,7 +58,8 @@ typedef enum lmh_status {
   LMH_ERR_UNSUPPORTED_DEVICE = 2,
   LMH_ERR_WORKSPACE_TOO_SMALL = 3,
   LMH_ERR_ALIGNMENT = 4,
-  LMH_ERR_CUDA = 5
+  LMH_ERR_CUDA = 5,
+  LMH_ERR_SCRATCH_LIMIT = 6
 } lmh_status;
 
 #define LMH_IGNORE_INDEX (-100)
@@ -195,6 +196,36 @@ LMH_API lmh_status lmh_support_kl(const lmh_shape* shape, const lmh_bf16* H, con
  * call that used `workspace` into *errors (host). Each entry clears the word when it starts.
  */
 LMH_API lmh_status lmh_read_errors(const void* workspace, uint32_t* errors, void* stream);
+
+/*
+ * lmh_logprob_noalloc — the same per-row target log-probability and log-sum-exp as
+ * lmh_logprob, for callers that cannot allocate device memory. The pages have no counterpart
+ * of this entry.
+ *
+ * Who needs it: code that is handed its input and output buffers but may not call
+ * cudaMalloc on the call path, so it cannot provide the workspace lmh_logprob needs. Examples
+ * are a plugin inside an inference engine that owns and pre-reserves the whole device heap,
+ * and a hot loop that must not change a memory pool's accounting.
+ *
+ * What it does instead: its scratch (error word, label logits, per-tile partials) lives in
+ * one fixed 32 MiB array inside this library, which every GPU that loads the library keeps
+ * until the process exits. The call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine. Results are bit-identical to lmh_logprob's. The rows are split
+ * into chunks small enough for the array; the chunk plan does not change any log-prob bit.
+ *   - The first call on each device looks up the array's device address (with that device
+ *     current) and caches it. Make that first call before any stream capture.
+ *   - All calls share the one array, and it keeps the last call's contents. Calls whose work
+ *     overlaps on the GPU (other streams, other host threads, the same device) race on it and
+ *     give wrong results. Order such calls on one stream or synchronise between them.
+ *   - A shape whose plan does not fit the array even one row at a time (about 2.6 million
+ *     vocabulary entries per row, or fewer with very many rows) returns
+ *     LMH_ERR_SCRATCH_LIMIT before anything is enqueued.
+ * Arguments as lmh_logprob, without the workspace. The error word cannot be read back; use
+ * lmh_logprob where that matters.
+ */
+LMH_API lmh_status lmh_logprob_noalloc(const lmh_shape* shape, const lmh_bf16* H,
+                                       const lmh_bf16* W, const int32_t* labels, float* logprob,
+                                       float* lse, void* stream);
 
 /*
  * Measurement hook (not part of the method). lmh_profile_enable(1) makes every later call

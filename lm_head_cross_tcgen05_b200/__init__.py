@@ -4,7 +4,7 @@ The functions named ``lmh_*`` mirror the C ABI of ``include/lmh.h`` one to one: 
 torch CUDA tensors, check dtype / contiguity / device, and pass raw pointers and the
 current stream through ctypes. Every step of the computation runs in the library's CUDA
 kernels; there is no fallback path, and importing this package fails if ``liblmh.so`` has
-not been built (``python -m lm_head_cross_tcgen05_b200.build``).
+not been built (``python lm_head_cross_tcgen05_b200/build.py``).
 
 The lower-case helpers (``loss_fwd``, ``loss_bwd``, ``logprob``, ``support_logprob``,
 ``support_kl``) allocate the outputs and the workspace with torch and call the same entries.

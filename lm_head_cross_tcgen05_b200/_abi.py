@@ -14,7 +14,8 @@ c_int64, c_uint32, c_int, c_size_t, c_void_p = (ctypes.c_int64, ctypes.c_uint32,
 
 LMH_OK = 0
 STATUS_NAMES = {0: "LMH_OK", 1: "LMH_ERR_INVALID_ARG", 2: "LMH_ERR_UNSUPPORTED_DEVICE",
-                3: "LMH_ERR_WORKSPACE_TOO_SMALL", 4: "LMH_ERR_ALIGNMENT", 5: "LMH_ERR_CUDA"}
+                3: "LMH_ERR_WORKSPACE_TOO_SMALL", 4: "LMH_ERR_ALIGNMENT", 5: "LMH_ERR_CUDA",
+                6: "LMH_ERR_SCRATCH_LIMIT"}
 
 IGNORE_INDEX = -100
 DEVERR_LABEL_RANGE, DEVERR_TIMEOUT, DEVERR_NONFINITE = 0x1, 0x2, 0x4
@@ -38,6 +39,7 @@ _SIGS = {
     "lmh_support_logprob": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6 + [c_size_t, _P]),
     "lmh_support_kl": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 9 + [c_size_t, _P]),
     "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),
+    "lmh_logprob_noalloc": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6),
     "lmh_profile_enable": (c_int, [c_int]),
     "lmh_profile_read": (c_int, [c_int, ctypes.POINTER(ctypes.c_int32),
                                  ctypes.POINTER(ctypes.c_float)]),
@@ -57,13 +59,15 @@ _lib = None
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
+        hint = "run `python lm_head_cross_tcgen05_b200/build.py` (this package has no fallback path)"
         if not os.path.exists(LIB_PATH):
-            raise ImportError(
-                f"{LIB_PATH} is not built; run `python -m lm_head_cross_tcgen05_b200.build` "
-                "(this package has no fallback path)")
+            raise ImportError(f"{LIB_PATH} is not built; {hint}")
         L = ctypes.CDLL(LIB_PATH)
         for name, (res, args) in _SIGS.items():
-            f = getattr(L, name)
+            try:
+                f = getattr(L, name)
+            except AttributeError:
+                raise ImportError(f"{LIB_PATH} lacks {name}: it is older than its sources; {hint}")
             f.restype, f.argtypes = res, args
         _lib = L
     return _lib

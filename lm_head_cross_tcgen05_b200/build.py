@@ -1,6 +1,9 @@
 """Builds liblmh.so (the C ABI of include/lmh.h) in-tree for sm_100a with nvcc.
 
-    python -m lm_head_cross_tcgen05_b200.build [--force] [--verbose-ptxas]
+    python lm_head_cross_tcgen05_b200/build.py [--force] [--verbose-ptxas]
+
+Run it as a script (or load it by path, as __graft_entry__.build() does): importing the
+package would load the library this script is about to build.
 """
 from __future__ import annotations
 

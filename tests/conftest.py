@@ -8,7 +8,18 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _ensure_built():
+    # build (or rebuild) the in-tree library before any test imports the package
+    import importlib.util
+    path = os.path.join(ROOT, "lm_head_cross_tcgen05_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_lmh_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
 def pytest_configure(config):
+    _ensure_built()
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: full-size workloads (minutes)")
 
