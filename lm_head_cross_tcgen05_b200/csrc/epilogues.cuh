@@ -79,6 +79,9 @@ struct TargetCursor<kCands> {
   }
 };
 
+// kStream: the data is read once, much later (the chunk's softmax / gradient buffer): store
+// with the streaming hint so it does not push reused operands out of L2.
+template <bool kStream = false>
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32],
                                               int nvec) {
   // nvec: how many of the four 8-column vectors to write (the rest lie past the row end)
@@ -91,7 +94,7 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&
       w.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
       w.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
       w.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-      d4[u] = w;
+      if (kStream) __stcs(d4 + u, w); else d4[u] = w;
     }
   }
 }
@@ -178,7 +181,7 @@ struct EpiStats {
       if (kStoreP && rv) {
         const long long rem = p.ldp - col0;
         const int nvec = rem >= 32 ? 4 : (rem > 0 ? static_cast<int>(rem >> 3) : 0);
-        store_bf16x32(prow + col0, v, nvec);
+        store_bf16x32<true>(prow + col0, v, nvec);
       }
     }
     if (rv) {
@@ -238,7 +241,7 @@ struct EpiGrad {
       if (rv) {
         const long long rem = p.ldp - col0;
         const int nvec = rem >= 32 ? 4 : (rem > 0 ? static_cast<int>(rem >> 3) : 0);
-        store_bf16x32(prow + col0, v, nvec);
+        store_bf16x32<true>(prow + col0, v, nvec);
       }
     }
   }

@@ -1,69 +1,85 @@
-// gemm.cuh — persistent, warp-specialised bf16 GEMM on the sm_100a tensor cores.
+// gemm.cuh — persistent, warp-specialised bf16 GEMM on the sm_100a tensor cores, run by CTA
+// pairs (clusters of 2) that share one 256 x 256 output tile per MMA (tcgen05 cta_group::2).
 //
-// One CTA per SM (grid = min(tiles, SMs)); each CTA walks the output tiles
-// t = blockIdx.x, blockIdx.x + gridDim.x, ... in a fixed order. Every output tile is owned
-// by exactly one CTA and its K loop runs in ascending order, so the fp32 result of a tile
-// does not depend on which CTA ran it or on the SM count: the GEMM is deterministic with no
-// cross-CTA reduction.
+// Each CTA of a pair owns 128 of the tile's 256 rows: it stages its 128 rows of A and its 128
+// rows (of 256) of B in its own shared memory, and its half of the fp32 accumulator lives in
+// its own TMEM. The pair's rank-0 CTA issues the MMAs, which read the operand halves of both
+// CTAs. Per SM this halves the B operand traffic of a 128 x 256 single-CTA tile.
 //
-// Roles (192 threads):
-//   warp 0, lane 0  TMA producer: 128-byte-swizzled operand tiles into a STAGES-deep ring.
-//   warp 1, lane 0  MMA issuer: tcgen05.mma (M=128, N=256, K=16 per instruction) into one of
-//                   two TMEM accumulators (2 x 256 fp32 columns = all 512 TMEM columns), so
-//                   the epilogue of tile i overlaps the main loop of tile i+1.
-//   warps 2..5      epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//                   32*(w%4) .. +31, i.e. tile rows), then the fused math of `Epi`.
+// Persistent schedule: grid = 2 x (number of co-resident pairs); pair p walks the tiles
+// p, p + pairs, ... of a fixed, grouped order (group_m row tiles at a time, rows fastest).
+// Every output tile is owned by one pair and its K loop runs in ascending order, so the fp32
+// result of a tile does not depend on which SMs ran it or how many there are: the GEMM is
+// deterministic without any cross-CTA reduction.
 //
-// Operand layouts: A is [M, K] and B is [N, K] in the tensor core's view. Each may sit in
-// global memory K-major (K contiguous: box 64 x rows) or MN-major (M or N contiguous: boxes
-// of 64 MN x 64 K); the MMA reads MN-major operands through the descriptor's transpose bit,
-// so no operand is ever transposed in memory.
+// Roles (192 threads per CTA):
+//   warp 0, lane 0  TMA producer (both CTAs): its own operand halves into a STAGES-deep ring;
+//                   every load completes its bytes on the rank-0 CTA's `full` barrier.
+//   warp 1, lane 0  MMA issuer (rank 0 only): tcgen05.mma 256x256x16 into one of two TMEM
+//                   accumulators (2 x 256 fp32 columns = all 512), so the epilogue of tile i
+//                   overlaps the main loop of tile i+1; commits free the smem stage and signal
+//                   the accumulator in both CTAs (multicast commit, no multicast loads).
+//   warps 2..5      epilogue (both CTAs): tcgen05.ld of the CTA's accumulator half (warp w
+//                   reads TMEM lanes 32*(w%4) .. +31), then the fused math of `Epi`; releases
+//                   the accumulator with an arrival on the rank-0 CTA's `tmem_empty` barrier.
+//
+// Operand layouts: A is [M, K] and B is [N, K] in the tensor core's view. Each may be K-major
+// in global memory (K contiguous: box 64 x 128 rows) or MN-major (M or N contiguous: boxes of
+// 64 MN x 64 K); MN-major operands are read through the descriptor's transpose bit, so no
+// operand is ever transposed in memory.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace lmh {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KiB
-constexpr int B_STAGE_BYTES = BN * BK * 2;  // 32 KiB
+constexpr int BM = 128;   // accumulator rows per CTA (half of a pair tile)
+constexpr int PM = 256;   // rows per pair tile
+constexpr int BN = 256;   // columns per tile
+constexpr int BNH = 128;  // B rows staged per CTA
+constexpr int BK = 64;                       // K per pipeline stage
+constexpr int KSUB = BK / 64;                // 128-byte-wide K sub-tiles of a K-major stage
+constexpr int STAGES = 6;
+constexpr int A_STAGE_BYTES = BM * BK * 2;
+constexpr int B_STAGE_BYTES = BNH * BK * 2;
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x 64 (K) box: 8 KiB
+constexpr int A_SUB_BYTES = BM * 128;        // one K-major sub-tile of A (rows x 64 K)
+constexpr int B_SUB_BYTES = BNH * 128;
+constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x BK (K) box
 constexpr int GEMM_THREADS = 192;
 constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + slack to 1 KiB-align
 constexpr uint32_t TMEM_COLS = 512;
 
 struct GemmGrid {
-  int m_tiles;
-  int n_tiles;
-  int k_blocks;     // ceil(K / 64)
-  int n_fastest;    // tile order: 0 -> consecutive tiles walk M, 1 -> walk N
-  uint32_t* err;    // device error word
+  int m_tiles;   // pair tiles along M (256 rows each)
+  int n_tiles;   // tiles along N (256 columns each)
+  int k_blocks;  // ceil(K / 64)
+  int group_m;   // tile order: group_m row tiles at a time, rows fastest within a group
+  int hint_a;    // L2 eviction priority of A's loads (L2Hint)
+  int hint_b;    // L2 eviction priority of B's loads
+  uint32_t* err; // device error word
 };
 
 __device__ __forceinline__ void tile_coords(const GemmGrid& g, int t, int& mb, int& nb) {
-  if (g.n_fastest) {
-    nb = t % g.n_tiles;
-    mb = t / g.n_tiles;
-  } else {
-    mb = t % g.m_tiles;
-    nb = t / g.m_tiles;
-  }
+  const int per_group = g.group_m * g.n_tiles;
+  const int grp = t / per_group;
+  const int rem = t - grp * per_group;
+  const int m0 = grp * g.group_m;
+  const int gm = min(g.group_m, g.m_tiles - m0);
+  mb = m0 + rem % gm;
+  nb = rem / gm;
 }
 
 template <class Epi>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB, const GemmGrid g,
                    const typename Epi::Params ep) {
   extern __shared__ uint8_t dsmem[];
-  __shared__ __align__(8) uint64_t full_bar[STAGES];
-  __shared__ __align__(8) uint64_t empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t tfull_bar[2];
-  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];   // rank 0: operands of a stage landed
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];  // both: the stage was read by the MMAs
+  __shared__ __align__(8) uint64_t tfull_bar[2];       // both: accumulator b is complete
+  __shared__ __align__(8) uint64_t tempty_bar[2];      // rank 0: both CTAs drained accumulator b
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
@@ -71,6 +87,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint32_t smem_base = (smem_u32(dsmem) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
   const int num_tiles = g.m_tiles * g.n_tiles;
 
   if (threadIdx.x == 0) {
@@ -80,15 +99,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tfull_bar[b]), 1);
-      mbar_init(smem_u32(&tempty_bar[b]), 4);
+      mbar_init(smem_u32(&tempty_bar[b]), 8);  // 4 epilogue warps x 2 CTAs
     }
     mbar_init(smem_u32(&drain_bar), 1);
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), TMEM_COLS);
+  if (warp == 1) tmem_alloc_pair(smem_u32(&tmem_slot), TMEM_COLS);
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
 
@@ -97,10 +116,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
+      const uint64_t pol_a = l2_policy(g.hint_a);
+      const uint64_t pol_b = l2_policy(g.hint_b);
       uint32_t kbg = 0;
-      for (int t = blockIdx.x; t < num_tiles && !abort_flag; t += gridDim.x) {
+      for (int t = pair; t < num_tiles && !abort_flag; t += npairs) {
         int mb, nb;
         tile_coords(g, t, mb, nb);
+        const int arow = mb * PM + static_cast<int>(rank) * BM;    // this CTA's A rows
+        const int brow = nb * BN + static_cast<int>(rank) * BNH;   // this CTA's B rows
         for (int kb = 0; kb < g.k_blocks; ++kb, ++kbg) {
           const uint32_t s = kbg % STAGES;
           const uint32_t ph = (kbg / STAGES) & 1u;
@@ -108,34 +131,40 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             abort_flag = 1;
             break;
           }
-          const uint32_t fb = smem_u32(&full_bar[s]);
+          const uint32_t lfull = map_to_rank(smem_u32(&full_bar[s]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * STAGE_BYTES);
           const uint32_t a_dst = smem_base + s * STAGE_BYTES;
           const uint32_t b_dst = a_dst + A_STAGE_BYTES;
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
           if (!Epi::kAMajorMN) {
-            tma_load_2d(a_dst, &tmA, fb, kb * BK, mb * BM);
+#pragma unroll
+            for (int j = 0; j < KSUB; ++j)
+              tma_load_2d_pair(a_dst + j * A_SUB_BYTES, &tmA, lfull, kb * BK + 64 * j, arow, pol_a);
           } else {
 #pragma unroll
             for (int j = 0; j < BM / 64; ++j)
-              tma_load_2d(a_dst + j * MN_BLOCK_BYTES, &tmA, fb, mb * BM + 64 * j, kb * BK);
+              tma_load_2d_pair(a_dst + j * MN_BLOCK_BYTES, &tmA, lfull, arow + 64 * j, kb * BK,
+                               pol_a);
           }
           if (!Epi::kBMajorMN) {
-            tma_load_2d(b_dst, &tmB, fb, kb * BK, nb * BN);
+#pragma unroll
+            for (int j = 0; j < KSUB; ++j)
+              tma_load_2d_pair(b_dst + j * B_SUB_BYTES, &tmB, lfull, kb * BK + 64 * j, brow, pol_b);
           } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(b_dst + j * MN_BLOCK_BYTES, &tmB, fb, nb * BN + 64 * j, kb * BK);
+            for (int j = 0; j < BNH / 64; ++j)
+              tma_load_2d_pair(b_dst + j * MN_BLOCK_BYTES, &tmB, lfull, brow + 64 * j, kb * BK,
+                               pol_b);
           }
         }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc_bf16(BM, BN, Epi::kAMajorMN, Epi::kBMajorMN);
+    // ------------------------------------------------------------------ MMA issuer (rank 0)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = make_idesc_bf16(PM, BN, Epi::kAMajorMN, Epi::kBMajorMN);
       uint32_t kbg = 0;
       int it = 0;
-      for (int t = blockIdx.x; t < num_tiles && !abort_flag; t += gridDim.x, ++it) {
+      for (int t = pair; t < num_tiles && !abort_flag; t += npairs, ++it) {
         const int b = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         if (!mbar_wait(smem_u32(&tempty_bar[b]), (use & 1u) ^ 1u, g.err)) {
@@ -157,24 +186,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t b_base = a_base + A_STAGE_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t adesc = Epi::kAMajorMN
-                                       ? make_sw128_desc(a_base + k * 2048, MN_BLOCK_BYTES, 1024)
-                                       : make_sw128_desc(a_base + k * 32, 16, 1024);
-            const uint64_t bdesc = Epi::kBMajorMN
-                                       ? make_sw128_desc(b_base + k * 2048, MN_BLOCK_BYTES, 1024)
-                                       : make_sw128_desc(b_base + k * 32, 16, 1024);
-            mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+            // K-major: sub-tile k/4, 32-byte step inside its 128-byte rows; MN-major: 16 rows
+            const uint64_t adesc =
+                Epi::kAMajorMN
+                    ? make_sw128_desc(a_base + k * 2048, MN_BLOCK_BYTES, 1024)
+                    : make_sw128_desc(a_base + (k >> 2) * A_SUB_BYTES + (k & 3) * 32, 16, 1024);
+            const uint64_t bdesc =
+                Epi::kBMajorMN
+                    ? make_sw128_desc(b_base + k * 2048, MN_BLOCK_BYTES, 1024)
+                    : make_sw128_desc(b_base + (k >> 2) * B_SUB_BYTES + (k & 3) * 32, 16, 1024);
+            mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
           }
-          mma_commit(smem_u32(&empty_bar[s]));  // frees the smem stage once read
+          mma_commit_pair(smem_u32(&empty_bar[s]), 0x3);  // both CTAs may refill stage s
         }
         if (!ok) {
           abort_flag = 1;
           break;
         }
-        mma_commit(smem_u32(&tfull_bar[b]));  // accumulator b is complete
+        mma_commit_pair(smem_u32(&tfull_bar[b]), 0x3);  // accumulator b done in both CTAs
       }
       // No MMA may still be writing TMEM when the columns are released.
-      mma_commit(smem_u32(&drain_bar));
+      mma_commit_pair_local(smem_u32(&drain_bar));
       mbar_wait(smem_u32(&drain_bar), 0, g.err);
     }
   } else {
@@ -182,7 +214,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int q = warp & 3;  // the TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
     int it = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+    for (int t = pair; t < num_tiles; t += npairs, ++it) {
       const int b = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       bool ok = !abort_flag && mbar_wait(smem_u32(&tfull_bar[b]), use & 1u, g.err);
@@ -196,17 +228,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       tile_coords(g, t, mb, nb);
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
-      Epi::tile(ep, mb, nb, taddr, row_in_tile);
+      Epi::tile(ep, mb * 2 + static_cast<int>(rank), nb, taddr, row_in_tile);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[b]));
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty_bar[b]), 0));
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // MMAs drained in rank 0, accumulator reads done in both CTAs
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
 }
 
 }  // namespace lmh

@@ -200,31 +200,60 @@ bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
 }
 
 // ------------------------------------------------------------------------ launches
+// Tile orders and L2 priorities of the three contractions.
+struct GemmOrder {
+  int group_m;  // pair-row tiles per group (rows fastest inside a group)
+  int hint_a, hint_b;
+};
+
 template <class Epi>
 lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap& b,
-                       int64_t M, int64_t Ncols, int64_t K, int n_fastest, uint32_t* err,
+                       int64_t M, int64_t Ncols, int64_t K, GemmOrder order, uint32_t* err,
                        const typename Epi::Params& ep, cudaStream_t st) {
   static std::atomic<uint64_t> attr_done{0};
+  static std::atomic<int> pairs_cache[64];
   const uint64_t bit = 1ull << dev;
   if (!(attr_done.load() & bit)) {
     if (cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GEMM_SMEM_BYTES) != cudaSuccess)
       return LMH_ERR_CUDA;
+    // how many CTA pairs can be resident at once (one CTA per SM)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sms / 2 * 2));
+    cfg.blockDim = dim3(GEMM_THREADS);
+    cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, gemm_tc_kernel<Epi>, &cfg) != cudaSuccess ||
+        nclusters < 1) {
+      cudaGetLastError();
+      nclusters = sms / 2;
+    }
+    pairs_cache[dev].store(nclusters);
     attr_done.fetch_or(bit);
   }
   GemmGrid g;
-  g.m_tiles = static_cast<int>(cdiv(M, BM));
+  g.m_tiles = static_cast<int>(cdiv(M, PM));
   g.n_tiles = static_cast<int>(cdiv(Ncols, BN));
   g.k_blocks = static_cast<int>(cdiv(K, BK));
-  g.n_fastest = n_fastest;
+  g.group_m = order.group_m < 1 ? g.m_tiles : (order.group_m < g.m_tiles ? order.group_m : g.m_tiles);
+  g.hint_a = order.hint_a;
+  g.hint_b = order.hint_b;
   g.err = err;
   const int64_t tiles = static_cast<int64_t>(g.m_tiles) * g.n_tiles;
   if (tiles <= 0) return LMH_OK;
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  const int64_t pairs_max = pairs_cache[dev].load();
+  const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
   ProfScope ps(Epi::kId, st);
-  gemm_tc_kernel<Epi><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(a, b, g, ep);
+  gemm_tc_kernel<Epi><<<2 * pairs, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(a, b, g, ep);
   return cudaGetLastError() == cudaSuccess ? LMH_OK : LMH_ERR_CUDA;
 }
+
+// logits: all row tiles of a vocabulary tile before the next one
+constexpr GemmOrder kOrderLogits{0, kL2Normal, kL2Normal};
+// dH: eight 256-row tiles at a time across all hidden tiles
+constexpr GemmOrder kOrderDH{8, kL2Normal, kL2Normal};
+// dW: one 256-word vocabulary tile across all hidden tiles
+constexpr GemmOrder kOrderDW{1, kL2Normal, kL2Normal};
 
 #define LMH_TRY(x)                      \
   do {                                  \
@@ -259,7 +288,7 @@ template <int TK, bool kStoreP>
 lmh_status run_stats(const Plan& P, int dev, int sms, const lmh_bf16* H, const lmh_bf16* W,
                      const Targets& tg, int64_t r0, int rows, const Ws& ws, cudaStream_t st) {
   CUtensorMap ta, tb;
-  if (!tmap_2d(&ta, H + r0 * P.d, P.d, rows, P.d, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BN))
+  if (!tmap_2d(&ta, H + r0 * P.d, P.d, rows, P.d, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BNH))
     return LMH_ERR_CUDA;
   typename EpiStats<TK, kStoreP>::Params ep;
   ep.rows = rows;
@@ -273,8 +302,8 @@ lmh_status run_stats(const Plan& P, int dev, int sms, const lmh_bf16* H, const l
   ep.part_s = ws.at<float>(P.o_ps);
   ep.part_i = ws.at<int32_t>(P.o_pi);
   ep.P = kStoreP ? ws.at<__nv_bfloat16>(P.o_gbuf) : nullptr;
-  return launch_gemm<EpiStats<TK, kStoreP>>(dev, sms, ta, tb, rows, P.V, P.d, 0, &ws.h->err, ep,
-                                           st);
+  return launch_gemm<EpiStats<TK, kStoreP>>(dev, sms, ta, tb, rows, P.V, P.d, kOrderLogits,
+                                           &ws.h->err, ep, st);
 }
 
 lmh_status run_finalize(const Plan& P, int kind, int64_t r0, int rows, const int32_t* labels,
@@ -313,18 +342,18 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
   const __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
   if (dH) {
     CUtensorMap ta, tb;
-    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, 64))
+    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BK))
       return LMH_ERR_CUDA;
     EpiDH::Params ep;
     ep.rows = rows;
     ep.row0 = r0;
     ep.d = static_cast<int>(P.d);
     ep.dH = reinterpret_cast<__nv_bfloat16*>(dH);
-    LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, rows, P.d, P.V, 1, &ws.h->err, ep, st));
+    LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, rows, P.d, P.V, kOrderDH, &ws.h->err, ep, st));
   }
   if (dW || dW_acc) {
     CUtensorMap ta, tb;
-    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, 64) || !tmap_2d(&tb, H + r0 * P.d, P.d, rows, P.d, 64))
+    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BK) || !tmap_2d(&tb, H + r0 * P.d, P.d, rows, P.d, BK))
       return LMH_ERR_CUDA;
     EpiDW::Params ep;
     ep.V = static_cast<int>(P.V);
@@ -341,7 +370,7 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
       ep.acc_mode = 0;
     }
     ep.out = (dW && last) ? reinterpret_cast<__nv_bfloat16*>(dW) : nullptr;
-    LMH_TRY(launch_gemm<EpiDW>(dev, sms, ta, tb, P.V, P.d, rows, 1, &ws.h->err, ep, st));
+    LMH_TRY(launch_gemm<EpiDW>(dev, sms, ta, tb, P.V, P.d, rows, kOrderDW, &ws.h->err, ep, st));
   }
   return LMH_OK;
 }
@@ -436,13 +465,13 @@ extern "C" lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, co
     if (fused) {
       __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
       const int64_t nv = P.Vp / 8;
-      const int64_t bx = cdiv(nv, 256);
+      const int64_t bx = cdiv(nv, kGbuildThreads * kGbuildVec);
       dim3 grid(static_cast<unsigned>(bx < 64 ? bx : 64),
                 static_cast<unsigned>(rows < 65535 ? rows : 65535));
       {
         ProfScope ps(KID_GBUILD, st);
-        gbuild_kernel<<<grid, 256, 0, st>>>(rows, P.Vp, static_cast<int>(P.T),
-                                            ws.at<float>(P.o_ps), G);
+        gbuild_kernel<<<grid, kGbuildThreads, 0, st>>>(rows, P.Vp, static_cast<int>(P.T),
+                                                       ws.at<float>(P.o_ps), G);
       }
       LMH_TRY(last_launch());
       {
@@ -601,18 +630,18 @@ extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_b
     const int64_t r0 = ci * P.c;
     const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
     CUtensorMap ta, tb;
-    if (!tmap_2d(&ta, H + r0 * P.d, P.d, rows, P.d, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BN))
+    if (!tmap_2d(&ta, H + r0 * P.d, P.d, rows, P.d, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BNH))
       return LMH_ERR_CUDA;
     if (cands) {
       EpiGrad<kCands>::Params ep{rows, r0, static_cast<int>(P.V), P.Vp, tg, lse, alpha, beta,
                                  ws.at<__nv_bfloat16>(P.o_gbuf)};
-      LMH_TRY(launch_gemm<EpiGrad<kCands>>(dev, sms, ta, tb, rows, P.V, P.d, 0, &ws.h->err, ep,
-                                           st));
+      LMH_TRY(launch_gemm<EpiGrad<kCands>>(dev, sms, ta, tb, rows, P.V, P.d, kOrderLogits,
+                                           &ws.h->err, ep, st));
     } else {
       EpiGrad<kLabel>::Params ep{rows, r0, static_cast<int>(P.V), P.Vp, tg, lse, alpha, beta,
                                  ws.at<__nv_bfloat16>(P.o_gbuf)};
-      LMH_TRY(launch_gemm<EpiGrad<kLabel>>(dev, sms, ta, tb, rows, P.V, P.d, 0, &ws.h->err, ep,
-                                           st));
+      LMH_TRY(launch_gemm<EpiGrad<kLabel>>(dev, sms, ta, tb, rows, P.V, P.d, kOrderLogits,
+                                           &ws.h->err, ep, st));
     }
     LMH_TRY(run_backward_gemms(P, dev, sms, H, W, r0, rows, static_cast<int>(ci), dH, dW, dW_acc,
                                ws, st));

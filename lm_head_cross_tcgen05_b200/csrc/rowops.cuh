@@ -189,24 +189,41 @@ __global__ void finalize_rows_kernel(const FinParams p) {
 
 // ---------------------------------------------------------------------------- G rescale
 // In place over the chunk's [rows, ldp] bf16 buffer: G = scale[row, t] * p~ (t = col / 256).
-// 16-byte vectors, fully coalesced; grid (x: vectors of a row, y: rows).
-__global__ void gbuild_kernel(int rows, long long ldp, int T, const float* __restrict__ scale,
-                              __nv_bfloat16* __restrict__ P) {
-  const long long nv = ldp >> 3;
+// Grid (x: spans of a row, y: rows). Each thread moves four 16-byte vectors a blockDim apart
+// (coalesced), issuing all four loads before any store.
+constexpr int kGbuildThreads = 256;
+constexpr int kGbuildVec = 4;
+
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 w, float f) {
+  float2 a = unpack_bf16x2(w.x), b = unpack_bf16x2(w.y), e = unpack_bf16x2(w.z),
+         g = unpack_bf16x2(w.w);
+  w.x = pack_bf16x2(a.x * f, a.y * f);
+  w.y = pack_bf16x2(b.x * f, b.y * f);
+  w.z = pack_bf16x2(e.x * f, e.y * f);
+  w.w = pack_bf16x2(g.x * f, g.y * f);
+  return w;
+}
+
+__global__ void __launch_bounds__(kGbuildThreads)
+    gbuild_kernel(int rows, long long ldp, int T, const float* __restrict__ scale,
+                  __nv_bfloat16* __restrict__ P) {
+  const long long nv = ldp >> 3;  // 16-byte vectors per row
+  const long long span = static_cast<long long>(kGbuildThreads) * kGbuildVec;
   for (long long r = blockIdx.y; r < rows; r += gridDim.y) {
     uint4* row4 = reinterpret_cast<uint4*>(P + r * ldp);
     const float* sc = scale + r * T;
-    for (long long c = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; c < nv;
-         c += static_cast<long long>(gridDim.x) * blockDim.x) {
-      const float f = sc[c >> 5];  // 32 vectors of 8 columns per 256-wide tile
-      uint4 w = row4[c];
-      float2 a = unpack_bf16x2(w.x), b = unpack_bf16x2(w.y), e = unpack_bf16x2(w.z),
-             g = unpack_bf16x2(w.w);
-      w.x = pack_bf16x2(a.x * f, a.y * f);
-      w.y = pack_bf16x2(b.x * f, b.y * f);
-      w.z = pack_bf16x2(e.x * f, e.y * f);
-      w.w = pack_bf16x2(g.x * f, g.y * f);
-      row4[c] = w;
+    for (long long c0 = blockIdx.x * span + threadIdx.x; c0 < nv; c0 += gridDim.x * span) {
+      uint4 w[kGbuildVec];
+#pragma unroll
+      for (int u = 0; u < kGbuildVec; ++u) {
+        const long long c = c0 + u * kGbuildThreads;
+        if (c < nv) w[u] = __ldcs(row4 + c);
+      }
+#pragma unroll
+      for (int u = 0; u < kGbuildVec; ++u) {
+        const long long c = c0 + u * kGbuildThreads;
+        if (c < nv) row4[c] = scale_bf16x8(w[u], sc[c >> 5]);  // 32 vectors per 256-wide tile
+      }
     }
   }
 }
