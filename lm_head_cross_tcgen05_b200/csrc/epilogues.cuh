@@ -1,6 +1,8 @@
 // epilogues.cuh — what each GEMM does with its fp32 accumulator tile (128 rows x 256
-// columns in TMEM). Each epilogue thread owns one tile row and reads it as eight 32-column
-// slices with tcgen05.ld; nothing here synchronises across threads.
+// columns of TMEM per CTA). Each epilogue thread owns one tile row and reads it as four
+// 64-column slabs (two tcgen05.ld of 32 columns each). bf16 outputs are staged per warp in
+// shared memory (32 rows x 64 columns, 128-byte swizzled) and written with one TMA store, so
+// global writes are full 128-byte lines instead of 32 scattered 16-byte pieces.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -10,7 +12,7 @@
 
 namespace lmh {
 
-constexpr int kSlices = BN / 32;
+constexpr int kSlabs = BN / 64;
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // ---------------------------------------------------------------------------- targets
@@ -79,52 +81,65 @@ struct TargetCursor<kCands> {
   }
 };
 
-// kStream: the data is read once, much later (the chunk's softmax / gradient buffer): store
-// with the streaming hint so it does not push reused operands out of L2.
-template <bool kStream = false>
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32],
-                                              int nvec) {
-  // nvec: how many of the four 8-column vectors to write (the rest lie past the row end)
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+// ---------------------------------------------------------------------------- staged store
+// The warp writes its 32 rows x 64 columns (a: columns 0..31, b: 32..63 of each thread's
+// row) into one of its two staging buffers and lane 0 stores the block at (x, y) of ctx.tmC.
+// A buffer is reused only after the store issued from it two calls earlier has finished
+// reading it. All lanes of the warp must call this together.
+__device__ __forceinline__ void stage_store_64(EpiCtx& c, const float (&a)[32],
+                                               const float (&b)[32], int x, int y,
+                                               bool do_store) {
+  const uint32_t buf = c.stage + (c.nstore & 1u) * EPI_BUF_BYTES;
+  if (c.lane == 0) bulk_wait_read_le1();
+  __syncwarp();
+  const uint32_t row = buf + static_cast<uint32_t>(c.lane) * 128u;
+  const uint32_t sw = static_cast<uint32_t>(c.lane & 7);
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    if (u < nvec) {
-      uint4 w;
-      w.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
-      w.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-      w.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-      w.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-      if (kStream) __stcs(d4 + u, w); else d4[u] = w;
-    }
+  for (int u = 0; u < 8; ++u) {
+    const float* v = u < 4 ? a : b;
+    const int o = (u & 3) * 8;
+    uint4 w;
+    w.x = pack_bf16x2(v[o + 0], v[o + 1]);
+    w.y = pack_bf16x2(v[o + 2], v[o + 3]);
+    w.z = pack_bf16x2(v[o + 4], v[o + 5]);
+    w.w = pack_bf16x2(v[o + 6], v[o + 7]);
+    st_shared_v4(row + ((static_cast<uint32_t>(u) ^ sw) << 4), w);  // 16-byte chunk swizzle
   }
+  fence_async_smem();
+  __syncwarp();
+  if (c.lane == 0 && do_store) {
+    tma_store_2d(c.tmC, buf, x, y);
+    bulk_commit();
+  }
+  ++c.nstore;
 }
 
 // ------------------------------------------------------------------ logits statistics
 // Forward epilogue of z = H_c W^T. Per (row, 256-wide vocabulary tile t) it writes the tile
 // maximum m_t, s_t = sum_v exp(z_v - m_t), the first column attaining m_t, and the logits at
-// the row's targets; with kStoreP it also stores p~ = exp(z - m_t) in bf16, which the fused
-// backward rescales into the softmax gradient. Columns >= V are masked to -inf.
+// the row's targets; with kStoreP it also stores p~ = exp(z - m_t) in bf16 (zero past V),
+// which the fused backward rescales into the softmax gradient. Columns >= V are masked.
+// ctx.tmC (kStoreP): the chunk's [rows, ldp] bf16 buffer.
 template <int TK, bool kStoreP>
 struct EpiStats {
   static constexpr int kId = kStoreP ? 3 : 2;  // gemm_logits_stats(_store)
-  static constexpr int kAMajorMN = 0;  // H chunk [rows, d], K-major
-  static constexpr int kBMajorMN = 0;  // W [V, d], K-major
+  static constexpr int kAMajorMN = 0;          // H chunk [rows, d], K-major
+  static constexpr int kBMajorMN = 0;          // W [V, d], K-major
   struct Params {
     int rows;           // rows of this chunk
     long long row0;     // global index of the chunk's first row
     int V;
     int T;              // vocabulary tiles, ceil(V / 256)
-    long long ldp;      // row stride of P (elements), round_up(V, 8)
+    long long ldp;      // row stride of the chunk buffer (elements), round_up(V, 8)
     Targets tg;
     float* zt;          // target logits: [N] (kLabel) or [N, K] by sorted index (kCands)
     float* part_m;      // [rows, T]
     float* part_s;      // [rows, T]
     int32_t* part_i;    // [rows, T]
-    __nv_bfloat16* P;   // [rows, ldp] (kStoreP)
   };
 
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
-                                              int rit) {
+                                              int rit, EpiCtx& ctx) {
     const int row = mb * BM + rit;
     const bool rv = row < p.rows;
     const long long grow = p.row0 + row;
@@ -137,7 +152,7 @@ struct EpiStats {
     float m = kNegInf;
     int am = n0;
 #pragma unroll 1
-    for (int sl = 0; sl < kSlices; ++sl) {
+    for (int sl = 0; sl < 2 * kSlabs; ++sl) {
       float v[32];
       tmem_ld32(taddr + sl * 32, v);
       const int col0 = n0 + sl * 32;
@@ -159,30 +174,26 @@ struct EpiStats {
       });
     }
 
-    // pass 2: sum of exp(z - m), optionally p~ = exp(z - m) to P
+    // pass 2: sum of exp(z - m); optionally p~ = exp(z - m) to the chunk buffer
     const float moff = -m * kLog2e;
     float s0 = 0.f, s1 = 0.f;
-    __nv_bfloat16* prow = kStoreP ? p.P + static_cast<long long>(row) * p.ldp : nullptr;
+    const int wrow = mb * BM + ctx.row_w;  // first chunk row of this warp
 #pragma unroll 1
-    for (int sl = 0; sl < kSlices; ++sl) {
-      float v[32];
-      tmem_ld32(taddr + sl * 32, v);
-      const int col0 = n0 + sl * 32;
+    for (int sb = 0; sb < kSlabs; ++sb) {
+      float a[32], b[32];
+      const int col0 = n0 + sb * 64;
+      tmem_ld32(taddr + sb * 64, a);
+      tmem_ld32(taddr + sb * 64 + 32, b);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float e = fast_exp2(fmaf(v[j], kLog2e, moff));
-        v[j] = (full || col0 + j < p.V) ? e : 0.f;
+        const float ea = fast_exp2(fmaf(a[j], kLog2e, moff));
+        const float eb = fast_exp2(fmaf(b[j], kLog2e, moff));
+        a[j] = (full || col0 + j < p.V) ? ea : 0.f;
+        b[j] = (full || col0 + 32 + j < p.V) ? eb : 0.f;
+        s0 += a[j];
+        s1 += b[j];
       }
-#pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        s0 += v[j];
-        s1 += v[j + 1];
-      }
-      if (kStoreP && rv) {
-        const long long rem = p.ldp - col0;
-        const int nvec = rem >= 32 ? 4 : (rem > 0 ? static_cast<int>(rem >> 3) : 0);
-        store_bf16x32<true>(prow + col0, v, nvec);
-      }
+      if (kStoreP) stage_store_64(ctx, a, b, col0, wrow, wrow < p.rows && col0 < p.ldp);
     }
     if (rv) {
       const long long o = static_cast<long long>(row) * p.T + nb;
@@ -195,7 +206,7 @@ struct EpiStats {
 
 // ------------------------------------------------------------------ softmax gradient
 // Backward epilogue with recomputed logits: G = alpha_i exp(z - lse_i) - beta at the row's
-// targets, written in bf16 to the chunk's G buffer (zero past column V).
+// targets, written in bf16 to the chunk's G buffer (zero past column V; ctx.tmC maps it).
 template <int TK>
 struct EpiGrad {
   static constexpr int kId = 4;  // gemm_logits_grad
@@ -210,67 +221,66 @@ struct EpiGrad {
     const float* lse;    // [N]
     const float* alpha;  // [N]
     const float* beta;   // [N] (kLabel) or [N, K] in sorted order (kCands)
-    __nv_bfloat16* P;    // [rows, ldp]
   };
 
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
-                                              int rit) {
+                                              int rit, EpiCtx& ctx) {
     const int row = mb * BM + rit;
     const bool rv = row < p.rows;
     const long long grow = p.row0 + row;
     const int n0 = nb * BN;
     const bool full = n0 + BN <= p.V;
-    const float a = rv ? p.alpha[grow] : 0.f;
+    const float al = rv ? p.alpha[grow] : 0.f;
     const float loff = rv ? -p.lse[grow] * kLog2e : 0.f;
     TargetCursor<TK> cur;
     if (rv) cur.init(p.tg, grow, n0, p.V); else cur.none();
-    __nv_bfloat16* prow = p.P + static_cast<long long>(row) * p.ldp;
+    const int wrow = mb * BM + ctx.row_w;
 #pragma unroll 1
-    for (int sl = 0; sl < kSlices; ++sl) {
-      float v[32];
-      tmem_ld32(taddr + sl * 32, v);
-      const int col0 = n0 + sl * 32;
+    for (int sb = 0; sb < kSlabs; ++sb) {
+      float a[32], b[32];
+      const int col0 = n0 + sb * 64;
+      tmem_ld32(taddr + sb * 64, a);
+      tmem_ld32(taddr + sb * 64 + 32, b);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float e = a * fast_exp2(fmaf(v[j], kLog2e, loff));
-        v[j] = (full || col0 + j < p.V) ? e : 0.f;
+        const float ea = al * fast_exp2(fmaf(a[j], kLog2e, loff));
+        const float eb = al * fast_exp2(fmaf(b[j], kLog2e, loff));
+        a[j] = (full || col0 + j < p.V) ? ea : 0.f;
+        b[j] = (full || col0 + 32 + j < p.V) ? eb : 0.f;
       }
       cur.slice(col0, [&](int j, int idx) {
-        v[j] -= (TK == kLabel) ? p.beta[grow] : p.beta[grow * p.tg.K + idx];
+        a[j] -= (TK == kLabel) ? p.beta[grow] : p.beta[grow * p.tg.K + idx];
       });
-      if (rv) {
-        const long long rem = p.ldp - col0;
-        const int nvec = rem >= 32 ? 4 : (rem > 0 ? static_cast<int>(rem >> 3) : 0);
-        store_bf16x32<true>(prow + col0, v, nvec);
-      }
+      cur.slice(col0 + 32, [&](int j, int idx) {
+        b[j] -= (TK == kLabel) ? p.beta[grow] : p.beta[grow * p.tg.K + idx];
+      });
+      stage_store_64(ctx, a, b, col0, wrow, wrow < p.rows && col0 < p.ldp);
     }
   }
 };
 
 // ------------------------------------------------------------------ dH = G W
+// ctx.tmC maps this chunk's rows of dH ([rows, d] at row r0).
 struct EpiDH {
-  static constexpr int kId = 5;  // gemm_dH
+  static constexpr int kId = 5;        // gemm_dH
   static constexpr int kAMajorMN = 0;  // G chunk [rows, V], K-major
   static constexpr int kBMajorMN = 1;  // W [V, d] read as [K = V, N = d], N contiguous
   struct Params {
     int rows;
-    long long row0;
     int d;
-    __nv_bfloat16* dH;  // [N, d]
   };
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
-                                              int rit) {
-    const int row = mb * BM + rit;
-    const bool rv = row < p.rows;
+                                              int rit, EpiCtx& ctx) {
     const int n0 = nb * BN;
-    __nv_bfloat16* out = p.dH + (p.row0 + row) * static_cast<long long>(p.d);
+    const int wrow = mb * BM + ctx.row_w;
 #pragma unroll 1
-    for (int sl = 0; sl < kSlices; ++sl) {
-      const int col0 = n0 + sl * 32;
-      if (col0 >= p.d) break;  // uniform across the warp
-      float v[32];
-      tmem_ld32(taddr + sl * 32, v);
-      if (rv) store_bf16x32(out + col0, v, 4);
+    for (int sb = 0; sb < kSlabs; ++sb) {
+      const int col0 = n0 + sb * 64;
+      if (col0 >= p.d) break;  // uniform across the warp (d is a multiple of 64)
+      float a[32], b[32];
+      tmem_ld32(taddr + sb * 64, a);
+      tmem_ld32(taddr + sb * 64 + 32, b);
+      stage_store_64(ctx, a, b, col0, wrow, wrow < p.rows);
     }
   }
 };
@@ -278,9 +288,9 @@ struct EpiDH {
 // ------------------------------------------------------------------ dW = G^T H_c
 // acc_mode 0: the tile sum is the whole dW; 1: acc = 0 + sum (first chunk into a fresh
 // internal accumulator); 2: acc += sum (the caller's or a later chunk). With `out` set the
-// bf16 cast of the resulting value is written as well (last chunk).
+// bf16 cast of the resulting value is stored as well (last chunk; ctx.tmC maps dW [V, d]).
 struct EpiDW {
-  static constexpr int kId = 6;  // gemm_dW
+  static constexpr int kId = 6;        // gemm_dW
   static constexpr int kAMajorMN = 1;  // G^T: G chunk [rows, V] read as [K = rows, M = V]
   static constexpr int kBMajorMN = 1;  // H chunk [rows, d] read as [K = rows, N = d]
   struct Params {
@@ -288,46 +298,52 @@ struct EpiDW {
     int d;
     float* acc;           // [V, d] or null
     int acc_mode;
-    __nv_bfloat16* out;   // [V, d] or null
+    int out;              // store the bf16 cast through ctx.tmC
   };
+  static __device__ __forceinline__ void rmw32(const Params& p, long long base, int col0,
+                                               float (&v)[32]) {
+    float4* a4 = reinterpret_cast<float4*>(p.acc + base + col0);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      float4 a;
+      if (p.acc_mode == 2) {
+        a = a4[u];
+        a.x += v[4 * u + 0];
+        a.y += v[4 * u + 1];
+        a.z += v[4 * u + 2];
+        a.w += v[4 * u + 3];
+      } else {
+        a.x = v[4 * u + 0] + 0.f;
+        a.y = v[4 * u + 1] + 0.f;
+        a.z = v[4 * u + 2] + 0.f;
+        a.w = v[4 * u + 3] + 0.f;
+      }
+      a4[u] = a;
+      v[4 * u + 0] = a.x;
+      v[4 * u + 1] = a.y;
+      v[4 * u + 2] = a.z;
+      v[4 * u + 3] = a.w;
+    }
+  }
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
-                                              int rit) {
+                                              int rit, EpiCtx& ctx) {
     const int vrow = mb * BM + rit;
     const bool vv = vrow < p.V;
     const int n0 = nb * BN;
     const long long base = static_cast<long long>(vrow) * p.d;
+    const int wrow = mb * BM + ctx.row_w;
 #pragma unroll 1
-    for (int sl = 0; sl < kSlices; ++sl) {
-      const int col0 = n0 + sl * 32;
+    for (int sb = 0; sb < kSlabs; ++sb) {
+      const int col0 = n0 + sb * 64;
       if (col0 >= p.d) break;
-      float v[32];
-      tmem_ld32(taddr + sl * 32, v);
-      if (!vv) continue;
-      if (p.acc_mode != 0) {
-        float4* a4 = reinterpret_cast<float4*>(p.acc + base + col0);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          float4 a;
-          if (p.acc_mode == 2) {
-            a = a4[u];
-            a.x += v[4 * u + 0];
-            a.y += v[4 * u + 1];
-            a.z += v[4 * u + 2];
-            a.w += v[4 * u + 3];
-          } else {
-            a.x = v[4 * u + 0] + 0.f;
-            a.y = v[4 * u + 1] + 0.f;
-            a.z = v[4 * u + 2] + 0.f;
-            a.w = v[4 * u + 3] + 0.f;
-          }
-          a4[u] = a;
-          v[4 * u + 0] = a.x;
-          v[4 * u + 1] = a.y;
-          v[4 * u + 2] = a.z;
-          v[4 * u + 3] = a.w;
-        }
+      float a[32], b[32];
+      tmem_ld32(taddr + sb * 64, a);
+      tmem_ld32(taddr + sb * 64 + 32, b);
+      if (p.acc_mode != 0 && vv) {
+        rmw32(p, base, col0, a);
+        rmw32(p, base, col0 + 32, b);
       }
-      if (p.out) store_bf16x32(p.out + base + col0, v, 4);
+      if (p.out) stage_store_64(ctx, a, b, col0, wrow, wrow < p.V);
     }
   }
 };

@@ -24,9 +24,9 @@
 //                   the accumulator with an arrival on the rank-0 CTA's `tmem_empty` barrier.
 //
 // Operand layouts: A is [M, K] and B is [N, K] in the tensor core's view. Each may be K-major
-// in global memory (K contiguous: box 64 x 128 rows) or MN-major (M or N contiguous: boxes of
-// 64 MN x 64 K); MN-major operands are read through the descriptor's transpose bit, so no
-// operand is ever transposed in memory.
+// in global memory (K contiguous: boxes of 64 K x 128 rows, two per stage) or MN-major (M or N
+// contiguous: boxes of 64 MN x 128 K); MN-major operands are read through the descriptor's
+// transpose bit, so no operand is ever transposed in memory.
 #pragma once
 
 #include "sm100.cuh"
@@ -37,9 +37,12 @@ constexpr int BM = 128;   // accumulator rows per CTA (half of a pair tile)
 constexpr int PM = 256;   // rows per pair tile
 constexpr int BN = 256;   // columns per tile
 constexpr int BNH = 128;  // B rows staged per CTA
-constexpr int BK = 64;                       // K per pipeline stage
+// K per pipeline stage: 128, i.e. 8 MMAs per barrier round trip. Each round trip (wait for
+// the stage, commit its release) costs the tensor pipe a roughly fixed bubble, so the deeper
+// stage runs about 18 % more MMAs per clock than a 64-deep one; 3 stages of 64 KiB per CTA.
+constexpr int BK = 128;
 constexpr int KSUB = BK / 64;                // 128-byte-wide K sub-tiles of a K-major stage
-constexpr int STAGES = 6;
+constexpr int STAGES = 3;
 constexpr int A_STAGE_BYTES = BM * BK * 2;
 constexpr int B_STAGE_BYTES = BNH * BK * 2;
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
@@ -47,13 +50,26 @@ constexpr int A_SUB_BYTES = BM * 128;        // one K-major sub-tile of A (rows 
 constexpr int B_SUB_BYTES = BNH * 128;
 constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x BK (K) box
 constexpr int GEMM_THREADS = 192;
-constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + slack to 1 KiB-align
+constexpr int EPI_BUF_BYTES = 32 * 128;                      // 32 rows x 64 bf16, 128B-swizzled
+constexpr int EPI_STAGE_BYTES = 4 * 2 * EPI_BUF_BYTES;       // two buffers per epilogue warp
+constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + 1024;  // + align slack
+
+// What an epilogue warp needs to stage bf16 output through shared memory and store it with
+// TMA: the output tensor map (bf16, box 64 columns x 32 rows, 128-byte swizzle), its two
+// staging buffers, and a running count of its stores (which selects the buffer).
+struct EpiCtx {
+  const CUtensorMap* tmC;
+  uint32_t stage;
+  int lane;
+  int row_w;         // first accumulator row of this warp within the CTA's 128
+  uint32_t nstore;
+};
 constexpr uint32_t TMEM_COLS = 512;
 
 struct GemmGrid {
   int m_tiles;   // pair tiles along M (256 rows each)
   int n_tiles;   // tiles along N (256 columns each)
-  int k_blocks;  // ceil(K / 64)
+  int k_blocks;  // ceil(K / BK)
   int group_m;   // tile order: group_m row tiles at a time, rows fastest within a group
   int hint_a;    // L2 eviction priority of A's loads (L2Hint)
   int hint_b;    // L2 eviction priority of B's loads
@@ -73,7 +89,8 @@ __device__ __forceinline__ void tile_coords(const GemmGrid& g, int t, int& mb, i
 template <class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
-                   const __grid_constant__ CUtensorMap tmB, const GemmGrid g,
+                   const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmC, const GemmGrid g,
                    const typename Epi::Params ep) {
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];   // rank 0: operands of a stage landed
@@ -213,6 +230,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // the TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
+    EpiCtx ctx{&tmC, smem_base + STAGES * STAGE_BYTES + (warp - 2) * 2 * EPI_BUF_BYTES, lane,
+               q * 32, 0u};
+    if (lane == 0) tma_prefetch_desc(&tmC);
     int it = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++it) {
       const int b = it & 1;
@@ -228,11 +248,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       tile_coords(g, t, mb, nb);
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
-      Epi::tile(ep, mb * 2 + static_cast<int>(rank), nb, taddr, row_in_tile);
+      Epi::tile(ep, mb * 2 + static_cast<int>(rank), nb, taddr, row_in_tile, ctx);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty_bar[b]), 0));
     }
+    if (lane == 0) bulk_wait_all();  // every staged output has reached global memory
   }
 
   tc_fence_before();
