@@ -30,6 +30,9 @@ Readings taken where the pages are silent (each is listed in the design doc):
 * the mean divides by the count of valid rows; with no valid row the loss is 0 and every
   gradient is 0.
 * a candidate id < 0 is padding: it has lp = 0 and takes no part in the KL or gradients.
+* temperature (the lm_head op commit's temperature stages: off, scalar, per row): every
+  quantity is computed on the tempered logits z_iv / tau_i, and the gradients carry the chain
+  rule factor 1 / tau_i. tau_i is a scalar, a per-row array, or None (off, the same as 1).
 
 Parity status: every function here is pinned by the tests in
 ``tests/test_oracle_pins.py`` (brute force, closed forms, finite differences, invariants).
@@ -73,9 +76,20 @@ def chunk_plan(N: int, chunk_rows: int, default_chunk: int = 4096):
     return [(r0, min(N, r0 + c)) for r0 in range(0, N, c)]
 
 
-def logits(H, W) -> np.ndarray:
-    """z = H W^T, the LM-head logits, in fp64 ([N, V])."""
-    return as_f64(H) @ as_f64(W).T
+def tau_rows(tau, N: int) -> np.ndarray:
+    """Per-row temperatures as an [N] fp64 array (None: all ones)."""
+    if tau is None:
+        return np.ones(N)
+    t = as_f64(tau)
+    return np.full(N, float(t)) if t.ndim == 0 else t.reshape(N)
+
+
+def logits(H, W, tau=None) -> np.ndarray:
+    """z = H W^T, the LM-head logits, in fp64 ([N, V]); with a temperature, z_iv / tau_i."""
+    z = as_f64(H) @ as_f64(W).T
+    if tau is not None:
+        z = z / tau_rows(tau, z.shape[0])[:, None]
+    return z
 
 
 def logsumexp_rows(z: np.ndarray) -> np.ndarray:
@@ -90,14 +104,14 @@ def valid_rows(labels, V: int):
     return (y >= 0) & (y < V), y >= V
 
 
-def ce_forward(H, W, labels) -> dict:
+def ce_forward(H, W, labels, tau=None) -> dict:
     """Cross-entropy forward: per-row loss, lse, target log-prob, argmax, count and mean.
 
     loss_i = lse_i - z_i,y_i and logprob_i = z_i,y_i - lse_i for valid rows, 0 for ignored
     rows; lse_i and argmax_i are reported for every row; mean = sum_valid loss / n_valid
     (0 when n_valid = 0).
     """
-    z = logits(H, W)
+    z = logits(H, W, tau)
     N, V = z.shape
     y = as_i64(labels)
     valid, oob = valid_rows(y, V)
@@ -167,29 +181,29 @@ def lm_head_backward(H, W, G: np.ndarray):
     return G @ as_f64(W), G.T @ as_f64(H)
 
 
-def ce_fused(H, W, labels, mean: bool = True) -> dict:
+def ce_fused(H, W, labels, mean: bool = True, tau=None) -> dict:
     """Forward CE plus dH, dW of the reduced loss (mean over valid rows, or sum)."""
-    f = ce_forward(H, W, labels)
+    f = ce_forward(H, W, labels, tau)
     N = f["z"].shape[0]
     if mean:
         g = np.full(N, 1.0 / f["n_valid"]) if f["n_valid"] else np.zeros(N)
     else:
         g = np.ones(N)
-    G = grad_logits(BWD_CE, f["z"], f["lse"], labels, g)
+    G = grad_logits(BWD_CE, f["z"], f["lse"], labels, g) / tau_rows(tau, N)[:, None]
     dH, dW = lm_head_backward(H, W, G)
     f.update(G=G, dH=dH, dW=dW, grad_rows=g)
     return f
 
 
-def logprob_forward(H, W, labels) -> dict:
+def logprob_forward(H, W, labels, tau=None) -> dict:
     """Per-row target log-prob z_i,y_i - lse_i (0 for ignored rows) and lse."""
-    f = ce_forward(H, W, labels)
+    f = ce_forward(H, W, labels, tau)
     return dict(logprob=f["logprob"], lse=f["lse"], z=f["z"])
 
 
-def support_logprob(H, W, ids) -> dict:
+def support_logprob(H, W, ids, tau=None) -> dict:
     """lp_ik = z_i,c_ik - lse_i: full-vocabulary log-probs at K candidate ids per row."""
-    z = logits(H, W)
+    z = logits(H, W, tau)
     N, V = z.shape
     c = as_i64(ids)
     lse = logsumexp_rows(z) if N else np.zeros(0)
@@ -200,9 +214,9 @@ def support_logprob(H, W, ids) -> dict:
     return dict(lp=lp, lse=lse, z=z, out_of_range=bool((c >= V).any()))
 
 
-def support_kl(H, W, ids, ref_logp) -> dict:
+def support_kl(H, W, ids, ref_logp, tau=None) -> dict:
     """KL_i = sum_k exp(r_ik) (r_ik - lp_ik) over valid candidates; mean over all N rows."""
-    s = support_logprob(H, W, ids)
+    s = support_logprob(H, W, ids, tau)
     c = as_i64(ids)
     V = s["z"].shape[1]
     r = as_f64(ref_logp).reshape(c.shape)
@@ -214,13 +228,13 @@ def support_kl(H, W, ids, ref_logp) -> dict:
     return s
 
 
-def backward(mode: int, H, W, targets, grad, ref_logp=None) -> dict:
+def backward(mode: int, H, W, targets, grad, ref_logp=None, tau=None) -> dict:
     """Standalone backward of one of the four row objectives: recompute z and lse, form G,
     contract. The library's backward takes lse from its forward; here it is recomputed,
-    which is the same value."""
-    z = logits(H, W)
+    which is the same value. With a temperature, G carries the factor 1 / tau_i."""
+    z = logits(H, W, tau)
     lse = logsumexp_rows(z) if z.shape[0] else np.zeros(0)
-    G = grad_logits(mode, z, lse, targets, grad, ref_logp)
+    G = grad_logits(mode, z, lse, targets, grad, ref_logp) / tau_rows(tau, z.shape[0])[:, None]
     dH, dW = lm_head_backward(H, W, G)
     return dict(G=G, dH=dH, dW=dW, lse=lse)
 

@@ -354,3 +354,49 @@ def test_gates_reject_two_percent_scale():
     assert rejects(check_rows, f["loss_rows"] * 1.02, f["loss_rows"])
     assert rejects(check_grad, f["dW"].T.copy().T[::-1], f["dW"])
     check_rows(f["lse"] + 0.5 * ATOL_ROW, f["lse"])
+
+
+# ---------------------------------------------------------------- temperature
+
+def test_fd_with_temperature_scalar_and_rows():
+    H, W = rand_problem(4, 3, 6, 21)
+    y = np.array([0, 5, -100, 2])
+    for tau in (0.7, np.array([0.5, 1.0, 2.0, 1.3])):
+        f = O.ce_fused(H, W, y, mean=True, tau=tau)
+
+        def L():
+            return O.ce_forward(H, W, y, tau)["loss_mean"]
+
+        assert_fd(f["dH"], fd_grad(L, H))
+        assert_fd(f["dW"], fd_grad(L, W))
+    ids = np.array([[0, 5, 3], [2, 2, -1], [1, 4, 0], [5, 3, 1]])
+    r = np.log(np.full((4, 3), 1.0 / 3.0))
+    tau = np.array([0.8, 1.5, 1.0, 0.6])
+    b = O.backward(O.BWD_SUPPORT_KL, H, W, ids, np.ones(4), r, tau=tau)
+
+    def Lk():
+        return float(O.support_kl(H, W, ids, r, tau)["kl_rows"].sum())
+
+    assert_fd(b["dH"], fd_grad(Lk, H))
+    assert_fd(b["dW"], fd_grad(Lk, W))
+
+
+def test_scalar_temperature_equals_scaled_weights():
+    H, W = rand_problem(5, 4, 9, 22)
+    y = np.array([1, 8, 0, -100, 3])
+    tau = 0.37
+    a = O.ce_fused(H, W, y, tau=tau)
+    b = O.ce_fused(H, W / tau, y)
+    np.testing.assert_allclose(a["loss_rows"], b["loss_rows"], atol=1e-13)
+    np.testing.assert_allclose(a["lse"], b["lse"], atol=1e-13)
+    np.testing.assert_allclose(a["dH"], b["dH"], atol=1e-13)
+    # d/dW of L(H (W/tau)^T) = (1/tau) dL/dW' at W' = W / tau
+    np.testing.assert_allclose(a["dW"], b["dW"] / tau, atol=1e-13)
+
+
+def test_temperature_one_is_off():
+    H, W = rand_problem(3, 4, 7, 23)
+    y = np.array([1, 2, 6])
+    a, b = O.ce_fused(H, W, y), O.ce_fused(H, W, y, tau=np.ones(3))
+    np.testing.assert_array_equal(a["dW"], b["dW"])
+    np.testing.assert_array_equal(a["loss_rows"], b["loss_rows"])
