@@ -239,6 +239,74 @@ def backward(mode: int, H, W, targets, grad, ref_logp=None, tau=None) -> dict:
     return dict(G=G, dH=dH, dW=dW, lse=lse)
 
 
+# ---------------------------------------------------------------- renormalised support set
+# The other reading of "candidate-restricted log-probabilities": log-probs normalised over the
+# row's distinct valid candidate ids (the support) instead of the whole vocabulary.
+
+def support_renorm_logprob(H, W, ids, tau=None) -> dict:
+    """lpK_ik = z_i,c_ik - log sum_{c in S_i} exp z_ic, S_i the distinct valid ids of row i;
+    lseK_i is that log-normaliser (0 for a row without candidates); padding slots get 0."""
+    z = logits(H, W, tau)
+    N, V = z.shape
+    c = as_i64(ids)
+    lp = np.zeros(c.shape)
+    lse = np.zeros(N)
+    for i in range(N):
+        S = sorted({int(v) for v in c[i] if 0 <= v < V})
+        if not S:
+            continue
+        zs = z[i, S]
+        m = zs.max()
+        lse[i] = m + np.log(np.exp(zs - m).sum())
+        for k in range(c.shape[1]):
+            if 0 <= c[i, k] < V:
+                lp[i, k] = z[i, c[i, k]] - lse[i]
+    return dict(lp=lp, lse=lse, z=z)
+
+
+def support_renorm_kl(H, W, ids, ref_logp, tau=None) -> dict:
+    """KL_i = sum_k exp(r_ik) (r_ik - lpK_ik) over valid slots; mean over all N rows."""
+    s = support_renorm_logprob(H, W, ids, tau)
+    c = as_i64(ids)
+    V = s["z"].shape[1]
+    r = as_f64(ref_logp).reshape(c.shape)
+    ok = (c >= 0) & (c < V)
+    kl = np.where(ok, np.exp(r) * (r - s["lp"]), 0.0).sum(axis=1)
+    N = c.shape[0]
+    s.update(kl_rows=kl, kl_mean=float(kl.sum() / N) if N else 0.0)
+    return s
+
+
+def backward_renorm(mode: int, H, W, ids, grad, ref_logp=None, tau=None) -> dict:
+    """Backward of sum_ik g_ik lpK_ik (BWD_SUPPORT_LOGPROB) or sum_i g_i KL_i (BWD_SUPPORT_KL)
+    over the renormalised support: with q = softmax of z over S_i,
+    dL/dz_ic = sum_{k: c_ik = c} w_ik - q_ic sum_k w_ik for c in S_i (w = g for log-probs,
+    w = -g_i exp(r_ik) for the KL), 0 outside S_i; times 1 / tau_i."""
+    s = support_renorm_logprob(H, W, ids, tau)
+    z, lse = s["z"], s["lse"]
+    N, V = z.shape
+    c = as_i64(ids)
+    K = c.shape[1]
+    if mode == BWD_SUPPORT_LOGPROB:
+        w = as_f64(grad).reshape(N, K)
+    elif mode == BWD_SUPPORT_KL:
+        w = -as_f64(grad).reshape(N)[:, None] * np.exp(as_f64(ref_logp).reshape(N, K))
+    else:
+        raise ValueError("renormalised backward exists for the support objectives only")
+    G = np.zeros_like(z)
+    for i in range(N):
+        S = sorted({int(v) for v in c[i] if 0 <= v < V})
+        if not S:
+            continue
+        q = np.exp(z[i, S] - lse[i])
+        wsum = sum(w[i, k] for k in range(K) if 0 <= c[i, k] < V)
+        for j, v in enumerate(S):
+            G[i, v] = sum(w[i, k] for k in range(K) if c[i, k] == v) - q[j] * wsum
+    G = G / tau_rows(tau, N)[:, None]
+    dH, dW = lm_head_backward(H, W, G)
+    return dict(G=G, dH=dH, dW=dW, lse=lse)
+
+
 def bf16_round(x: np.ndarray) -> np.ndarray:
     """Round fp64 -> fp32 -> bf16 (round to nearest even), returned as fp64 values."""
     f = np.asarray(x, dtype=np.float32)

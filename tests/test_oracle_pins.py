@@ -400,3 +400,50 @@ def test_temperature_one_is_off():
     a, b = O.ce_fused(H, W, y), O.ce_fused(H, W, y, tau=np.ones(3))
     np.testing.assert_array_equal(a["dW"], b["dW"])
     np.testing.assert_array_equal(a["loss_rows"], b["loss_rows"])
+
+
+# ---------------------------------------------------------------- renormalised support set
+
+def test_renorm_support_normalises_and_kl_identities():
+    H, W = rand_problem(3, 4, 10, 31)
+    ids = np.array([[1, 7, 3, 7], [0, 9, -1, 4], [2, 5, 6, 8]])   # a repeat and a padding slot
+    s = O.support_renorm_logprob(H, W, ids)
+    for i in range(3):
+        S = sorted({v for v in ids[i] if v >= 0})
+        tot = sum(np.exp(s["lp"][i, list(ids[i]).index(v)]) for v in S)
+        assert abs(tot - 1.0) < 1e-13
+    # against a brute-force softmax over the support, row 2
+    z = O.logits(H, W)[2, [2, 5, 6, 8]]
+    np.testing.assert_allclose(s["lp"][2], z - np.log(np.exp(z).sum()), atol=1e-13)
+    # KL = 0 against the model's own renormalised log-probs (distinct ids), >= 0 otherwise
+    ids_u = np.array([[1, 7, 3], [0, 9, 4], [2, 5, 6]])
+    lp = O.support_renorm_logprob(H, W, ids_u)["lp"]
+    np.testing.assert_allclose(O.support_renorm_kl(H, W, ids_u, lp)["kl_rows"], 0.0, atol=1e-14)
+    rng = np.random.default_rng(32)
+    r = rng.normal(size=ids_u.shape)
+    r -= np.log(np.exp(r).sum(axis=1, keepdims=True))
+    assert np.all(O.support_renorm_kl(H, W, ids_u, r)["kl_rows"] >= -1e-14)
+
+
+@pytest.mark.parametrize("tau", [None, np.array([0.6, 1.4, 1.0])])
+def test_fd_renorm_support(tau):
+    H, W = rand_problem(3, 4, 10, 33)
+    ids = np.array([[1, 7, 3, 7], [0, 9, -1, 4], [2, 5, 6, 8]])
+    gam = np.random.default_rng(34).normal(size=ids.shape)
+    b = O.backward_renorm(O.BWD_SUPPORT_LOGPROB, H, W, ids, gam, tau=tau)
+
+    def L():
+        lp = O.support_renorm_logprob(H, W, ids, tau)["lp"]
+        return float((lp * gam * (ids >= 0)).sum())
+
+    assert_fd(b["dH"], fd_grad(L, H))
+    assert_fd(b["dW"], fd_grad(L, W))
+    r = np.log(np.full(ids.shape, 0.25))
+    g = np.array([1.0, -0.5, 2.0])
+    b = O.backward_renorm(O.BWD_SUPPORT_KL, H, W, ids, g, r, tau=tau)
+
+    def Lk():
+        return float((O.support_renorm_kl(H, W, ids, r, tau)["kl_rows"] * g).sum())
+
+    assert_fd(b["dH"], fd_grad(Lk, H))
+    assert_fd(b["dW"], fd_grad(Lk, W))
