@@ -29,11 +29,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "LM-head+CE fwd+bwd TFLOP/s (6·N·V·d) and % of bf16 tensor peak, 1×B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# the sources of the GEMM kernels whose DRAM traffic profiles/traffic.json records
 KERNEL_SOURCES = ["lm_head_cross_tcgen05_b200/csrc/gemm.cuh",
                   "lm_head_cross_tcgen05_b200/csrc/epilogues.cuh",
-                  "lm_head_cross_tcgen05_b200/csrc/sm100.cuh",
-                  "lm_head_cross_tcgen05_b200/csrc/rowops.cuh",
-                  "lm_head_cross_tcgen05_b200/csrc/lmh_api.cu"]
+                  "lm_head_cross_tcgen05_b200/csrc/sm100.cuh"]
 
 
 def parse_args():
@@ -43,6 +42,11 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_vocab")
+    ap.add_argument("--entry", choices=["fused_ce", "ce_separate", "support_kl"],
+                    default="fused_ce",
+                    help="fused_ce: lmh_loss_fwd with dH/dW (the headline step); ce_separate: "
+                         "lmh_loss_fwd then lmh_loss_bwd (recomputed logits); support_kl: "
+                         "lmh_support_kl then lmh_loss_bwd of the mean KL")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -68,9 +72,15 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def workload_config(wl, chunk_rows, n_gpus):
-    return {"workload": f"{wl.name}: fused CE forward+backward, N={wl.N} d={wl.d} V={wl.V}, "
+ENTRY_TEXT = {"fused_ce": "fused CE forward+backward",
+              "ce_separate": "CE forward, then backward with recomputed logits",
+              "support_kl": "support-set KL forward (K candidates), then its backward"}
+
+
+def workload_config(wl, chunk_rows, n_gpus, entry="fused_ce"):
+    return {"workload": f"{wl.name}: {ENTRY_TEXT[entry]}, N={wl.N} d={wl.d} V={wl.V}, "
                         f"{wl.labels} labels, {wl.num_ignored} ignored rows, bf16 H/W",
+            "entry": entry,
             "N": wl.N, "d": wl.d, "V": wl.V, "chunk_rows": chunk_rows,
             "rows_per_gpu": wl.N, "total_rows": wl.N * n_gpus,
             "l2": "inputs larger than L2 (W alone is %.2f GB)" % (wl.V * wl.d * 2 / 1e9)}
@@ -277,10 +287,39 @@ def main():
                dW=torch.empty(V, d, dtype=bf, device=dev))
     stream = torch.cuda.current_stream()
 
-    def step(Hs=H, ys=y):
-        L.lmh_loss_fwd(shape, Hs, W, ys, out["loss_rows"], out["lse"], out["logprob"],
-                       out["argmax"], out["loss_mean"], out["n_valid"], None, out["dH"],
-                       out["dW"], None, workspace=ws, stream=stream)
+    if args.entry == "fused_ce":
+        def step(Hs=H, ys=y):
+            L.lmh_loss_fwd(shape, Hs, W, ys, out["loss_rows"], out["lse"], out["logprob"],
+                           out["argmax"], out["loss_mean"], out["n_valid"], None, out["dH"],
+                           out["dW"], None, workspace=ws, stream=stream)
+    elif args.entry == "ce_separate":
+        fshape = L.make_shape(N, d, V, 0, chunk, L.F_MEAN)
+        fws = L.workspace(fshape, L.ENTRY_LOSS_FWD, dev)
+        bshape = L.make_shape(N, d, V, 1, chunk, L.F_MEAN)
+        bws = L.workspace(bshape, L.ENTRY_LOSS_BWD, dev)
+
+        def step(Hs=H, ys=y):
+            L.lmh_loss_fwd(fshape, Hs, W, ys, out["loss_rows"], out["lse"], out["logprob"],
+                           out["argmax"], out["loss_mean"], out["n_valid"], workspace=fws,
+                           stream=stream)
+            # backward of the mean loss: no grad given, 1 / n_valid taken on the device
+            L.lmh_loss_bwd(bshape, L.BWD_CE, Hs, W, ys, out["lse"], None, None, out["dH"],
+                           out["dW"], None, workspace=bws, stream=stream)
+    else:
+        ids, ref = x["ids"], x["ref_logp"]
+        K = ids.shape[1]
+        sshape = L.make_shape(N, d, V, K, chunk, L.F_MEAN)
+        sws = L.workspace(sshape, L.ENTRY_SUPPORT_KL, dev)
+        bws = L.workspace(sshape, L.ENTRY_LOSS_BWD, dev)
+        kl_rows = torch.empty(N, dtype=f32, device=dev)
+        lp = torch.empty(N, K, dtype=f32, device=dev)
+
+        def step(Hs=H, ys=y):
+            L.lmh_support_kl(sshape, Hs, W, ids, ref, kl_rows, out["loss_mean"], lp, out["lse"],
+                             workspace=sws, stream=stream)
+            # backward of the mean KL: no grad given, 1 / N on the device
+            L.lmh_loss_bwd(sshape, L.BWD_SUPPORT_KL, Hs, W, ids, out["lse"], None, ref,
+                           out["dH"], out["dW"], None, workspace=bws, stream=stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -414,7 +453,7 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": workload_config(wl, chunk, world),
+                "config": workload_config(wl, chunk, world, args.entry),
                 "peak_frac": {"of_burst": value / world / peaks["bf16_tflops"],
                               "of_sustained": value / world / peaks["bf16_tflops_sustained"],
                               "peaks": peak_src},

@@ -68,11 +68,13 @@ typedef enum lmh_status {
 #define LMH_DEVERR_LABEL_RANGE 0x1u /* a label or candidate id was >= V          */
 #define LMH_DEVERR_TIMEOUT 0x2u     /* a bounded wait inside a kernel gave up     */
 #define LMH_DEVERR_NONFINITE 0x4u   /* a row's log-sum-exp came out inf or NaN    */
+#define LMH_DEVERR_TEMPERATURE 0x8u /* a per-row temperature was not finite and > 0 (used 1) */
 
 /* shape->flags */
 #define LMH_F_MEAN 0x1u         /* fused CE gradient is of the mean over valid rows    */
 #define LMH_F_FUSED_BWD 0x2u    /* sizing only: lmh_loss_fwd will also produce dH/dW   */
 #define LMH_F_DW_ACC_GIVEN 0x4u /* sizing only: the caller passes an fp32 dW_acc       */
+#define LMH_F_SUPPORT_RENORM 0x8u /* support entries: renormalise over the candidates   */
 
 /* entries, for lmh_workspace_size */
 #define LMH_ENTRY_LOSS_FWD 0
@@ -89,14 +91,23 @@ typedef enum lmh_status {
 
 #define LMH_MAX_K 1024 /* largest candidate count per row of the support entries */
 
+/*
+ * Temperature (miles-ext-kernels PR #14, lm_head op commit: temperature stages, tested off,
+ * scalar, per row and 1.0): every entry works on the tempered logits z_iv / tau_i with
+ * tau_i = temperature * row_temperature[i] (a factor that is 0 or absent counts as 1), and
+ * the gradients carry the chain-rule factor 1 / tau_i. With both off the results are bit for
+ * bit those without temperature. A per-row value that is not finite and > 0 is used as 1
+ * and flags LMH_DEVERR_TEMPERATURE.
+ */
 typedef struct lmh_shape {
-  int64_t N;          /* rows (tokens), >= 0                                     */
-  int64_t d;          /* hidden size, multiple of 64                             */
-  int64_t V;          /* vocabulary size, 1 .. 2^31 - 1                          */
-  int64_t K;          /* candidates per row for the support entries, 1..LMH_MAX_K */
-  int64_t chunk_rows; /* rows per chunk; 0 selects 4096                          */
-  uint32_t flags;     /* LMH_F_*                                                 */
-  uint32_t reserved;  /* must be 0                                               */
+  int64_t N;                    /* rows (tokens), >= 0                                 */
+  int64_t d;                    /* hidden size, multiple of 64                         */
+  int64_t V;                    /* vocabulary size, 1 .. 2^31 - 1                      */
+  int64_t K;                    /* candidates per row (support entries), 1..LMH_MAX_K  */
+  int64_t chunk_rows;           /* rows per chunk; 0 selects 4096                      */
+  uint32_t flags;               /* LMH_F_*                                             */
+  float temperature;            /* scalar temperature, finite and >= 0; 0 or 1: none   */
+  const float* row_temperature; /* device [N] per-row temperatures, or NULL            */
 } lmh_shape;
 
 /*
@@ -151,6 +162,9 @@ LMH_API lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, const
  *   LMH_BWD_SUPPORT_KL:      targets = ids [N, K]; grad [N] = dL/dKL_i; ref_logp [N, K];
  *                            alpha_i = g_i sum_k exp(r_ik), beta_ik = g_i exp(r_ik).
  * Candidate ids < 0 are padding and are skipped. lse [N] is the forward's output.
+ * grad may be NULL: every row term then has the weight 1, or 1 / count with LMH_F_MEAN in
+ * shape->flags (count: the valid rows of the labels for CE / LOGPROB, N for the support
+ * objectives), taken on the device without a host synchronisation.
  * dH, dW, dW_acc: as in lmh_loss_fwd (nullable; dW_acc accumulates in chunk order).
  */
 LMH_API lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,
@@ -185,6 +199,16 @@ LMH_API lmh_status lmh_support_logprob(const lmh_shape* shape, const lmh_bf16* H
  * with r = ref_logp the given reference log-probs.
  *   ids [N, K], ref_logp [N, K] fp32 in. kl_rows [N] fp32 out. kl_mean [1] fp32 out,
  *   nullable (mean over all N rows). lp [N, K] fp32 out, nullable. lse [N] out (required).
+ */
+/*
+ * LMH_F_SUPPORT_RENORM (the other reading of "candidate-restricted"): with this flag the
+ * support entries normalise over each row's distinct valid candidate ids instead of the whole
+ * vocabulary: lp_ik = z_i,c_ik - log sum_{distinct valid c} exp z_ic, and `lse` receives that
+ * log-normaliser (0 for a row without candidates). Only the K candidate logits are computed
+ * (K dot products per row). lmh_loss_bwd with LMH_BWD_SUPPORT_LOGPROB / LMH_BWD_SUPPORT_KL and
+ * the same flag takes that `lse` and forms the gradient on the candidates only: dH by a
+ * gather of W rows, dW by a scatter summed per vocabulary row in ascending row order (rows of
+ * dW with no candidate get 0, or keep dW_acc). chunk_rows plays no part in this path.
  */
 LMH_API lmh_status lmh_support_kl(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,
                           const int32_t* ids, const float* ref_logp, float* kl_rows,
@@ -226,6 +250,15 @@ LMH_API lmh_status lmh_read_errors(const void* workspace, uint32_t* errors, void
 LMH_API lmh_status lmh_logprob_noalloc(const lmh_shape* shape, const lmh_bf16* H,
                                        const lmh_bf16* W, const int32_t* labels, float* logprob,
                                        float* lse, void* stream);
+
+/*
+ * lmh_selftest_wait_timeout — failure-path self-test (not part of the method). Enqueues one
+ * thread that waits, with the bounded wait every kernel of this library uses, on an mbarrier
+ * that nothing arrives on. The wait gives up after timeout_ms (1..5000) and sets
+ * LMH_DEVERR_TIMEOUT in the workspace's error word (read it with lmh_read_errors); the
+ * context stays usable. workspace: at least 256 bytes, 256-byte aligned.
+ */
+LMH_API lmh_status lmh_selftest_wait_timeout(void* workspace, uint32_t timeout_ms, void* stream);
 
 /*
  * Measurement hook (not part of the method). lmh_profile_enable(1) makes every later call

@@ -17,18 +17,18 @@ from typing import Optional
 import torch
 
 from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEVERR_LABEL_RANGE,
-                   DEVERR_NONFINITE, DEVERR_TIMEOUT, ENTRY_LOGPROB, ENTRY_LOSS_BWD,
+                   DEVERR_NONFINITE, DEVERR_TEMPERATURE, DEVERR_TIMEOUT, ENTRY_LOGPROB, ENTRY_LOSS_BWD,
                    ENTRY_LOSS_FWD, ENTRY_SUPPORT_KL, ENTRY_SUPPORT_LOGPROB, F_DW_ACC_GIVEN,
-                   F_FUSED_BWD, F_MEAN, IGNORE_INDEX, MAX_K, STATUS_NAMES, lib, lmh_shape)
+                   F_FUSED_BWD, F_MEAN, F_SUPPORT_RENORM, IGNORE_INDEX, MAX_K, STATUS_NAMES, lib, lmh_shape)
 
 __all__ = [
     "lmh_shape", "make_shape", "lmh_workspace_size", "lmh_loss_fwd", "lmh_loss_bwd",
     "lmh_logprob", "lmh_support_logprob", "lmh_support_kl", "lmh_read_errors", "LmhError",
     "loss_fwd", "loss_bwd", "logprob", "support_logprob", "support_kl", "workspace",
     "IGNORE_INDEX", "BWD_CE", "BWD_LOGPROB", "BWD_SUPPORT_LOGPROB", "BWD_SUPPORT_KL",
-    "F_MEAN", "F_FUSED_BWD", "F_DW_ACC_GIVEN", "ENTRY_LOSS_FWD", "ENTRY_LOSS_BWD",
+    "F_MEAN", "F_FUSED_BWD", "F_DW_ACC_GIVEN", "F_SUPPORT_RENORM", "ENTRY_LOSS_FWD", "ENTRY_LOSS_BWD",
     "ENTRY_LOGPROB", "ENTRY_SUPPORT_LOGPROB", "ENTRY_SUPPORT_KL", "DEVERR_LABEL_RANGE",
-    "DEVERR_TIMEOUT", "DEVERR_NONFINITE", "MAX_K",
+    "DEVERR_TIMEOUT", "DEVERR_NONFINITE", "DEVERR_TEMPERATURE", "MAX_K",
 ]
 
 lib()  # load now: a missing library is an import error, never a silent fallback
@@ -40,9 +40,18 @@ class LmhError(RuntimeError):
         self.status = status
 
 
-def make_shape(N: int, d: int, V: int, K: int = 0, chunk_rows: int = 0,
-               flags: int = 0) -> lmh_shape:
-    return lmh_shape(int(N), int(d), int(V), int(K), int(chunk_rows), int(flags), 0)
+def make_shape(N: int, d: int, V: int, K: int = 0, chunk_rows: int = 0, flags: int = 0,
+               temperature=None) -> lmh_shape:
+    """temperature: None (off), a float (one temperature for every row) or a CUDA float32
+    tensor [N] of per-row temperatures (kept alive by the caller for the call)."""
+    scalar, rows = 0.0, None
+    if isinstance(temperature, torch.Tensor):
+        if temperature.numel() != int(N):
+            raise ValueError("per-row temperature must have N elements")
+        rows = _p(temperature, _f32, "temperature")
+    elif temperature is not None:
+        scalar = float(temperature)
+    return lmh_shape(int(N), int(d), int(V), int(K), int(chunk_rows), int(flags), scalar, rows)
 
 
 def _p(t: Optional[torch.Tensor], dtype=None, what: str = "tensor"):
@@ -145,7 +154,7 @@ def workspace(shape: lmh_shape, entry: int, device) -> torch.Tensor:
 
 def loss_fwd(H, W, labels, *, chunk_rows: int = 0, mean: bool = True, grads: bool = False,
              want_dH: bool = True, want_dW: bool = True, dW_acc=None, n_valid_given=None,
-             ws=None, stream=None) -> dict:
+             temperature=None, ws=None, stream=None) -> dict:
     """CE forward (loss_rows, lse, logprob, argmax, loss_mean, n_valid); with grads=True also
     dH / dW of the mean (or summed) loss, fused with the forward."""
     N, d = H.shape
@@ -153,7 +162,7 @@ def loss_fwd(H, W, labels, *, chunk_rows: int = 0, mean: bool = True, grads: boo
     dev = H.device
     flags = (F_MEAN if mean else 0) | (F_FUSED_BWD if grads else 0) | (
         F_DW_ACC_GIVEN if dW_acc is not None else 0)
-    shape = make_shape(N, d, V, 0, chunk_rows, flags)
+    shape = make_shape(N, d, V, 0, chunk_rows, flags, temperature)
     out = dict(loss_rows=torch.empty(N, dtype=_f32, device=dev),
                lse=torch.empty(N, dtype=_f32, device=dev),
                logprob=torch.empty(N, dtype=_f32, device=dev),
@@ -172,13 +181,17 @@ def loss_fwd(H, W, labels, *, chunk_rows: int = 0, mean: bool = True, grads: boo
 
 
 def loss_bwd(mode: int, H, W, targets, lse, grad, ref_logp=None, *, chunk_rows: int = 0,
-             want_dH: bool = True, want_dW: bool = True, dW_acc=None, ws=None,
-             stream=None) -> dict:
+             want_dH: bool = True, want_dW: bool = True, dW_acc=None, temperature=None,
+             mean: bool = False, renorm: bool = False, ws=None, stream=None) -> dict:
+    """Backward of one objective (LMH_BWD_*). grad=None: unit row weights, or 1 / count with
+    mean=True, taken on the device."""
     N, d = H.shape
     V = W.shape[0]
     K = targets.shape[1] if targets.dim() == 2 else 1
     dev = H.device
-    shape = make_shape(N, d, V, K, chunk_rows, F_DW_ACC_GIVEN if dW_acc is not None else 0)
+    flags = ((F_DW_ACC_GIVEN if dW_acc is not None else 0) | (F_MEAN if mean else 0)
+             | (F_SUPPORT_RENORM if renorm else 0))
+    shape = make_shape(N, d, V, K, chunk_rows, flags, temperature)
     out = dict(dH=torch.empty(N, d, dtype=_bf, device=dev) if want_dH else None,
                dW=torch.empty(V, d, dtype=_bf, device=dev) if want_dW else None)
     ws = workspace(shape, ENTRY_LOSS_BWD, dev) if ws is None else ws
@@ -188,9 +201,10 @@ def loss_bwd(mode: int, H, W, targets, lse, grad, ref_logp=None, *, chunk_rows: 
     return out
 
 
-def logprob(H, W, labels, *, chunk_rows: int = 0, ws=None, stream=None) -> dict:
+def logprob(H, W, labels, *, chunk_rows: int = 0, temperature=None, ws=None,
+            stream=None) -> dict:
     N, d = H.shape
-    shape = make_shape(N, d, W.shape[0], 0, chunk_rows)
+    shape = make_shape(N, d, W.shape[0], 0, chunk_rows, 0, temperature)
     out = dict(logprob=torch.empty(N, dtype=_f32, device=H.device),
                lse=torch.empty(N, dtype=_f32, device=H.device))
     ws = workspace(shape, ENTRY_LOGPROB, H.device) if ws is None else ws
@@ -199,10 +213,13 @@ def logprob(H, W, labels, *, chunk_rows: int = 0, ws=None, stream=None) -> dict:
     return out
 
 
-def support_logprob(H, W, ids, *, chunk_rows: int = 0, ws=None, stream=None) -> dict:
+def support_logprob(H, W, ids, *, chunk_rows: int = 0, temperature=None, renorm: bool = False,
+                    ws=None, stream=None) -> dict:
+    """renorm=True: log-probs normalised over each row's candidates (LMH_F_SUPPORT_RENORM)."""
     N, d = H.shape
     K = ids.shape[1]
-    shape = make_shape(N, d, W.shape[0], K, chunk_rows)
+    shape = make_shape(N, d, W.shape[0], K, chunk_rows, F_SUPPORT_RENORM if renorm else 0,
+                       temperature)
     out = dict(lp=torch.empty(N, K, dtype=_f32, device=H.device),
                lse=torch.empty(N, dtype=_f32, device=H.device))
     ws = workspace(shape, ENTRY_SUPPORT_LOGPROB, H.device) if ws is None else ws
@@ -211,10 +228,12 @@ def support_logprob(H, W, ids, *, chunk_rows: int = 0, ws=None, stream=None) -> 
     return out
 
 
-def support_kl(H, W, ids, ref_logp, *, chunk_rows: int = 0, ws=None, stream=None) -> dict:
+def support_kl(H, W, ids, ref_logp, *, chunk_rows: int = 0, temperature=None,
+               renorm: bool = False, ws=None, stream=None) -> dict:
     N, d = H.shape
     K = ids.shape[1]
-    shape = make_shape(N, d, W.shape[0], K, chunk_rows)
+    shape = make_shape(N, d, W.shape[0], K, chunk_rows, F_SUPPORT_RENORM if renorm else 0,
+                       temperature)
     dev = H.device
     out = dict(kl_rows=torch.empty(N, dtype=_f32, device=dev),
                kl_mean=torch.empty(1, dtype=_f32, device=dev),

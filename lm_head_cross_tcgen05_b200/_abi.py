@@ -18,8 +18,8 @@ STATUS_NAMES = {0: "LMH_OK", 1: "LMH_ERR_INVALID_ARG", 2: "LMH_ERR_UNSUPPORTED_D
                 6: "LMH_ERR_SCRATCH_LIMIT"}
 
 IGNORE_INDEX = -100
-DEVERR_LABEL_RANGE, DEVERR_TIMEOUT, DEVERR_NONFINITE = 0x1, 0x2, 0x4
-F_MEAN, F_FUSED_BWD, F_DW_ACC_GIVEN = 0x1, 0x2, 0x4
+DEVERR_LABEL_RANGE, DEVERR_TIMEOUT, DEVERR_NONFINITE, DEVERR_TEMPERATURE = 0x1, 0x2, 0x4, 0x8
+F_MEAN, F_FUSED_BWD, F_DW_ACC_GIVEN, F_SUPPORT_RENORM = 0x1, 0x2, 0x4, 0x8
 ENTRY_LOSS_FWD, ENTRY_LOSS_BWD, ENTRY_LOGPROB, ENTRY_SUPPORT_LOGPROB, ENTRY_SUPPORT_KL = range(5)
 BWD_CE, BWD_LOGPROB, BWD_SUPPORT_LOGPROB, BWD_SUPPORT_KL = range(4)
 MAX_K = 1024
@@ -27,7 +27,8 @@ MAX_K = 1024
 
 class lmh_shape(ctypes.Structure):
     _fields_ = [("N", c_int64), ("d", c_int64), ("V", c_int64), ("K", c_int64),
-                ("chunk_rows", c_int64), ("flags", c_uint32), ("reserved", c_uint32)]
+                ("chunk_rows", c_int64), ("flags", c_uint32), ("temperature", ctypes.c_float),
+                ("row_temperature", c_void_p)]
 
 
 _P = c_void_p
@@ -40,6 +41,7 @@ _SIGS = {
     "lmh_support_kl": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 9 + [c_size_t, _P]),
     "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),
     "lmh_logprob_noalloc": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6),
+    "lmh_selftest_wait_timeout": (c_int, [_P, c_uint32, _P]),
     "lmh_profile_enable": (c_int, [c_int]),
     "lmh_profile_read": (c_int, [c_int, ctypes.POINTER(ctypes.c_int32),
                                  ctypes.POINTER(ctypes.c_float)]),

@@ -136,6 +136,7 @@ struct EpiStats {
     float* part_m;      // [rows, T]
     float* part_s;      // [rows, T]
     int32_t* part_i;    // [rows, T]
+    Temperature temp;   // logits are z / tau_i
   };
 
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
@@ -145,10 +146,11 @@ struct EpiStats {
     const long long grow = p.row0 + row;
     const int n0 = nb * BN;
     const bool full = n0 + BN <= p.V;
+    const float it = rv ? inv_temperature(p.temp, grow) : 1.f;
     TargetCursor<TK> cur;
     if (rv) cur.init(p.tg, grow, n0, p.V); else cur.none();
 
-    // pass 1: maximum, its first column, target logits
+    // pass 1: maximum, its first column, target logits (of the tempered logits)
     float m = kNegInf;
     int am = n0;
 #pragma unroll 1
@@ -156,6 +158,8 @@ struct EpiStats {
       float v[32];
       tmem_ld32(taddr + sl * 32, v);
       const int col0 = n0 + sl * 32;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= it;
       if (!full) {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
@@ -176,6 +180,7 @@ struct EpiStats {
 
     // pass 2: sum of exp(z - m); optionally p~ = exp(z - m) to the chunk buffer
     const float moff = -m * kLog2e;
+    const float sc = it * kLog2e;
     float s0 = 0.f, s1 = 0.f;
     const int wrow = mb * BM + ctx.row_w;  // first chunk row of this warp
 #pragma unroll 1
@@ -186,8 +191,8 @@ struct EpiStats {
       tmem_ld32(taddr + sb * 64 + 32, b);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float ea = fast_exp2(fmaf(a[j], kLog2e, moff));
-        const float eb = fast_exp2(fmaf(b[j], kLog2e, moff));
+        const float ea = fast_exp2(fmaf(a[j], sc, moff));
+        const float eb = fast_exp2(fmaf(b[j], sc, moff));
         a[j] = (full || col0 + j < p.V) ? ea : 0.f;
         b[j] = (full || col0 + 32 + j < p.V) ? eb : 0.f;
         s0 += a[j];
@@ -221,6 +226,7 @@ struct EpiGrad {
     const float* lse;    // [N]
     const float* alpha;  // [N]
     const float* beta;   // [N] (kLabel) or [N, K] in sorted order (kCands)
+    Temperature temp;    // logits are z / tau_i (alpha and beta carry the 1 / tau_i factor)
   };
 
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
@@ -232,6 +238,7 @@ struct EpiGrad {
     const bool full = n0 + BN <= p.V;
     const float al = rv ? p.alpha[grow] : 0.f;
     const float loff = rv ? -p.lse[grow] * kLog2e : 0.f;
+    const float sc = (rv ? inv_temperature(p.temp, grow) : 1.f) * kLog2e;
     TargetCursor<TK> cur;
     if (rv) cur.init(p.tg, grow, n0, p.V); else cur.none();
     const int wrow = mb * BM + ctx.row_w;
@@ -243,8 +250,8 @@ struct EpiGrad {
       tmem_ld32(taddr + sb * 64 + 32, b);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float ea = al * fast_exp2(fmaf(a[j], kLog2e, loff));
-        const float eb = al * fast_exp2(fmaf(b[j], kLog2e, loff));
+        const float ea = al * fast_exp2(fmaf(a[j], sc, loff));
+        const float eb = al * fast_exp2(fmaf(b[j], sc, loff));
         a[j] = (full || col0 + j < p.V) ? ea : 0.f;
         b[j] = (full || col0 + 32 + j < p.V) ? eb : 0.f;
       }

@@ -13,6 +13,7 @@
 #include "epilogues.cuh"
 #include "gemm.cuh"
 #include "rowops.cuh"
+#include "sparse.cuh"
 
 using namespace lmh;
 
@@ -31,21 +32,29 @@ struct Plan {
   bool cands;   // per-row candidate lists (support entries, candidate backward)
   bool gbuf;    // chunk softmax / gradient buffer
   bool acc;     // internal fp32 dW accumulator
+  bool renorm;  // support entries renormalised over the candidate set (sparse path)
   size_t o_zt, o_sorted, o_nuniq, o_rank, o_pm, o_ps, o_pi, o_alpha, o_beta, o_gbuf, o_acc;
+  size_t o_gu, o_cnt, o_off, o_fill, o_prow, o_pslot;  // sparse backward
   size_t total;
+  Temperature temp;  // logits are z / tau_i
 };
 
 bool shape_ok(const lmh_shape* s) {
   if (!s) return false;
   if (s->N < 0 || s->d <= 0 || (s->d % 64) != 0 || s->V <= 0 || s->V > 0x7fffffffLL)
     return false;
-  if (s->d > (1LL << 24) || s->chunk_rows < 0 || s->reserved != 0) return false;
+  if (s->d > (1LL << 24) || s->chunk_rows < 0) return false;
+  if (!(s->temperature >= 0.f && s->temperature < 3.0e38f)) return false;  // NaN fails too
+  if ((reinterpret_cast<uintptr_t>(s->row_temperature) & 3u) != 0) return false;
   return true;
 }
 
 // fused: the entry keeps a [c, Vp] bf16 buffer; need_acc: an fp32 [V, d] accumulator.
 Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   Plan p{};
+  const float t = s->temperature;
+  p.temp.inv_scalar = (t > 0.f && t != 1.f) ? 1.f / t : 1.f;
+  p.temp.rows = s->row_temperature;
   p.N = s->N;
   p.d = s->d;
   p.V = s->V;
@@ -57,9 +66,12 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   p.cands = (entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL ||
              entry == LMH_ENTRY_LOSS_BWD);
   p.K = p.cands ? (s->K > 0 ? s->K : 1) : 1;
-  p.gbuf = (entry == LMH_ENTRY_LOSS_BWD) || (entry == LMH_ENTRY_LOSS_FWD && fused);
+  p.renorm = p.cands && (s->flags & LMH_F_SUPPORT_RENORM);
+  p.gbuf = !p.renorm &&
+           ((entry == LMH_ENTRY_LOSS_BWD) || (entry == LMH_ENTRY_LOSS_FWD && fused));
   p.acc = p.gbuf && dw_without_acc && p.nchunks > 1;
   const bool stats = entry != LMH_ENTRY_LOSS_BWD;
+  const bool partials = stats && !p.renorm;
   size_t o = sizeof(WsHeader);
   auto take = [&](size_t bytes) {
     const size_t at = o;
@@ -67,18 +79,25 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
     return at;
   };
   const size_t N = static_cast<size_t>(p.N);
-  p.o_zt = stats ? take(N * p.K * 4) : 0;
+  p.o_zt = (stats || p.renorm) ? take(N * p.K * 4) : 0;
   p.o_sorted = p.cands ? take(N * p.K * 4) : 0;
   p.o_nuniq = p.cands ? take(N * 4) : 0;
   p.o_rank = p.cands ? take(N * p.K * 4) : 0;
   const size_t cT = static_cast<size_t>(p.c) * p.T;
-  p.o_pm = stats ? take(cT * 4) : 0;
-  p.o_ps = stats ? take(cT * 4) : 0;
-  p.o_pi = stats ? take(cT * 4) : 0;
+  p.o_pm = partials ? take(cT * 4) : 0;
+  p.o_ps = partials ? take(cT * 4) : 0;
+  p.o_pi = partials ? take(cT * 4) : 0;
   p.o_alpha = (entry == LMH_ENTRY_LOSS_BWD) ? take(N * 4) : 0;
   p.o_beta = (entry == LMH_ENTRY_LOSS_BWD) ? take(N * p.K * 4) : 0;
   p.o_gbuf = p.gbuf ? take(static_cast<size_t>(p.c) * p.Vp * 2) : 0;
   p.o_acc = p.acc ? take(static_cast<size_t>(p.V) * p.d * 4) : 0;
+  const bool sparse_bwd = p.renorm && entry == LMH_ENTRY_LOSS_BWD;
+  p.o_gu = sparse_bwd ? take(N * p.K * 4) : 0;
+  p.o_cnt = sparse_bwd ? take(static_cast<size_t>(p.V) * 4) : 0;
+  p.o_off = sparse_bwd ? take((static_cast<size_t>(p.V) + 1) * 4) : 0;
+  p.o_fill = sparse_bwd ? take(static_cast<size_t>(p.V) * 4) : 0;
+  p.o_prow = sparse_bwd ? take(N * p.K * 4) : 0;
+  p.o_pslot = sparse_bwd ? take(N * p.K * 4) : 0;
   p.total = o;
   return p;
 }
@@ -119,12 +138,14 @@ lmh_status current_device(int* dev_out, int* sms) {
 enum KernelId {
   KID_COUNT_LABELS, KID_PREP_CANDS, KID_GEMM_LOGITS, KID_GEMM_LOGITS_P, KID_GEMM_GRAD,
   KID_GEMM_DH, KID_GEMM_DW, KID_FINALIZE, KID_GBUILD, KID_FIX_LABELS, KID_MEAN,
-  KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_COUNT
+  KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_SUPPORT_DOTS, KID_SUPPORT_LSE,
+  KID_SUPPORT_DH, KID_SUPPORT_DW, KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "count_labels", "prep_cands", "gemm_logits_stats", "gemm_logits_stats_store",
     "gemm_logits_grad", "gemm_dH", "gemm_dW", "row_finalize", "gbuild", "fix_labels",
-    "mean", "support_out", "bwd_coef", "cast_bf16"};
+    "mean", "support_out", "bwd_coef", "cast_bf16", "support_dots", "support_lse",
+    "support_grad_dh", "support_dw"};
 
 struct ProfRec {
   int id;
@@ -316,6 +337,7 @@ lmh_status run_stats(const Plan& P, int dev, int sms, const lmh_bf16* H, const l
   ep.part_m = ws.at<float>(P.o_pm);
   ep.part_s = ws.at<float>(P.o_ps);
   ep.part_i = ws.at<int32_t>(P.o_pi);
+  ep.temp = P.temp;
   return launch_gemm<EpiStats<TK, kStoreP>>(dev, sms, ta, tb, tc, rows, P.V, P.d, kOrderLogits,
                                            &ws.h->err, ep, st);
 }
@@ -342,6 +364,7 @@ lmh_status run_finalize(const Plan& P, int kind, int64_t r0, int rows, const int
   f.mean = mean;
   f.n_given = n_given;
   f.h = ws.h;
+  f.temp = P.temp;
   const int warps = 8;
   ProfScope ps(KID_FINALIZE, st);
   finalize_rows_kernel<<<static_cast<unsigned>(cdiv(rows, warps)), 32 * warps, 0, st>>>(f);
@@ -416,6 +439,61 @@ lmh_status prep_cands(const Plan& P, const int32_t* ids, const Ws& ws, cudaStrea
   prep_cands_kernel<<<static_cast<unsigned>(blocks), threads, 3 * P.K * sizeof(int32_t), st>>>(
       ids, P.N, static_cast<int>(P.K), static_cast<int>(P.V), ws.at<int32_t>(P.o_sorted),
       ws.at<int32_t>(P.o_nuniq), ws.at<int32_t>(P.o_rank), ws.h);
+  return last_launch();
+}
+
+// Logits of each row's distinct candidates (renormalised support entries): zt [N, K].
+lmh_status support_logits(const Plan& P, const lmh_bf16* H, const lmh_bf16* W, const Ws& ws,
+                          cudaStream_t st) {
+  ProfScope ps(KID_SUPPORT_DOTS, st);
+  const int64_t blocks = P.N < 65535 ? P.N : 65535;
+  support_dots_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      P.N, static_cast<int>(P.K), static_cast<int>(P.d),
+      reinterpret_cast<const __nv_bfloat16*>(H), reinterpret_cast<const __nv_bfloat16*>(W),
+      ws.at<int32_t>(P.o_sorted), ws.at<int32_t>(P.o_nuniq), P.temp, ws.at<float>(P.o_zt));
+  return last_launch();
+}
+
+// Backward of the renormalised support objectives: G on the candidates only, dH by a gather
+// of W rows, dW by a scatter whose pairs are grouped by id and summed in row order.
+lmh_status sparse_backward(const Plan& P, const lmh_bf16* H, const lmh_bf16* W, const float* lse,
+                           lmh_bf16* dH, lmh_bf16* dW, float* dW_acc, const Ws& ws,
+                           cudaStream_t st) {
+  const int K = static_cast<int>(P.K), d = static_cast<int>(P.d), V = static_cast<int>(P.V);
+  LMH_TRY(support_logits(P, H, W, ws, st));
+  const int64_t rblocks = P.N < 65535 ? P.N : 65535;
+  {
+    ProfScope ps(KID_SUPPORT_DH, st);
+    support_grad_dh_kernel<<<static_cast<unsigned>(rblocks), 256, K * sizeof(float), st>>>(
+        P.N, K, d, reinterpret_cast<const __nv_bfloat16*>(W), ws.at<int32_t>(P.o_sorted),
+        ws.at<int32_t>(P.o_nuniq), ws.at<float>(P.o_zt), lse, ws.at<float>(P.o_alpha),
+        ws.at<float>(P.o_beta), ws.at<float>(P.o_gu), reinterpret_cast<__nv_bfloat16*>(dH));
+  }
+  LMH_TRY(last_launch());
+  if (!dW && !dW_acc) return LMH_OK;
+  if (cudaMemsetAsync(ws.at<int32_t>(P.o_cnt), 0, size_t(V) * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(ws.at<int32_t>(P.o_fill), 0, size_t(V) * 4, st) != cudaSuccess)
+    return LMH_ERR_CUDA;
+  ProfScope ps(KID_SUPPORT_DW, st);
+  const int64_t pb = cdiv(P.N * K, 256);
+  const unsigned pblocks = static_cast<unsigned>(pb < 4096 ? pb : 4096);
+  support_count_kernel<<<pblocks, 256, 0, st>>>(P.N, K, ws.at<int32_t>(P.o_sorted),
+                                                ws.at<int32_t>(P.o_nuniq), ws.at<int32_t>(P.o_cnt));
+  LMH_TRY(last_launch());
+  scan_kernel<<<1, 1024, 0, st>>>(V, ws.at<int32_t>(P.o_cnt), ws.at<int32_t>(P.o_off));
+  LMH_TRY(last_launch());
+  support_place_kernel<<<pblocks, 256, 0, st>>>(
+      P.N, K, ws.at<int32_t>(P.o_sorted), ws.at<int32_t>(P.o_nuniq), ws.at<int32_t>(P.o_off),
+      ws.at<int32_t>(P.o_fill), ws.at<int32_t>(P.o_prow), ws.at<int32_t>(P.o_pslot));
+  LMH_TRY(last_launch());
+  support_sort_buckets_kernel<<<static_cast<unsigned>(cdiv(V, 256)), 256, 0, st>>>(
+      V, ws.at<int32_t>(P.o_off), ws.at<int32_t>(P.o_prow), ws.at<int32_t>(P.o_pslot));
+  LMH_TRY(last_launch());
+  const int64_t vblocks = V < 65535 ? V : 65535;
+  support_dw_kernel<<<static_cast<unsigned>(vblocks), 256, 0, st>>>(
+      V, K, d, reinterpret_cast<const __nv_bfloat16*>(H), ws.at<int32_t>(P.o_off),
+      ws.at<int32_t>(P.o_prow), ws.at<int32_t>(P.o_pslot), ws.at<float>(P.o_gu), dW_acc,
+      dW_acc ? 2 : 0, reinterpret_cast<__nv_bfloat16*>(dW));
   return last_launch();
 }
 
@@ -498,7 +576,7 @@ extern "C" lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, co
         ProfScope ps(KID_FIX_LABELS, st);
         fix_labels_kernel<<<static_cast<unsigned>(cdiv(rows, 256)), 256, 0, st>>>(
             rows, r0, static_cast<int>(P.V), P.Vp, labels, ws.at<float>(P.o_zt), lse, mean,
-            n_valid_given, ws.h, G);
+            n_valid_given, ws.h, P.temp, G);
       }
       LMH_TRY(last_launch());
       LMH_TRY(run_backward_gemms(P, dev, sms, H, W, r0, rows, static_cast<int>(ci), dH, dW,
@@ -561,16 +639,24 @@ static lmh_status support_fwd(const lmh_shape* shape, int entry, const lmh_bf16*
     return LMH_OK;
   }
   LMH_TRY(prep_cands(P, ids, ws, st));
-  Targets tg{};
-  tg.sorted = ws.at<int32_t>(P.o_sorted);
-  tg.nuniq = ws.at<int32_t>(P.o_nuniq);
-  tg.K = static_cast<int>(P.K);
-  for (int64_t ci = 0; ci < P.nchunks; ++ci) {
-    const int64_t r0 = ci * P.c;
-    const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
-    LMH_TRY((run_stats<kCands, false>(P, dev, sms, H, W, tg, r0, rows, ws, st)));
-    LMH_TRY(run_finalize(P, 2, r0, rows, nullptr, lse, nullptr, nullptr, nullptr, 0, 0, nullptr,
-                         ws, st));
+  if (P.renorm) {
+    LMH_TRY(support_logits(P, H, W, ws, st));
+    ProfScope ps(KID_SUPPORT_LSE, st);
+    support_lse_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
+        P.N, static_cast<int>(P.K), ws.at<int32_t>(P.o_nuniq), ws.at<float>(P.o_zt), lse, ws.h);
+    LMH_TRY(last_launch());
+  } else {
+    Targets tg{};
+    tg.sorted = ws.at<int32_t>(P.o_sorted);
+    tg.nuniq = ws.at<int32_t>(P.o_nuniq);
+    tg.K = static_cast<int>(P.K);
+    for (int64_t ci = 0; ci < P.nchunks; ++ci) {
+      const int64_t r0 = ci * P.c;
+      const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
+      LMH_TRY((run_stats<kCands, false>(P, dev, sms, H, W, tg, r0, rows, ws, st)));
+      LMH_TRY(run_finalize(P, 2, r0, rows, nullptr, lse, nullptr, nullptr, nullptr, 0, 0,
+                           nullptr, ws, st));
+    }
   }
   {
     ProfScope ps(KID_SUPPORT_OUT, st);
@@ -614,10 +700,12 @@ extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_b
     return LMH_ERR_INVALID_ARG;
   const bool cands = mode >= LMH_BWD_SUPPORT_LOGPROB;
   if (cands && (shape->K < 1 || shape->K > LMH_MAX_K)) return LMH_ERR_INVALID_ARG;
-  const Plan P = make_plan(shape, LMH_ENTRY_LOSS_BWD, true, dW && !dW_acc);
+  lmh_shape sh = *shape;  // the renormalised path exists for the support objectives only
+  if (!cands) sh.flags &= ~LMH_F_SUPPORT_RENORM;
+  const Plan P = make_plan(&sh, LMH_ENTRY_LOSS_BWD, true, dW && !dW_acc);
   int dev, sms;
   LMH_TRY(common_checks(shape, H, W, workspace, workspace_bytes, P.total, &dev, &sms));
-  if (P.N > 0 && (!targets || !lse || !grad)) return LMH_ERR_INVALID_ARG;
+  if (P.N > 0 && (!targets || !lse)) return LMH_ERR_INVALID_ARG;
   if (mode == LMH_BWD_SUPPORT_KL && P.N > 0 && !ref_logp) return LMH_ERR_INVALID_ARG;
   if (!aligned16(dH) || !aligned16(dW) || !aligned16(dW_acc)) return LMH_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -643,9 +731,11 @@ extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_b
     bwd_coef_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
       mode, P.N, cands ? static_cast<int>(P.K) : 1, static_cast<int>(P.V), targets, grad,
       ref_logp, cands ? ws.at<int32_t>(P.o_rank) : nullptr,
-      cands ? ws.at<int32_t>(P.o_nuniq) : nullptr, alpha, beta);
+      cands ? ws.at<int32_t>(P.o_nuniq) : nullptr, P.temp,
+      (shape->flags & LMH_F_MEAN) ? 1 : 0, ws.h, alpha, beta);
   }
   LMH_TRY(last_launch());
+  if (P.renorm) return sparse_backward(P, H, W, lse, dH, dW, dW_acc, ws, st);
   for (int64_t ci = 0; ci < P.nchunks; ++ci) {
     const int64_t r0 = ci * P.c;
     const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
@@ -654,11 +744,13 @@ extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_b
         !tmap_out(&tc, ws.at<__nv_bfloat16>(P.o_gbuf), P.Vp, rows, P.Vp))
       return LMH_ERR_CUDA;
     if (cands) {
-      EpiGrad<kCands>::Params ep{rows, r0, static_cast<int>(P.V), P.Vp, tg, lse, alpha, beta};
+      EpiGrad<kCands>::Params ep{rows, r0, static_cast<int>(P.V), P.Vp, tg, lse, alpha, beta,
+                                 P.temp};
       LMH_TRY(launch_gemm<EpiGrad<kCands>>(dev, sms, ta, tb, tc, rows, P.V, P.d, kOrderLogits,
                                            &ws.h->err, ep, st));
     } else {
-      EpiGrad<kLabel>::Params ep{rows, r0, static_cast<int>(P.V), P.Vp, tg, lse, alpha, beta};
+      EpiGrad<kLabel>::Params ep{rows, r0, static_cast<int>(P.V), P.Vp, tg, lse, alpha, beta,
+                                 P.temp};
       LMH_TRY(launch_gemm<EpiGrad<kLabel>>(dev, sms, ta, tb, tc, rows, P.V, P.d, kOrderLogits,
                                            &ws.h->err, ep, st));
     }
@@ -675,6 +767,19 @@ extern "C" lmh_status lmh_read_errors(const void* workspace, uint32_t* errors, v
   if (cudaMemcpy(errors, workspace, 4, cudaMemcpyDeviceToHost) != cudaSuccess)
     return LMH_ERR_CUDA;
   return LMH_OK;
+}
+
+extern "C" lmh_status lmh_selftest_wait_timeout(void* workspace, uint32_t timeout_ms,
+                                                void* stream) {
+  if (!workspace || timeout_ms < 1 || timeout_ms > 5000) return LMH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return LMH_ERR_ALIGNMENT;
+  int dev, sms;
+  LMH_TRY(current_device(&dev, &sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  wait_selftest_kernel<<<1, 32, 0, st>>>(&ws.h->err, uint64_t(timeout_ms) * 1000000ull);
+  return last_launch();
 }
 
 extern "C" lmh_status lmh_profile_enable(int on) {

@@ -139,6 +139,7 @@ struct FinParams {
   int mean;
   const int32_t* n_given;
   WsHeader* h;
+  Temperature temp;
 };
 
 __global__ void finalize_rows_kernel(const FinParams p) {
@@ -164,6 +165,7 @@ __global__ void finalize_rows_kernel(const FinParams p) {
   if (lane == 0) {
     p.lse[grow] = lse;
     if (!isfinite(lse)) atomicOr(&p.h->err, kErrNonFinite);
+    if (p.temp.rows && !temperature_ok(p.temp.rows[grow])) atomicOr(&p.h->err, kErrTemperature);
   }
   bool valid = false;
   if (p.kind <= 1) {
@@ -181,7 +183,7 @@ __global__ void finalize_rows_kernel(const FinParams p) {
     if (lane == 0) p.argmax[grow] = (tfirst < p.T) ? p.part_i[static_cast<long long>(row) * p.T + tfirst] : 0;
   }
   if (p.write_scale) {
-    const float a = row_weight(valid, p.mean, p.n_given, p.h);
+    const float a = row_weight(valid, p.mean, p.n_given, p.h) * inv_temperature(p.temp, grow);
     const float loff = -lse * kLog2e;
     for (int t = lane; t < p.T; t += 32) ps[t] = a * fast_exp2(fmaf(pm[t], kLog2e, loff));
   }
@@ -233,13 +235,13 @@ __global__ void fix_labels_kernel(int rows, long long row0, int V, long long ldp
                                   const int32_t* __restrict__ labels,
                                   const float* __restrict__ zt, const float* __restrict__ lse,
                                   int mean, const int32_t* n_given, const WsHeader* h,
-                                  __nv_bfloat16* __restrict__ P) {
+                                  Temperature temp, __nv_bfloat16* __restrict__ P) {
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= rows) return;
   const long long g = row0 + r;
   const int y = labels[g];
   if (y < 0 || y >= V) return;
-  const float a = row_weight(true, mean, n_given, h);
+  const float a = row_weight(true, mean, n_given, h) * inv_temperature(temp, g);
   const float v = a * fast_exp2(fmaf(zt[g], kLog2e, -lse[g] * kLog2e)) - a;
   P[r * ldp + y] = __float2bfloat16_rn(v);
 }
@@ -293,20 +295,30 @@ __global__ void support_out_kernel(long long N, int K, const int32_t* __restrict
 // ---------------------------------------------------------------------------- backward
 // alpha_i and beta (per label, or per sorted candidate id summed over repeated slots) of
 // G = alpha P - sum beta e_t for the four objectives; one warp per row.
+// Without `grad` every row term has the weight 1, or 1 / count with `mean` (count: the valid
+// rows of the labels for CE / LOGPROB, N for the support objectives).
 __global__ void bwd_coef_kernel(int mode, long long N, int K, int V,
                                 const int32_t* __restrict__ targets,
                                 const float* __restrict__ grad, const float* __restrict__ ref,
                                 const int32_t* __restrict__ rank,
-                                const int32_t* __restrict__ nuniq, float* __restrict__ alpha,
+                                const int32_t* __restrict__ nuniq, Temperature temp, int mean,
+                                WsHeader* h, float* __restrict__ alpha,
                                 float* __restrict__ beta) {
   const int lane = threadIdx.x & 31;
   const long long i = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5);
   if (i >= N) return;
+  const float it = inv_temperature(temp, i);  // chain-rule factor of the tempered logits
+  if (lane == 0 && temp.rows && !temperature_ok(temp.rows[i])) atomicOr(&h->err, kErrTemperature);
+  float unit = 1.f;  // weight of a row term when no grad is given
+  if (mean) {
+    const long long cnt = (mode <= 1) ? h->n_valid : N;
+    unit = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
+  }
   if (mode <= 1) {  // CE / LOGPROB over labels
     if (lane == 0) {
       const int y = targets[i];
       const bool ok = (y >= 0 && y < V);
-      const float g = ok ? grad[i] : 0.f;
+      const float g = ok ? (grad ? grad[i] : unit) * it : 0.f;
       const float a = (mode == 0) ? g : -g;
       alpha[i] = a;
       beta[i] = a;
@@ -315,11 +327,11 @@ __global__ void bwd_coef_kernel(int mode, long long N, int K, int V,
   }
   // support: weight w_k = gamma_ik (SUPPORT_LOGPROB, alpha = -sum, beta = -w) or
   // g_i exp(r_ik) (SUPPORT_KL, alpha = sum, beta = w)
-  const float gi = (mode == 3) ? grad[i] : 0.f;
+  const float gi = (mode == 3) ? (grad ? grad[i] : unit) * it : 0.f;
   float sum = 0.f;
   for (int k = lane; k < K; k += 32) {
     if (rank[i * K + k] < 0) continue;
-    sum += (mode == 2) ? grad[i * K + k] : gi * expf(ref[i * K + k]);
+    sum += (mode == 2) ? (grad ? grad[i * K + k] : unit) * it : gi * expf(ref[i * K + k]);
   }
   sum = warp_sum(sum);
   if (lane == 0) alpha[i] = (mode == 2) ? -sum : sum;
@@ -328,10 +340,23 @@ __global__ void bwd_coef_kernel(int mode, long long N, int K, int V,
     float b = 0.f;
     for (int k = 0; k < K; ++k) {
       if (rank[i * K + k] != r) continue;
-      b += (mode == 2) ? grad[i * K + k] : gi * expf(ref[i * K + k]);
+      b += (mode == 2) ? (grad ? grad[i * K + k] : unit) * it : gi * expf(ref[i * K + k]);
     }
     beta[i * K + r] = (mode == 2) ? -b : b;
   }
+}
+
+// ---------------------------------------------------------------------------- self-test
+// One thread waits on an mbarrier that nothing ever arrives on, with the same bounded wait
+// the GEMMs use: the wait gives up after timeout_ns and records kErrTimeout.
+__global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, err, timeout_ns);
 }
 
 // ---------------------------------------------------------------------------- dW cast

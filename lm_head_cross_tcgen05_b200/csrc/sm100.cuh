@@ -13,6 +13,7 @@ namespace lmh {
 constexpr uint32_t kErrLabelRange = 0x1u;
 constexpr uint32_t kErrTimeout = 0x2u;
 constexpr uint32_t kErrNonFinite = 0x4u;
+constexpr uint32_t kErrTemperature = 0x8u;
 
 // Every wait inside a kernel gives up after this long, sets kErrTimeout and lets the
 // kernel wind down instead of spinning forever.
@@ -61,13 +62,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase of parity `parity` to complete. Returns false (after setting the
-// timeout bit in *err) if it has not completed within kWaitTimeoutNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
+// timeout bit in *err) if it has not completed within timeout_ns.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* err,
+                                          uint64_t timeout_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > timeout_ns) {
       atomicOr(err, kErrTimeout);
       return false;
     }
@@ -310,6 +312,22 @@ __device__ __forceinline__ void mma_commit_pair_local(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
       : "memory");
+}
+
+// ---------------------------------------------------------------------------- temperature
+// Inverse temperature of a row: 1 / (scalar * per-row), a factor of 0 or absent being 1.
+// A per-row value that is not finite and > 0 counts as 1 (the row finalize flags it).
+struct Temperature {
+  float inv_scalar;   // 1 / scalar temperature (1 when off)
+  const float* rows;  // [N] per-row temperatures or null
+};
+
+__device__ __forceinline__ bool temperature_ok(float t) { return t > 0.f && t < 3.0e38f; }
+
+__device__ __forceinline__ float inv_temperature(const Temperature& t, long long grow) {
+  if (!t.rows) return t.inv_scalar;
+  const float r = t.rows[grow];
+  return temperature_ok(r) ? t.inv_scalar / r : t.inv_scalar;
 }
 
 // ---------------------------------------------------------------------------- math

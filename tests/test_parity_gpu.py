@@ -219,3 +219,122 @@ def test_host_rejections():
         L.lmh_loss_fwd(bad, x["H"], x["W"], x["labels"], lr, lse, workspace=ws)
     with pytest.raises(L.LmhError, match="ALIGNMENT"):
         L.lmh_loss_fwd(shape, x["H"], x["W"], x["labels"], lr, lse, workspace=ws[8:])
+
+
+def _temps(kind, N, seed=3):
+    if kind == "scalar":
+        return 0.7, 0.7
+    if kind == "rows":
+        g = torch.Generator().manual_seed(seed)
+        t = torch.rand(N, generator=g, dtype=torch.float32) * 1.5 + 0.5
+        return t.cuda(), t.double().numpy()
+    return 1.0, None
+
+
+@pytest.mark.parametrize("kind", ["scalar", "rows", "one"])
+def test_temperature_ce_logprob_and_backward(kind):
+    N, d, V = 300, 192, 1000
+    x, xc = device_inputs(_wl(N, d, V, 5))
+    t_dev, t_ref = _temps(kind, N)
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=128, grads=True, temperature=t_dev)
+    ref = O.ce_fused(xc["H"], xc["W"], xc["labels"], tau=t_ref)
+    check_ce_fused(out, ref)
+    lp = L.logprob(x["H"], x["W"], x["labels"], temperature=t_dev)
+    check_rows(lp["logprob"], ref["logprob"], what="logprob")
+    n = int(out["n_valid"].item())
+    grad = torch.full((N,), 1.0 / n, device="cuda")
+    b = L.loss_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], out["lse"], grad, chunk_rows=100,
+                   temperature=t_dev)
+    check_grad(b["dH"], ref["dH"], "dH (recompute, tempered)")
+    check_grad(b["dW"], ref["dW"], "dW (recompute, tempered)")
+    if kind == "one":
+        plain = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=128, grads=True)
+        assert digest(plain["dW"], plain["dH"], plain["lse"]) == digest(out["dW"], out["dH"], out["lse"])
+
+
+@pytest.mark.parametrize("kind", ["scalar", "rows"])
+def test_temperature_support_kl(kind):
+    N, d, V, K = 200, 128, 3000, 16
+    x, xc = _support_inputs(N, d, V, K, 91)
+    t_dev, t_ref = _temps(kind, N, seed=8)
+    kl = L.support_kl(x["H"], x["W"], x["ids"], x["ref_logp"], temperature=t_dev)
+    ref = O.support_kl(xc["H"], xc["W"], xc["ids"], xc["ref_logp"], tau=t_ref)
+    check_rows(kl["kl_rows"], ref["kl_rows"], what="kl_rows")
+    check_rows(kl["lp"], ref["lp"], what="lp")
+    grad = torch.full((N,), 1.0 / N, device="cuda")
+    b = L.loss_bwd(L.BWD_SUPPORT_KL, x["H"], x["W"], x["ids"], kl["lse"], grad, x["ref_logp"],
+                   temperature=t_dev)
+    rb = O.backward(O.BWD_SUPPORT_KL, xc["H"], xc["W"], xc["ids"], np.full(N, 1.0 / N),
+                    xc["ref_logp"], tau=t_ref)
+    check_grad(b["dH"], rb["dH"], "dH")
+    check_grad(b["dW"], rb["dW"], "dW")
+
+
+def test_invalid_row_temperature_is_flagged_and_used_as_one():
+    N = 130
+    x, xc = device_inputs(_wl(N, 64, 300, 0))
+    t = torch.ones(N, device="cuda")
+    t[5] = 0.0
+    t[9] = float("nan")
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], temperature=t)
+    assert L.lmh_read_errors(out["workspace"]) & L.DEVERR_TEMPERATURE
+    ref = O.ce_forward(xc["H"], xc["W"], xc["labels"])
+    check_rows(out["loss_rows"], ref["loss_rows"], what="loss_rows")
+
+
+def test_backward_without_grad_uses_device_count():
+    N, d, V = 300, 192, 1000
+    x, xc = device_inputs(_wl(N, d, V, 5))
+    f = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    n = int(f["n_valid"].item())
+    explicit = L.loss_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], f["lse"],
+                          torch.full((N,), 1.0 / n, device="cuda"))
+    implicit = L.loss_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], f["lse"], None, mean=True)
+    assert torch.equal(explicit["dW"], implicit["dW"]) and torch.equal(explicit["dH"], implicit["dH"])
+    ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
+    check_grad(implicit["dW"], ref["dW"], "dW mean, no grad")
+    # the sum objective: unit weights
+    s = L.loss_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], f["lse"], None, mean=False)
+    rs = O.ce_fused(xc["H"], xc["W"], xc["labels"], mean=False)
+    check_grad(s["dH"], rs["dH"], "dH sum, no grad")
+    # support KL, mean over N rows
+    xs, xsc = _support_inputs(N, d, V, 8, 55)
+    kl = L.support_kl(xs["H"], xs["W"], xs["ids"], xs["ref_logp"])
+    a = L.loss_bwd(L.BWD_SUPPORT_KL, xs["H"], xs["W"], xs["ids"], kl["lse"],
+                   torch.full((N,), 1.0 / N, device="cuda"), xs["ref_logp"])
+    b = L.loss_bwd(L.BWD_SUPPORT_KL, xs["H"], xs["W"], xs["ids"], kl["lse"], None, xs["ref_logp"],
+                   mean=True)
+    assert torch.equal(a["dW"], b["dW"]) and torch.equal(a["dH"], b["dH"])
+
+
+@pytest.mark.parametrize("tau_kind", ["off", "rows"])
+def test_renorm_support_forward_and_backward(tau_kind):
+    N, d, V, K = 260, 192, 3000, 16
+    x, xc = _support_inputs(N, d, V, K, 123)
+    t_dev, t_ref = (None, None) if tau_kind == "off" else _temps("rows", N, seed=12)
+    lp = L.support_logprob(x["H"], x["W"], x["ids"], renorm=True, temperature=t_dev)
+    kl = L.support_kl(x["H"], x["W"], x["ids"], x["ref_logp"], renorm=True, temperature=t_dev)
+    ref = O.support_renorm_kl(xc["H"], xc["W"], xc["ids"], xc["ref_logp"], tau=t_ref)
+    check_rows(lp["lp"], ref["lp"], what="lp renorm")
+    check_rows(lp["lse"], ref["lse"], what="lse over the support")
+    check_rows(kl["kl_rows"], ref["kl_rows"], what="kl renorm")
+    assert torch.equal(kl["lp"], lp["lp"])
+    g = torch.Generator().manual_seed(4)
+    gam = torch.randn(N, K, generator=g) / N
+    b = L.loss_bwd(L.BWD_SUPPORT_LOGPROB, x["H"], x["W"], x["ids"], lp["lse"], gam.cuda(),
+                   renorm=True, temperature=t_dev)
+    rb = O.backward_renorm(O.BWD_SUPPORT_LOGPROB, xc["H"], xc["W"], xc["ids"], gam, tau=t_ref)
+    check_grad(b["dH"], rb["dH"], "dH renorm logprob")
+    check_grad(b["dW"], rb["dW"], "dW renorm logprob")
+    acc = torch.zeros(V, d, device="cuda")
+    bk = L.loss_bwd(L.BWD_SUPPORT_KL, x["H"], x["W"], x["ids"], kl["lse"], None, x["ref_logp"],
+                    mean=True, renorm=True, temperature=t_dev, dW_acc=acc)
+    rk = O.backward_renorm(O.BWD_SUPPORT_KL, xc["H"], xc["W"], xc["ids"], np.full(N, 1.0 / N),
+                           xc["ref_logp"], tau=t_ref)
+    check_grad(bk["dH"], rk["dH"], "dH renorm KL")
+    check_grad(acc, rk["dW"], "dW_acc renorm KL")
+    assert torch.equal(bk["dW"], acc.to(torch.bfloat16))
+    # bitwise repeats (the scatter is summed in a fixed row order)
+    b2 = L.loss_bwd(L.BWD_SUPPORT_LOGPROB, x["H"], x["W"], x["ids"], lp["lse"], gam.cuda(),
+                    renorm=True, temperature=t_dev)
+    assert torch.equal(b2["dW"], b["dW"]) and torch.equal(b2["dH"], b["dH"])
