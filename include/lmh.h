@@ -27,9 +27,11 @@
  *   value). A label >= V is out of range: the row is treated as ignored and the device
  *   error word gets LMH_DEVERR_LABEL_RANGE (no trap; read it with lmh_read_errors).
  * - Rows are processed in chunks of shape->chunk_rows rows (0 selects 4096, the default of
- *   the same commit's --cake-lm-head-chunk-size), in ascending order. The chunk plan only
- *   changes the summation order of dW across chunks; every other output is independent
- *   of it bit for bit.
+ *   the same commit's --cake-lm-head-chunk-size), in ascending order. The chunk plan changes
+ *   the summation order of dW across chunks and, for chunks too small to fill the GPU with
+ *   dH tiles (fewer than 384 tiles of 256 x 256), of dH, whose vocabulary sum is then split
+ *   into up to 8 ranges added in a fixed order. The forward outputs (loss, lse, log-probs,
+ *   argmax, counts) do not depend on it; no output depends on the GPU's SM count.
  * - Return value: LMH_OK, or an error found on the host before anything was enqueued
  *   (invalid argument, misalignment, short workspace, unsupported device), or
  *   LMH_ERR_CUDA when a launch failed. Errors found on the device go to the error word.
@@ -139,6 +141,8 @@ LMH_API size_t lmh_workspace_size(const lmh_shape* shape, int entry);
  *     sum_i loss_i (not set), reusing the forward's softmax instead of recomputing logits.
  *     dW_acc, if given, is incremented by this call's dW in chunk order (zero it first for
  *     a fresh gradient) and dW, if given, receives its round-to-nearest-even bf16 cast.
+ *     Each increment is one fp32 add per element and chunk, rounded to nearest even, with
+ *     subnormal operands and sums (below 2^-126) flushed to zero.
  *     Without dW_acc and with one chunk, dW is the bf16 cast of the fp32 tile sums.
  */
 LMH_API lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,

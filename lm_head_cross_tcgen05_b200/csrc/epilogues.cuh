@@ -114,6 +114,35 @@ __device__ __forceinline__ void stage_store_64(EpiCtx& c, const float (&a)[32],
   ++c.nstore;
 }
 
+// The fp32 counterpart: the warp's 32 rows x 32 columns (v of each thread's row, 128 bytes)
+// go through one staging buffer to a TMA store, or with `reduce` to a TMA add into the
+// destination, at (x, y) of ctx.tmC (fp32, box 32 columns x 32 rows, 128-byte swizzle).
+__device__ __forceinline__ void stage_f32_32(EpiCtx& c, const float (&v)[32], int x, int y,
+                                             bool do_op, bool reduce) {
+  const uint32_t buf = c.stage + (c.nstore & 1u) * EPI_BUF_BYTES;
+  if (c.lane == 0) bulk_wait_read_le1();
+  __syncwarp();
+  const uint32_t row = buf + static_cast<uint32_t>(c.lane) * 128u;
+  const uint32_t sw = static_cast<uint32_t>(c.lane & 7);
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    uint4 w;
+    w.x = __float_as_uint(v[u * 4 + 0]);
+    w.y = __float_as_uint(v[u * 4 + 1]);
+    w.z = __float_as_uint(v[u * 4 + 2]);
+    w.w = __float_as_uint(v[u * 4 + 3]);
+    st_shared_v4(row + ((static_cast<uint32_t>(u) ^ sw) << 4), w);
+  }
+  fence_async_smem();
+  __syncwarp();
+  if (c.lane == 0 && do_op) {
+    if (reduce) tma_reduce_add_2d(c.tmC, buf, x, y);
+    else tma_store_2d(c.tmC, buf, x, y);
+    bulk_commit();
+  }
+  ++c.nstore;
+}
+
 // ------------------------------------------------------------------ logits statistics
 // Forward epilogue of z = H_c W^T. Per (row, 256-wide vocabulary tile t) it writes the tile
 // maximum m_t, s_t = sum_v exp(z_v - m_t), the first column attaining m_t, and the logits at
@@ -267,7 +296,9 @@ struct EpiGrad {
 };
 
 // ------------------------------------------------------------------ dH = G W
-// ctx.tmC maps this chunk's rows of dH ([rows, d] at row r0).
+// ctx.tmC maps this chunk's rows of dH ([rows, d] at row r0). With K (= V) split, each unit
+// writes its fp32 partial to part[split][row][col] instead; a fixed-order reduction over the
+// splits then produces dH.
 struct EpiDH {
   static constexpr int kId = 5;        // gemm_dH
   static constexpr int kAMajorMN = 0;  // G chunk [rows, V], K-major
@@ -275,11 +306,13 @@ struct EpiDH {
   struct Params {
     int rows;
     int d;
+    float* part;  // [splits, rows, d] fp32, or null when K is not split
   };
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
                                               int rit, EpiCtx& ctx) {
     const int n0 = nb * BN;
     const int wrow = mb * BM + ctx.row_w;
+    const int row = mb * BM + rit;
 #pragma unroll 1
     for (int sb = 0; sb < kSlabs; ++sb) {
       const int col0 = n0 + sb * 64;
@@ -287,15 +320,34 @@ struct EpiDH {
       float a[32], b[32];
       tmem_ld32(taddr + sb * 64, a);
       tmem_ld32(taddr + sb * 64 + 32, b);
-      stage_store_64(ctx, a, b, col0, wrow, wrow < p.rows);
+      if (p.part) {
+        if (row < p.rows) {
+          float4* o = reinterpret_cast<float4*>(
+              p.part + (static_cast<long long>(ctx.split) * p.rows + row) * p.d + col0);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float* v = u < 8 ? a : b;
+            const int q = (u & 7) * 4;
+            __stcs(o + u, make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]));
+          }
+        }
+      } else {
+        stage_store_64(ctx, a, b, col0, wrow, wrow < p.rows);
+      }
     }
   }
 };
 
 // ------------------------------------------------------------------ dW = G^T H_c
-// acc_mode 0: the tile sum is the whole dW; 1: acc = 0 + sum (first chunk into a fresh
-// internal accumulator); 2: acc += sum (the caller's or a later chunk). With `out` set the
-// bf16 cast of the resulting value is stored as well (last chunk; ctx.tmC maps dW [V, d]).
+// acc_mode 0: the tile sum is the whole dW, stored in bf16 (ctx.tmC: bf16 dW [V, d]).
+// acc_mode 1: acc = 0 + sum (first chunk into a fresh internal accumulator; 0 + x turns -0
+// into +0 exactly as an add into a zeroed buffer would), stored in fp32.
+// acc_mode 2: acc += sum, one fp32 add per element done by the TMA unit at L2.
+// In modes 1 and 2 ctx.tmC maps the fp32 accumulator [V, d]; every element has one owner tile
+// per launch and the launches of a call run in chunk order, so the accumulation order is fixed.
+// The accumulator never passes through registers: the epilogue only writes, and the DRAM
+// read-modify-write runs at L2 asynchronously instead of as 16-byte loads that each wait for
+// memory. The bf16 cast of the final accumulator is a separate pass after the last chunk.
 struct EpiDW {
   static constexpr int kId = 6;        // gemm_dW
   static constexpr int kAMajorMN = 1;  // G^T: G chunk [rows, V] read as [K = rows, M = V]
@@ -303,54 +355,33 @@ struct EpiDW {
   struct Params {
     int V;
     int d;
-    float* acc;           // [V, d] or null
     int acc_mode;
-    int out;              // store the bf16 cast through ctx.tmC
   };
-  static __device__ __forceinline__ void rmw32(const Params& p, long long base, int col0,
-                                               float (&v)[32]) {
-    float4* a4 = reinterpret_cast<float4*>(p.acc + base + col0);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      float4 a;
-      if (p.acc_mode == 2) {
-        a = a4[u];
-        a.x += v[4 * u + 0];
-        a.y += v[4 * u + 1];
-        a.z += v[4 * u + 2];
-        a.w += v[4 * u + 3];
-      } else {
-        a.x = v[4 * u + 0] + 0.f;
-        a.y = v[4 * u + 1] + 0.f;
-        a.z = v[4 * u + 2] + 0.f;
-        a.w = v[4 * u + 3] + 0.f;
-      }
-      a4[u] = a;
-      v[4 * u + 0] = a.x;
-      v[4 * u + 1] = a.y;
-      v[4 * u + 2] = a.z;
-      v[4 * u + 3] = a.w;
-    }
-  }
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
                                               int rit, EpiCtx& ctx) {
-    const int vrow = mb * BM + rit;
-    const bool vv = vrow < p.V;
     const int n0 = nb * BN;
-    const long long base = static_cast<long long>(vrow) * p.d;
     const int wrow = mb * BM + ctx.row_w;
+    const bool wv = wrow < p.V;  // rows past V are clipped by the tensor map
 #pragma unroll 1
     for (int sb = 0; sb < kSlabs; ++sb) {
       const int col0 = n0 + sb * 64;
-      if (col0 >= p.d) break;
+      if (col0 >= p.d) break;  // uniform across the warp (d is a multiple of 64)
       float a[32], b[32];
       tmem_ld32(taddr + sb * 64, a);
       tmem_ld32(taddr + sb * 64 + 32, b);
-      if (p.acc_mode != 0 && vv) {
-        rmw32(p, base, col0, a);
-        rmw32(p, base, col0 + 32, b);
+      if (p.acc_mode == 0) {
+        stage_store_64(ctx, a, b, col0, wrow, wv);
+      } else {
+        if (p.acc_mode == 1) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            a[j] = __fadd_rn(0.f, a[j]);
+            b[j] = __fadd_rn(0.f, b[j]);
+          }
+        }
+        stage_f32_32(ctx, a, col0, wrow, wv, p.acc_mode == 2);
+        stage_f32_32(ctx, b, col0 + 32, wrow, wv, p.acc_mode == 2);
       }
-      if (p.out) stage_store_64(ctx, a, b, col0, wrow, wrow < p.V);
     }
   }
 };

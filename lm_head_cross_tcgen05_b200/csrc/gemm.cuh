@@ -6,8 +6,10 @@
 // its own TMEM. The pair's rank-0 CTA issues the MMAs, which read the operand halves of both
 // CTAs. Per SM this halves the B operand traffic of a 128 x 256 single-CTA tile.
 //
-// Persistent schedule: grid = 2 x (number of co-resident pairs); pair p walks the tiles
-// p, p + pairs, ... of a fixed, grouped order (group_m row tiles at a time, rows fastest).
+// Persistent schedule: grid = 2 x (number of co-resident pairs); pair p walks the work units
+// p, p + pairs, ... of a fixed, grouped order (group_m row tiles at a time, rows fastest). A
+// work unit is an output tile, or a tile and one of k_splits consecutive K ranges when a
+// launch has too few tiles to fill the GPU (its epilogue then writes an fp32 partial).
 // Every output tile is owned by one pair and its K loop runs in ascending order, so the fp32
 // result of a tile does not depend on which SMs ran it or how many there are: the GEMM is
 // deterministic without any cross-CTA reduction.
@@ -63,6 +65,7 @@ struct EpiCtx {
   int lane;
   int row_w;         // first accumulator row of this warp within the CTA's 128
   uint32_t nstore;
+  int split;         // K range of the current work unit (0 unless K is split)
 };
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -70,13 +73,19 @@ struct GemmGrid {
   int m_tiles;   // pair tiles along M (256 rows each)
   int n_tiles;   // tiles along N (256 columns each)
   int k_blocks;  // ceil(K / BK)
+  int k_splits;  // K split into this many consecutive ranges (work units = tiles x splits)
   int group_m;   // tile order: group_m row tiles at a time, rows fastest within a group
   int hint_a;    // L2 eviction priority of A's loads (L2Hint)
   int hint_b;    // L2 eviction priority of B's loads
   uint32_t* err; // device error word
 };
 
-__device__ __forceinline__ void tile_coords(const GemmGrid& g, int t, int& mb, int& nb) {
+// Work unit u = split * tiles + tile: the split's K blocks are [kb0, kb1).
+__device__ __forceinline__ void unit_coords(const GemmGrid& g, int u, int& mb, int& nb, int& split,
+                                            int& kb0, int& kb1) {
+  const int tiles = g.m_tiles * g.n_tiles;
+  split = u / tiles;
+  int t = u - split * tiles;
   const int per_group = g.group_m * g.n_tiles;
   const int grp = t / per_group;
   const int rem = t - grp * per_group;
@@ -84,6 +93,8 @@ __device__ __forceinline__ void tile_coords(const GemmGrid& g, int t, int& mb, i
   const int gm = min(g.group_m, g.m_tiles - m0);
   mb = m0 + rem % gm;
   nb = rem / gm;
+  kb0 = static_cast<int>(static_cast<long long>(g.k_blocks) * split / g.k_splits);
+  kb1 = static_cast<int>(static_cast<long long>(g.k_blocks) * (split + 1) / g.k_splits);
 }
 
 template <class Epi>
@@ -107,7 +118,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  const int num_tiles = g.m_tiles * g.n_tiles;
+  const int num_tiles = g.m_tiles * g.n_tiles * g.k_splits;  // work units
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -137,11 +148,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       const uint64_t pol_b = l2_policy(g.hint_b);
       uint32_t kbg = 0;
       for (int t = pair; t < num_tiles && !abort_flag; t += npairs) {
-        int mb, nb;
-        tile_coords(g, t, mb, nb);
+        int mb, nb, sp, kb0, kb1;
+        unit_coords(g, t, mb, nb, sp, kb0, kb1);
         const int arow = mb * PM + static_cast<int>(rank) * BM;    // this CTA's A rows
         const int brow = nb * BN + static_cast<int>(rank) * BNH;   // this CTA's B rows
-        for (int kb = 0; kb < g.k_blocks; ++kb, ++kbg) {
+        for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
           const uint32_t s = kbg % STAGES;
           const uint32_t ph = (kbg / STAGES) & 1u;
           if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, g.err)) {
@@ -189,9 +200,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           break;
         }
         tc_fence_after();
+        int mb, nb, sp, kb0, kb1;
+        unit_coords(g, t, mb, nb, sp, kb0, kb1);
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
         bool ok = true;
-        for (int kb = 0; kb < g.k_blocks; ++kb, ++kbg) {
+        for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
           const uint32_t s = kbg % STAGES;
           const uint32_t ph = (kbg / STAGES) & 1u;
           if (!mbar_wait(smem_u32(&full_bar[s]), ph, g.err)) {
@@ -212,7 +225,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                 Epi::kBMajorMN
                     ? make_sw128_desc(b_base + k * 2048, MN_BLOCK_BYTES, 1024)
                     : make_sw128_desc(b_base + (k >> 2) * B_SUB_BYTES + (k & 3) * 32, 16, 1024);
-            mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+            mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
           }
           mma_commit_pair(smem_u32(&empty_bar[s]), 0x3);  // both CTAs may refill stage s
         }
@@ -231,7 +244,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     const int q = warp & 3;  // the TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
     EpiCtx ctx{&tmC, smem_base + STAGES * STAGE_BYTES + (warp - 2) * 2 * EPI_BUF_BYTES, lane,
-               q * 32, 0u};
+               q * 32, 0u, 0};
     if (lane == 0) tma_prefetch_desc(&tmC);
     int it = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++it) {
@@ -244,8 +257,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         break;
       }
       tc_fence_after();
-      int mb, nb;
-      tile_coords(g, t, mb, nb);
+      int mb, nb, sp, kb0, kb1;
+      unit_coords(g, t, mb, nb, sp, kb0, kb1);
+      ctx.split = sp;
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
       Epi::tile(ep, mb * 2 + static_cast<int>(rank), nb, taddr, row_in_tile, ctx);

@@ -35,6 +35,7 @@ struct Plan {
   bool renorm;  // support entries renormalised over the candidate set (sparse path)
   size_t o_zt, o_sorted, o_nuniq, o_rank, o_pm, o_ps, o_pi, o_alpha, o_beta, o_gbuf, o_acc;
   size_t o_gu, o_cnt, o_off, o_fill, o_prow, o_pslot;  // sparse backward
+  size_t o_dhpart;                                     // split-K partials of dH
   size_t total;
   Temperature temp;  // logits are z / tau_i
 };
@@ -47,6 +48,20 @@ bool shape_ok(const lmh_shape* s) {
   if (!(s->temperature >= 0.f && s->temperature < 3.0e38f)) return false;  // NaN fails too
   if ((reinterpret_cast<uintptr_t>(s->row_temperature) & 3u) != 0) return false;
   return true;
+}
+
+// K splits of the dH GEMM of a chunk with `rows` rows. Chunks with too few output tiles to keep
+// every SM busy (fewer than 384 pair tiles) split the vocabulary into up to 8 ranges, aiming at
+// 512 work units; each range keeps at least 8 K blocks. The rule reads the shape only (never
+// the SM count), so the result bits do not depend on the GPU's size.
+int dh_splits(int64_t rows, int64_t d, int64_t V) {
+  const int64_t tiles = cdiv(rows, PM) * cdiv(d, BN);
+  if (tiles >= 384) return 1;
+  int64_t sp = cdiv(512, tiles);
+  const int64_t by_k = cdiv(V, BK) / 8;
+  if (sp > 8) sp = 8;
+  if (sp > by_k) sp = by_k;
+  return sp < 1 ? 1 : static_cast<int>(sp);
 }
 
 // fused: the entry keeps a [c, Vp] bf16 buffer; need_acc: an fp32 [V, d] accumulator.
@@ -91,6 +106,13 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   p.o_beta = (entry == LMH_ENTRY_LOSS_BWD) ? take(N * p.K * 4) : 0;
   p.o_gbuf = p.gbuf ? take(static_cast<size_t>(p.c) * p.Vp * 2) : 0;
   p.o_acc = p.acc ? take(static_cast<size_t>(p.V) * p.d * 4) : 0;
+  if (p.gbuf && p.nchunks > 0) {  // the largest split-K partial of any chunk
+    const int64_t last = p.N - (p.nchunks - 1) * p.c;
+    const int64_t a = dh_splits(p.c, p.d, p.V) > 1 ? dh_splits(p.c, p.d, p.V) * p.c : 0;
+    const int64_t b = dh_splits(last, p.d, p.V) > 1 ? dh_splits(last, p.d, p.V) * last : 0;
+    const int64_t r = a > b ? a : b;
+    p.o_dhpart = r ? take(static_cast<size_t>(r) * p.d * 4) : 0;
+  }
   const bool sparse_bwd = p.renorm && entry == LMH_ENTRY_LOSS_BWD;
   p.o_gu = sparse_bwd ? take(N * p.K * 4) : 0;
   p.o_cnt = sparse_bwd ? take(static_cast<size_t>(p.V) * 4) : 0;
@@ -139,13 +161,13 @@ enum KernelId {
   KID_COUNT_LABELS, KID_PREP_CANDS, KID_GEMM_LOGITS, KID_GEMM_LOGITS_P, KID_GEMM_GRAD,
   KID_GEMM_DH, KID_GEMM_DW, KID_FINALIZE, KID_GBUILD, KID_FIX_LABELS, KID_MEAN,
   KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_SUPPORT_DOTS, KID_SUPPORT_LSE,
-  KID_SUPPORT_DH, KID_SUPPORT_DW, KID_COUNT
+  KID_SUPPORT_DH, KID_SUPPORT_DW, KID_SPLIT_SUM, KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "count_labels", "prep_cands", "gemm_logits_stats", "gemm_logits_stats_store",
     "gemm_logits_grad", "gemm_dH", "gemm_dW", "row_finalize", "gbuild", "fix_labels",
     "mean", "support_out", "bwd_coef", "cast_bf16", "support_dots", "support_lse",
-    "support_grad_dh", "support_dw"};
+    "support_grad_dh", "support_dw", "split_sum"};
 
 struct ProfRec {
   int id;
@@ -225,6 +247,20 @@ bool tmap_out(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
   return tmap_2d(m, base, inner, outer, ld, 32);
 }
 
+// Accumulator map of the dW epilogue's staged fp32 stores and adds: fp32 [outer, inner] with
+// row stride `ld` elements, box 32 x 32 rows, 128-byte swizzle.
+bool tmap_acc(CUtensorMap* m, const float* base, uint64_t inner, uint64_t outer, uint64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------------ launches
 // Tile orders and L2 priorities of the three contractions.
 struct GemmOrder {
@@ -236,7 +272,7 @@ template <class Epi>
 lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap& b,
                        const CUtensorMap& c, int64_t M, int64_t Ncols, int64_t K,
                        GemmOrder order, uint32_t* err, const typename Epi::Params& ep,
-                       cudaStream_t st) {
+                       cudaStream_t st, int k_splits = 1) {
   static std::atomic<uint64_t> attr_done{0};
   static std::atomic<int> pairs_cache[64];
   const uint64_t bit = 1ull << dev;
@@ -262,11 +298,12 @@ lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap
   g.m_tiles = static_cast<int>(cdiv(M, PM));
   g.n_tiles = static_cast<int>(cdiv(Ncols, BN));
   g.k_blocks = static_cast<int>(cdiv(K, BK));
+  g.k_splits = k_splits;
   g.group_m = order.group_m < 1 ? g.m_tiles : (order.group_m < g.m_tiles ? order.group_m : g.m_tiles);
   g.hint_a = order.hint_a;
   g.hint_b = order.hint_b;
   g.err = err;
-  const int64_t tiles = static_cast<int64_t>(g.m_tiles) * g.n_tiles;
+  const int64_t tiles = static_cast<int64_t>(g.m_tiles) * g.n_tiles * k_splits;
   if (tiles <= 0) return LMH_OK;
   const int64_t pairs_max = pairs_cache[dev].load();
   const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
@@ -371,6 +408,16 @@ lmh_status run_finalize(const Plan& P, int kind, int64_t r0, int rows, const int
   return last_launch();
 }
 
+// dW = bf16(acc) over [V, d] (V * d is a multiple of 4; both buffers 16-byte aligned).
+lmh_status cast_dw(const Plan& P, const float* acc, lmh_bf16* dW, cudaStream_t st) {
+  ProfScope ps(KID_CAST, st);
+  const int64_t n4 = P.V * P.d / 4;
+  const int64_t blocks = cdiv(n4, 256);
+  cast_bf16_kernel<<<static_cast<unsigned>(blocks < 8192 ? blocks : 8192), 256, 0, st>>>(
+      acc, n4, reinterpret_cast<__nv_bfloat16*>(dW));
+  return last_launch();
+}
+
 // dH = G W and dW (+)= G^T H_c for one chunk whose G sits in the workspace buffer.
 lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H,
                               const lmh_bf16* W, int64_t r0, int rows, int chunk_idx,
@@ -385,35 +432,33 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
     EpiDH::Params ep;
     ep.rows = rows;
     ep.d = static_cast<int>(P.d);
+    const int sp = dh_splits(rows, P.d, P.V);
+    ep.part = sp > 1 ? ws.at<float>(P.o_dhpart) : nullptr;
     LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, tc, rows, P.d, P.V, kOrderDH, &ws.h->err, ep,
-                               st));
+                               st, sp));
+    if (sp > 1) {
+      ProfScope ps(KID_SPLIT_SUM, st);
+      const int64_t blocks = cdiv(static_cast<int64_t>(rows) * P.d / 2, 256);
+      split_sum_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(
+          sp, rows, static_cast<int>(P.d), ws.at<float>(P.o_dhpart),
+          reinterpret_cast<__nv_bfloat16*>(dH + r0 * P.d));
+      LMH_TRY(last_launch());
+    }
   }
   if (dW || dW_acc) {
     CUtensorMap ta, tb, tc;
     if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BK) || !tmap_2d(&tb, H + r0 * P.d, P.d, rows, P.d, BK))
       return LMH_ERR_CUDA;
-    const bool last = chunk_idx == P.nchunks - 1;
-    if (dW && last) {
-      if (!tmap_out(&tc, dW, P.d, P.V, P.d)) return LMH_ERR_CUDA;
-    } else {
-      tc = tb;  // not used without the bf16 store
-    }
+    float* acc = dW_acc ? dW_acc : (P.acc ? ws.at<float>(P.o_acc) : nullptr);
     EpiDW::Params ep;
     ep.V = static_cast<int>(P.V);
     ep.d = static_cast<int>(P.d);
-    if (dW_acc) {
-      ep.acc = dW_acc;
-      ep.acc_mode = 2;
-    } else if (P.acc) {
-      ep.acc = ws.at<float>(P.o_acc);
-      ep.acc_mode = chunk_idx == 0 ? 1 : 2;
-    } else {
-      ep.acc = nullptr;
-      ep.acc_mode = 0;
-    }
-    ep.out = (dW && last) ? 1 : 0;
+    ep.acc_mode = !acc ? 0 : (dW_acc || chunk_idx > 0) ? 2 : 1;
+    if (!(acc ? tmap_acc(&tc, acc, P.d, P.V, P.d) : tmap_out(&tc, dW, P.d, P.V, P.d)))
+      return LMH_ERR_CUDA;
     LMH_TRY(launch_gemm<EpiDW>(dev, sms, ta, tb, tc, P.V, P.d, rows, kOrderDW, &ws.h->err, ep,
                                st));
+    if (acc && dW && chunk_idx == P.nchunks - 1) LMH_TRY(cast_dw(P, acc, dW, st));
   }
   return LMH_OK;
 }
@@ -504,11 +549,7 @@ lmh_status empty_call(const Plan& P, float* mean_out, int32_t* nvalid_out, lmh_b
   if (nvalid_out && cudaMemsetAsync(nvalid_out, 0, 4, st) != cudaSuccess) return LMH_ERR_CUDA;
   if (dW) {
     const int64_t n = P.V * P.d;
-    if (dW_acc) {
-      ProfScope ps(KID_CAST, st);
-      cast_bf16_kernel<<<1024, 256, 0, st>>>(dW_acc, n, reinterpret_cast<__nv_bfloat16*>(dW));
-      return last_launch();
-    }
+    if (dW_acc) return cast_dw(P, dW_acc, dW, st);
     if (cudaMemsetAsync(dW, 0, n * 2, st) != cudaSuccess) return LMH_ERR_CUDA;
   }
   return LMH_OK;

@@ -346,6 +346,25 @@ __global__ void bwd_coef_kernel(int mode, long long N, int K, int V,
   }
 }
 
+// ---------------------------------------------------------------------------- split-K sum
+// dH[r, j] = bf16(sum over s = 0, 1, ... of part[s, r, j]): the fixed-order reduction of the
+// split dH GEMM's fp32 partials. Pairs of columns per thread, grid-stride.
+__global__ void split_sum_kernel(int splits, long long rows, int d, const float* __restrict__ part,
+                                 __nv_bfloat16* __restrict__ out) {
+  const long long n2 = rows * d / 2;
+  const long long plane = rows * d;
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < n2;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float2 acc = __ldcs(reinterpret_cast<const float2*>(part) + e);
+    for (int sp = 1; sp < splits; ++sp) {
+      const float2 v = __ldcs(reinterpret_cast<const float2*>(part + sp * plane) + e);
+      acc.x += v.x;
+      acc.y += v.y;
+    }
+    reinterpret_cast<uint32_t*>(out)[e] = pack_bf16x2(acc.x, acc.y);
+  }
+}
+
 // ---------------------------------------------------------------------------- self-test
 // One thread waits on an mbarrier that nothing ever arrives on, with the same bounded wait
 // the GEMMs use: the wait gives up after timeout_ns and records kErrTimeout.
@@ -360,11 +379,16 @@ __global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
 }
 
 // ---------------------------------------------------------------------------- dW cast
-__global__ void cast_bf16_kernel(const float* __restrict__ src, long long n,
+// dst = bf16(src) over n4 groups of 4 elements (round to nearest even).
+__global__ void cast_bf16_kernel(const float* __restrict__ src, long long n4,
                                  __nv_bfloat16* __restrict__ dst) {
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x)
-    dst[i] = __float2bfloat16_rn(src[i]);
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+  uint2* d4 = reinterpret_cast<uint2*>(dst);
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 v = __ldcs(s4 + i);
+    __stcs(d4 + i, make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w)));
+  }
 }
 
 }  // namespace lmh

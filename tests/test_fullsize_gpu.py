@@ -101,7 +101,11 @@ def test_large_vocab_fused_matches_recompute_and_chunking(large_vocab):
     check_grad(b["dH"], f64(out["dH"]), "dH recompute vs fused")
     del b
     c = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=3000, grads=True)
-    assert torch.equal(c["dH"], out["dH"]) and torch.equal(c["lse"], out["lse"])
+    # the forward outputs never depend on the chunk plan; dH of 3000-row chunks is summed over
+    # vocabulary ranges (too few tiles to fill the GPU) and dW over chunks: same values to
+    # rounding
+    assert torch.equal(c["lse"], out["lse"]) and torch.equal(c["loss_rows"], out["loss_rows"])
+    check_grad(c["dH"], f64(out["dH"]), "dH 3 chunks vs 1")
     check_grad(c["dW"], ref_dw, "dW 3 chunks vs 1")
 
 

@@ -338,3 +338,36 @@ def test_renorm_support_forward_and_backward(tau_kind):
     b2 = L.loss_bwd(L.BWD_SUPPORT_LOGPROB, x["H"], x["W"], x["ids"], lp["lse"], gam.cuda(),
                     renorm=True, temperature=t_dev)
     assert torch.equal(b2["dW"], b["dW"]) and torch.equal(b2["dH"], b["dH"])
+
+
+def test_single_word_vocabulary():
+    # V = 1: every valid row has loss 0, lse = its only logit, and zero gradients
+    N, d = 50, 64
+    x, xc = device_inputs(_wl(N, d, 1, 0))
+    y = torch.zeros(N, dtype=torch.int32, device="cuda")
+    y[3] = -100
+    out = L.loss_fwd(x["H"], x["W"], y, grads=True, chunk_rows=16)
+    ref = O.ce_fused(xc["H"], xc["W"], y.cpu())
+    check_ce_fused(out, ref)
+    assert torch.count_nonzero(out["argmax"]) == 0
+    assert torch.count_nonzero(out["dW"]) == 0 and torch.count_nonzero(out["dH"]) == 0
+
+
+def test_maximum_candidate_count():
+    N, d, V, K = 40, 64, 5000, L.MAX_K
+    x, xc = _support_inputs(N, d, V, K, 31)
+    kl = L.support_kl(x["H"], x["W"], x["ids"], x["ref_logp"])
+    ref = O.support_kl(xc["H"], xc["W"], xc["ids"], xc["ref_logp"])
+    check_rows(kl["kl_rows"], ref["kl_rows"], what="kl_rows K=1024")
+    check_rows(kl["lp"], ref["lp"], what="lp K=1024")
+    b = L.loss_bwd(L.BWD_SUPPORT_KL, x["H"], x["W"], x["ids"], kl["lse"], None, x["ref_logp"],
+                   mean=True)
+    rb = O.backward(O.BWD_SUPPORT_KL, xc["H"], xc["W"], xc["ids"], np.full(N, 1.0 / N),
+                    xc["ref_logp"])
+    check_grad(b["dW"], rb["dW"], "dW K=1024")
+    r = L.support_logprob(x["H"], x["W"], x["ids"], renorm=True)
+    rr = O.support_renorm_logprob(xc["H"], xc["W"], xc["ids"])
+    check_rows(r["lp"], rr["lp"], what="renorm lp K=1024")
+    with pytest.raises((ValueError, L.LmhError)):
+        ids = torch.zeros(N, K + 1, dtype=torch.int32, device="cuda")
+        L.support_logprob(x["H"], x["W"], ids)
