@@ -169,65 +169,73 @@ def gpu_id_for_smi(torch, dev) -> str:
 
 # ----------------------------------------------------------------------------- oracle timing
 
-def oracle_sample(wl, target_s: float):
-    """Times the fp64 oracle's fused forward+backward on the first n rows of the workload
-    (full V and d), with n chosen so that the run takes about target_s seconds."""
-    import threadpoolctl
-
+def oracle_runner(wl, entry):
+    """The oracle's work for one step of `entry` on the first n rows of the workload (full V
+    and d): run(n) does it, `what` names it. Both CE entries compute forward, dH and dW; the
+    support entry computes the candidate log-probs, the KL and its backward."""
     from oracle import lmh_oracle as O
     from workloads import make_inputs
     x = make_inputs(wl.scaled(N=min(wl.N, 4096)), device="cpu")
+    if entry == "support_kl":
+        def run(n):
+            O.support_kl(x["H"][:n], x["W"], x["ids"][:n], x["ref_logp"][:n])
+            g = [1.0 / wl.N] * n
+            O.backward(O.BWD_SUPPORT_KL, x["H"][:n], x["W"], x["ids"][:n], g,
+                       x["ref_logp"][:n])
+        return run, "fp64 numpy oracle support_kl + backward (dH, dW)"
 
     def run(n):
-        t = time.perf_counter()
         O.ce_fused(x["H"][:n], x["W"], x["labels"][:n])
-        return time.perf_counter() - t
+    return run, "fp64 numpy oracle ce_fused (forward, dH, dW)"
 
-    # t(n) = a + b n: a is the per-call fp64 widening of W, b the per-row work
-    t8, t40 = run(8), run(40)
-    b = max((t40 - t8) / 32.0, 1e-6)
-    a = max(t8 - 8 * b, 0.0)
-    n = int(max(8, min(1024, (target_s - a) / b)))
-    t = run(n)
-    info = threadpoolctl.threadpool_info()
-    cores = max([i.get("num_threads", 1) for i in info] + [1])
-    return n, t, cores
+
+def _timed(fn, n):
+    t = time.perf_counter()
+    fn(n)
+    return time.perf_counter() - t
+
+
+def _rows_for(fn, target_s, n0, n1, cap=1024):
+    """Rows that take about target_s seconds, from t(n) = a + b n at two calibration sizes
+    (a is the per-call fp64 widening of W, b the per-row work)."""
+    t0, t1 = _timed(fn, n0), _timed(fn, n1)
+    b = max((t1 - t0) / float(n1 - n0), 1e-6)
+    a = max(t0 - n0 * b, 0.0)
+    return int(max(n0, min(cap, (target_s - a) / b)))
+
+
+def _cores():
+    import threadpoolctl
+    return max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+
+
+def oracle_sample(wl, target_s: float, entry="fused_ce"):
+    """Times the fp64 oracle's step on the first n rows of the workload (full V and d), with
+    n chosen so that the run takes about target_s seconds."""
+    run, what = oracle_runner(wl, entry)
+    n = _rows_for(run, target_s, 8, 40)
+    return n, _timed(run, n), _cores(), what
 
 
 def run_reference(args, wl, n_gpus):
     """The oracle as it stands, on the host cores, steps of a bounded sample."""
-    import threadpoolctl
-
-    from oracle import lmh_oracle as O
-    from workloads import make_inputs
-    x = make_inputs(wl.scaled(N=min(wl.N, 4096)), device="cpu")
+    run, what = oracle_runner(wl, args.entry)
     budget = 150.0 / max(1, args.steps + args.warmup)       # seconds per step
-
-    def run(n):
-        t = time.perf_counter()
-        O.ce_fused(x["H"][:n], x["W"], x["labels"][:n])
-        return time.perf_counter() - t
-
-    t4, t20 = run(4), run(20)
-    b = max((t20 - t4) / 16.0, 1e-6)
-    a = max(t4 - 4 * b, 0.0)
-    n = int(max(4, min(1024, (budget - a) / b)))
+    n = _rows_for(run, budget, 4, 20)
     for _ in range(args.warmup):
-        O.ce_fused(x["H"][:n], x["W"], x["labels"][:n])
+        run(n)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        O.ce_fused(x["H"][:n], x["W"], x["labels"][:n])
+        run(n)
     dt = (time.perf_counter() - t0) / max(1, args.steps)
     value = 6.0 * n * wl.V * wl.d / dt / 1e12
-    cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
-    sample = (f"first {n} rows of {wl.name} (full V={wl.V}, d={wl.d}) per step, "
-              f"fp64 numpy oracle ce_fused (forward, dH, dW)")
+    sample = f"first {n} rows of {wl.name} (full V={wl.V}, d={wl.d}) per step, {what}"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": n_gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(wl, wl.N, 1),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
+            "config": workload_config(wl, wl.chunk_rows or wl.N, 1, args.entry),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -287,9 +295,11 @@ def main():
                dW=torch.empty(V, d, dtype=bf, device=dev))
     stream = torch.cuda.current_stream()
 
+    # the step's per-batch inputs (W is model state and stays resident)
+    batch = {"H": H, "labels": y}
     if args.entry == "fused_ce":
-        def step(Hs=H, ys=y):
-            L.lmh_loss_fwd(shape, Hs, W, ys, out["loss_rows"], out["lse"], out["logprob"],
+        def step(b=batch):
+            L.lmh_loss_fwd(shape, b["H"], W, b["labels"], out["loss_rows"], out["lse"], out["logprob"],
                            out["argmax"], out["loss_mean"], out["n_valid"], None, out["dH"],
                            out["dW"], None, workspace=ws, stream=stream)
     elif args.entry == "ce_separate":
@@ -298,28 +308,30 @@ def main():
         bshape = L.make_shape(N, d, V, 1, chunk, L.F_MEAN)
         bws = L.workspace(bshape, L.ENTRY_LOSS_BWD, dev)
 
-        def step(Hs=H, ys=y):
-            L.lmh_loss_fwd(fshape, Hs, W, ys, out["loss_rows"], out["lse"], out["logprob"],
+        def step(b=batch):
+            L.lmh_loss_fwd(fshape, b["H"], W, b["labels"], out["loss_rows"], out["lse"],
+                           out["logprob"],
                            out["argmax"], out["loss_mean"], out["n_valid"], workspace=fws,
                            stream=stream)
             # backward of the mean loss: no grad given, 1 / n_valid taken on the device
-            L.lmh_loss_bwd(bshape, L.BWD_CE, Hs, W, ys, out["lse"], None, None, out["dH"],
-                           out["dW"], None, workspace=bws, stream=stream)
+            L.lmh_loss_bwd(bshape, L.BWD_CE, b["H"], W, b["labels"], out["lse"], None, None,
+                           out["dH"], out["dW"], None, workspace=bws, stream=stream)
     else:
-        ids, ref = x["ids"], x["ref_logp"]
-        K = ids.shape[1]
+        batch = {"H": H, "ids": x["ids"], "ref_logp": x["ref_logp"]}
+        K = batch["ids"].shape[1]
         sshape = L.make_shape(N, d, V, K, chunk, L.F_MEAN)
         sws = L.workspace(sshape, L.ENTRY_SUPPORT_KL, dev)
         bws = L.workspace(sshape, L.ENTRY_LOSS_BWD, dev)
         kl_rows = torch.empty(N, dtype=f32, device=dev)
         lp = torch.empty(N, K, dtype=f32, device=dev)
 
-        def step(Hs=H, ys=y):
-            L.lmh_support_kl(sshape, Hs, W, ids, ref, kl_rows, out["loss_mean"], lp, out["lse"],
-                             workspace=sws, stream=stream)
+        def step(b=batch):
+            L.lmh_support_kl(sshape, b["H"], W, b["ids"], b["ref_logp"], kl_rows,
+                             out["loss_mean"], lp, out["lse"], workspace=sws, stream=stream)
             # backward of the mean KL: no grad given, 1 / N on the device
-            L.lmh_loss_bwd(sshape, L.BWD_SUPPORT_KL, Hs, W, ids, out["lse"], None, ref,
-                           out["dH"], out["dW"], None, workspace=bws, stream=stream)
+            L.lmh_loss_bwd(sshape, L.BWD_SUPPORT_KL, b["H"], W, b["ids"], out["lse"], None,
+                           b["ref_logp"], out["dH"], out["dW"], None, workspace=bws,
+                           stream=stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -346,14 +358,14 @@ def main():
     # per-kernel device times of the timed region (event pairs on the launching stream)
     import ctypes
     cap = 64 * args.steps + 64
-    ids = (ctypes.c_int32 * cap)()
-    mss = (ctypes.c_float * cap)()
-    n_rec = lib().lmh_profile_read(cap, ids, mss)
+    kid_buf = (ctypes.c_int32 * cap)()
+    ms_buf = (ctypes.c_float * cap)()
+    n_rec = lib().lmh_profile_read(cap, kid_buf, ms_buf)
     per = {}
     for i in range(n_rec):
-        name = lib().lmh_kernel_name(ids[i]).decode()
+        name = lib().lmh_kernel_name(kid_buf[i]).decode()
         c, t = per.get(name, (0, 0.0))
-        per[name] = (c + 1, t + mss[i])
+        per[name] = (c + 1, t + ms_buf[i])
     kernels = {k: {"launches": c, "total_ms": t, "avg_ms": t / c,
                    "share": t / max(1e-9, sum(v[1] for v in per.values()))}
                for k, (c, t) in sorted(per.items(), key=lambda kv: -kv[1][1])}
@@ -389,34 +401,33 @@ def main():
     # end to end through the public API: pinned host batch in, loss out, every step
     e2e = None
     if not args.no_e2e:
-        # every step uploads its batch (H, labels) from pinned host memory and reads back its
-        # mean loss and valid count; the upload of step i+1 runs on a copy stream while step i
-        # computes (two device buffers), as a training loop would overlap it
-        Hh = H.cpu().pin_memory()
-        yh = y.cpu().pin_memory()
-        Hd = [torch.empty_like(H) for _ in range(2)]
-        yd = [torch.empty_like(y) for _ in range(2)]
+        # every step uploads its batch (H and labels, or H, candidate ids and reference
+        # log-probs) from pinned host memory and reads back its mean loss (and valid count);
+        # the upload of step i+1 runs on a copy stream while step i computes (two device
+        # buffers), as a training loop would overlap it
+        host = {k: v.cpu().pin_memory() for k, v in batch.items()}
+        dbuf = [{k: torch.empty_like(v) for k, v in batch.items()} for _ in range(2)]
+        reads = [out["loss_mean"]] + ([out["n_valid"]] if args.entry != "support_kl" else [])
+        reads_h = [torch.empty_like(t, device="cpu").pin_memory() for t in reads]
         ready = [torch.cuda.Event() for _ in range(2)]
         free = [torch.cuda.Event() for _ in range(2)]
-        loss_h = torch.empty(1, dtype=f32).pin_memory()
-        nv_h = torch.empty(1, dtype=i32).pin_memory()
         copy_stream = torch.cuda.Stream(device=dev)
 
         def upload(i):
             b = i % 2
             with torch.cuda.stream(copy_stream):
                 copy_stream.wait_event(free[b])
-                Hd[b].copy_(Hh, non_blocking=True)
-                yd[b].copy_(yh, non_blocking=True)
+                for k, v in host.items():
+                    dbuf[b][k].copy_(v, non_blocking=True)
                 ready[b].record(copy_stream)
 
         def compute(i):
             b = i % 2
             stream.wait_event(ready[b])
-            step(Hd[b], yd[b])
+            step(dbuf[b])
             free[b].record(stream)
-            loss_h.copy_(out["loss_mean"], non_blocking=True)
-            nv_h.copy_(out["n_valid"], non_blocking=True)
+            for th, td in zip(reads_h, reads):
+                th.copy_(td, non_blocking=True)
 
         def run(n):
             copy_stream.wait_stream(stream)
@@ -434,19 +445,20 @@ def main():
         barrier()
         ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / args.steps
         e2e = {"value": job_tflops(flops_step, world, ms_e2e), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": Hh.numel() * 2 + yh.numel() * 4,
-               "d2h_bytes_per_step": 8, "ms_per_step": ms_e2e,
-               "note": "every step copies its H and labels in from pinned host memory (on a copy "
-                       "stream, overlapped with the previous step) and reads its mean loss and "
-                       "valid count back; W stays resident as model state"}
+               "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in reads_h),
+               "ms_per_step": ms_e2e,
+               "note": f"every step copies its {', '.join(host)} in from pinned host memory (on "
+                       "a copy stream, overlapped with the previous step) and reads its mean "
+                       "back; W stays resident as model state"}
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, t, cores = oracle_sample(wl, args.cpu_seconds)
+        n, t, cores, what = oracle_sample(wl, args.cpu_seconds, args.entry)
         cpu_baseline = {"value": 6.0 * n * V * d / t / 1e12, "unit": "TFLOP/s", "cores": cores,
                         "kind": "oracle",
-                        "sample": f"first {n} rows of {wl.name} (full V={V}, d={d}): fp64 "
-                                  f"numpy oracle ce_fused (forward, dH, dW), {t:.1f} s"}
+                        "sample": f"first {n} rows of {wl.name} (full V={V}, d={d}): {what}, "
+                                  f"{t:.1f} s"}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,

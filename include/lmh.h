@@ -141,8 +141,7 @@ LMH_API size_t lmh_workspace_size(const lmh_shape* shape, int entry);
  *     sum_i loss_i (not set), reusing the forward's softmax instead of recomputing logits.
  *     dW_acc, if given, is incremented by this call's dW in chunk order (zero it first for
  *     a fresh gradient) and dW, if given, receives its round-to-nearest-even bf16 cast.
- *     Each increment is one fp32 add per element and chunk, rounded to nearest even, with
- *     subnormal operands and sums (below 2^-126) flushed to zero.
+ *     Each increment is one IEEE fp32 add per element and chunk, rounded to nearest even.
  *     Without dW_acc and with one chunk, dW is the bf16 cast of the fp32 tile sums.
  */
 LMH_API lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,

@@ -340,14 +340,19 @@ struct EpiDH {
 
 // ------------------------------------------------------------------ dW = G^T H_c
 // acc_mode 0: the tile sum is the whole dW, stored in bf16 (ctx.tmC: bf16 dW [V, d]).
-// acc_mode 1: acc = 0 + sum (first chunk into a fresh internal accumulator; 0 + x turns -0
-// into +0 exactly as an add into a zeroed buffer would), stored in fp32.
+// acc_mode 1: acc = 0 + sum (first chunk), stored in fp32.
 // acc_mode 2: acc += sum, one fp32 add per element done by the TMA unit at L2.
-// In modes 1 and 2 ctx.tmC maps the fp32 accumulator [V, d]; every element has one owner tile
-// per launch and the launches of a call run in chunk order, so the accumulation order is fixed.
-// The accumulator never passes through registers: the epilogue only writes, and the DRAM
-// read-modify-write runs at L2 asynchronously instead of as 16-byte loads that each wait for
-// memory. The bf16 cast of the final accumulator is a separate pass after the last chunk.
+// acc_mode 3: dW = bf16(acc + sum) (last chunk of an internal accumulator, which is not
+//             written back): the accumulator block is loaded by TMA into the warp's staging
+//             buffers, added in registers, and the bf16 result stored through ctx.tmC.
+// In modes 1 and 2 ctx.tmC maps the fp32 accumulator [V, d]; in mode 3 ctx.tmD does (fp32,
+// box 32 x 32 rows, 128-byte swizzle) and ctx.tmC maps bf16 dW. Every
+// element has one owner tile per launch and the launches of a call run in chunk order, so the
+// accumulation order is fixed. Every add (modes 1 and 3 in registers, mode 2 in the TMA unit)
+// is an IEEE fp32 add rounded to nearest even, so an internal accumulator gives the same bits
+// as a zeroed caller-owned one. The accumulator is never read by 16-byte register loads that
+// wait on DRAM one row at a time: writes are staged stores and L2 reduce-adds, and the one
+// read (mode 3) is a TMA block load.
 struct EpiDW {
   static constexpr int kId = 6;        // gemm_dW
   static constexpr int kAMajorMN = 1;  // G^T: G chunk [rows, V] read as [K = rows, M = V]
@@ -361,7 +366,7 @@ struct EpiDW {
                                               int rit, EpiCtx& ctx) {
     const int n0 = nb * BN;
     const int wrow = mb * BM + ctx.row_w;
-    const bool wv = wrow < p.V;  // rows past V are clipped by the tensor map
+    const bool wv = wrow < p.V;  // rows past V are clipped by the tensor maps
 #pragma unroll 1
     for (int sb = 0; sb < kSlabs; ++sb) {
       const int col0 = n0 + sb * 64;
@@ -371,6 +376,10 @@ struct EpiDW {
       tmem_ld32(taddr + sb * 64 + 32, b);
       if (p.acc_mode == 0) {
         stage_store_64(ctx, a, b, col0, wrow, wv);
+      } else if (p.acc_mode == 3) {
+        if (!wv) continue;  // warp-uniform: nothing of this block exists
+        add_loaded_64(ctx, col0, wrow, a, b);
+        stage_store_64(ctx, a, b, col0, wrow, true);
       } else {
         if (p.acc_mode == 1) {
 #pragma unroll
@@ -383,6 +392,39 @@ struct EpiDW {
         stage_f32_32(ctx, b, col0 + 32, wrow, wv, p.acc_mode == 2);
       }
     }
+  }
+  // a (+)= acc[wrow + lane, col0 .. col0+31], b (+)= acc[.., col0+32 .. col0+63], the 32 x 64
+  // fp32 block loaded by TMA into the warp's two staging buffers (zero past V).
+  static __device__ __forceinline__ void add_loaded_64(EpiCtx& c, int col0, int wrow,
+                                                       float (&a)[32], float (&b)[32]) {
+    const uint32_t b0 = c.stage, b1 = c.stage + EPI_BUF_BYTES;
+    if (c.lane == 0) {
+      bulk_wait_read_all();  // earlier staged stores have finished reading both buffers
+      mbar_arrive_expect_tx(c.bar, 2 * EPI_BUF_BYTES);
+      tma_load_2d(b0, c.tmD, c.bar, col0, wrow);
+      tma_load_2d(b1, c.tmD, c.bar, col0 + 32, wrow);
+    }
+    __syncwarp();
+    // bounded: on expiry the error word is set; wait once more for the copies in flight
+    if (!mbar_wait(c.bar, c.bar_phase, c.err)) mbar_wait(c.bar, c.bar_phase, c.err);
+    c.bar_phase ^= 1u;
+    const uint32_t sw = static_cast<uint32_t>(c.lane & 7);
+    const uint32_t off = static_cast<uint32_t>(c.lane) * 128u;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t ch = ((static_cast<uint32_t>(u) ^ sw) << 4) + off;
+      const uint4 x = ld_shared_v4(b0 + ch);
+      const uint4 y = ld_shared_v4(b1 + ch);
+      a[u * 4 + 0] = __fadd_rn(__uint_as_float(x.x), a[u * 4 + 0]);
+      a[u * 4 + 1] = __fadd_rn(__uint_as_float(x.y), a[u * 4 + 1]);
+      a[u * 4 + 2] = __fadd_rn(__uint_as_float(x.z), a[u * 4 + 2]);
+      a[u * 4 + 3] = __fadd_rn(__uint_as_float(x.w), a[u * 4 + 3]);
+      b[u * 4 + 0] = __fadd_rn(__uint_as_float(y.x), b[u * 4 + 0]);
+      b[u * 4 + 1] = __fadd_rn(__uint_as_float(y.y), b[u * 4 + 1]);
+      b[u * 4 + 2] = __fadd_rn(__uint_as_float(y.z), b[u * 4 + 2]);
+      b[u * 4 + 3] = __fadd_rn(__uint_as_float(y.w), b[u * 4 + 3]);
+    }
+    __syncwarp();  // every lane has read both buffers before the bf16 staging reuses one
   }
 };
 

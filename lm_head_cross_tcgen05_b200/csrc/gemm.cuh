@@ -61,11 +61,15 @@ constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + 1024;  
 // staging buffers, and a running count of its stores (which selects the buffer).
 struct EpiCtx {
   const CUtensorMap* tmC;
+  const CUtensorMap* tmD;  // a second map some epilogues read through (else tmC again)
   uint32_t stage;
   int lane;
   int row_w;         // first accumulator row of this warp within the CTA's 128
   uint32_t nstore;
   int split;         // K range of the current work unit (0 unless K is split)
+  uint32_t bar;      // this warp's mbarrier for TMA loads into its staging buffers
+  uint32_t bar_phase;
+  uint32_t* err;
 };
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -101,7 +105,8 @@ template <class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmC, const GemmGrid g,
+                   const __grid_constant__ CUtensorMap tmC,
+                   const __grid_constant__ CUtensorMap tmD, const GemmGrid g,
                    const typename Epi::Params ep) {
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];   // rank 0: operands of a stage landed
@@ -109,6 +114,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   __shared__ __align__(8) uint64_t tfull_bar[2];       // both: accumulator b is complete
   __shared__ __align__(8) uint64_t tempty_bar[2];      // rank 0: both CTAs drained accumulator b
   __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ __align__(8) uint64_t epi_bar[4];         // epilogue warp w-2: its staged loads
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
 
@@ -130,6 +136,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(smem_u32(&tempty_bar[b]), 8);  // 4 epilogue warps x 2 CTAs
     }
     mbar_init(smem_u32(&drain_bar), 1);
+    for (int w = 0; w < 4; ++w) mbar_init(smem_u32(&epi_bar[w]), 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -243,8 +250,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // the TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
-    EpiCtx ctx{&tmC, smem_base + STAGES * STAGE_BYTES + (warp - 2) * 2 * EPI_BUF_BYTES, lane,
-               q * 32, 0u, 0};
+    EpiCtx ctx{&tmC, &tmD, smem_base + STAGES * STAGE_BYTES + (warp - 2) * 2 * EPI_BUF_BYTES, lane,
+               q * 32, 0u, 0, smem_u32(&epi_bar[warp - 2]), 0u, g.err};
     if (lane == 0) tma_prefetch_desc(&tmC);
     int it = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++it) {

@@ -52,15 +52,17 @@ bool shape_ok(const lmh_shape* s) {
 
 // K splits of the dH GEMM of a chunk with `rows` rows. Chunks with too few output tiles to keep
 // every SM busy (fewer than 384 pair tiles) split the vocabulary into up to 8 ranges, aiming at
-// 512 work units; each range keeps at least 8 K blocks. The rule reads the shape only (never
-// the SM count), so the result bits do not depend on the GPU's size.
+// 512 work units. Each split costs a write and a read of an fp32 [rows, d] partial, i.e. 8 / V
+// bytes per flop of the GEMM: a range must span at least 32768 vocabulary rows, which keeps
+// that traffic near 3 % of the GEMM's time (at V = 32000 no split pays). The rule reads the
+// shape only (never the SM count), so the result bits do not depend on the GPU's size.
 int dh_splits(int64_t rows, int64_t d, int64_t V) {
   const int64_t tiles = cdiv(rows, PM) * cdiv(d, BN);
   if (tiles >= 384) return 1;
   int64_t sp = cdiv(512, tiles);
-  const int64_t by_k = cdiv(V, BK) / 8;
+  const int64_t by_v = V / 32768;
   if (sp > 8) sp = 8;
-  if (sp > by_k) sp = by_k;
+  if (sp > by_v) sp = by_v;
   return sp < 1 ? 1 : static_cast<int>(sp);
 }
 
@@ -272,7 +274,7 @@ template <class Epi>
 lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap& b,
                        const CUtensorMap& c, int64_t M, int64_t Ncols, int64_t K,
                        GemmOrder order, uint32_t* err, const typename Epi::Params& ep,
-                       cudaStream_t st, int k_splits = 1) {
+                       cudaStream_t st, int k_splits = 1, const CUtensorMap* d = nullptr) {
   static std::atomic<uint64_t> attr_done{0};
   static std::atomic<int> pairs_cache[64];
   const uint64_t bit = 1ull << dev;
@@ -308,7 +310,8 @@ lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap
   const int64_t pairs_max = pairs_cache[dev].load();
   const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
   ProfScope ps(Epi::kId, st);
-  gemm_tc_kernel<Epi><<<2 * pairs, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(a, b, c, g, ep);
+  gemm_tc_kernel<Epi><<<2 * pairs, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(a, b, c, d ? *d : c,
+                                                                        g, ep);
   return cudaGetLastError() == cudaSuccess ? LMH_OK : LMH_ERR_CUDA;
 }
 
@@ -449,16 +452,30 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
     CUtensorMap ta, tb, tc;
     if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BK) || !tmap_2d(&tb, H + r0 * P.d, P.d, rows, P.d, BK))
       return LMH_ERR_CUDA;
+    // Internal accumulator (several chunks, no caller dW_acc): store, add, ..., and the last
+    // chunk adds and casts in its epilogue without writing the sum back. Caller's dW_acc:
+    // add in every chunk, then cast it. One chunk without dW_acc: bf16 tile sums directly.
+    const bool last = chunk_idx == P.nchunks - 1;
     float* acc = dW_acc ? dW_acc : (P.acc ? ws.at<float>(P.o_acc) : nullptr);
     EpiDW::Params ep;
     ep.V = static_cast<int>(P.V);
     ep.d = static_cast<int>(P.d);
-    ep.acc_mode = !acc ? 0 : (dW_acc || chunk_idx > 0) ? 2 : 1;
-    if (!(acc ? tmap_acc(&tc, acc, P.d, P.V, P.d) : tmap_out(&tc, dW, P.d, P.V, P.d)))
-      return LMH_ERR_CUDA;
+    if (!acc) ep.acc_mode = 0;
+    else if (dW_acc) ep.acc_mode = 2;
+    else ep.acc_mode = chunk_idx == 0 ? 1 : (last ? 3 : 2);
+    CUtensorMap td;  // mode 3: the accumulator, read by the epilogue
+    bool ok;
+    if (ep.acc_mode == 0) {
+      ok = tmap_out(&tc, dW, P.d, P.V, P.d);
+    } else if (ep.acc_mode == 3) {
+      ok = tmap_out(&tc, dW, P.d, P.V, P.d) && tmap_acc(&td, acc, P.d, P.V, P.d);
+    } else {
+      ok = tmap_acc(&tc, acc, P.d, P.V, P.d);
+    }
+    if (!ok) return LMH_ERR_CUDA;
     LMH_TRY(launch_gemm<EpiDW>(dev, sms, ta, tb, tc, P.V, P.d, rows, kOrderDW, &ws.h->err, ep,
-                               st));
-    if (acc && dW && chunk_idx == P.nchunks - 1) LMH_TRY(cast_dw(P, acc, dW, st));
+                               st, 1, ep.acc_mode == 3 ? &td : nullptr));
+    if (dW_acc && dW && last) LMH_TRY(cast_dw(P, acc, dW, st));
   }
   return LMH_OK;
 }

@@ -169,6 +169,22 @@ def test_dW_is_bf16_cast_of_fp32_accumulator():
     assert torch.equal(o3["dW"], o["dW"])
 
 
+@pytest.mark.parametrize("chunk", [0, 16])
+def test_dW_accumulate_is_ieee_add(chunk):
+    # H = 0 makes every dW contribution zero, so the accumulator must come back unchanged:
+    # subnormal values are neither flushed by the add nor by the cast's input
+    x, _ = device_inputs(_wl(64, 128, 700, 0))
+    H = torch.zeros_like(x["H"])
+    acc = torch.full((700, 128), 1e-39, dtype=torch.float32, device="cuda")
+    acc[::2] = -3.5e-40
+    acc[1::7] = 1.25
+    before = acc.clone()
+    o = L.loss_fwd(H, x["W"], x["labels"], chunk_rows=chunk, grads=True, dW_acc=acc)
+    assert torch.equal(acc, before)
+    assert torch.equal(o["dW"], before.to(torch.bfloat16))
+    assert torch.count_nonzero(o["dH"]) > 0  # dH = G W does not vanish
+
+
 def test_no_valid_rows_and_empty_call():
     x, xc = device_inputs(_wl(140, 64, 500, 0))
     y = torch.full_like(x["labels"], -100)
@@ -371,3 +387,51 @@ def test_maximum_candidate_count():
     with pytest.raises((ValueError, L.LmhError)):
         ids = torch.zeros(N, K + 1, dtype=torch.int32, device="cuda")
         L.support_logprob(x["H"], x["W"], ids)
+
+
+def _kernels_launched(fn):
+    """Names of the library kernels that fn() launched (the library's own launch record)."""
+    import ctypes
+    from lm_head_cross_tcgen05_b200._abi import lib
+    lib().lmh_profile_read(0, None, None)  # drop any earlier records
+    lib().lmh_profile_enable(1)
+    try:
+        fn()
+        torch.cuda.synchronize()
+    finally:
+        lib().lmh_profile_enable(0)
+    cap = 4096
+    kid, ms = (ctypes.c_int32 * cap)(), (ctypes.c_float * cap)()
+    n = lib().lmh_profile_read(cap, kid, ms)
+    return [lib().lmh_kernel_name(kid[i]).decode() for i in range(n)]
+
+
+@pytest.mark.parametrize("N,d,V,ign,splits", [
+    (300, 320, 70000, 5, 2),     # 4 dH tiles: V split in 2 ranges, the last K block ragged
+    (130, 128, 132072, 0, 4),    # 1 dH tile: V split in 4 ranges
+])
+def test_dh_split_over_vocabulary(N, d, V, ign, splits):
+    # chunks with few dH tiles and a large V sum dH over vocabulary ranges in a fixed order
+    x, xc = device_inputs(_wl(N, d, V, ign))
+    res = {}
+
+    def run():
+        res["o"] = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    names = _kernels_launched(run)
+    assert names.count("split_sum") == 1 and names.count("gemm_dH") == 1
+    out = res["o"]
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    check_ce_fused(out, O.ce_fused(xc["H"], xc["W"], xc["labels"]))
+    again = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    assert torch.equal(again["dH"], out["dH"]) and torch.equal(again["dW"], out["dW"])
+    # the same problem split across row chunks sums dW in chunk order: same values to rounding
+    ch = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=128, grads=True)
+    assert torch.equal(ch["lse"], out["lse"])
+    check_grad(ch["dH"], out["dH"], "dH chunked vs split")
+
+
+def test_no_split_when_vocabulary_is_small():
+    # V = 32000: the fp32 partials would cost more than the fuller waves give back
+    x, _ = device_inputs(_wl(256, 256, 32000, 0))
+    names = _kernels_launched(lambda: L.loss_fwd(x["H"], x["W"], x["labels"], grads=True))
+    assert "split_sum" not in names and names.count("gemm_dH") == 1
