@@ -42,11 +42,13 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_vocab")
-    ap.add_argument("--entry", choices=["fused_ce", "ce_separate", "support_kl"],
+    ap.add_argument("--entry", choices=["fused_ce", "ce_separate", "support_kl",
+                                        "vocab_parallel"],
                     default="fused_ce",
                     help="fused_ce: lmh_loss_fwd with dH/dW (the headline step); ce_separate: "
                          "lmh_loss_fwd then lmh_loss_bwd (recomputed logits); support_kl: "
-                         "lmh_support_kl then lmh_loss_bwd of the mean KL")
+                         "lmh_support_kl then lmh_loss_bwd of the mean KL; vocab_parallel: one "
+                         "CE problem with W split over the GPUs (strong scaling)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -74,15 +76,19 @@ def source_hash() -> str:
 
 ENTRY_TEXT = {"fused_ce": "fused CE forward+backward",
               "ce_separate": "CE forward, then backward with recomputed logits",
-              "support_kl": "support-set KL forward (K candidates), then its backward"}
+              "support_kl": "support-set KL forward (K candidates), then its backward",
+              "vocab_parallel": "vocabulary-parallel CE forward, then backward with recomputed "
+                                "logits (W split over the GPUs)"}
 
 
 def workload_config(wl, chunk_rows, n_gpus, entry="fused_ce"):
+    vp = entry == "vocab_parallel"
     return {"workload": f"{wl.name}: {ENTRY_TEXT[entry]}, N={wl.N} d={wl.d} V={wl.V}, "
                         f"{wl.labels} labels, {wl.num_ignored} ignored rows, bf16 H/W",
             "entry": entry,
             "N": wl.N, "d": wl.d, "V": wl.V, "chunk_rows": chunk_rows,
-            "rows_per_gpu": wl.N, "total_rows": wl.N * n_gpus,
+            "parallelism": (f"vocab-parallel over {n_gpus}" if vp else f"replicas x{n_gpus}"),
+            "rows_per_gpu": wl.N, "total_rows": wl.N if vp else wl.N * n_gpus,
             "l2": "inputs larger than L2 (W alone is %.2f GB)" % (wl.V * wl.d * 2 / 1e9)}
 
 
@@ -278,7 +284,9 @@ def main():
     def max_over_ranks(v: float) -> float:
         return reduce_max(v, world, dev)
 
-    x = make_inputs(wl, device=dev, seed=replica_seed(wl, rank))
+    vp_entry = args.entry == "vocab_parallel"
+    # replicas draw one batch per rank; the vocabulary-parallel ranks share one problem
+    x = make_inputs(wl, device=dev, seed=wl.seed if vp_entry else replica_seed(wl, rank))
     H, W, y = x["H"], x["W"], x["labels"]
     N, d, V = wl.N, wl.d, wl.V
     chunk = wl.chunk_rows or N
@@ -316,6 +324,16 @@ def main():
             # backward of the mean loss: no grad given, 1 / n_valid taken on the device
             L.lmh_loss_bwd(bshape, L.BWD_CE, b["H"], W, b["labels"], out["lse"], None, None,
                            out["dH"], out["dW"], None, workspace=bws, stream=stream)
+    elif vp_entry:
+        from lm_head_cross_tcgen05_b200.vocab_parallel import VocabParallelCE
+        vp = VocabParallelCE(V, chunk_rows=chunk)      # the default group when world > 1
+        W_shard = W[vp.v0:vp.v1].contiguous()
+
+        def step(b=batch):
+            f = vp.forward(b["H"], W_shard, b["labels"])
+            vp.backward(b["H"], W_shard, b["labels"], f["lse"])
+            out["loss_mean"].copy_(f["loss_mean"])
+            out["n_valid"].copy_(f["n_valid"])
     else:
         batch = {"H": H, "ids": x["ids"], "ref_logp": x["ref_logp"]}
         K = batch["ids"].shape[1]
@@ -353,7 +371,8 @@ def main():
     ms_total = max_over_ranks(e0.elapsed_time(e1))
     ms_step = ms_total / args.steps
     flops_step = 6.0 * N * V * d
-    value = job_tflops(flops_step, world, ms_step)
+    jobs = 1 if vp_entry else world          # problems solved per step by the whole job
+    value = job_tflops(flops_step, jobs, ms_step)
 
     # per-kernel device times of the timed region (event pairs on the launching stream)
     import ctypes
@@ -373,7 +392,8 @@ def main():
     peaks, peak_src = load_peaks()
     roofline = None
     if dom:
-        gemm_flops = 2.0 * chunk * V * d      # one GEMM launch over one chunk
+        V_gemm = (vp.v1 - vp.v0) if vp_entry else V     # the vocabulary one GEMM spans
+        gemm_flops = 2.0 * chunk * V_gemm * d           # one GEMM launch over one chunk
         hbm_bytes = {"gbuild": 4.0 * chunk * ((V + 7) // 8 * 8)}
         if dom.startswith("gemm"):
             ach = gemm_flops / (kernels[dom]["avg_ms"] / 1e3) / 1e12
@@ -444,7 +464,7 @@ def main():
         e1.record(stream)
         barrier()
         ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / args.steps
-        e2e = {"value": job_tflops(flops_step, world, ms_e2e), "unit": "TFLOP/s",
+        e2e = {"value": job_tflops(flops_step, jobs, ms_e2e), "unit": "TFLOP/s",
                "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in reads_h),
                "ms_per_step": ms_e2e,
@@ -463,8 +483,8 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16", "data": "synthetic",
+                "higher_is_better": True, "scaling": "strong" if vp_entry else "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": workload_config(wl, chunk, world, args.entry),
                 "peak_frac": {"of_burst": value / world / peaks["bf16_tflops"],
                               "of_sustained": value / world / peaks["bf16_tflops_sustained"],

@@ -84,6 +84,9 @@ typedef enum lmh_status {
 #define LMH_ENTRY_LOGPROB 2
 #define LMH_ENTRY_SUPPORT_LOGPROB 3
 #define LMH_ENTRY_SUPPORT_KL 4
+#define LMH_ENTRY_VP_PARTIALS 5 /* vocabulary-parallel entries, below */
+#define LMH_ENTRY_VP_COMBINE 6
+#define LMH_ENTRY_VP_BWD 7
 
 /* objectives of lmh_loss_bwd */
 #define LMH_BWD_CE 0              /* L = sum_i g_i loss_i                                */
@@ -217,6 +220,74 @@ LMH_API lmh_status lmh_support_kl(const lmh_shape* shape, const lmh_bf16* H, con
                           const int32_t* ids, const float* ref_logp, float* kl_rows,
                           float* kl_mean, float* lp, float* lse, void* workspace,
                           size_t workspace_bytes, void* stream);
+
+/*
+ * Vocabulary-parallel cross entropy. The pages run the head at tensor-parallel size 1 only
+ * (miles-ext-kernels PR #14, lm_head op commit: the validate hook's startup checks). These
+ * entries split the same definitions over R ranks that each hold a contiguous row range
+ * [v0, v0 + V_r) of W (the shard); every rank passes the whole H, the global labels and the
+ * same chunk_rows, temperature and flags. Per step:
+ *   1. lmh_vp_partials on every rank: a 4-word record per row over the rank's shard.
+ *   2. The caller gathers the records of all ranks, in rank order, into [R, N, 4].
+ *   3. lmh_vp_combine (any rank, or every rank): lse, loss, log-prob, argmax and the mean, as
+ *      lmh_loss_fwd gives them for the whole vocabulary, combined over the ranks in ascending
+ *      order.
+ *   4. lmh_vp_loss_bwd on every rank with the combined lse: the rank's fp32 contribution to
+ *      dH (the sum over its shard) and its shard's dW. dW needs no exchange.
+ *   5. The caller sums the dH contributions with lmh_vp_reduce_rows, in rank order (for
+ *      example: each rank gathers one row slice from every rank, reduces it, and the bf16
+ *      slices are gathered back).
+ * With a fixed R and shard plan every output is bitwise reproducible. Against the one-device
+ * entries the lse is combined in a different grouping (tiles within a shard, then shards), so
+ * the values agree to fp32 rounding, not bit for bit. Label rules as lmh_loss_fwd, against the
+ * full vocabulary V_total.
+ *
+ * lmh_vp_partials: shard->V = V_r (the shard's rows of W), shard->N, d, chunk_rows, flags,
+ *   temperature as for lmh_logprob. W_shard [V_r, d] bf16. records [N, 4] out, 16-byte
+ *   aligned: { lse_r (fp32) = log sum over the shard of exp z_iv; max_r (fp32) = the shard's
+ *   largest logit; arg_r (int32 bits) = the smallest global id attaining it; zy_r (fp32) =
+ *   the label's logit if 0 <= y_i - v0 < V_r, else -inf }. Requires 0 <= v0 and
+ *   v0 + V_r <= V_total. Workspace: lmh_workspace_size(shard, LMH_ENTRY_VP_PARTIALS).
+ */
+LMH_API lmh_status lmh_vp_partials(const lmh_shape* shard, int64_t v0, int64_t V_total,
+                                   const lmh_bf16* H, const lmh_bf16* W_shard,
+                                   const int32_t* labels, float* records, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
+ * lmh_vp_combine: shape->N rows, shape->V = V_total, shape->d as the shards'. records
+ * [R, N, 4] in (the ranks' records in rank order, 16-byte aligned). Outputs as lmh_loss_fwd:
+ * loss_rows, lse (required), logprob, argmax, loss_mean, n_valid (nullable), n_valid_given
+ * (nullable). A valid row whose label logit no record holds sets LMH_DEVERR_NONFINITE.
+ * Workspace: lmh_workspace_size(shape, LMH_ENTRY_VP_COMBINE) (256 bytes).
+ */
+LMH_API lmh_status lmh_vp_combine(const lmh_shape* shape, int R, const float* records,
+                                  const int32_t* labels, float* loss_rows, float* lse,
+                                  float* logprob, int32_t* argmax, float* loss_mean,
+                                  int32_t* n_valid, const int32_t* n_valid_given, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
+ * lmh_vp_loss_bwd: the shard's part of lmh_loss_bwd (mode LMH_BWD_CE or LMH_BWD_LOGPROB; grad
+ * nullable as there, with the count over the full vocabulary). lse [N] is the combined one.
+ * dH_part [N, d] fp32 out (nullable): sum over the shard's columns of G_iv W_v, to be summed
+ * over the ranks. dW_shard [V_r, d] bf16 out and dW_acc_shard [V_r, d] fp32 in/out (nullable,
+ * as dW and dW_acc of lmh_loss_bwd). Workspace: lmh_workspace_size(shard, LMH_ENTRY_VP_BWD)
+ * (with LMH_F_DW_ACC_GIVEN in shard->flags if dW_acc_shard is passed).
+ */
+LMH_API lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t v0,
+                                   int64_t V_total, const lmh_bf16* H, const lmh_bf16* W_shard,
+                                   const int32_t* labels, const float* lse, const float* grad,
+                                   float* dH_part, lmh_bf16* dW_shard, float* dW_acc_shard,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * lmh_vp_reduce_rows: out[j] = bf16(sum_{r = 0..R-1} parts[r, j]) over rows x d elements, the
+ * R fp32 contributions added in ascending r (round to nearest even). parts [R, rows, d] fp32,
+ * out [rows, d] bf16, both 16-byte aligned; d a multiple of 64. No workspace.
+ */
+LMH_API lmh_status lmh_vp_reduce_rows(int R, int64_t rows, int64_t d, const float* parts,
+                                      lmh_bf16* out, void* stream);
 
 /*
  * lmh_read_errors — synchronises `stream`, then copies the device error word of the last

@@ -18,7 +18,8 @@ import torch
 
 from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEVERR_LABEL_RANGE,
                    DEVERR_NONFINITE, DEVERR_TEMPERATURE, DEVERR_TIMEOUT, ENTRY_LOGPROB, ENTRY_LOSS_BWD,
-                   ENTRY_LOSS_FWD, ENTRY_SUPPORT_KL, ENTRY_SUPPORT_LOGPROB, F_DW_ACC_GIVEN,
+                   ENTRY_LOSS_FWD, ENTRY_SUPPORT_KL, ENTRY_SUPPORT_LOGPROB, ENTRY_VP_BWD,
+                   ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN,
                    F_FUSED_BWD, F_MEAN, F_SUPPORT_RENORM, IGNORE_INDEX, MAX_K, STATUS_NAMES, lib, lmh_shape)
 
 __all__ = [
@@ -29,6 +30,8 @@ __all__ = [
     "F_MEAN", "F_FUSED_BWD", "F_DW_ACC_GIVEN", "F_SUPPORT_RENORM", "ENTRY_LOSS_FWD", "ENTRY_LOSS_BWD",
     "ENTRY_LOGPROB", "ENTRY_SUPPORT_LOGPROB", "ENTRY_SUPPORT_KL", "DEVERR_LABEL_RANGE",
     "DEVERR_TIMEOUT", "DEVERR_NONFINITE", "DEVERR_TEMPERATURE", "MAX_K",
+    "lmh_vp_partials", "lmh_vp_combine", "lmh_vp_loss_bwd", "lmh_vp_reduce_rows",
+    "ENTRY_VP_PARTIALS", "ENTRY_VP_COMBINE", "ENTRY_VP_BWD",
 ]
 
 lib()  # load now: a missing library is an import error, never a silent fallback
@@ -134,6 +137,47 @@ def lmh_support_kl(shape, H, W, ids, ref_logp, kl_rows, kl_mean=None, lp=None, l
                               _p(lp, _f32, "lp"), _p(lse, _f32, "lse"),
                               _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
     _ok("lmh_support_kl", st)
+
+
+def lmh_vp_partials(shard, v0, V_total, H, W_shard, labels, records, *, workspace,
+                    stream=None) -> None:
+    st = lib().lmh_vp_partials(ctypes.byref(shard), int(v0), int(V_total), _p(H, _bf, "H"),
+                               _p(W_shard, _bf, "W_shard"), _p(labels, _i32, "labels"),
+                               _p(records, _f32, "records"), _p(workspace, _u8, "workspace"),
+                               workspace.numel(), _s(stream))
+    _ok("lmh_vp_partials", st)
+
+
+def lmh_vp_combine(shape, R, records, labels, loss_rows, lse, logprob=None, argmax=None,
+                   loss_mean=None, n_valid=None, n_valid_given=None, *, workspace,
+                   stream=None) -> None:
+    st = lib().lmh_vp_combine(ctypes.byref(shape), int(R), _p(records, _f32, "records"),
+                              _p(labels, _i32, "labels"), _p(loss_rows, _f32, "loss_rows"),
+                              _p(lse, _f32, "lse"), _p(logprob, _f32, "logprob"),
+                              _p(argmax, _i32, "argmax"), _p(loss_mean, _f32, "loss_mean"),
+                              _p(n_valid, _i32, "n_valid"),
+                              _p(n_valid_given, _i32, "n_valid_given"),
+                              _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
+    _ok("lmh_vp_combine", st)
+
+
+def lmh_vp_loss_bwd(shard, mode, v0, V_total, H, W_shard, labels, lse, grad=None, dH_part=None,
+                    dW_shard=None, dW_acc_shard=None, *, workspace, stream=None) -> None:
+    st = lib().lmh_vp_loss_bwd(ctypes.byref(shard), int(mode), int(v0), int(V_total),
+                               _p(H, _bf, "H"), _p(W_shard, _bf, "W_shard"),
+                               _p(labels, _i32, "labels"), _p(lse, _f32, "lse"),
+                               _p(grad, _f32, "grad"), _p(dH_part, _f32, "dH_part"),
+                               _p(dW_shard, _bf, "dW_shard"), _p(dW_acc_shard, _f32, "dW_acc_shard"),
+                               _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
+    _ok("lmh_vp_loss_bwd", st)
+
+
+def lmh_vp_reduce_rows(parts, out, stream=None) -> None:
+    """parts [R, rows, d] fp32 -> out [rows, d] bf16, summed in ascending R."""
+    R, rows, d = parts.shape
+    st = lib().lmh_vp_reduce_rows(int(R), int(rows), int(d), _p(parts, _f32, "parts"),
+                                  _p(out, _bf, "out"), _s(stream))
+    _ok("lmh_vp_reduce_rows", st)
 
 
 def lmh_read_errors(workspace: torch.Tensor, stream=None) -> int:

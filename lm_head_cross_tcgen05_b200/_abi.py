@@ -21,6 +21,7 @@ IGNORE_INDEX = -100
 DEVERR_LABEL_RANGE, DEVERR_TIMEOUT, DEVERR_NONFINITE, DEVERR_TEMPERATURE = 0x1, 0x2, 0x4, 0x8
 F_MEAN, F_FUSED_BWD, F_DW_ACC_GIVEN, F_SUPPORT_RENORM = 0x1, 0x2, 0x4, 0x8
 ENTRY_LOSS_FWD, ENTRY_LOSS_BWD, ENTRY_LOGPROB, ENTRY_SUPPORT_LOGPROB, ENTRY_SUPPORT_KL = range(5)
+ENTRY_VP_PARTIALS, ENTRY_VP_COMBINE, ENTRY_VP_BWD = 5, 6, 7
 BWD_CE, BWD_LOGPROB, BWD_SUPPORT_LOGPROB, BWD_SUPPORT_KL = range(4)
 MAX_K = 1024
 
@@ -39,6 +40,12 @@ _SIGS = {
     "lmh_logprob": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6 + [c_size_t, _P]),
     "lmh_support_logprob": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6 + [c_size_t, _P]),
     "lmh_support_kl": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 9 + [c_size_t, _P]),
+    "lmh_vp_partials": (c_int, [ctypes.POINTER(lmh_shape), c_int64, c_int64] + [_P] * 5
+                        + [c_size_t, _P]),
+    "lmh_vp_combine": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 10 + [c_size_t, _P]),
+    "lmh_vp_loss_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int, c_int64, c_int64] + [_P] * 9
+                        + [c_size_t, _P]),
+    "lmh_vp_reduce_rows": (c_int, [c_int, c_int64, c_int64, _P, _P, _P]),
     "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),
     "lmh_logprob_noalloc": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6),
     "lmh_selftest_wait_timeout": (c_int, [_P, c_uint32, _P]),

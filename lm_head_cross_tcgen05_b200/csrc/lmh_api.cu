@@ -14,6 +14,7 @@
 #include "gemm.cuh"
 #include "rowops.cuh"
 #include "sparse.cuh"
+#include "vp.cuh"
 
 using namespace lmh;
 
@@ -36,6 +37,7 @@ struct Plan {
   size_t o_zt, o_sorted, o_nuniq, o_rank, o_pm, o_ps, o_pi, o_alpha, o_beta, o_gbuf, o_acc;
   size_t o_gu, o_cnt, o_off, o_fill, o_prow, o_pslot;  // sparse backward
   size_t o_dhpart;                                     // split-K partials of dH
+  size_t o_lloc;                                       // vocab-parallel: shard-local labels
   size_t total;
   Temperature temp;  // logits are z / tau_i
 };
@@ -80,14 +82,15 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   const int64_t c = s->chunk_rows > 0 ? s->chunk_rows : kDefaultChunk;
   p.c = p.N > 0 ? (c < p.N ? c : p.N) : 0;
   p.nchunks = p.N > 0 ? cdiv(p.N, p.c) : 0;
+  const bool vp_bwd = entry == LMH_ENTRY_VP_BWD;
+  const bool bwd = entry == LMH_ENTRY_LOSS_BWD || vp_bwd;
   p.cands = (entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL ||
              entry == LMH_ENTRY_LOSS_BWD);
   p.K = p.cands ? (s->K > 0 ? s->K : 1) : 1;
   p.renorm = p.cands && (s->flags & LMH_F_SUPPORT_RENORM);
-  p.gbuf = !p.renorm &&
-           ((entry == LMH_ENTRY_LOSS_BWD) || (entry == LMH_ENTRY_LOSS_FWD && fused));
+  p.gbuf = !p.renorm && (bwd || (entry == LMH_ENTRY_LOSS_FWD && fused));
   p.acc = p.gbuf && dw_without_acc && p.nchunks > 1;
-  const bool stats = entry != LMH_ENTRY_LOSS_BWD;
+  const bool stats = !bwd && entry != LMH_ENTRY_VP_COMBINE;
   const bool partials = stats && !p.renorm;
   size_t o = sizeof(WsHeader);
   auto take = [&](size_t bytes) {
@@ -104,11 +107,12 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   p.o_pm = partials ? take(cT * 4) : 0;
   p.o_ps = partials ? take(cT * 4) : 0;
   p.o_pi = partials ? take(cT * 4) : 0;
-  p.o_alpha = (entry == LMH_ENTRY_LOSS_BWD) ? take(N * 4) : 0;
-  p.o_beta = (entry == LMH_ENTRY_LOSS_BWD) ? take(N * p.K * 4) : 0;
+  p.o_alpha = bwd ? take(N * 4) : 0;
+  p.o_beta = bwd ? take(N * p.K * 4) : 0;
+  p.o_lloc = (vp_bwd || entry == LMH_ENTRY_VP_PARTIALS) ? take(N * 4) : 0;
   p.o_gbuf = p.gbuf ? take(static_cast<size_t>(p.c) * p.Vp * 2) : 0;
   p.o_acc = p.acc ? take(static_cast<size_t>(p.V) * p.d * 4) : 0;
-  if (p.gbuf && p.nchunks > 0) {  // the largest split-K partial of any chunk
+  if (p.gbuf && p.nchunks > 0 && !vp_bwd) {  // the largest split-K partial of any chunk
     const int64_t last = p.N - (p.nchunks - 1) * p.c;
     const int64_t a = dh_splits(p.c, p.d, p.V) > 1 ? dh_splits(p.c, p.d, p.V) * p.c : 0;
     const int64_t b = dh_splits(last, p.d, p.V) > 1 ? dh_splits(last, p.d, p.V) * last : 0;
@@ -163,13 +167,15 @@ enum KernelId {
   KID_COUNT_LABELS, KID_PREP_CANDS, KID_GEMM_LOGITS, KID_GEMM_LOGITS_P, KID_GEMM_GRAD,
   KID_GEMM_DH, KID_GEMM_DW, KID_FINALIZE, KID_GBUILD, KID_FIX_LABELS, KID_MEAN,
   KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_SUPPORT_DOTS, KID_SUPPORT_LSE,
-  KID_SUPPORT_DH, KID_SUPPORT_DW, KID_SPLIT_SUM, KID_COUNT
+  KID_SUPPORT_DH, KID_SUPPORT_DW, KID_SPLIT_SUM, KID_VP_LABELS, KID_VP_FINALIZE,
+  KID_VP_COMBINE, KID_VP_REDUCE, KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "count_labels", "prep_cands", "gemm_logits_stats", "gemm_logits_stats_store",
     "gemm_logits_grad", "gemm_dH", "gemm_dW", "row_finalize", "gbuild", "fix_labels",
     "mean", "support_out", "bwd_coef", "cast_bf16", "support_dots", "support_lse",
-    "support_grad_dh", "support_dw", "split_sum"};
+    "support_grad_dh", "support_dw", "split_sum", "vp_local_labels", "vp_finalize",
+    "vp_combine", "vp_reduce_rows"};
 
 struct ProfRec {
   int id;
@@ -422,12 +428,23 @@ lmh_status cast_dw(const Plan& P, const float* acc, lmh_bf16* dW, cudaStream_t s
 }
 
 // dH = G W and dW (+)= G^T H_c for one chunk whose G sits in the workspace buffer.
+// With dH_f32 (vocabulary-parallel shards) dH's rows go to it in fp32 instead, unsplit.
 lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H,
                               const lmh_bf16* W, int64_t r0, int rows, int chunk_idx,
                               lmh_bf16* dH, lmh_bf16* dW, float* dW_acc, const Ws& ws,
-                              cudaStream_t st) {
+                              cudaStream_t st, float* dH_f32 = nullptr) {
   const __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
-  if (dH) {
+  if (dH_f32) {
+    CUtensorMap ta, tb;
+    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BK))
+      return LMH_ERR_CUDA;
+    EpiDH::Params ep;
+    ep.rows = rows;
+    ep.d = static_cast<int>(P.d);
+    ep.part = dH_f32 + r0 * P.d;  // split 0 of a one-split partial: the rows themselves
+    LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, ta, rows, P.d, P.V, kOrderDH, &ws.h->err, ep,
+                               st, 1));
+  } else if (dH) {
     CUtensorMap ta, tb, tc;
     if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BK) ||
         !tmap_out(&tc, dH + r0 * P.d, P.d, rows, P.d))
@@ -577,7 +594,7 @@ lmh_status empty_call(const Plan& P, float* mean_out, int32_t* nvalid_out, lmh_b
 // ============================================================================ C ABI
 
 extern "C" size_t lmh_workspace_size(const lmh_shape* shape, int entry) {
-  if (!shape_ok(shape) || entry < LMH_ENTRY_LOSS_FWD || entry > LMH_ENTRY_SUPPORT_KL) return 0;
+  if (!shape_ok(shape) || entry < LMH_ENTRY_LOSS_FWD || entry > LMH_ENTRY_VP_BWD) return 0;
   if ((entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL) &&
       (shape->K < 1 || shape->K > LMH_MAX_K))
     return 0;
@@ -816,6 +833,180 @@ extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_b
                                ws, st));
   }
   return LMH_OK;
+}
+
+// ============================================================================ vocab-parallel
+namespace {
+
+lmh_status vp_args_ok(const lmh_shape* shard, int64_t v0, int64_t V_total) {
+  if (!shape_ok(shard) || v0 < 0 || V_total <= 0 || V_total > 0x7fffffffLL ||
+      v0 + shard->V > V_total)
+    return LMH_ERR_INVALID_ARG;
+  return LMH_OK;
+}
+
+lmh_status vp_local_labels(const Plan& P, const int32_t* labels, int64_t v0, const Ws& ws,
+                           cudaStream_t st) {
+  const int64_t blocks = cdiv(P.N, 256);
+  ProfScope ps(KID_VP_LABELS, st);
+  vp_local_labels_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 256, 0, st>>>(
+      P.N, labels, v0, P.V, ws.at<int32_t>(P.o_lloc));
+  return last_launch();
+}
+
+// Valid rows of the full vocabulary (0 <= y < V_total) into the header; flags y >= V_total.
+lmh_status count_labels_total(const Plan& P, const int32_t* labels, int64_t V_total,
+                              const Ws& ws, cudaStream_t st) {
+  const int64_t blocks = cdiv(P.N, 256);
+  ProfScope ps(KID_COUNT_LABELS, st);
+  count_labels_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 256, 0, st>>>(
+      labels, P.N, static_cast<int>(V_total), ws.h);
+  return last_launch();
+}
+
+}  // namespace
+
+extern "C" lmh_status lmh_vp_partials(const lmh_shape* shard, int64_t v0, int64_t V_total,
+                                      const lmh_bf16* H, const lmh_bf16* W_shard,
+                                      const int32_t* labels, float* records, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  LMH_TRY(vp_args_ok(shard, v0, V_total));
+  const Plan P = make_plan(shard, LMH_ENTRY_VP_PARTIALS, false, false);
+  int dev, sms;
+  LMH_TRY(common_checks(shard, H, W_shard, workspace, workspace_bytes, P.total, &dev, &sms));
+  if (P.N > 0 && (!labels || !records)) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(records)) return LMH_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return LMH_OK;
+  LMH_TRY(vp_local_labels(P, labels, v0, ws, st));
+  Targets tg{};
+  tg.labels = ws.at<int32_t>(P.o_lloc);
+  tg.K = 1;
+  for (int64_t ci = 0; ci < P.nchunks; ++ci) {
+    const int64_t r0 = ci * P.c;
+    const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
+    LMH_TRY((run_stats<kLabel, false>(P, dev, sms, H, W_shard, tg, r0, rows, ws, st)));
+    ProfScope ps(KID_VP_FINALIZE, st);
+    vp_finalize_kernel<<<static_cast<unsigned>(cdiv(rows, 8)), 256, 0, st>>>(
+        rows, r0, static_cast<int>(P.T), v0, ws.at<float>(P.o_pm), ws.at<float>(P.o_ps),
+        ws.at<int32_t>(P.o_pi), ws.at<int32_t>(P.o_lloc), ws.at<float>(P.o_zt), P.temp, ws.h,
+        reinterpret_cast<float4*>(records));
+    LMH_TRY(last_launch());
+  }
+  return LMH_OK;
+}
+
+extern "C" lmh_status lmh_vp_combine(const lmh_shape* shape, int R, const float* records,
+                                     const int32_t* labels, float* loss_rows, float* lse,
+                                     float* logprob, int32_t* argmax, float* loss_mean,
+                                     int32_t* n_valid, const int32_t* n_valid_given,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (!shape_ok(shape) || R < 1) return LMH_ERR_INVALID_ARG;
+  const Plan P = make_plan(shape, LMH_ENTRY_VP_COMBINE, false, false);
+  if (!workspace) return LMH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return LMH_ERR_ALIGNMENT;
+  if (workspace_bytes < P.total) return LMH_ERR_WORKSPACE_TOO_SMALL;
+  if (P.N > 0 && (!records || !labels || !loss_rows || !lse)) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(records)) return LMH_ERR_ALIGNMENT;
+  int dev, sms;
+  LMH_TRY(current_device(&dev, &sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return empty_call(P, loss_mean, n_valid, nullptr, nullptr, st);
+  LMH_TRY(count_labels_total(P, labels, P.V, ws, st));
+  {
+    const int64_t blocks = cdiv(P.N, 256);
+    ProfScope ps(KID_VP_COMBINE, st);
+    vp_combine_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(
+        P.N, R, static_cast<int>(P.V), reinterpret_cast<const float4*>(records), labels, lse,
+        loss_rows, logprob, argmax, ws.h);
+  }
+  LMH_TRY(last_launch());
+  if (loss_mean) {
+    ProfScope ps(KID_MEAN, st);
+    mean_kernel<<<1, 1024, 0, st>>>(loss_rows, P.N, 1, n_valid_given, ws.h, loss_mean);
+    LMH_TRY(last_launch());
+  }
+  if (n_valid &&
+      cudaMemcpyAsync(n_valid, &ws.h->n_valid, 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return LMH_ERR_CUDA;
+  return LMH_OK;
+}
+
+extern "C" lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t v0,
+                                      int64_t V_total, const lmh_bf16* H,
+                                      const lmh_bf16* W_shard, const int32_t* labels,
+                                      const float* lse, const float* grad, float* dH_part,
+                                      lmh_bf16* dW_shard, float* dW_acc_shard, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  LMH_TRY(vp_args_ok(shard, v0, V_total));
+  if (mode != LMH_BWD_CE && mode != LMH_BWD_LOGPROB) return LMH_ERR_INVALID_ARG;
+  lmh_shape sh = *shard;
+  sh.flags &= ~LMH_F_SUPPORT_RENORM;
+  sh.K = 1;
+  const Plan P = make_plan(&sh, LMH_ENTRY_VP_BWD, true, dW_shard && !dW_acc_shard);
+  int dev, sms;
+  LMH_TRY(common_checks(&sh, H, W_shard, workspace, workspace_bytes, P.total, &dev, &sms));
+  if (P.N > 0 && (!labels || !lse)) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(dH_part) || !aligned16(dW_shard) || !aligned16(dW_acc_shard))
+    return LMH_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return empty_call(P, nullptr, nullptr, dW_shard, dW_acc_shard, st);
+  if (!dH_part && !dW_shard && !dW_acc_shard) return LMH_OK;
+  LMH_TRY(count_labels_total(P, labels, V_total, ws, st));
+  LMH_TRY(vp_local_labels(P, labels, v0, ws, st));
+  float* alpha = ws.at<float>(P.o_alpha);
+  float* beta = ws.at<float>(P.o_beta);
+  {
+    // the row coefficients see the global label (valid rows over the full vocabulary); the
+    // one-hot term lands in this shard only if the label is one of its columns
+    ProfScope ps(KID_BWD_COEF, st);
+    bwd_coef_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
+        mode, P.N, 1, static_cast<int>(V_total), labels, grad, nullptr, nullptr, nullptr, P.temp,
+        (sh.flags & LMH_F_MEAN) ? 1 : 0, ws.h, alpha, beta);
+  }
+  LMH_TRY(last_launch());
+  Targets tg{};
+  tg.labels = ws.at<int32_t>(P.o_lloc);
+  tg.K = 1;
+  for (int64_t ci = 0; ci < P.nchunks; ++ci) {
+    const int64_t r0 = ci * P.c;
+    const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
+    CUtensorMap ta, tb, tc;
+    if (!tmap_2d(&ta, H + r0 * P.d, P.d, rows, P.d, BM) ||
+        !tmap_2d(&tb, W_shard, P.d, P.V, P.d, BNH) ||
+        !tmap_out(&tc, ws.at<__nv_bfloat16>(P.o_gbuf), P.Vp, rows, P.Vp))
+      return LMH_ERR_CUDA;
+    EpiGrad<kLabel>::Params ep{rows, r0, static_cast<int>(P.V), P.Vp, tg, lse, alpha, beta,
+                               P.temp};
+    LMH_TRY(launch_gemm<EpiGrad<kLabel>>(dev, sms, ta, tb, tc, rows, P.V, P.d, kOrderLogits,
+                                         &ws.h->err, ep, st));
+    LMH_TRY(run_backward_gemms(P, dev, sms, H, W_shard, r0, rows, static_cast<int>(ci), nullptr,
+                               dW_shard, dW_acc_shard, ws, st, dH_part));
+  }
+  return LMH_OK;
+}
+
+extern "C" lmh_status lmh_vp_reduce_rows(int R, int64_t rows, int64_t d, const float* parts,
+                                         lmh_bf16* out, void* stream) {
+  if (R < 1 || rows < 0 || d <= 0 || (d % 64) != 0) return LMH_ERR_INVALID_ARG;
+  if (rows == 0) return LMH_OK;
+  if (!parts || !out) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(parts) || !aligned16(out)) return LMH_ERR_ALIGNMENT;
+  int dev, sms;
+  LMH_TRY(current_device(&dev, &sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t n4 = rows * d / 4;
+  const int64_t blocks = cdiv(n4, 256);
+  ProfScope ps(KID_VP_REDUCE, st);
+  vp_reduce_rows_kernel<<<static_cast<unsigned>(blocks < 8192 ? blocks : 8192), 256, 0, st>>>(
+      R, n4, reinterpret_cast<const float4*>(parts), reinterpret_cast<__nv_bfloat16*>(out));
+  return last_launch();
 }
 
 extern "C" lmh_status lmh_read_errors(const void* workspace, uint32_t* errors, void* stream) {

@@ -1,0 +1,175 @@
+"""Vocabulary-parallel cross entropy over the ranks of a torch.distributed process group.
+
+Each of the R ranks holds a contiguous row range of W (its shard, from ``shard_plan``) and the
+whole batch (H, labels). The pages run the head at tensor-parallel size 1 only
+(miles-ext-kernels PR #14, lm_head op commit: the validate hook's startup checks). This module
+splits the same definitions over ranks, with one exchange per direction:
+
+forward
+    every rank reduces each row over its shard to a 4-word record (``lmh_vp_partials``); the
+    records are all-gathered in rank order (N x 16 bytes per rank) and every rank combines them
+    in ascending rank order (``lmh_vp_combine``), so all ranks hold the same lse, loss,
+    log-prob, argmax and mean.
+backward
+    every rank forms G on its shard with the combined lse and contracts it
+    (``lmh_vp_loss_bwd``): its shard's dW (no exchange) and an fp32 contribution to dH. The
+    contributions are summed in a fixed order: an all-to-all hands rank j the rows of slice j
+    from every rank, rank j adds them in ascending rank order (``lmh_vp_reduce_rows``), and an
+    all-gather returns the bf16 slices to every rank.
+
+With a fixed R every result is bitwise reproducible: no floating-point value is reduced by a
+collective, only moved. The compute steps run in the library's CUDA kernels through
+``CudaOps``; ``VocabParallelCE`` takes any object with the same four methods, which is how its
+exchange logic is tested on CPU ranks.
+"""
+from __future__ import annotations
+
+from typing import List, Optional, Tuple
+
+import torch
+import torch.distributed as dist
+
+from . import (BWD_CE, ENTRY_VP_BWD, ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN,
+               F_MEAN, lmh_vp_combine, lmh_vp_loss_bwd, lmh_vp_partials, lmh_vp_reduce_rows,
+               make_shape, workspace)
+
+__all__ = ["shard_plan", "row_slices", "CudaOps", "VocabParallelCE"]
+
+
+def shard_plan(V: int, R: int) -> List[Tuple[int, int]]:
+    """The R contiguous vocabulary ranges [v0, v1) that cover [0, V), in rank order. Sizes are
+    equal up to the last range, rounded up to the 256-wide logits tile when a range holds at
+    least one tile; every range is non-empty (so V >= R is required)."""
+    if R < 1 or V < R:
+        raise ValueError(f"cannot split V={V} into {R} non-empty ranges")
+    per = -(-V // R)
+    if per >= 256:
+        tiled = -(-per // 256) * 256
+        if (R - 1) * tiled < V:  # every range keeps at least one word
+            per = tiled
+    return [(min(r * per, V), min((r + 1) * per, V)) for r in range(R)]
+
+
+def row_slices(N: int, R: int) -> List[Tuple[int, int]]:
+    """The rows [a, b) whose dH rank j reduces: N split as evenly as possible, in order."""
+    base, extra = divmod(N, R)
+    out, a = [], 0
+    for j in range(R):
+        b = a + base + (1 if j < extra else 0)
+        out.append((a, b))
+        a = b
+    return out
+
+
+class CudaOps:
+    """The library's vocabulary-parallel entries on CUDA tensors (outputs allocated here)."""
+
+    def partials(self, H, W_shard, labels, v0, V_total, chunk_rows=0, temperature=None):
+        N, d = H.shape
+        shard = make_shape(N, d, W_shard.shape[0], 0, chunk_rows, 0, temperature)
+        ws = workspace(shard, ENTRY_VP_PARTIALS, H.device)
+        rec = torch.empty(N, 4, dtype=torch.float32, device=H.device)
+        lmh_vp_partials(shard, v0, V_total, H, W_shard, labels, rec, workspace=ws)
+        return rec
+
+    def combine(self, records, labels, V_total, d, n_valid_given=None):
+        R, N, _ = records.shape
+        shape = make_shape(N, d, V_total, 0, 0, 0)
+        ws = workspace(shape, ENTRY_VP_COMBINE, records.device)
+        f32, dev = torch.float32, records.device
+        out = dict(loss_rows=torch.empty(N, dtype=f32, device=dev),
+                   lse=torch.empty(N, dtype=f32, device=dev),
+                   logprob=torch.empty(N, dtype=f32, device=dev),
+                   argmax=torch.empty(N, dtype=torch.int32, device=dev),
+                   loss_mean=torch.empty(1, dtype=f32, device=dev),
+                   n_valid=torch.empty(1, dtype=torch.int32, device=dev))
+        lmh_vp_combine(shape, R, records, labels, out["loss_rows"], out["lse"], out["logprob"],
+                       out["argmax"], out["loss_mean"], out["n_valid"], n_valid_given,
+                       workspace=ws)
+        return out
+
+    def backward(self, mode, H, W_shard, labels, lse, grad, v0, V_total, chunk_rows=0,
+                 mean=True, temperature=None, dW_acc=None, want_dW=True):
+        N, d = H.shape
+        Vr = W_shard.shape[0]
+        flags = (F_MEAN if mean else 0) | (F_DW_ACC_GIVEN if dW_acc is not None else 0)
+        shard = make_shape(N, d, Vr, 0, chunk_rows, flags, temperature)
+        ws = workspace(shard, ENTRY_VP_BWD, H.device)
+        dH_part = torch.empty(N, d, dtype=torch.float32, device=H.device)
+        dW = torch.empty(Vr, d, dtype=torch.bfloat16, device=H.device) if want_dW else None
+        lmh_vp_loss_bwd(shard, mode, v0, V_total, H, W_shard, labels, lse, grad, dH_part, dW,
+                        dW_acc, workspace=ws)
+        return dH_part, dW
+
+    def reduce_rows(self, parts):
+        out = torch.empty(parts.shape[1], parts.shape[2], dtype=torch.bfloat16,
+                          device=parts.device)
+        lmh_vp_reduce_rows(parts, out)
+        return out
+
+
+class VocabParallelCE:
+    """Cross entropy (and the per-row log-prob objective) with W split over the ranks of
+    ``group``. Every rank calls ``forward`` and ``backward`` with its own shard
+    ``W[v0:v1]`` (``self.v0``, ``self.v1``) and the same H, labels and options. Without an
+    initialised process group it runs as the only rank (R = 1, no collective)."""
+
+    def __init__(self, V_total: int, group=None, chunk_rows: int = 0, mean: bool = True,
+                 temperature=None, ops=None):
+        self.group = group
+        self.distributed = dist.is_available() and dist.is_initialized()
+        self.R = dist.get_world_size(group) if self.distributed else 1
+        self.rank = dist.get_rank(group) if self.distributed else 0
+        self.V_total = int(V_total)
+        self.v0, self.v1 = shard_plan(self.V_total, self.R)[self.rank]
+        self.chunk_rows = chunk_rows
+        self.mean = mean
+        self.temperature = temperature
+        self.ops = ops if ops is not None else CudaOps()
+
+    def _check_shard(self, W_shard):
+        if W_shard.shape[0] != self.v1 - self.v0:
+            raise ValueError(f"rank {self.rank} holds rows [{self.v0}, {self.v1}) of W, "
+                             f"got {W_shard.shape[0]} rows")
+
+    def forward(self, H, W_shard, labels, n_valid_given=None) -> dict:
+        """loss_rows, lse, logprob, argmax, loss_mean, n_valid: the same on every rank."""
+        self._check_shard(W_shard)
+        N, d = H.shape
+        rec = self.ops.partials(H, W_shard, labels, self.v0, self.V_total, self.chunk_rows,
+                                self.temperature)
+        if self.R == 1:
+            every = rec.reshape(-1)
+        else:
+            every = torch.empty(self.R * N * 4, dtype=rec.dtype, device=rec.device)
+            dist.all_gather_into_tensor(every, rec.reshape(-1).contiguous(), group=self.group)
+        return self.ops.combine(every.view(self.R, N, 4), labels, self.V_total, d, n_valid_given)
+
+    def backward(self, H, W_shard, labels, lse, grad=None, mode: int = BWD_CE,
+                 dW_acc: Optional[torch.Tensor] = None, want_dW: bool = True) -> dict:
+        """dH [N, d] (the same on every rank) and this rank's dW shard [v1 - v0, d]."""
+        self._check_shard(W_shard)
+        N, d = H.shape
+        dH_part, dW = self.ops.backward(mode, H, W_shard, labels, lse, grad, self.v0,
+                                        self.V_total, self.chunk_rows, self.mean,
+                                        self.temperature, dW_acc, want_dW)
+        return dict(dH=self._sum_rows(dH_part), dW=dW)
+
+    def _sum_rows(self, part: torch.Tensor) -> torch.Tensor:
+        """sum over ranks of part [N, d], added in ascending rank order, on every rank."""
+        N, d = part.shape
+        if self.R == 1:
+            return self.ops.reduce_rows(part.view(1, N, d))
+        sl = row_slices(N, self.R)
+        sizes = [b - a for a, b in sl]
+        mine = sizes[self.rank]
+        recv = torch.empty(self.R * mine, d, dtype=part.dtype, device=part.device)
+        dist.all_to_all_single(recv, part.contiguous(), output_split_sizes=[mine] * self.R,
+                               input_split_sizes=sizes, group=self.group)
+        red = self.ops.reduce_rows(recv.view(self.R, mine, d))
+        top = max(sizes)
+        pad = torch.zeros(top, d, dtype=red.dtype, device=red.device)
+        pad[:mine] = red
+        every = torch.empty(self.R * top, d, dtype=red.dtype, device=red.device)
+        dist.all_gather_into_tensor(every, pad, group=self.group)
+        return torch.cat([every[j * top: j * top + sizes[j]] for j in range(self.R)])

@@ -28,7 +28,8 @@ def test_invalid_shapes_size_zero():
     assert ws(10, 64, 0) == 0
     assert ws(10, 64, 100, K=0, entry=L.ENTRY_SUPPORT_KL) == 0
     assert ws(10, 64, 100, K=L.MAX_K + 1, entry=L.ENTRY_SUPPORT_LOGPROB) == 0
-    assert ws(10, 64, 100, entry=7) == 0
+    assert ws(10, 64, 100, entry=8) == 0
+    assert ws(10, 64, 100, entry=-1) == 0
 
 
 def test_chunk_buffer_term():
@@ -75,3 +76,28 @@ def test_host_argument_errors_without_gpu():
     st = lib.lmh_loss_bwd(ctypes.byref(shape), 9, *([None] * 10), 0, None)
     assert st == 1
     assert lib.lmh_read_errors(None, None, None) == 1
+
+
+def test_vocab_parallel_sizes():
+    # combine: the header only; partials: a shard-local label buffer on top of the log-prob
+    # entry's plan; shard backward: the standalone backward's plan without dH split partials
+    assert ws(1000, 64, 5000, entry=L.ENTRY_VP_COMBINE) == 256
+    assert ws(1000, 64, 5000, entry=L.ENTRY_VP_PARTIALS) == \
+        ws(1000, 64, 5000, entry=L.ENTRY_LOGPROB) + 4096
+    N, d, Vr = 2048, 5120, 151936 // 4     # few dH tiles, large V: one-device plan would split
+    assert ws(N, d, Vr, chunk=N, entry=L.ENTRY_VP_BWD) < ws(N, d, Vr, chunk=N, entry=L.ENTRY_LOSS_BWD)
+
+
+def test_vocab_parallel_host_errors_without_gpu():
+    lib = _abi.lib()
+    shard = L.make_shape(4, 64, 100)
+    P = [None] * 5
+    # shard past the vocabulary, negative offset, empty vocabulary: refused before any CUDA call
+    assert lib.lmh_vp_partials(ctypes.byref(shard), 50, 120, *P, 0, None) == 1
+    assert lib.lmh_vp_partials(ctypes.byref(shard), -1, 120, *P, 0, None) == 1
+    assert lib.lmh_vp_loss_bwd(ctypes.byref(shard), 0, 0, 0, *([None] * 9), 0, None) == 1
+    assert lib.lmh_vp_loss_bwd(ctypes.byref(shard), 2, 0, 100, *([None] * 9), 0, None) == 1
+    assert lib.lmh_vp_combine(ctypes.byref(shard), 0, *([None] * 10), 0, None) == 1
+    assert lib.lmh_vp_reduce_rows(2, 4, 96, None, None, None) == 1     # d not a multiple of 64
+    assert lib.lmh_vp_reduce_rows(0, 4, 64, None, None, None) == 1
+    assert lib.lmh_vp_reduce_rows(2, 0, 64, None, None, None) == 0     # nothing to do

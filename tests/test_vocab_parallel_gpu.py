@@ -1,0 +1,158 @@
+"""GPU parity of the vocabulary-parallel entries (through the C ABI) against the fp64 oracle.
+
+One GPU stands in for R ranks: the R shards' steps run one after another and the exchange is a
+concatenation in rank order. No kernel of one shard waits for another shard, so this runs the
+same device code each rank would run, in the same order of additions. (The exchange logic of
+VocabParallelCE itself is covered on CPU ranks over gloo, and on one rank here.)"""
+from __future__ import annotations
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import lm_head_cross_tcgen05_b200 as L
+from lm_head_cross_tcgen05_b200.vocab_parallel import CudaOps, VocabParallelCE, shard_plan
+from tests.gpu_common import O, check_ce_fused, check_grad, check_rows, device_inputs
+from workloads import ragged
+
+pytestmark = pytest.mark.gpu
+
+
+def _wl(N, d, V, ign):
+    return ragged(N, d, V, n_ignored=ign, seed=3000 + N + d + V)
+
+
+def _emulate(x, V, R, chunk=0, tau=None, mode=L.BWD_CE, grad=None, mean=True):
+    H, W, y = x["H"], x["W"], x["labels"]
+    d = H.shape[1]
+    ops = CudaOps()
+    plan = shard_plan(V, R)
+    recs = [ops.partials(H, W[a:b], y, a, V, chunk, tau) for a, b in plan]
+    f = ops.combine(torch.stack(recs), y, V, d)
+    parts, dWs = [], []
+    for a, b in plan:
+        p, w = ops.backward(mode, H, W[a:b], y, f["lse"], grad, a, V, chunk, mean, tau)
+        parts.append(p)
+        dWs.append(w)
+    f["dH"] = ops.reduce_rows(torch.stack(parts))
+    f["dW"] = torch.cat(dWs)
+    torch.cuda.synchronize()
+    return f
+
+
+@pytest.mark.parametrize("N,d,V,ign,R,chunk", [
+    (300, 192, 1000, 5, 2, 0),       # 2 shards of 500 words: ragged vocabulary tiles
+    (129, 64, 4100, 3, 3, 100),      # 3 shards of 1367/1367/1366, two row chunks
+    (200, 512, 70000, 10, 4, 128),   # 4 shards of 17664 (+ 17008), several K blocks
+    (64, 256, 2048, 8, 8, 0),        # the tiny workload on 8 shards of 256
+])
+def test_vocab_parallel_matches_oracle(N, d, V, ign, R, chunk):
+    x, xc = device_inputs(_wl(N, d, V, ign))
+    out = _emulate(x, V, R, chunk)
+    ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
+    check_ce_fused(out, ref)
+    again = _emulate(x, V, R, chunk)
+    for k in ("lse", "loss_rows", "logprob", "argmax", "loss_mean", "dH", "dW"):
+        assert torch.equal(again[k], out[k]), k
+    one = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=chunk, grads=True)
+    assert torch.equal(one["argmax"], out["argmax"])
+    assert (one["lse"] - out["lse"]).abs().max().item() < 1e-4   # fp32 grouping differs
+
+
+@pytest.mark.parametrize("kind", ["scalar", "rows"])
+def test_vocab_parallel_temperature_and_logprob_objective(kind):
+    N, d, V = 150, 128, 3000
+    x, xc = device_inputs(_wl(N, d, V, 6))
+    if kind == "scalar":
+        tau, tau_ref = 0.8, 0.8
+    else:
+        t = torch.linspace(0.5, 1.5, N, dtype=torch.float32)
+        tau, tau_ref = t.cuda(), t.numpy()
+    g = torch.linspace(-1.0, 1.0, N, dtype=torch.float32)
+    out = _emulate(x, V, 3, 64, tau, mode=L.BWD_LOGPROB, grad=g.cuda())
+    lp = O.logprob_forward(xc["H"], xc["W"], xc["labels"], tau=tau_ref)
+    check_rows(out["logprob"], lp["logprob"], what="logprob")
+    check_rows(out["lse"], lp["lse"], what="lse")
+    ref = O.backward(O.BWD_LOGPROB, xc["H"], xc["W"], xc["labels"], g.numpy(), tau=tau_ref)
+    check_grad(out["dH"], ref["dH"], "dH")
+    check_grad(out["dW"], ref["dW"], "dW")
+
+
+def test_vocab_parallel_label_errors_and_ignored_rows():
+    N, d, V = 96, 64, 1200
+    x, xc = device_inputs(_wl(N, d, V, 0))
+    y = x["labels"].clone()
+    y[:10] = -100
+    y[10] = -7
+    y[11] = V + 5                      # out of range: flagged, row ignored
+    xs = dict(x, labels=y)
+    ops = CudaOps()
+    plan = shard_plan(V, 2)
+    recs = torch.stack([ops.partials(x["H"], x["W"][a:b], y, a, V) for a, b in plan])
+    shape = L.make_shape(N, d, V)
+    ws = L.workspace(shape, L.ENTRY_VP_COMBINE, "cuda")
+    f32 = torch.float32
+    loss, lse = torch.empty(N, dtype=f32, device="cuda"), torch.empty(N, dtype=f32, device="cuda")
+    nv = torch.empty(1, dtype=torch.int32, device="cuda")
+    L.lmh_vp_combine(shape, 2, recs, y, loss, lse, n_valid=nv, workspace=ws)
+    assert L.lmh_read_errors(ws) & L.DEVERR_LABEL_RANGE
+    assert int(nv.item()) == N - 12
+    assert torch.all(loss[:12] == 0)
+    out = _emulate(xs, V, 2)
+    ref = O.ce_fused(xc["H"], xc["W"], y.cpu())
+    check_rows(out["loss_rows"], ref["loss_rows"], what="loss_rows")
+    check_grad(out["dH"], ref["dH"], "dH")
+    check_grad(out["dW"], ref["dW"], "dW")
+
+
+def test_vocab_parallel_caller_accumulator_and_host_rejections():
+    N, d, V = 80, 64, 900
+    x, xc = device_inputs(_wl(N, d, V, 2))
+    plan = shard_plan(V, 2)
+    ops = CudaOps()
+    f = ops.combine(torch.stack([ops.partials(x["H"], x["W"][a:b], x["labels"], a, V)
+                                 for a, b in plan]), x["labels"], V, d)
+    accs = []
+    for a, b in plan:
+        acc = torch.zeros(b - a, d, dtype=torch.float32, device="cuda")
+        _, dw = ops.backward(L.BWD_CE, x["H"], x["W"][a:b], x["labels"], f["lse"], None, a, V,
+                             32, True, None, acc)
+        assert torch.equal(dw, acc.to(torch.bfloat16))
+        accs.append(acc)
+    ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
+    check_grad(torch.cat(accs), ref["dW"], "dW_acc shards")
+    # a shard that runs past V_total, and a negative offset, are refused before any launch
+    shard = L.make_shape(N, d, plan[1][1] - plan[1][0])
+    ws = L.workspace(shard, L.ENTRY_VP_PARTIALS, "cuda")
+    rec = torch.empty(N, 4, dtype=torch.float32, device="cuda")
+    for v0 in (V - 10, -1):
+        with pytest.raises(L.LmhError):
+            L.lmh_vp_partials(shard, v0, V, x["H"], x["W"][plan[1][0]:], x["labels"], rec,
+                              workspace=ws)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_vocab_parallel_class_on_one_rank():
+    # the class's collectives over one NCCL rank: the same results as the one-device entries
+    import torch.distributed as dist
+    N, d, V = 130, 128, 2100
+    x, xc = device_inputs(_wl(N, d, V, 4))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        vp = VocabParallelCE(V)
+        f = vp.forward(x["H"], x["W"], x["labels"])
+        b = vp.backward(x["H"], x["W"], x["labels"], f["lse"])
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
+    check_ce_fused(dict(f, dH=b["dH"], dW=b["dW"]), ref)
