@@ -77,6 +77,7 @@ typedef enum lmh_status {
 #define LMH_F_FUSED_BWD 0x2u    /* sizing only: lmh_loss_fwd will also produce dH/dW   */
 #define LMH_F_DW_ACC_GIVEN 0x4u /* sizing only: the caller passes an fp32 dW_acc       */
 #define LMH_F_SUPPORT_RENORM 0x8u /* support entries: renormalise over the candidates   */
+#define LMH_F_GRAD_SCALAR 0x10u   /* backward: grad is one float shared by every term    */
 
 /* entries, for lmh_workspace_size */
 #define LMH_ENTRY_LOSS_FWD 0
@@ -170,7 +171,9 @@ LMH_API lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, const
  * Candidate ids < 0 are padding and are skipped. lse [N] is the forward's output.
  * grad may be NULL: every row term then has the weight 1, or 1 / count with LMH_F_MEAN in
  * shape->flags (count: the valid rows of the labels for CE / LOGPROB, N for the support
- * objectives), taken on the device without a host synchronisation.
+ * objectives), taken on the device without a host synchronisation. With LMH_F_GRAD_SCALAR,
+ * grad points to one float g (device memory, e.g. the upstream gradient of a summed or
+ * averaged loss) and every term has the weight g, or g / count with LMH_F_MEAN.
  * dH, dW, dW_acc: as in lmh_loss_fwd (nullable; dW_acc accumulates in chunk order).
  */
 LMH_API lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,

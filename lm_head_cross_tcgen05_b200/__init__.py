@@ -19,7 +19,7 @@ import torch
 from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEVERR_LABEL_RANGE,
                    DEVERR_NONFINITE, DEVERR_TEMPERATURE, DEVERR_TIMEOUT, ENTRY_LOGPROB, ENTRY_LOSS_BWD,
                    ENTRY_LOSS_FWD, ENTRY_SUPPORT_KL, ENTRY_SUPPORT_LOGPROB, ENTRY_VP_BWD,
-                   ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN,
+                   ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN, F_GRAD_SCALAR,
                    F_FUSED_BWD, F_MEAN, F_SUPPORT_RENORM, IGNORE_INDEX, MAX_K, STATUS_NAMES, lib, lmh_shape)
 
 __all__ = [
@@ -31,7 +31,7 @@ __all__ = [
     "ENTRY_LOGPROB", "ENTRY_SUPPORT_LOGPROB", "ENTRY_SUPPORT_KL", "DEVERR_LABEL_RANGE",
     "DEVERR_TIMEOUT", "DEVERR_NONFINITE", "DEVERR_TEMPERATURE", "MAX_K",
     "lmh_vp_partials", "lmh_vp_combine", "lmh_vp_loss_bwd", "lmh_vp_reduce_rows",
-    "ENTRY_VP_PARTIALS", "ENTRY_VP_COMBINE", "ENTRY_VP_BWD",
+    "ENTRY_VP_PARTIALS", "ENTRY_VP_COMBINE", "ENTRY_VP_BWD", "F_GRAD_SCALAR",
 ]
 
 lib()  # load now: a missing library is an import error, never a silent fallback
@@ -226,15 +226,17 @@ def loss_fwd(H, W, labels, *, chunk_rows: int = 0, mean: bool = True, grads: boo
 
 def loss_bwd(mode: int, H, W, targets, lse, grad, ref_logp=None, *, chunk_rows: int = 0,
              want_dH: bool = True, want_dW: bool = True, dW_acc=None, temperature=None,
-             mean: bool = False, renorm: bool = False, ws=None, stream=None) -> dict:
+             mean: bool = False, renorm: bool = False, scalar_grad: bool = False, ws=None,
+             stream=None) -> dict:
     """Backward of one objective (LMH_BWD_*). grad=None: unit row weights, or 1 / count with
-    mean=True, taken on the device."""
+    mean=True, taken on the device. scalar_grad=True: grad is a one-element device tensor g
+    that multiplies every term's weight (LMH_F_GRAD_SCALAR)."""
     N, d = H.shape
     V = W.shape[0]
     K = targets.shape[1] if targets.dim() == 2 else 1
     dev = H.device
     flags = ((F_DW_ACC_GIVEN if dW_acc is not None else 0) | (F_MEAN if mean else 0)
-             | (F_SUPPORT_RENORM if renorm else 0))
+             | (F_SUPPORT_RENORM if renorm else 0) | (F_GRAD_SCALAR if scalar_grad else 0))
     shape = make_shape(N, d, V, K, chunk_rows, flags, temperature)
     out = dict(dH=torch.empty(N, d, dtype=_bf, device=dev) if want_dH else None,
                dW=torch.empty(V, d, dtype=_bf, device=dev) if want_dW else None)

@@ -19,7 +19,7 @@ STATUS_NAMES = {0: "LMH_OK", 1: "LMH_ERR_INVALID_ARG", 2: "LMH_ERR_UNSUPPORTED_D
 
 IGNORE_INDEX = -100
 DEVERR_LABEL_RANGE, DEVERR_TIMEOUT, DEVERR_NONFINITE, DEVERR_TEMPERATURE = 0x1, 0x2, 0x4, 0x8
-F_MEAN, F_FUSED_BWD, F_DW_ACC_GIVEN, F_SUPPORT_RENORM = 0x1, 0x2, 0x4, 0x8
+F_MEAN, F_FUSED_BWD, F_DW_ACC_GIVEN, F_SUPPORT_RENORM, F_GRAD_SCALAR = 0x1, 0x2, 0x4, 0x8, 0x10
 ENTRY_LOSS_FWD, ENTRY_LOSS_BWD, ENTRY_LOGPROB, ENTRY_SUPPORT_LOGPROB, ENTRY_SUPPORT_KL = range(5)
 ENTRY_VP_PARTIALS, ENTRY_VP_COMBINE, ENTRY_VP_BWD = 5, 6, 7
 BWD_CE, BWD_LOGPROB, BWD_SUPPORT_LOGPROB, BWD_SUPPORT_KL = range(4)

@@ -782,6 +782,7 @@ extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_b
   LMH_TRY(common_checks(shape, H, W, workspace, workspace_bytes, P.total, &dev, &sms));
   if (P.N > 0 && (!targets || !lse)) return LMH_ERR_INVALID_ARG;
   if (mode == LMH_BWD_SUPPORT_KL && P.N > 0 && !ref_logp) return LMH_ERR_INVALID_ARG;
+  if ((shape->flags & LMH_F_GRAD_SCALAR) && !grad) return LMH_ERR_INVALID_ARG;
   if (!aligned16(dH) || !aligned16(dW) || !aligned16(dW_acc)) return LMH_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
@@ -807,7 +808,8 @@ extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_b
       mode, P.N, cands ? static_cast<int>(P.K) : 1, static_cast<int>(P.V), targets, grad,
       ref_logp, cands ? ws.at<int32_t>(P.o_rank) : nullptr,
       cands ? ws.at<int32_t>(P.o_nuniq) : nullptr, P.temp,
-      (shape->flags & LMH_F_MEAN) ? 1 : 0, ws.h, alpha, beta);
+      (shape->flags & LMH_F_MEAN) ? 1 : 0, (shape->flags & LMH_F_GRAD_SCALAR) ? 1 : 0, ws.h,
+      alpha, beta);
   }
   LMH_TRY(last_launch());
   if (P.renorm) return sparse_backward(P, H, W, lse, dH, dW, dW_acc, ws, st);
@@ -951,6 +953,7 @@ extern "C" lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t 
   int dev, sms;
   LMH_TRY(common_checks(&sh, H, W_shard, workspace, workspace_bytes, P.total, &dev, &sms));
   if (P.N > 0 && (!labels || !lse)) return LMH_ERR_INVALID_ARG;
+  if ((sh.flags & LMH_F_GRAD_SCALAR) && !grad) return LMH_ERR_INVALID_ARG;
   if (!aligned16(dH_part) || !aligned16(dW_shard) || !aligned16(dW_acc_shard))
     return LMH_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -968,7 +971,8 @@ extern "C" lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t 
     ProfScope ps(KID_BWD_COEF, st);
     bwd_coef_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
         mode, P.N, 1, static_cast<int>(V_total), labels, grad, nullptr, nullptr, nullptr, P.temp,
-        (sh.flags & LMH_F_MEAN) ? 1 : 0, ws.h, alpha, beta);
+        (sh.flags & LMH_F_MEAN) ? 1 : 0, (sh.flags & LMH_F_GRAD_SCALAR) ? 1 : 0, ws.h, alpha,
+        beta);
   }
   LMH_TRY(last_launch());
   Targets tg{};

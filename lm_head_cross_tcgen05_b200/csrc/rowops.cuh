@@ -296,23 +296,28 @@ __global__ void support_out_kernel(long long N, int K, const int32_t* __restrict
 // alpha_i and beta (per label, or per sorted candidate id summed over repeated slots) of
 // G = alpha P - sum beta e_t for the four objectives; one warp per row.
 // Without `grad` every row term has the weight 1, or 1 / count with `mean` (count: the valid
-// rows of the labels for CE / LOGPROB, N for the support objectives).
+// rows of the labels for CE / LOGPROB, N for the support objectives); with `scalar` grad[0]
+// multiplies that weight instead of grad holding one weight per term.
 __global__ void bwd_coef_kernel(int mode, long long N, int K, int V,
                                 const int32_t* __restrict__ targets,
                                 const float* __restrict__ grad, const float* __restrict__ ref,
                                 const int32_t* __restrict__ rank,
                                 const int32_t* __restrict__ nuniq, Temperature temp, int mean,
-                                WsHeader* h, float* __restrict__ alpha,
+                                int scalar, WsHeader* h, float* __restrict__ alpha,
                                 float* __restrict__ beta) {
   const int lane = threadIdx.x & 31;
   const long long i = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5);
   if (i >= N) return;
   const float it = inv_temperature(temp, i);  // chain-rule factor of the tempered logits
   if (lane == 0 && temp.rows && !temperature_ok(temp.rows[i])) atomicOr(&h->err, kErrTemperature);
-  float unit = 1.f;  // weight of a row term when no grad is given
+  float unit = 1.f;  // weight of a row term when no per-term grad is given
   if (mean) {
     const long long cnt = (mode <= 1) ? h->n_valid : N;
     unit = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
+  }
+  if (scalar) {
+    unit *= grad[0];
+    grad = nullptr;
   }
   if (mode <= 1) {  // CE / LOGPROB over labels
     if (lane == 0) {
