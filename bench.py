@@ -77,8 +77,8 @@ def source_hash() -> str:
 ENTRY_TEXT = {"fused_ce": "fused CE forward+backward",
               "ce_separate": "CE forward, then backward with recomputed logits",
               "support_kl": "support-set KL forward (K candidates), then its backward",
-              "vocab_parallel": "vocabulary-parallel CE forward, then backward with recomputed "
-                                "logits (W split over the GPUs)"}
+              "vocab_parallel": "vocabulary-parallel fused CE forward+backward (W split over "
+                                "the GPUs)"}
 
 
 def workload_config(wl, chunk_rows, n_gpus, entry="fused_ce"):
@@ -330,8 +330,7 @@ def main():
         W_shard = W[vp.v0:vp.v1].contiguous()
 
         def step(b=batch):
-            f = vp.forward(b["H"], W_shard, b["labels"])
-            vp.backward(b["H"], W_shard, b["labels"], f["lse"])
+            f = vp.forward_backward(b["H"], W_shard, b["labels"])   # fused: 3 GEMMs per shard
             out["loss_mean"].copy_(f["loss_mean"])
             out["n_valid"].copy_(f["n_valid"])
     else:

@@ -251,6 +251,9 @@ LMH_API lmh_status lmh_support_kl(const lmh_shape* shape, const lmh_bf16* H, con
  *   largest logit; arg_r (int32 bits) = the smallest global id attaining it; zy_r (fp32) =
  *   the label's logit if 0 <= y_i - v0 < V_r, else -inf }. Requires 0 <= v0 and
  *   v0 + V_r <= V_total. Workspace: lmh_workspace_size(shard, LMH_ENTRY_VP_PARTIALS).
+ *   With LMH_F_FUSED_BWD in shard->flags the call also keeps the shard's softmax numerators
+ *   p~ = exp(z - m_t) and tile maxima in the workspace for lmh_vp_fused_bwd (all rows in one
+ *   chunk: chunk_rows >= N, else LMH_ERR_INVALID_ARG; size the workspace with the flag).
  */
 LMH_API lmh_status lmh_vp_partials(const lmh_shape* shard, int64_t v0, int64_t V_total,
                                    const lmh_bf16* H, const lmh_bf16* W_shard,
@@ -283,6 +286,22 @@ LMH_API lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t v0,
                                    const int32_t* labels, const float* lse, const float* grad,
                                    float* dH_part, lmh_bf16* dW_shard, float* dW_acc_shard,
                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * lmh_vp_fused_bwd: the shard's backward of the summed loss (or of the mean over the valid
+ * rows of all ranks with LMH_F_MEAN) from the p~ that lmh_vp_partials kept, as lmh_loss_fwd's
+ * fused path does on one device: G = alpha_i exp(m_t - lse_i) p~ minus alpha_i at the label,
+ * with the combined lse. Three GEMMs per step instead of the four of partials + lmh_vp_loss_bwd.
+ * Call it with the same shard, flags and workspace as that lmh_vp_partials call, after it and
+ * before the workspace is reused. n_valid_given (nullable) as in lmh_loss_fwd. Outputs as
+ * lmh_vp_loss_bwd.
+ */
+LMH_API lmh_status lmh_vp_fused_bwd(const lmh_shape* shard, int64_t v0, int64_t V_total,
+                                    const lmh_bf16* H, const lmh_bf16* W_shard,
+                                    const int32_t* labels, const float* lse,
+                                    const int32_t* n_valid_given, float* dH_part,
+                                    lmh_bf16* dW_shard, float* dW_acc_shard, void* workspace,
+                                    size_t workspace_bytes, void* stream);
 
 /*
  * lmh_vp_reduce_rows: out[j] = bf16(sum_{r = 0..R-1} parts[r, j]) over rows x d elements, the

@@ -30,7 +30,8 @@ __all__ = [
     "F_MEAN", "F_FUSED_BWD", "F_DW_ACC_GIVEN", "F_SUPPORT_RENORM", "ENTRY_LOSS_FWD", "ENTRY_LOSS_BWD",
     "ENTRY_LOGPROB", "ENTRY_SUPPORT_LOGPROB", "ENTRY_SUPPORT_KL", "DEVERR_LABEL_RANGE",
     "DEVERR_TIMEOUT", "DEVERR_NONFINITE", "DEVERR_TEMPERATURE", "MAX_K",
-    "lmh_vp_partials", "lmh_vp_combine", "lmh_vp_loss_bwd", "lmh_vp_reduce_rows",
+    "lmh_vp_partials", "lmh_vp_combine", "lmh_vp_loss_bwd", "lmh_vp_fused_bwd",
+    "lmh_vp_reduce_rows",
     "ENTRY_VP_PARTIALS", "ENTRY_VP_COMBINE", "ENTRY_VP_BWD", "F_GRAD_SCALAR",
 ]
 
@@ -170,6 +171,18 @@ def lmh_vp_loss_bwd(shard, mode, v0, V_total, H, W_shard, labels, lse, grad=None
                                _p(dW_shard, _bf, "dW_shard"), _p(dW_acc_shard, _f32, "dW_acc_shard"),
                                _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
     _ok("lmh_vp_loss_bwd", st)
+
+
+def lmh_vp_fused_bwd(shard, v0, V_total, H, W_shard, labels, lse, n_valid_given=None,
+                     dH_part=None, dW_shard=None, dW_acc_shard=None, *, workspace,
+                     stream=None) -> None:
+    st = lib().lmh_vp_fused_bwd(ctypes.byref(shard), int(v0), int(V_total), _p(H, _bf, "H"),
+                                _p(W_shard, _bf, "W_shard"), _p(labels, _i32, "labels"),
+                                _p(lse, _f32, "lse"), _p(n_valid_given, _i32, "n_valid_given"),
+                                _p(dH_part, _f32, "dH_part"), _p(dW_shard, _bf, "dW_shard"),
+                                _p(dW_acc_shard, _f32, "dW_acc_shard"),
+                                _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
+    _ok("lmh_vp_fused_bwd", st)
 
 
 def lmh_vp_reduce_rows(parts, out, stream=None) -> None:

@@ -45,6 +45,8 @@ _SIGS = {
     "lmh_vp_combine": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 10 + [c_size_t, _P]),
     "lmh_vp_loss_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int, c_int64, c_int64] + [_P] * 9
                         + [c_size_t, _P]),
+    "lmh_vp_fused_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int64, c_int64] + [_P] * 9
+                         + [c_size_t, _P]),
     "lmh_vp_reduce_rows": (c_int, [c_int, c_int64, c_int64, _P, _P, _P]),
     "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),
     "lmh_logprob_noalloc": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6),

@@ -88,7 +88,9 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
              entry == LMH_ENTRY_LOSS_BWD);
   p.K = p.cands ? (s->K > 0 ? s->K : 1) : 1;
   p.renorm = p.cands && (s->flags & LMH_F_SUPPORT_RENORM);
-  p.gbuf = !p.renorm && (bwd || (entry == LMH_ENTRY_LOSS_FWD && fused));
+  const bool fwd_fused =
+      fused && (entry == LMH_ENTRY_LOSS_FWD || entry == LMH_ENTRY_VP_PARTIALS);
+  p.gbuf = !p.renorm && (bwd || fwd_fused);
   p.acc = p.gbuf && dw_without_acc && p.nchunks > 1;
   const bool stats = !bwd && entry != LMH_ENTRY_VP_COMBINE;
   const bool partials = stats && !p.renorm;
@@ -112,7 +114,8 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   p.o_lloc = (vp_bwd || entry == LMH_ENTRY_VP_PARTIALS) ? take(N * 4) : 0;
   p.o_gbuf = p.gbuf ? take(static_cast<size_t>(p.c) * p.Vp * 2) : 0;
   p.o_acc = p.acc ? take(static_cast<size_t>(p.V) * p.d * 4) : 0;
-  if (p.gbuf && p.nchunks > 0 && !vp_bwd) {  // the largest split-K partial of any chunk
+  const bool vp = vp_bwd || entry == LMH_ENTRY_VP_PARTIALS;  // dH leaves in fp32, unsplit
+  if (p.gbuf && p.nchunks > 0 && !vp) {  // the largest split-K partial of any chunk
     const int64_t last = p.N - (p.nchunks - 1) * p.c;
     const int64_t a = dh_splits(p.c, p.d, p.V) > 1 ? dh_splits(p.c, p.d, p.V) * p.c : 0;
     const int64_t b = dh_splits(last, p.d, p.V) > 1 ? dh_splits(last, p.d, p.V) * last : 0;
@@ -168,14 +171,14 @@ enum KernelId {
   KID_GEMM_DH, KID_GEMM_DW, KID_FINALIZE, KID_GBUILD, KID_FIX_LABELS, KID_MEAN,
   KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_SUPPORT_DOTS, KID_SUPPORT_LSE,
   KID_SUPPORT_DH, KID_SUPPORT_DW, KID_SPLIT_SUM, KID_VP_LABELS, KID_VP_FINALIZE,
-  KID_VP_COMBINE, KID_VP_REDUCE, KID_COUNT
+  KID_VP_COMBINE, KID_VP_REDUCE, KID_VP_SCALE, KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "count_labels", "prep_cands", "gemm_logits_stats", "gemm_logits_stats_store",
     "gemm_logits_grad", "gemm_dH", "gemm_dW", "row_finalize", "gbuild", "fix_labels",
     "mean", "support_out", "bwd_coef", "cast_bf16", "support_dots", "support_lse",
     "support_grad_dh", "support_dw", "split_sum", "vp_local_labels", "vp_finalize",
-    "vp_combine", "vp_reduce_rows"};
+    "vp_combine", "vp_reduce_rows", "vp_scale"};
 
 struct ProfRec {
   int id;
@@ -598,7 +601,8 @@ extern "C" size_t lmh_workspace_size(const lmh_shape* shape, int entry) {
   if ((entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL) &&
       (shape->K < 1 || shape->K > LMH_MAX_K))
     return 0;
-  const bool fused = entry == LMH_ENTRY_LOSS_FWD && (shape->flags & LMH_F_FUSED_BWD);
+  const bool fused = (entry == LMH_ENTRY_LOSS_FWD || entry == LMH_ENTRY_VP_PARTIALS) &&
+                     (shape->flags & LMH_F_FUSED_BWD);
   const bool want_acc = !(shape->flags & LMH_F_DW_ACC_GIVEN);
   return make_plan(shape, entry, fused, want_acc).total;
 }
@@ -873,10 +877,12 @@ extern "C" lmh_status lmh_vp_partials(const lmh_shape* shard, int64_t v0, int64_
                                       const int32_t* labels, float* records, void* workspace,
                                       size_t workspace_bytes, void* stream) {
   LMH_TRY(vp_args_ok(shard, v0, V_total));
-  const Plan P = make_plan(shard, LMH_ENTRY_VP_PARTIALS, false, false);
+  const bool fused = (shard->flags & LMH_F_FUSED_BWD) != 0;
+  const Plan P = make_plan(shard, LMH_ENTRY_VP_PARTIALS, fused, false);
   int dev, sms;
   LMH_TRY(common_checks(shard, H, W_shard, workspace, workspace_bytes, P.total, &dev, &sms));
   if (P.N > 0 && (!labels || !records)) return LMH_ERR_INVALID_ARG;
+  if (fused && P.nchunks > 1) return LMH_ERR_INVALID_ARG;  // p~ of every row is kept
   if (!aligned16(records)) return LMH_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
@@ -889,7 +895,11 @@ extern "C" lmh_status lmh_vp_partials(const lmh_shape* shard, int64_t v0, int64_
   for (int64_t ci = 0; ci < P.nchunks; ++ci) {
     const int64_t r0 = ci * P.c;
     const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
-    LMH_TRY((run_stats<kLabel, false>(P, dev, sms, H, W_shard, tg, r0, rows, ws, st)));
+    if (fused) {
+      LMH_TRY((run_stats<kLabel, true>(P, dev, sms, H, W_shard, tg, r0, rows, ws, st)));
+    } else {
+      LMH_TRY((run_stats<kLabel, false>(P, dev, sms, H, W_shard, tg, r0, rows, ws, st)));
+    }
     ProfScope ps(KID_VP_FINALIZE, st);
     vp_finalize_kernel<<<static_cast<unsigned>(cdiv(rows, 8)), 256, 0, st>>>(
         rows, r0, static_cast<int>(P.T), v0, ws.at<float>(P.o_pm), ws.at<float>(P.o_ps),
@@ -994,6 +1004,61 @@ extern "C" lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t 
                                dW_shard, dW_acc_shard, ws, st, dH_part));
   }
   return LMH_OK;
+}
+
+extern "C" lmh_status lmh_vp_fused_bwd(const lmh_shape* shard, int64_t v0, int64_t V_total,
+                                       const lmh_bf16* H, const lmh_bf16* W_shard,
+                                       const int32_t* labels, const float* lse,
+                                       const int32_t* n_valid_given, float* dH_part,
+                                       lmh_bf16* dW_shard, float* dW_acc_shard, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  LMH_TRY(vp_args_ok(shard, v0, V_total));
+  if (!(shard->flags & LMH_F_FUSED_BWD)) return LMH_ERR_INVALID_ARG;
+  const Plan P = make_plan(shard, LMH_ENTRY_VP_PARTIALS, true, false);
+  int dev, sms;
+  LMH_TRY(common_checks(shard, H, W_shard, workspace, workspace_bytes, P.total, &dev, &sms));
+  if (P.nchunks > 1) return LMH_ERR_INVALID_ARG;
+  if (P.N > 0 && (!labels || !lse)) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(dH_part) || !aligned16(dW_shard) || !aligned16(dW_acc_shard))
+    return LMH_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return empty_call(P, nullptr, nullptr, dW_shard, dW_acc_shard, st);
+  if (!dH_part && !dW_shard && !dW_acc_shard) return LMH_OK;
+  const int mean = (shard->flags & LMH_F_MEAN) ? 1 : 0;
+  const int rows = static_cast<int>(P.N);
+  LMH_TRY(count_labels_total(P, labels, V_total, ws, st));
+  LMH_TRY(vp_local_labels(P, labels, v0, ws, st));
+  {
+    // s_t of each (row, tile) becomes alpha_i exp(m_t - lse_i) with the combined lse
+    ProfScope ps(KID_VP_SCALE, st);
+    vp_scale_kernel<<<static_cast<unsigned>(cdiv(rows, 8)), 256, 0, st>>>(
+        rows, static_cast<int>(P.T), static_cast<int>(V_total), labels, lse,
+        ws.at<float>(P.o_pm), mean, n_valid_given, ws.h, P.temp, ws.at<float>(P.o_ps));
+  }
+  LMH_TRY(last_launch());
+  __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
+  {
+    const int64_t nv = P.Vp / 8;
+    const int64_t bx = cdiv(nv, kGbuildThreads * kGbuildVec);
+    dim3 grid(static_cast<unsigned>(bx < 64 ? bx : 64),
+              static_cast<unsigned>(rows < 65535 ? rows : 65535));
+    ProfScope ps(KID_GBUILD, st);
+    gbuild_kernel<<<grid, kGbuildThreads, 0, st>>>(rows, P.Vp, static_cast<int>(P.T),
+                                                   ws.at<float>(P.o_ps), G);
+  }
+  LMH_TRY(last_launch());
+  {
+    // the one-hot term, in the shard that holds the label's column
+    ProfScope ps(KID_FIX_LABELS, st);
+    fix_labels_kernel<<<static_cast<unsigned>(cdiv(rows, 256)), 256, 0, st>>>(
+        rows, 0, static_cast<int>(P.V), P.Vp, ws.at<int32_t>(P.o_lloc), ws.at<float>(P.o_zt),
+        lse, mean, n_valid_given, ws.h, P.temp, G);
+  }
+  LMH_TRY(last_launch());
+  return run_backward_gemms(P, dev, sms, H, W_shard, 0, rows, 0, nullptr, dW_shard,
+                            dW_acc_shard, ws, st, dH_part);
 }
 
 extern "C" lmh_status lmh_vp_reduce_rows(int R, int64_t rows, int64_t d, const float* parts,

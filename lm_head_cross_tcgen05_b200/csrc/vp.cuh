@@ -104,6 +104,25 @@ __global__ void vp_combine_kernel(long long N, int R, int V, const float4* __res
   }
 }
 
+// Fused backward of a shard, one warp per row: the tile factors that turn the stored
+// p~ = exp(z - m_t) into the softmax gradient with the combined lse,
+//   s_t = alpha_i exp(m_t - lse_i),  alpha_i = weight of row i / tau_i,
+// the weight being 1 (sum) or 1 / count (mean) for rows with 0 <= y_i < V (all ranks' count).
+__global__ void vp_scale_kernel(int rows, int T, int V, const int32_t* __restrict__ labels,
+                                const float* __restrict__ lse, const float* __restrict__ part_m,
+                                int mean, const int32_t* n_given, const WsHeader* h,
+                                Temperature temp, float* __restrict__ part_s) {
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int y = labels[row];
+  const float a = row_weight(y >= 0 && y < V, mean, n_given, h) * inv_temperature(temp, row);
+  const float loff = -lse[row] * kLog2e;
+  const float* pm = part_m + static_cast<long long>(row) * T;
+  float* ps = part_s + static_cast<long long>(row) * T;
+  for (int t = lane; t < T; t += 32) ps[t] = a * fast_exp2(fmaf(pm[t], kLog2e, loff));
+}
+
 // out[j] = bf16(sum_{r = 0..R-1} parts[r][j]) over n elements (a multiple of 4), the ranks'
 // fp32 contributions added in ascending rank order.
 __global__ void vp_reduce_rows_kernel(int R, long long n4, const float4* __restrict__ parts,

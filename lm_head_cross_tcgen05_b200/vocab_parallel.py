@@ -11,8 +11,10 @@ forward
     in ascending rank order (``lmh_vp_combine``), so all ranks hold the same lse, loss,
     log-prob, argmax and mean.
 backward
-    every rank forms G on its shard with the combined lse and contracts it
-    (``lmh_vp_loss_bwd``): its shard's dW (no exchange) and an fp32 contribution to dH. The
+    every rank forms G on its shard with the combined lse and contracts it: from recomputed
+    logits (``lmh_vp_loss_bwd``), or, in ``forward_backward``, from the softmax numerators its
+    forward kept (``lmh_vp_fused_bwd``, one GEMM fewer). This gives the shard's dW (no
+    exchange) and an fp32 contribution to dH. The
     contributions are summed in a fixed order: an all-to-all hands rank j the rows of slice j
     from every rank, rank j adds them in ascending rank order (``lmh_vp_reduce_rows``), and an
     all-gather returns the bf16 slices to every rank.
@@ -30,8 +32,8 @@ import torch
 import torch.distributed as dist
 
 from . import (BWD_CE, ENTRY_VP_BWD, ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN,
-               F_MEAN, lmh_vp_combine, lmh_vp_loss_bwd, lmh_vp_partials, lmh_vp_reduce_rows,
-               make_shape, workspace)
+               F_FUSED_BWD, F_MEAN, lmh_vp_combine, lmh_vp_fused_bwd, lmh_vp_loss_bwd,
+               lmh_vp_partials, lmh_vp_reduce_rows, make_shape, workspace)
 
 __all__ = ["shard_plan", "row_slices", "CudaOps", "VocabParallelCE"]
 
@@ -71,6 +73,27 @@ class CudaOps:
         rec = torch.empty(N, 4, dtype=torch.float32, device=H.device)
         lmh_vp_partials(shard, v0, V_total, H, W_shard, labels, rec, workspace=ws)
         return rec
+
+    def partials_fused(self, H, W_shard, labels, v0, V_total, mean=True, temperature=None):
+        """partials() that also keeps p~ for fused_backward; all rows form one chunk."""
+        N, d = H.shape
+        flags = F_FUSED_BWD | (F_MEAN if mean else 0)
+        shard = make_shape(N, d, W_shard.shape[0], 0, max(N, 1), flags, temperature)
+        ws = workspace(shard, ENTRY_VP_PARTIALS, H.device)
+        rec = torch.empty(N, 4, dtype=torch.float32, device=H.device)
+        lmh_vp_partials(shard, v0, V_total, H, W_shard, labels, rec, workspace=ws)
+        return rec, (shard, ws)
+
+    def fused_backward(self, state, H, W_shard, labels, lse, v0, V_total, n_valid_given=None,
+                       dW_acc=None, want_dW=True):
+        shard, ws = state
+        N, d = H.shape
+        dH_part = torch.empty(N, d, dtype=torch.float32, device=H.device)
+        dW = (torch.empty(W_shard.shape[0], d, dtype=torch.bfloat16, device=H.device)
+              if want_dW else None)
+        lmh_vp_fused_bwd(shard, v0, V_total, H, W_shard, labels, lse, n_valid_given, dH_part,
+                         dW, dW_acc, workspace=ws)
+        return dH_part, dW
 
     def combine(self, records, labels, V_total, d, n_valid_given=None):
         R, N, _ = records.shape
@@ -132,18 +155,36 @@ class VocabParallelCE:
             raise ValueError(f"rank {self.rank} holds rows [{self.v0}, {self.v1}) of W, "
                              f"got {W_shard.shape[0]} rows")
 
-    def forward(self, H, W_shard, labels, n_valid_given=None) -> dict:
-        """loss_rows, lse, logprob, argmax, loss_mean, n_valid: the same on every rank."""
-        self._check_shard(W_shard)
-        N, d = H.shape
-        rec = self.ops.partials(H, W_shard, labels, self.v0, self.V_total, self.chunk_rows,
-                                self.temperature)
+    def _combine(self, rec, labels, d, n_valid_given):
+        N = rec.shape[0]
         if self.R == 1:
             every = rec.reshape(-1)
         else:
             every = torch.empty(self.R * N * 4, dtype=rec.dtype, device=rec.device)
             dist.all_gather_into_tensor(every, rec.reshape(-1).contiguous(), group=self.group)
         return self.ops.combine(every.view(self.R, N, 4), labels, self.V_total, d, n_valid_given)
+
+    def forward(self, H, W_shard, labels, n_valid_given=None) -> dict:
+        """loss_rows, lse, logprob, argmax, loss_mean, n_valid: the same on every rank."""
+        self._check_shard(W_shard)
+        rec = self.ops.partials(H, W_shard, labels, self.v0, self.V_total, self.chunk_rows,
+                                self.temperature)
+        return self._combine(rec, labels, H.shape[1], n_valid_given)
+
+    def forward_backward(self, H, W_shard, labels, n_valid_given=None,
+                         dW_acc: Optional[torch.Tensor] = None, want_dW: bool = True) -> dict:
+        """forward() plus dH and this rank's dW of the loss (mean or sum), in one pass: the
+        backward reuses the forward's softmax numerators instead of recomputing the logits.
+        All rows form one chunk (chunk_rows is not used)."""
+        self._check_shard(W_shard)
+        rec, state = self.ops.partials_fused(H, W_shard, labels, self.v0, self.V_total,
+                                             self.mean, self.temperature)
+        out = self._combine(rec, labels, H.shape[1], n_valid_given)
+        dH_part, dW = self.ops.fused_backward(state, H, W_shard, labels, out["lse"], self.v0,
+                                              self.V_total, n_valid_given, dW_acc, want_dW)
+        out["dH"] = self._sum_rows(dH_part)
+        out["dW"] = dW
+        return out
 
     def backward(self, H, W_shard, labels, lse, grad=None, mode: int = BWD_CE,
                  dW_acc: Optional[torch.Tensor] = None, want_dW: bool = True) -> dict:

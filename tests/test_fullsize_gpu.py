@@ -187,3 +187,26 @@ def test_support_workload_sampled_rows():
                     ref[rows].cpu())
     check_grad(b["dH"][rows], rb["dH"], "dH rows (KL)")
     check_dw_properties(b["dW"])
+
+
+def test_many_chunks_and_large_row_indices():
+    # 131149 rows in 33 default-size chunks (32 x 4096 + 77): the dW accumulator is stored,
+    # added 31 times and finally added and cast in the epilogue; row indices pass 2^17 and
+    # per-row partial offsets pass 2^20. The full fp64 oracle still fits (V = 300).
+    from workloads import ragged
+    wl = ragged(131149, 64, 300, n_ignored=1000, seed=4500)
+    x = make_inputs(wl, device="cuda")
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    torch.cuda.synchronize()
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    xc = {k: v.cpu() for k, v in x.items()}
+    ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
+    check_rows(out["loss_rows"], ref["loss_rows"], what="loss_rows")
+    check_rows(out["lse"], ref["lse"], what="lse")
+    check_rows(out["loss_mean"], np.array([ref["loss_mean"]]), what="loss_mean")
+    assert int(out["n_valid"].item()) == ref["n_valid"]
+    check_argmax(out["argmax"], ref["z"])
+    check_grad(out["dH"], ref["dH"], "dH")
+    check_grad(out["dW"], ref["dW"], "dW")
+    again = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    assert torch.equal(again["dW"], out["dW"]) and torch.equal(again["dH"], out["dH"])

@@ -62,6 +62,10 @@ def _worker(rank, world, port, q, case):
         Ws = W[vp.v0:vp.v1]
         f = vp.forward(H, Ws, y)
         b = vp.backward(H, Ws, y, f["lse"])
+        fb = vp.forward_backward(H, Ws, y)
+        assert np.array_equal(fb["lse"].numpy(), f["lse"].numpy())
+        assert np.allclose(fb["dH"].numpy(), b["dH"].numpy(), rtol=1e-12, atol=1e-15)
+        assert np.allclose(fb["dW"].numpy(), b["dW"].numpy(), rtol=1e-12, atol=1e-15)
         ref = O.ce_fused(H, W, y, tau=tau)
         res = dict(rank=rank, v=(vp.v0, vp.v1),
                    lse=np.abs(f["lse"].numpy() - ref["lse"]).max(),

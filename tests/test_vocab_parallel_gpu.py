@@ -43,6 +43,67 @@ def _emulate(x, V, R, chunk=0, tau=None, mode=L.BWD_CE, grad=None, mean=True):
     return f
 
 
+def _emulate_fused(x, V, R, tau=None, mean=True, n_given=None):
+    H, W, y = x["H"], x["W"], x["labels"]
+    ops = CudaOps()
+    plan = shard_plan(V, R)
+    recs, states = zip(*[ops.partials_fused(H, W[a:b], y, a, V, mean, tau) for a, b in plan])
+    f = ops.combine(torch.stack(recs), y, V, H.shape[1], n_given)
+    parts, dWs = zip(*[ops.fused_backward(st, H, W[a:b], y, f["lse"], a, V, n_given)
+                       for st, (a, b) in zip(states, plan)])
+    f["dH"] = ops.reduce_rows(torch.stack(parts))
+    f["dW"] = torch.cat(dWs)
+    torch.cuda.synchronize()
+    return f
+
+
+@pytest.mark.parametrize("N,d,V,ign,R", [
+    (300, 192, 1000, 5, 2),
+    (200, 512, 70000, 10, 4),
+    (64, 256, 2048, 8, 8),
+])
+def test_vocab_parallel_fused_matches_oracle_and_recompute(N, d, V, ign, R):
+    x, xc = device_inputs(_wl(N, d, V, ign))
+    out = _emulate_fused(x, V, R)
+    check_ce_fused(out, O.ce_fused(xc["H"], xc["W"], xc["labels"]))
+    rec = _emulate(x, V, R)
+    assert torch.equal(out["lse"], rec["lse"]) and torch.equal(out["argmax"], rec["argmax"])
+    check_grad(out["dH"], rec["dH"], "dH fused vs recompute")
+    check_grad(out["dW"], rec["dW"], "dW fused vs recompute")
+    again = _emulate_fused(x, V, R)
+    assert torch.equal(again["dH"], out["dH"]) and torch.equal(again["dW"], out["dW"])
+
+
+def test_vocab_parallel_fused_sum_row_temperature_given_count():
+    N, d, V = 140, 128, 2600
+    x, xc = device_inputs(_wl(N, d, V, 6))
+    t = torch.linspace(0.6, 1.4, N, dtype=torch.float32)
+    out = _emulate_fused(x, V, 3, tau=t.cuda(), mean=False)
+    check_ce_fused(out, O.ce_fused(xc["H"], xc["W"], xc["labels"], mean=False, tau=t.numpy()))
+    n = torch.tensor([50], dtype=torch.int32, device="cuda")
+    out = _emulate_fused(x, V, 2, n_given=n)
+    f = O.ce_forward(xc["H"], xc["W"], xc["labels"])
+    g = np.where(xc["labels"].numpy() >= 0, 1.0 / 50, 0.0)
+    ref = O.backward(O.BWD_CE, xc["H"], xc["W"], xc["labels"], g)
+    check_rows(out["loss_mean"], np.array([f["loss_rows"].sum() / 50]), what="mean, given count")
+    check_grad(out["dH"], ref["dH"], "dH given count")
+    check_grad(out["dW"], ref["dW"], "dW given count")
+
+
+def test_vocab_parallel_fused_needs_one_chunk():
+    N, d, V = 300, 64, 800
+    x, _ = device_inputs(_wl(N, d, V, 0))
+    shard = L.make_shape(N, d, 400, 0, 128, L.F_FUSED_BWD)   # 3 chunks
+    ws = L.workspace(shard, L.ENTRY_VP_PARTIALS, "cuda")
+    rec = torch.empty(N, 4, dtype=torch.float32, device="cuda")
+    with pytest.raises(L.LmhError):
+        L.lmh_vp_partials(shard, 0, V, x["H"], x["W"][:400], x["labels"], rec, workspace=ws)
+    plain = L.make_shape(N, d, 400, 0, N, 0)                  # fused backward needs the flag
+    with pytest.raises(L.LmhError):
+        L.lmh_vp_fused_bwd(plain, 0, V, x["H"], x["W"][:400], x["labels"],
+                           torch.zeros(N, dtype=torch.float32, device="cuda"), workspace=ws)
+
+
 @pytest.mark.parametrize("N,d,V,ign,R,chunk", [
     (300, 192, 1000, 5, 2, 0),       # 2 shards of 500 words: ragged vocabulary tiles
     (129, 64, 4100, 3, 3, 100),      # 3 shards of 1367/1367/1366, two row chunks
@@ -151,8 +212,10 @@ def test_vocab_parallel_class_on_one_rank():
         vp = VocabParallelCE(V)
         f = vp.forward(x["H"], x["W"], x["labels"])
         b = vp.backward(x["H"], x["W"], x["labels"], f["lse"])
+        fb = vp.forward_backward(x["H"], x["W"], x["labels"])
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
     ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
     check_ce_fused(dict(f, dH=b["dH"], dW=b["dW"]), ref)
+    check_ce_fused(fb, ref)

@@ -59,6 +59,19 @@ class OracleOps:
         dH, dW = O.lm_head_backward(H, W_shard, G)
         return _t(dH), (_t(dW) if want_dW else None)
 
+    def partials_fused(self, H, W_shard, labels, v0, V_total, mean=True, temperature=None):
+        return self.partials(H, W_shard, labels, v0, V_total, 0, temperature), \
+            dict(mean=mean, temperature=temperature)
+
+    def fused_backward(self, state, H, W_shard, labels, lse, v0, V_total, n_valid_given=None,
+                       dW_acc=None, want_dW=True):
+        grad = None
+        if n_valid_given is not None:
+            n = int(n_valid_given)
+            grad = np.full(len(O.as_i64(labels)), (1.0 / n if n else 0.0) if state["mean"] else 1.0)
+        return self.backward(0, H, W_shard, labels, lse, grad, v0, V_total, 0, state["mean"],
+                             state["temperature"], dW_acc, want_dW)
+
     def reduce_rows(self, parts):
         out = parts[0].clone()
         for r in range(1, parts.shape[0]):
