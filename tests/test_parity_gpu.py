@@ -435,3 +435,20 @@ def test_no_split_when_vocabulary_is_small():
     x, _ = device_inputs(_wl(256, 256, 32000, 0))
     names = _kernels_launched(lambda: L.loss_fwd(x["H"], x["W"], x["labels"], grads=True))
     assert "split_sum" not in names and names.count("gemm_dH") == 1
+
+
+@pytest.mark.parametrize("N,d,V,ign,chunk", [
+    (256, 8192, 3000, 4, 0),      # 64 K blocks per logits tile, 32 dH column tiles
+    (8, 128, 200000, 1, 0),       # 782 vocabulary tiles, dH split into 6 ranges, dW K = 8 rows
+    (520, 64, 70001, 0, 200),     # minimum d, V one past a multiple of 8, 3 chunks
+])
+def test_extreme_aspect_ratios(N, d, V, ign, chunk):
+    x, xc = device_inputs(_wl(N, d, V, ign))
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=chunk, grads=True)
+    torch.cuda.synchronize()
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    check_ce_fused(out, O.ce_fused(xc["H"], xc["W"], xc["labels"]))
+    lse = out["lse"]
+    b = L.loss_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], lse, None, chunk_rows=chunk, mean=True)
+    check_grad(b["dH"], out["dH"], "dH recompute vs fused")
+    check_grad(b["dW"], out["dW"], "dW recompute vs fused")
