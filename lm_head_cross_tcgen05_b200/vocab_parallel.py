@@ -209,8 +209,15 @@ class VocabParallelCE:
                                input_split_sizes=sizes, group=self.group)
         red = self.ops.reduce_rows(recv.view(self.R, mine, d))
         top = max(sizes)
-        pad = torch.zeros(top, d, dtype=red.dtype, device=red.device)
-        pad[:mine] = red
+        if top == 0:
+            return red
+        if mine == top:
+            pad = red
+        else:  # slices differ by one row at most: gather equal blocks, drop the padding
+            pad = torch.zeros(top, d, dtype=red.dtype, device=red.device)
+            pad[:mine] = red
         every = torch.empty(self.R * top, d, dtype=red.dtype, device=red.device)
-        dist.all_gather_into_tensor(every, pad, group=self.group)
+        dist.all_gather_into_tensor(every, pad.contiguous(), group=self.group)
+        if all(n == top for n in sizes):
+            return every
         return torch.cat([every[j * top: j * top + sizes[j]] for j in range(self.R)])

@@ -86,6 +86,8 @@ def _worker(rank, world, port, q, case):
 @pytest.mark.parametrize("world,case", [
     (2, (37, 64, 700, 5, None)),       # ragged rows over 2 ranks, a shard of 350 words
     (3, (20, 64, 1030, 3, 0.7)),       # 3 ranks, shards 344/344/342, scalar temperature
+    (2, (40, 64, 512, 0, None)),       # rows divide evenly: no padding in the dH gather
+    (3, (2, 64, 900, 0, None)),        # fewer rows than ranks: one rank reduces no row
 ])
 def test_vocab_parallel_exchange_gloo(world, case):
     ctx = mp.get_context("spawn")
