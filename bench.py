@@ -49,6 +49,8 @@ def parse_args():
                          "lmh_loss_fwd then lmh_loss_bwd (recomputed logits); support_kl: "
                          "lmh_support_kl then lmh_loss_bwd of the mean KL; vocab_parallel: one "
                          "CE problem with W split over the GPUs (strong scaling)")
+    ap.add_argument("--chunk-rows", type=int, default=0,
+                    help="rows per chunk (the memory budget); 0: the workload's own plan")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -289,7 +291,7 @@ def main():
     x = make_inputs(wl, device=dev, seed=wl.seed if vp_entry else replica_seed(wl, rank))
     H, W, y = x["H"], x["W"], x["labels"]
     N, d, V = wl.N, wl.d, wl.V
-    chunk = wl.chunk_rows or N
+    chunk = args.chunk_rows or wl.chunk_rows or N
     shape = L.make_shape(N, d, V, 0, chunk, L.F_MEAN | L.F_FUSED_BWD)
     ws = L.workspace(shape, L.ENTRY_LOSS_FWD, dev)
     f32, i32, bf = torch.float32, torch.int32, torch.bfloat16
@@ -326,6 +328,7 @@ def main():
                            out["dH"], out["dW"], None, workspace=bws, stream=stream)
     elif vp_entry:
         from lm_head_cross_tcgen05_b200.vocab_parallel import VocabParallelCE
+        chunk = N                                   # the fused step runs all rows as one chunk
         vp = VocabParallelCE(V, chunk_rows=chunk)      # the default group when world > 1
         W_shard = W[vp.v0:vp.v1].contiguous()
 
