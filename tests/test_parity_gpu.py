@@ -452,3 +452,41 @@ def test_extreme_aspect_ratios(N, d, V, ign, chunk):
     b = L.loss_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], lse, None, chunk_rows=chunk, mean=True)
     check_grad(b["dH"], out["dH"], "dH recompute vs fused")
     check_grad(b["dW"], out["dW"], "dW recompute vs fused")
+
+
+_DIGEST_SCRIPT = r"""
+import sys
+sys.path.insert(0, {root!r})
+import torch
+import lm_head_cross_tcgen05_b200 as L
+from tests.gpu_common import digest
+from workloads import make_inputs, ragged
+x = {{k: v.cuda() for k, v in
+      make_inputs(ragged(520, 256, 5000, n_ignored=9, seed=1000 + 520 + 256 + 5000)).items()}}
+o = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=200, grads=True)
+s = L.support_kl(x["H"], x["W"], torch.stack([x["labels"].clamp(min=0), x["labels"].clamp(min=0) + 1], 1),
+                 torch.full((520, 2), -0.7, device="cuda"))
+print(digest(o["loss_rows"], o["lse"], o["argmax"], o["dH"], o["dW"], s["kl_rows"], s["lp"]))
+"""
+
+
+def test_same_bits_in_a_new_process():
+    # the pages' determinism contract: a fresh process (new context, new allocations,
+    # first-call setup) gives the same bits as this one
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    script = _DIGEST_SCRIPT.format(root=root)
+    here = subprocess.run([sys.executable, "-c", script], capture_output=True, text=True,
+                          timeout=300, cwd=root)
+    assert here.returncode == 0, here.stderr[-2000:]
+    again = subprocess.run([sys.executable, "-c", script], capture_output=True, text=True,
+                           timeout=300, cwd=root)
+    assert again.returncode == 0, again.stderr[-2000:]
+    x = device_inputs(_wl(520, 256, 5000, 9))[0]
+    o = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=200, grads=True)
+    ids = torch.stack([x["labels"].clamp(min=0), x["labels"].clamp(min=0) + 1], 1)
+    s = L.support_kl(x["H"], x["W"], ids, torch.full((520, 2), -0.7, device="cuda"))
+    mine = digest(o["loss_rows"], o["lse"], o["argmax"], o["dH"], o["dW"], s["kl_rows"], s["lp"])
+    assert here.stdout.strip().splitlines()[-1] == again.stdout.strip().splitlines()[-1] == mine
