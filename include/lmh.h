@@ -17,7 +17,9 @@
  * - H [N, d] and W [V, d] are bf16, row-major and contiguous (row stride d elements);
  *   lmh_bf16 is the raw 16-bit pattern. d must be a positive multiple of 64.
  * - Every pointer argument is a DEVICE pointer unless marked "host", 16-byte aligned, and
- *   owned by the caller. The library never allocates device memory, never frees it, and
+ *   owned by the caller. The library sees no buffer sizes: each buffer must hold what the
+ *   shape declares for it (the sizes given below); a smaller one is read or written past
+ *   its end. The Python binding checks every size before the call. The library never allocates device memory, never frees it, and
  *   never synchronises the host: each call only enqueues work on `stream` (a cudaStream_t;
  *   NULL is the legacy default stream) and returns.
  * - The workspace must hold at least lmh_workspace_size(shape, entry) bytes, be 256-byte

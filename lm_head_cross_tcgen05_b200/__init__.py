@@ -70,6 +70,14 @@ def _p(t: Optional[torch.Tensor], dtype=None, what: str = "tensor"):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _fits(**named) -> None:
+    """Each named (tensor, elements) pair: the tensor, when given, holds at least that many
+    elements, so no kernel can index past its allocation for the shape the call declares."""
+    for what, (t, n) in named.items():
+        if t is not None and t.numel() < int(n):
+            raise ValueError(f"{what} has {t.numel()} elements; the shape needs {int(n)}")
+
+
 def _s(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -93,6 +101,11 @@ def lmh_workspace_size(shape: lmh_shape, entry: int) -> int:
 def lmh_loss_fwd(shape, H, W, labels, loss_rows, lse, logprob=None, argmax=None, loss_mean=None,
                  n_valid=None, n_valid_given=None, dH=None, dW=None, dW_acc=None, *, workspace,
                  stream=None) -> None:
+    N, d, V = shape.N, shape.d, shape.V
+    _fits(H=(H, N * d), W=(W, V * d), labels=(labels, N), loss_rows=(loss_rows, N),
+          lse=(lse, N), logprob=(logprob, N), argmax=(argmax, N), loss_mean=(loss_mean, 1),
+          n_valid=(n_valid, 1), n_valid_given=(n_valid_given, 1), dH=(dH, N * d),
+          dW=(dW, V * d), dW_acc=(dW_acc, V * d))
     st = lib().lmh_loss_fwd(
         ctypes.byref(shape), _p(H, _bf, "H"), _p(W, _bf, "W"), _p(labels, _i32, "labels"),
         _p(loss_rows, _f32, "loss_rows"), _p(lse, _f32, "lse"), _p(logprob, _f32, "logprob"),
@@ -105,6 +118,12 @@ def lmh_loss_fwd(shape, H, W, labels, loss_rows, lse, logprob=None, argmax=None,
 
 def lmh_loss_bwd(shape, mode, H, W, targets, lse, grad, ref_logp=None, dH=None, dW=None,
                  dW_acc=None, *, workspace, stream=None) -> None:
+    N, d, V, K = shape.N, shape.d, shape.V, max(shape.K, 1)
+    cands = int(mode) in (BWD_SUPPORT_LOGPROB, BWD_SUPPORT_KL)
+    g = 1 if shape.flags & F_GRAD_SCALAR else (N * K if int(mode) == BWD_SUPPORT_LOGPROB else N)
+    _fits(H=(H, N * d), W=(W, V * d), targets=(targets, N * K if cands else N), lse=(lse, N),
+          grad=(grad, g), ref_logp=(ref_logp, N * K), dH=(dH, N * d), dW=(dW, V * d),
+          dW_acc=(dW_acc, V * d))
     st = lib().lmh_loss_bwd(
         ctypes.byref(shape), int(mode), _p(H, _bf, "H"), _p(W, _bf, "W"),
         _p(targets, _i32, "targets"), _p(lse, _f32, "lse"), _p(grad, _f32, "grad"),
@@ -115,6 +134,8 @@ def lmh_loss_bwd(shape, mode, H, W, targets, lse, grad, ref_logp=None, dH=None, 
 
 
 def lmh_logprob(shape, H, W, labels, logprob, lse, *, workspace, stream=None) -> None:
+    N, d, V = shape.N, shape.d, shape.V
+    _fits(H=(H, N * d), W=(W, V * d), labels=(labels, N), logprob=(logprob, N), lse=(lse, N))
     st = lib().lmh_logprob(ctypes.byref(shape), _p(H, _bf, "H"), _p(W, _bf, "W"),
                            _p(labels, _i32, "labels"), _p(logprob, _f32, "logprob"),
                            _p(lse, _f32, "lse"), _p(workspace, _u8, "workspace"),
@@ -123,6 +144,8 @@ def lmh_logprob(shape, H, W, labels, logprob, lse, *, workspace, stream=None) ->
 
 
 def lmh_support_logprob(shape, H, W, ids, lp, lse, *, workspace, stream=None) -> None:
+    N, d, V, K = shape.N, shape.d, shape.V, shape.K
+    _fits(H=(H, N * d), W=(W, V * d), ids=(ids, N * K), lp=(lp, N * K), lse=(lse, N))
     st = lib().lmh_support_logprob(ctypes.byref(shape), _p(H, _bf, "H"), _p(W, _bf, "W"),
                                    _p(ids, _i32, "ids"), _p(lp, _f32, "lp"), _p(lse, _f32, "lse"),
                                    _p(workspace, _u8, "workspace"), workspace.numel(),
@@ -132,6 +155,9 @@ def lmh_support_logprob(shape, H, W, ids, lp, lse, *, workspace, stream=None) ->
 
 def lmh_support_kl(shape, H, W, ids, ref_logp, kl_rows, kl_mean=None, lp=None, lse=None, *,
                    workspace, stream=None) -> None:
+    N, d, V, K = shape.N, shape.d, shape.V, shape.K
+    _fits(H=(H, N * d), W=(W, V * d), ids=(ids, N * K), ref_logp=(ref_logp, N * K),
+          kl_rows=(kl_rows, N), kl_mean=(kl_mean, 1), lp=(lp, N * K), lse=(lse, N))
     st = lib().lmh_support_kl(ctypes.byref(shape), _p(H, _bf, "H"), _p(W, _bf, "W"),
                               _p(ids, _i32, "ids"), _p(ref_logp, _f32, "ref_logp"),
                               _p(kl_rows, _f32, "kl_rows"), _p(kl_mean, _f32, "kl_mean"),
@@ -142,6 +168,9 @@ def lmh_support_kl(shape, H, W, ids, ref_logp, kl_rows, kl_mean=None, lp=None, l
 
 def lmh_vp_partials(shard, v0, V_total, H, W_shard, labels, records, *, workspace,
                     stream=None) -> None:
+    N, d = shard.N, shard.d
+    _fits(H=(H, N * d), W_shard=(W_shard, shard.V * d), labels=(labels, N),
+          records=(records, N * 4))
     st = lib().lmh_vp_partials(ctypes.byref(shard), int(v0), int(V_total), _p(H, _bf, "H"),
                                _p(W_shard, _bf, "W_shard"), _p(labels, _i32, "labels"),
                                _p(records, _f32, "records"), _p(workspace, _u8, "workspace"),
@@ -152,6 +181,10 @@ def lmh_vp_partials(shard, v0, V_total, H, W_shard, labels, records, *, workspac
 def lmh_vp_combine(shape, R, records, labels, loss_rows, lse, logprob=None, argmax=None,
                    loss_mean=None, n_valid=None, n_valid_given=None, *, workspace,
                    stream=None) -> None:
+    N = shape.N
+    _fits(records=(records, int(R) * N * 4), labels=(labels, N), loss_rows=(loss_rows, N),
+          lse=(lse, N), logprob=(logprob, N), argmax=(argmax, N), loss_mean=(loss_mean, 1),
+          n_valid=(n_valid, 1), n_valid_given=(n_valid_given, 1))
     st = lib().lmh_vp_combine(ctypes.byref(shape), int(R), _p(records, _f32, "records"),
                               _p(labels, _i32, "labels"), _p(loss_rows, _f32, "loss_rows"),
                               _p(lse, _f32, "lse"), _p(logprob, _f32, "logprob"),
@@ -164,6 +197,10 @@ def lmh_vp_combine(shape, R, records, labels, loss_rows, lse, logprob=None, argm
 
 def lmh_vp_loss_bwd(shard, mode, v0, V_total, H, W_shard, labels, lse, grad=None, dH_part=None,
                     dW_shard=None, dW_acc_shard=None, *, workspace, stream=None) -> None:
+    N, d, Vr = shard.N, shard.d, shard.V
+    _fits(H=(H, N * d), W_shard=(W_shard, Vr * d), labels=(labels, N), lse=(lse, N),
+          grad=(grad, 1 if shard.flags & F_GRAD_SCALAR else N), dH_part=(dH_part, N * d),
+          dW_shard=(dW_shard, Vr * d), dW_acc_shard=(dW_acc_shard, Vr * d))
     st = lib().lmh_vp_loss_bwd(ctypes.byref(shard), int(mode), int(v0), int(V_total),
                                _p(H, _bf, "H"), _p(W_shard, _bf, "W_shard"),
                                _p(labels, _i32, "labels"), _p(lse, _f32, "lse"),
@@ -176,6 +213,10 @@ def lmh_vp_loss_bwd(shard, mode, v0, V_total, H, W_shard, labels, lse, grad=None
 def lmh_vp_fused_bwd(shard, v0, V_total, H, W_shard, labels, lse, n_valid_given=None,
                      dH_part=None, dW_shard=None, dW_acc_shard=None, *, workspace,
                      stream=None) -> None:
+    N, d, Vr = shard.N, shard.d, shard.V
+    _fits(H=(H, N * d), W_shard=(W_shard, Vr * d), labels=(labels, N), lse=(lse, N),
+          n_valid_given=(n_valid_given, 1), dH_part=(dH_part, N * d),
+          dW_shard=(dW_shard, Vr * d), dW_acc_shard=(dW_acc_shard, Vr * d))
     st = lib().lmh_vp_fused_bwd(ctypes.byref(shard), int(v0), int(V_total), _p(H, _bf, "H"),
                                 _p(W_shard, _bf, "W_shard"), _p(labels, _i32, "labels"),
                                 _p(lse, _f32, "lse"), _p(n_valid_given, _i32, "n_valid_given"),
@@ -188,6 +229,7 @@ def lmh_vp_fused_bwd(shard, v0, V_total, H, W_shard, labels, lse, n_valid_given=
 def lmh_vp_reduce_rows(parts, out, stream=None) -> None:
     """parts [R, rows, d] fp32 -> out [rows, d] bf16, summed in ascending R."""
     R, rows, d = parts.shape
+    _fits(out=(out, rows * d))
     st = lib().lmh_vp_reduce_rows(int(R), int(rows), int(d), _p(parts, _f32, "parts"),
                                   _p(out, _bf, "out"), _s(stream))
     _ok("lmh_vp_reduce_rows", st)

@@ -101,3 +101,27 @@ def test_vocab_parallel_host_errors_without_gpu():
     assert lib.lmh_vp_reduce_rows(2, 4, 96, None, None, None) == 1     # d not a multiple of 64
     assert lib.lmh_vp_reduce_rows(0, 4, 64, None, None, None) == 1
     assert lib.lmh_vp_reduce_rows(2, 0, 64, None, None, None) == 0     # nothing to do
+
+
+def test_binding_rejects_tensors_smaller_than_the_shape():
+    # a W with fewer columns than shape.d would let the tensor maps read past its allocation:
+    # the binding refuses it before any pointer reaches the library
+    import torch
+    shape = L.make_shape(4, 64, 100)
+    H = torch.zeros(4, 64, dtype=torch.bfloat16)
+    W = torch.zeros(100, 32, dtype=torch.bfloat16)
+    y = torch.zeros(4, dtype=torch.int32)
+    f = torch.zeros(4, dtype=torch.float32)
+    ws = torch.zeros(1 << 16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="W has 3200 elements"):
+        L.lmh_loss_fwd(shape, H, W, y, f, f, workspace=ws)
+    with pytest.raises(ValueError, match="lse has"):
+        L.lmh_logprob(shape, H, torch.zeros(100, 64, dtype=torch.bfloat16), y, f,
+                      torch.zeros(3), workspace=ws)
+    sup = L.make_shape(4, 64, 100, K=8)
+    with pytest.raises(ValueError, match="ids has"):
+        L.lmh_support_logprob(sup, H, torch.zeros(100, 64, dtype=torch.bfloat16),
+                              torch.zeros(4, 4, dtype=torch.int32),
+                              torch.zeros(4, 8), f, workspace=ws)
+    with pytest.raises(ValueError, match="records has"):
+        L.lmh_vp_combine(shape, 3, torch.zeros(2, 4, 4), y, f, f, workspace=ws)
