@@ -230,9 +230,13 @@ def test_host_rejections():
     lr, lse = torch.empty(64, device="cuda"), torch.empty(64, device="cuda")
     with pytest.raises(L.LmhError, match="WORKSPACE_TOO_SMALL"):
         L.lmh_loss_fwd(shape, x["H"], x["W"], x["labels"], lr, lse, workspace=ws[:100])
-    bad = L.make_shape(64, 96, 300)
+    bad = L.make_shape(64, 96, 300)     # d not a multiple of 64: refused by the library
+    H96 = torch.zeros(64, 96, dtype=torch.bfloat16, device="cuda")
+    W96 = torch.zeros(300, 96, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(L.LmhError, match="INVALID_ARG"):
-        L.lmh_loss_fwd(bad, x["H"], x["W"], x["labels"], lr, lse, workspace=ws)
+        L.lmh_loss_fwd(bad, H96, W96, x["labels"], lr, lse, workspace=ws)
+    with pytest.raises(ValueError, match="W has"):  # too small for the shape: the binding
+        L.lmh_loss_fwd(shape, x["H"], x["W"][:200], x["labels"], lr, lse, workspace=ws)
     with pytest.raises(L.LmhError, match="ALIGNMENT"):
         L.lmh_loss_fwd(shape, x["H"], x["W"], x["labels"], lr, lse, workspace=ws[8:])
 
