@@ -43,11 +43,13 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_vocab")
     ap.add_argument("--entry", choices=["fused_ce", "ce_separate", "support_kl",
-                                        "vocab_parallel"],
+                                        "support_kl_separate", "vocab_parallel"],
                     default="fused_ce",
                     help="fused_ce: lmh_loss_fwd with dH/dW (the headline step); ce_separate: "
                          "lmh_loss_fwd then lmh_loss_bwd (recomputed logits); support_kl: "
-                         "lmh_support_kl then lmh_loss_bwd of the mean KL; vocab_parallel: one "
+                         "lmh_support_kl_fwd_bwd (the mean KL's forward and backward in one "
+                         "pass); support_kl_separate: lmh_support_kl then lmh_loss_bwd; "
+                         "vocab_parallel: one "
                          "CE problem with W split over the GPUs (strong scaling)")
     ap.add_argument("--chunk-rows", type=int, default=0,
                     help="rows per chunk (the memory budget); 0: the workload's own plan")
@@ -78,7 +80,9 @@ def source_hash() -> str:
 
 ENTRY_TEXT = {"fused_ce": "fused CE forward+backward",
               "ce_separate": "CE forward, then backward with recomputed logits",
-              "support_kl": "support-set KL forward (K candidates), then its backward",
+              "support_kl": "support-set KL forward (K candidates) and its backward, fused",
+              "support_kl_separate": "support-set KL forward (K candidates), then its backward "
+                                     "with recomputed logits",
               "vocab_parallel": "vocabulary-parallel fused CE forward+backward (W split over "
                                 "the GPUs)"}
 
@@ -184,7 +188,7 @@ def oracle_runner(wl, entry):
     from oracle import lmh_oracle as O
     from workloads import make_inputs
     x = make_inputs(wl.scaled(N=min(wl.N, 4096)), device="cpu")
-    if entry == "support_kl":
+    if entry.startswith("support_kl"):
         def run(n):
             O.support_kl(x["H"][:n], x["W"], x["ids"][:n], x["ref_logp"][:n])
             g = [1.0 / wl.N] * n
@@ -340,18 +344,28 @@ def main():
         batch = {"H": H, "ids": x["ids"], "ref_logp": x["ref_logp"]}
         K = batch["ids"].shape[1]
         sshape = L.make_shape(N, d, V, K, chunk, L.F_MEAN)
-        sws = L.workspace(sshape, L.ENTRY_SUPPORT_KL, dev)
-        bws = L.workspace(sshape, L.ENTRY_LOSS_BWD, dev)
         kl_rows = torch.empty(N, dtype=f32, device=dev)
         lp = torch.empty(N, K, dtype=f32, device=dev)
+        if args.entry == "support_kl":
+            fshape = L.make_shape(N, d, V, K, chunk, L.F_MEAN | L.F_FUSED_BWD)
+            fws = L.workspace(fshape, L.ENTRY_SUPPORT_KL, dev)
 
-        def step(b=batch):
-            L.lmh_support_kl(sshape, b["H"], W, b["ids"], b["ref_logp"], kl_rows,
-                             out["loss_mean"], lp, out["lse"], workspace=sws, stream=stream)
-            # backward of the mean KL: no grad given, 1 / N on the device
-            L.lmh_loss_bwd(sshape, L.BWD_SUPPORT_KL, b["H"], W, b["ids"], out["lse"], None,
-                           b["ref_logp"], out["dH"], out["dW"], None, workspace=bws,
-                           stream=stream)
+            def step(b=batch):
+                # forward and the mean KL's backward in one pass (3 GEMMs per chunk)
+                L.lmh_support_kl_fwd_bwd(fshape, b["H"], W, b["ids"], b["ref_logp"], kl_rows,
+                                         out["loss_mean"], lp, out["lse"], out["dH"],
+                                         out["dW"], None, workspace=fws, stream=stream)
+        else:
+            sws = L.workspace(sshape, L.ENTRY_SUPPORT_KL, dev)
+            bws = L.workspace(sshape, L.ENTRY_LOSS_BWD, dev)
+
+            def step(b=batch):
+                L.lmh_support_kl(sshape, b["H"], W, b["ids"], b["ref_logp"], kl_rows,
+                                 out["loss_mean"], lp, out["lse"], workspace=sws, stream=stream)
+                # backward of the mean KL: no grad given, 1 / N on the device
+                L.lmh_loss_bwd(sshape, L.BWD_SUPPORT_KL, b["H"], W, b["ids"], out["lse"], None,
+                               b["ref_logp"], out["dH"], out["dW"], None, workspace=bws,
+                               stream=stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -417,7 +431,9 @@ def main():
             with open(tpath) as fh:
                 tr = json.load(fh)
             ent = tr.get(dom)
-            if ent and ent.get("source_hash") == source_hash():
+            if (ent and ent.get("source_hash") == source_hash()
+                    and ent.get("workload") == wl.name and ent.get("entry") == args.entry
+                    and chunk == (wl.chunk_rows or N)):
                 roofline["traffic"] = ent["bytes_per_launch"]
 
     # end to end through the public API: pinned host batch in, loss out, every step
@@ -429,7 +445,8 @@ def main():
         # buffers), as a training loop would overlap it
         host = {k: v.cpu().pin_memory() for k, v in batch.items()}
         dbuf = [{k: torch.empty_like(v) for k, v in batch.items()} for _ in range(2)]
-        reads = [out["loss_mean"]] + ([out["n_valid"]] if args.entry != "support_kl" else [])
+        reads = [out["loss_mean"]] + ([out["n_valid"]] if not args.entry.startswith("support")
+                                      else [])
         reads_h = [torch.empty_like(t, device="cpu").pin_memory() for t in reads]
         ready = [torch.cuda.Event() for _ in range(2)]
         free = [torch.cuda.Event() for _ in range(2)]

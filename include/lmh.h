@@ -314,6 +314,27 @@ LMH_API lmh_status lmh_vp_reduce_rows(int R, int64_t rows, int64_t d, const floa
                                       lmh_bf16* out, void* stream);
 
 /*
+ * lmh_support_kl_fwd_bwd — lmh_support_kl plus the backward of the mean KL (LMH_F_MEAN:
+ * weight 1 / N per row) or of the summed KL, in one pass that reuses the forward's softmax as
+ * lmh_loss_fwd's fused path does. The KL's coefficients (alpha_i = g_i sum_k exp(r_ik),
+ * beta_ic = g_i sum over the slots of c of exp(r_ik)) depend on the reference log-probs only,
+ * so the forward's softmax numerators p~ = exp(z - m_t) are kept per chunk, scaled into
+ * alpha_i P by the row finalize, and the candidate columns rewritten from their fp32 logits.
+ * Three GEMMs per chunk instead of the four of lmh_support_kl followed by lmh_loss_bwd.
+ *   Arguments as lmh_support_kl (kl_rows, lse and ref_logp required), plus dH, dW, dW_acc as
+ *   in lmh_loss_fwd (all null: the forward alone). Workspace: lmh_workspace_size(shape,
+ *   LMH_ENTRY_SUPPORT_KL) with LMH_F_FUSED_BWD (and LMH_F_DW_ACC_GIVEN) in shape->flags.
+ *   LMH_F_SUPPORT_RENORM is refused (LMH_ERR_INVALID_ARG): that reading's backward is the
+ *   sparse path of lmh_loss_bwd, which has no logits GEMM to save.
+ */
+LMH_API lmh_status lmh_support_kl_fwd_bwd(const lmh_shape* shape, const lmh_bf16* H,
+                                          const lmh_bf16* W, const int32_t* ids,
+                                          const float* ref_logp, float* kl_rows, float* kl_mean,
+                                          float* lp, float* lse, lmh_bf16* dH, lmh_bf16* dW,
+                                          float* dW_acc, void* workspace,
+                                          size_t workspace_bytes, void* stream);
+
+/*
  * lmh_read_errors — synchronises `stream`, then copies the device error word of the last
  * call that used `workspace` into *errors (host). Each entry clears the word when it starts.
  */

@@ -24,7 +24,8 @@ from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEV
 
 __all__ = [
     "lmh_shape", "make_shape", "lmh_workspace_size", "lmh_loss_fwd", "lmh_loss_bwd",
-    "lmh_logprob", "lmh_support_logprob", "lmh_support_kl", "lmh_read_errors", "LmhError",
+    "lmh_logprob", "lmh_support_logprob", "lmh_support_kl", "lmh_support_kl_fwd_bwd",
+    "lmh_read_errors", "LmhError",
     "loss_fwd", "loss_bwd", "logprob", "support_logprob", "support_kl", "workspace",
     "IGNORE_INDEX", "BWD_CE", "BWD_LOGPROB", "BWD_SUPPORT_LOGPROB", "BWD_SUPPORT_KL",
     "F_MEAN", "F_FUSED_BWD", "F_DW_ACC_GIVEN", "F_SUPPORT_RENORM", "ENTRY_LOSS_FWD", "ENTRY_LOSS_BWD",
@@ -164,6 +165,22 @@ def lmh_support_kl(shape, H, W, ids, ref_logp, kl_rows, kl_mean=None, lp=None, l
                               _p(lp, _f32, "lp"), _p(lse, _f32, "lse"),
                               _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
     _ok("lmh_support_kl", st)
+
+
+def lmh_support_kl_fwd_bwd(shape, H, W, ids, ref_logp, kl_rows, kl_mean=None, lp=None,
+                           lse=None, dH=None, dW=None, dW_acc=None, *, workspace,
+                           stream=None) -> None:
+    N, d, V, K = shape.N, shape.d, shape.V, shape.K
+    _fits(H=(H, N * d), W=(W, V * d), ids=(ids, N * K), ref_logp=(ref_logp, N * K),
+          kl_rows=(kl_rows, N), kl_mean=(kl_mean, 1), lp=(lp, N * K), lse=(lse, N),
+          dH=(dH, N * d), dW=(dW, V * d), dW_acc=(dW_acc, V * d))
+    st = lib().lmh_support_kl_fwd_bwd(
+        ctypes.byref(shape), _p(H, _bf, "H"), _p(W, _bf, "W"), _p(ids, _i32, "ids"),
+        _p(ref_logp, _f32, "ref_logp"), _p(kl_rows, _f32, "kl_rows"),
+        _p(kl_mean, _f32, "kl_mean"), _p(lp, _f32, "lp"), _p(lse, _f32, "lse"),
+        _p(dH, _bf, "dH"), _p(dW, _bf, "dW"), _p(dW_acc, _f32, "dW_acc"),
+        _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
+    _ok("lmh_support_kl_fwd_bwd", st)
 
 
 def lmh_vp_partials(shard, v0, V_total, H, W_shard, labels, records, *, workspace,
@@ -330,18 +347,30 @@ def support_logprob(H, W, ids, *, chunk_rows: int = 0, temperature=None, renorm:
 
 
 def support_kl(H, W, ids, ref_logp, *, chunk_rows: int = 0, temperature=None,
-               renorm: bool = False, ws=None, stream=None) -> dict:
+               renorm: bool = False, grads: bool = False, mean: bool = True, dW_acc=None,
+               ws=None, stream=None) -> dict:
+    """KL(ref || model) over the candidates (kl_rows, kl_mean, lp, lse). grads=True: also dH
+    and dW of the mean (or summed) KL in the same pass (lmh_support_kl_fwd_bwd)."""
     N, d = H.shape
-    K = ids.shape[1]
-    shape = make_shape(N, d, W.shape[0], K, chunk_rows, F_SUPPORT_RENORM if renorm else 0,
-                       temperature)
+    V, K = W.shape[0], ids.shape[1]
+    flags = (F_SUPPORT_RENORM if renorm else 0) | (F_FUSED_BWD | (F_MEAN if mean else 0)
+                                                   if grads else 0) | (
+        F_DW_ACC_GIVEN if dW_acc is not None else 0)
+    shape = make_shape(N, d, V, K, chunk_rows, flags, temperature)
     dev = H.device
     out = dict(kl_rows=torch.empty(N, dtype=_f32, device=dev),
                kl_mean=torch.empty(1, dtype=_f32, device=dev),
                lp=torch.empty(N, K, dtype=_f32, device=dev),
                lse=torch.empty(N, dtype=_f32, device=dev))
     ws = workspace(shape, ENTRY_SUPPORT_KL, dev) if ws is None else ws
-    lmh_support_kl(shape, H, W, ids, ref_logp, out["kl_rows"], out["kl_mean"], out["lp"],
-                   out["lse"], workspace=ws, stream=stream)
+    if grads:
+        out["dH"] = torch.empty(N, d, dtype=_bf, device=dev)
+        out["dW"] = torch.empty(V, d, dtype=_bf, device=dev)
+        lmh_support_kl_fwd_bwd(shape, H, W, ids, ref_logp, out["kl_rows"], out["kl_mean"],
+                               out["lp"], out["lse"], out["dH"], out["dW"], dW_acc,
+                               workspace=ws, stream=stream)
+    else:
+        lmh_support_kl(shape, H, W, ids, ref_logp, out["kl_rows"], out["kl_mean"], out["lp"],
+                       out["lse"], workspace=ws, stream=stream)
     out["workspace"] = ws
     return out

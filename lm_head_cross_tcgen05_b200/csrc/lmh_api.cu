@@ -88,8 +88,8 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
              entry == LMH_ENTRY_LOSS_BWD);
   p.K = p.cands ? (s->K > 0 ? s->K : 1) : 1;
   p.renorm = p.cands && (s->flags & LMH_F_SUPPORT_RENORM);
-  const bool fwd_fused =
-      fused && (entry == LMH_ENTRY_LOSS_FWD || entry == LMH_ENTRY_VP_PARTIALS);
+  const bool fwd_fused = fused && (entry == LMH_ENTRY_LOSS_FWD || entry == LMH_ENTRY_VP_PARTIALS ||
+                                   entry == LMH_ENTRY_SUPPORT_KL);
   p.gbuf = !p.renorm && (bwd || fwd_fused);
   p.acc = p.gbuf && dw_without_acc && p.nchunks > 1;
   const bool stats = !bwd && entry != LMH_ENTRY_VP_COMBINE;
@@ -109,8 +109,9 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   p.o_pm = partials ? take(cT * 4) : 0;
   p.o_ps = partials ? take(cT * 4) : 0;
   p.o_pi = partials ? take(cT * 4) : 0;
-  p.o_alpha = bwd ? take(N * 4) : 0;
-  p.o_beta = bwd ? take(N * p.K * 4) : 0;
+  const bool coef = bwd || (fwd_fused && entry == LMH_ENTRY_SUPPORT_KL);
+  p.o_alpha = coef ? take(N * 4) : 0;
+  p.o_beta = coef ? take(N * p.K * 4) : 0;
   p.o_lloc = (vp_bwd || entry == LMH_ENTRY_VP_PARTIALS) ? take(N * 4) : 0;
   p.o_gbuf = p.gbuf ? take(static_cast<size_t>(p.c) * p.Vp * 2) : 0;
   p.o_acc = p.acc ? take(static_cast<size_t>(p.V) * p.d * 4) : 0;
@@ -171,14 +172,14 @@ enum KernelId {
   KID_GEMM_DH, KID_GEMM_DW, KID_FINALIZE, KID_GBUILD, KID_FIX_LABELS, KID_MEAN,
   KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_SUPPORT_DOTS, KID_SUPPORT_LSE,
   KID_SUPPORT_DH, KID_SUPPORT_DW, KID_SPLIT_SUM, KID_VP_LABELS, KID_VP_FINALIZE,
-  KID_VP_COMBINE, KID_VP_REDUCE, KID_VP_SCALE, KID_COUNT
+  KID_VP_COMBINE, KID_VP_REDUCE, KID_VP_SCALE, KID_FIX_CANDS, KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "count_labels", "prep_cands", "gemm_logits_stats", "gemm_logits_stats_store",
     "gemm_logits_grad", "gemm_dH", "gemm_dW", "row_finalize", "gbuild", "fix_labels",
     "mean", "support_out", "bwd_coef", "cast_bf16", "support_dots", "support_lse",
     "support_grad_dh", "support_dw", "split_sum", "vp_local_labels", "vp_finalize",
-    "vp_combine", "vp_reduce_rows", "vp_scale"};
+    "vp_combine", "vp_reduce_rows", "vp_scale", "fix_cands"};
 
 struct ProfRec {
   int id;
@@ -393,7 +394,8 @@ lmh_status run_stats(const Plan& P, int dev, int sms, const lmh_bf16* H, const l
 
 lmh_status run_finalize(const Plan& P, int kind, int64_t r0, int rows, const int32_t* labels,
                         float* lse, float* loss, float* logprob, int32_t* argmax, int write_scale,
-                        int mean, const int32_t* n_given, const Ws& ws, cudaStream_t st) {
+                        int mean, const int32_t* n_given, const Ws& ws, cudaStream_t st,
+                        const float* alpha = nullptr) {
   FinParams f;
   f.rows = rows;
   f.row0 = r0;
@@ -414,6 +416,7 @@ lmh_status run_finalize(const Plan& P, int kind, int64_t r0, int rows, const int
   f.n_given = n_given;
   f.h = ws.h;
   f.temp = P.temp;
+  f.alpha = alpha;
   const int warps = 8;
   ProfScope ps(KID_FINALIZE, st);
   finalize_rows_kernel<<<static_cast<unsigned>(cdiv(rows, warps)), 32 * warps, 0, st>>>(f);
@@ -601,7 +604,8 @@ extern "C" size_t lmh_workspace_size(const lmh_shape* shape, int entry) {
   if ((entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL) &&
       (shape->K < 1 || shape->K > LMH_MAX_K))
     return 0;
-  const bool fused = (entry == LMH_ENTRY_LOSS_FWD || entry == LMH_ENTRY_VP_PARTIALS) &&
+  const bool fused = (entry == LMH_ENTRY_LOSS_FWD || entry == LMH_ENTRY_VP_PARTIALS ||
+                      entry == LMH_ENTRY_SUPPORT_KL) &&
                      (shape->flags & LMH_F_FUSED_BWD);
   const bool want_acc = !(shape->flags & LMH_F_DW_ACC_GIVEN);
   return make_plan(shape, entry, fused, want_acc).total;
@@ -768,6 +772,90 @@ extern "C" lmh_status lmh_support_kl(const lmh_shape* shape, const lmh_bf16* H,
                                      size_t workspace_bytes, void* stream) {
   return support_fwd(shape, LMH_ENTRY_SUPPORT_KL, H, W, ids, ref_logp, lp, kl_rows, kl_mean, lse,
                      workspace, workspace_bytes, stream);
+}
+
+extern "C" lmh_status lmh_support_kl_fwd_bwd(const lmh_shape* shape, const lmh_bf16* H,
+                                             const lmh_bf16* W, const int32_t* ids,
+                                             const float* ref_logp, float* kl_rows,
+                                             float* kl_mean, float* lp, float* lse,
+                                             lmh_bf16* dH, lmh_bf16* dW, float* dW_acc,
+                                             void* workspace, size_t workspace_bytes,
+                                             void* stream) {
+  if (!shape_ok(shape) || shape->K < 1 || shape->K > LMH_MAX_K) return LMH_ERR_INVALID_ARG;
+  if (shape->flags & LMH_F_SUPPORT_RENORM) return LMH_ERR_INVALID_ARG;  // sparse path: two calls
+  const bool grads = dH || dW || dW_acc;
+  const Plan P = make_plan(shape, LMH_ENTRY_SUPPORT_KL, grads, dW && !dW_acc);
+  int dev, sms;
+  LMH_TRY(common_checks(shape, H, W, workspace, workspace_bytes, P.total, &dev, &sms));
+  if (P.N > 0 && (!ids || !lse || !ref_logp || !kl_rows)) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(dH) || !aligned16(dW) || !aligned16(dW_acc)) return LMH_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return empty_call(P, kl_mean, nullptr, dW, dW_acc, st);
+  LMH_TRY(prep_cands(P, ids, ws, st));
+  const int K = static_cast<int>(P.K);
+  float* alpha = grads ? ws.at<float>(P.o_alpha) : nullptr;
+  float* beta = grads ? ws.at<float>(P.o_beta) : nullptr;
+  if (grads) {
+    // the KL's coefficients depend on the reference log-probs only, not on lse: alpha_i =
+    // g_i sum_k exp(r_ik), beta_ic = g_i sum_{k: c_ik = c} exp(r_ik), g_i = 1 / N or 1
+    ProfScope ps(KID_BWD_COEF, st);
+    bwd_coef_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
+        LMH_BWD_SUPPORT_KL, P.N, K, static_cast<int>(P.V), ids, nullptr, ref_logp,
+        ws.at<int32_t>(P.o_rank), ws.at<int32_t>(P.o_nuniq), P.temp,
+        (shape->flags & LMH_F_MEAN) ? 1 : 0, 0, ws.h, alpha, beta);
+  }
+  LMH_TRY(last_launch());
+  Targets tg{};
+  tg.sorted = ws.at<int32_t>(P.o_sorted);
+  tg.nuniq = ws.at<int32_t>(P.o_nuniq);
+  tg.K = K;
+  for (int64_t ci = 0; ci < P.nchunks; ++ci) {
+    const int64_t r0 = ci * P.c;
+    const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
+    if (!grads) {
+      LMH_TRY((run_stats<kCands, false>(P, dev, sms, H, W, tg, r0, rows, ws, st)));
+      LMH_TRY(run_finalize(P, 2, r0, rows, nullptr, lse, nullptr, nullptr, nullptr, 0, 0,
+                           nullptr, ws, st));
+      continue;
+    }
+    LMH_TRY((run_stats<kCands, true>(P, dev, sms, H, W, tg, r0, rows, ws, st)));
+    LMH_TRY(run_finalize(P, 2, r0, rows, nullptr, lse, nullptr, nullptr, nullptr, 1, 0, nullptr,
+                         ws, st, alpha));
+    __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
+    {
+      const int64_t nv = P.Vp / 8;
+      const int64_t bx = cdiv(nv, kGbuildThreads * kGbuildVec);
+      dim3 grid(static_cast<unsigned>(bx < 64 ? bx : 64),
+                static_cast<unsigned>(rows < 65535 ? rows : 65535));
+      ProfScope ps(KID_GBUILD, st);
+      gbuild_kernel<<<grid, kGbuildThreads, 0, st>>>(rows, P.Vp, static_cast<int>(P.T),
+                                                     ws.at<float>(P.o_ps), G);
+    }
+    LMH_TRY(last_launch());
+    {
+      ProfScope ps(KID_FIX_CANDS, st);
+      fix_cands_kernel<<<static_cast<unsigned>(cdiv(rows, 8)), 256, 0, st>>>(
+          rows, r0, K, P.Vp, ws.at<int32_t>(P.o_sorted), ws.at<int32_t>(P.o_nuniq),
+          ws.at<float>(P.o_zt), lse, alpha, beta, G);
+    }
+    LMH_TRY(last_launch());
+    LMH_TRY(run_backward_gemms(P, dev, sms, H, W, r0, rows, static_cast<int>(ci), dH, dW, dW_acc,
+                               ws, st));
+  }
+  {
+    ProfScope ps(KID_SUPPORT_OUT, st);
+    support_out_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
+        P.N, K, ws.at<int32_t>(P.o_rank), ws.at<float>(P.o_zt), lse, ref_logp, lp, kl_rows);
+  }
+  LMH_TRY(last_launch());
+  if (kl_mean) {
+    ProfScope ps(KID_MEAN, st);
+    mean_kernel<<<1, 1024, 0, st>>>(kl_rows, P.N, 0, nullptr, ws.h, kl_mean);
+    LMH_TRY(last_launch());
+  }
+  return LMH_OK;
 }
 
 extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,

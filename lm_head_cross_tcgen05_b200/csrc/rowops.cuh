@@ -140,6 +140,7 @@ struct FinParams {
   const int32_t* n_given;
   WsHeader* h;
   Temperature temp;
+  const float* alpha;  // write_scale: alpha_i given per row (it includes 1 / tau_i), or null
 };
 
 __global__ void finalize_rows_kernel(const FinParams p) {
@@ -183,7 +184,8 @@ __global__ void finalize_rows_kernel(const FinParams p) {
     if (lane == 0) p.argmax[grow] = (tfirst < p.T) ? p.part_i[static_cast<long long>(row) * p.T + tfirst] : 0;
   }
   if (p.write_scale) {
-    const float a = row_weight(valid, p.mean, p.n_given, p.h) * inv_temperature(p.temp, grow);
+    const float a = p.alpha ? p.alpha[grow]
+                            : row_weight(valid, p.mean, p.n_given, p.h) * inv_temperature(p.temp, grow);
     const float loff = -lse * kLog2e;
     for (int t = lane; t < p.T; t += 32) ps[t] = a * fast_exp2(fmaf(pm[t], kLog2e, loff));
   }
@@ -244,6 +246,29 @@ __global__ void fix_labels_kernel(int rows, long long row0, int V, long long ldp
   const float a = row_weight(true, mean, n_given, h) * inv_temperature(temp, g);
   const float v = a * fast_exp2(fmaf(zt[g], kLog2e, -lse[g] * kLog2e)) - a;
   P[r * ldp + y] = __float2bfloat16_rn(v);
+}
+
+// Candidate columns of each row (fused support backward), one warp per row:
+// G = alpha_i exp(z_ic - lse_i) - beta_ic at every distinct valid candidate c, from the fp32
+// logit (zt and beta are indexed by the sorted candidate position).
+__global__ void fix_cands_kernel(int rows, long long row0, int K, long long ldp,
+                                 const int32_t* __restrict__ sorted,
+                                 const int32_t* __restrict__ nuniq,
+                                 const float* __restrict__ zt, const float* __restrict__ lse,
+                                 const float* __restrict__ alpha,
+                                 const float* __restrict__ beta,
+                                 __nv_bfloat16* __restrict__ P) {
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const long long g = row0 + r;
+  const int nu = nuniq[g];
+  const float a = alpha[g], loff = -lse[g] * kLog2e;
+  for (int u = lane; u < nu; u += 32) {
+    const long long o = g * K + u;
+    const float v = a * fast_exp2(fmaf(zt[o], kLog2e, loff)) - beta[o];
+    P[r * ldp + sorted[o]] = __float2bfloat16_rn(v);
+  }
 }
 
 // ---------------------------------------------------------------------------- means

@@ -494,3 +494,54 @@ def test_same_bits_in_a_new_process():
     s = L.support_kl(x["H"], x["W"], ids, torch.full((520, 2), -0.7, device="cuda"))
     mine = digest(o["loss_rows"], o["lse"], o["argmax"], o["dH"], o["dW"], s["kl_rows"], s["lp"])
     assert here.stdout.strip().splitlines()[-1] == again.stdout.strip().splitlines()[-1] == mine
+
+
+@pytest.mark.parametrize("N,d,V,K,chunk,tau", [
+    (200, 192, 3000, 16, 0, None),
+    (300, 128, 5000, 8, 128, "rows"),   # three chunks: the internal dW accumulator
+    (64, 256, 2048, 64, 0, "scalar"),
+])
+def test_support_kl_fused_backward(N, d, V, K, chunk, tau):
+    x, xc = device_inputs(ragged(N, d, V, seed=4800 + N, K=K))
+    ids = x["ids"].clone()
+    ids[0, -1] = -1                      # padding
+    ids[1, 1] = ids[1, 0]                # a repeated id counts once per slot
+    ids_c = ids.cpu()
+    t_dev, t_ref = _temps(tau, N) if tau else (None, None)
+    out = L.support_kl(x["H"], x["W"], ids, x["ref_logp"], chunk_rows=chunk, temperature=t_dev,
+                       grads=True)
+    torch.cuda.synchronize()
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    rk = O.support_kl(xc["H"], xc["W"], ids_c, xc["ref_logp"], tau=t_ref)
+    check_rows(out["kl_rows"], rk["kl_rows"], what="kl_rows")
+    check_rows(out["kl_mean"], np.array([rk["kl_mean"]]), what="kl_mean")
+    check_rows(out["lp"], rk["lp"], what="lp")
+    check_rows(out["lse"], rk["lse"], what="lse")
+    ref = O.backward(O.BWD_SUPPORT_KL, xc["H"], xc["W"], ids_c, np.full(N, 1.0 / N),
+                     xc["ref_logp"], tau=t_ref)
+    check_grad(out["dH"], ref["dH"], "dH")
+    check_grad(out["dW"], ref["dW"], "dW")
+    # the two-call path: the same forward bits, the same gradients to rounding
+    f = L.support_kl(x["H"], x["W"], ids, x["ref_logp"], chunk_rows=chunk, temperature=t_dev)
+    assert torch.equal(f["kl_rows"], out["kl_rows"]) and torch.equal(f["lse"], out["lse"])
+    b = L.loss_bwd(L.BWD_SUPPORT_KL, x["H"], x["W"], ids, f["lse"], None, x["ref_logp"],
+                   chunk_rows=chunk, temperature=t_dev, mean=True)
+    check_grad(out["dH"], b["dH"], "dH fused vs two calls")
+    check_grad(out["dW"], b["dW"], "dW fused vs two calls")
+    again = L.support_kl(x["H"], x["W"], ids, x["ref_logp"], chunk_rows=chunk,
+                         temperature=t_dev, grads=True)
+    assert torch.equal(again["dH"], out["dH"]) and torch.equal(again["dW"], out["dW"])
+
+
+def test_support_kl_fused_sum_caller_accumulator_and_renorm_refused():
+    N, d, V, K = 120, 128, 1500, 8
+    x, xc = device_inputs(ragged(N, d, V, seed=4900, K=K))
+    acc = torch.zeros(V, d, dtype=torch.float32, device="cuda")
+    out = L.support_kl(x["H"], x["W"], x["ids"], x["ref_logp"], chunk_rows=50, grads=True,
+                       mean=False, dW_acc=acc)
+    ref = O.backward(O.BWD_SUPPORT_KL, xc["H"], xc["W"], xc["ids"], np.ones(N), xc["ref_logp"])
+    check_grad(acc, ref["dW"], "dW_acc")
+    assert torch.equal(out["dW"], acc.to(torch.bfloat16))
+    check_grad(out["dH"], ref["dH"], "dH")
+    with pytest.raises(L.LmhError, match="INVALID_ARG"):
+        L.support_kl(x["H"], x["W"], x["ids"], x["ref_logp"], grads=True, renorm=True)
