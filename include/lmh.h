@@ -90,6 +90,7 @@ typedef enum lmh_status {
 #define LMH_ENTRY_VP_PARTIALS 5 /* vocabulary-parallel entries, below */
 #define LMH_ENTRY_VP_COMBINE 6
 #define LMH_ENTRY_VP_BWD 7
+#define LMH_ENTRY_LOSS_FWD_BWD 8
 
 /* objectives of lmh_loss_bwd */
 #define LMH_BWD_CE 0              /* L = sum_i g_i loss_i                                */
@@ -182,6 +183,26 @@ LMH_API lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_bf16
                         const lmh_bf16* W, const int32_t* targets, const float* lse,
                         const float* grad, const float* ref_logp, lmh_bf16* dH, lmh_bf16* dW,
                         float* dW_acc, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * lmh_loss_fwd_bwd — lmh_loss_fwd with the fused backward of a weighted row objective known
+ * before the call: L = sum_i w_i loss_i (mode LMH_BWD_CE) or L = sum_i w_i logprob_i (mode
+ * LMH_BWD_LOGPROB), e.g. a policy-gradient loss whose per-row weights (advantages) are fixed
+ * before the forward (FlashInfer PR #8059, description: "the CE and policy losses"). The
+ * weights are those of lmh_loss_bwd: w_i = grad[i]; one shared grad[0] with
+ * LMH_F_GRAD_SCALAR; 1 with grad NULL; each times 1 / count with LMH_F_MEAN, the count
+ * being *n_valid_given if given, else the valid rows. Ignored rows get 0. The forward outputs
+ * are those of lmh_loss_fwd (loss_mean is always the mean loss); dH, dW, dW_acc as there.
+ * The softmax is reused as in lmh_loss_fwd's fused path: three GEMMs per chunk.
+ * Workspace: lmh_workspace_size(shape, LMH_ENTRY_LOSS_FWD_BWD) with LMH_F_FUSED_BWD.
+ */
+LMH_API lmh_status lmh_loss_fwd_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,
+                                    const lmh_bf16* W, const int32_t* labels, const float* grad,
+                                    float* loss_rows, float* lse, float* logprob,
+                                    int32_t* argmax, float* loss_mean, int32_t* n_valid,
+                                    const int32_t* n_valid_given, lmh_bf16* dH, lmh_bf16* dW,
+                                    float* dW_acc, void* workspace, size_t workspace_bytes,
+                                    void* stream);
 
 /*
  * lmh_logprob — per-row target log-probability (FlashInfer PR #8059, description:

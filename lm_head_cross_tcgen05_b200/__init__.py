@@ -19,7 +19,8 @@ import torch
 from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEVERR_LABEL_RANGE,
                    DEVERR_NONFINITE, DEVERR_TEMPERATURE, DEVERR_TIMEOUT, ENTRY_LOGPROB, ENTRY_LOSS_BWD,
                    ENTRY_LOSS_FWD, ENTRY_SUPPORT_KL, ENTRY_SUPPORT_LOGPROB, ENTRY_VP_BWD,
-                   ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN, F_GRAD_SCALAR,
+                   ENTRY_LOSS_FWD_BWD, ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN,
+                   F_GRAD_SCALAR,
                    F_FUSED_BWD, F_MEAN, F_SUPPORT_RENORM, IGNORE_INDEX, MAX_K, STATUS_NAMES, lib, lmh_shape)
 
 __all__ = [
@@ -34,6 +35,7 @@ __all__ = [
     "lmh_vp_partials", "lmh_vp_combine", "lmh_vp_loss_bwd", "lmh_vp_fused_bwd",
     "lmh_vp_reduce_rows",
     "ENTRY_VP_PARTIALS", "ENTRY_VP_COMBINE", "ENTRY_VP_BWD", "F_GRAD_SCALAR",
+    "ENTRY_LOSS_FWD_BWD", "lmh_loss_fwd_bwd", "loss_fwd_bwd",
 ]
 
 lib()  # load now: a missing library is an import error, never a silent fallback
@@ -132,6 +134,26 @@ def lmh_loss_bwd(shape, mode, H, W, targets, lse, grad, ref_logp=None, dH=None, 
         _p(dW_acc, _f32, "dW_acc"), _p(workspace, _u8, "workspace"), workspace.numel(),
         _s(stream))
     _ok("lmh_loss_bwd", st)
+
+
+def lmh_loss_fwd_bwd(shape, mode, H, W, labels, grad, loss_rows, lse, logprob=None,
+                     argmax=None, loss_mean=None, n_valid=None, n_valid_given=None, dH=None,
+                     dW=None, dW_acc=None, *, workspace, stream=None) -> None:
+    N, d, V = shape.N, shape.d, shape.V
+    _fits(H=(H, N * d), W=(W, V * d), labels=(labels, N),
+          grad=(grad, 1 if shape.flags & F_GRAD_SCALAR else N), loss_rows=(loss_rows, N),
+          lse=(lse, N), logprob=(logprob, N), argmax=(argmax, N), loss_mean=(loss_mean, 1),
+          n_valid=(n_valid, 1), n_valid_given=(n_valid_given, 1), dH=(dH, N * d),
+          dW=(dW, V * d), dW_acc=(dW_acc, V * d))
+    st = lib().lmh_loss_fwd_bwd(
+        ctypes.byref(shape), int(mode), _p(H, _bf, "H"), _p(W, _bf, "W"),
+        _p(labels, _i32, "labels"), _p(grad, _f32, "grad"), _p(loss_rows, _f32, "loss_rows"),
+        _p(lse, _f32, "lse"), _p(logprob, _f32, "logprob"), _p(argmax, _i32, "argmax"),
+        _p(loss_mean, _f32, "loss_mean"), _p(n_valid, _i32, "n_valid"),
+        _p(n_valid_given, _i32, "n_valid_given"), _p(dH, _bf, "dH"), _p(dW, _bf, "dW"),
+        _p(dW_acc, _f32, "dW_acc"), _p(workspace, _u8, "workspace"), workspace.numel(),
+        _s(stream))
+    _ok("lmh_loss_fwd_bwd", st)
 
 
 def lmh_logprob(shape, H, W, labels, logprob, lse, *, workspace, stream=None) -> None:
@@ -292,6 +314,34 @@ def loss_fwd(H, W, labels, *, chunk_rows: int = 0, mean: bool = True, grads: boo
     lmh_loss_fwd(shape, H, W, labels, out["loss_rows"], out["lse"], out["logprob"],
                  out["argmax"], out["loss_mean"], out["n_valid"], n_valid_given,
                  out.get("dH"), out.get("dW"), dW_acc, workspace=ws, stream=stream)
+    out["workspace"] = ws
+    return out
+
+
+def loss_fwd_bwd(mode: int, H, W, labels, grad=None, *, chunk_rows: int = 0,
+                 mean: bool = False, scalar_grad: bool = False, dW_acc=None,
+                 n_valid_given=None, temperature=None, ws=None, stream=None) -> dict:
+    """Forward outputs plus dH, dW of L = sum_i w_i l_i (l = loss for BWD_CE, log-prob for
+    BWD_LOGPROB; w from grad as in loss_bwd) in one pass: the fused path for objectives whose
+    row weights are known before the forward, such as policy-gradient losses."""
+    N, d = H.shape
+    V = W.shape[0]
+    dev = H.device
+    flags = (F_FUSED_BWD | (F_MEAN if mean else 0) | (F_GRAD_SCALAR if scalar_grad else 0)
+             | (F_DW_ACC_GIVEN if dW_acc is not None else 0))
+    shape = make_shape(N, d, V, 0, chunk_rows, flags, temperature)
+    out = dict(loss_rows=torch.empty(N, dtype=_f32, device=dev),
+               lse=torch.empty(N, dtype=_f32, device=dev),
+               logprob=torch.empty(N, dtype=_f32, device=dev),
+               argmax=torch.empty(N, dtype=_i32, device=dev),
+               loss_mean=torch.empty(1, dtype=_f32, device=dev),
+               n_valid=torch.empty(1, dtype=_i32, device=dev),
+               dH=torch.empty(N, d, dtype=_bf, device=dev),
+               dW=torch.empty(V, d, dtype=_bf, device=dev))
+    ws = workspace(shape, ENTRY_LOSS_FWD_BWD, dev) if ws is None else ws
+    lmh_loss_fwd_bwd(shape, mode, H, W, labels, grad, out["loss_rows"], out["lse"],
+                     out["logprob"], out["argmax"], out["loss_mean"], out["n_valid"],
+                     n_valid_given, out["dH"], out["dW"], dW_acc, workspace=ws, stream=stream)
     out["workspace"] = ws
     return out
 

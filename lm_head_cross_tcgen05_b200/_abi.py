@@ -21,7 +21,7 @@ IGNORE_INDEX = -100
 DEVERR_LABEL_RANGE, DEVERR_TIMEOUT, DEVERR_NONFINITE, DEVERR_TEMPERATURE = 0x1, 0x2, 0x4, 0x8
 F_MEAN, F_FUSED_BWD, F_DW_ACC_GIVEN, F_SUPPORT_RENORM, F_GRAD_SCALAR = 0x1, 0x2, 0x4, 0x8, 0x10
 ENTRY_LOSS_FWD, ENTRY_LOSS_BWD, ENTRY_LOGPROB, ENTRY_SUPPORT_LOGPROB, ENTRY_SUPPORT_KL = range(5)
-ENTRY_VP_PARTIALS, ENTRY_VP_COMBINE, ENTRY_VP_BWD = 5, 6, 7
+ENTRY_VP_PARTIALS, ENTRY_VP_COMBINE, ENTRY_VP_BWD, ENTRY_LOSS_FWD_BWD = 5, 6, 7, 8
 BWD_CE, BWD_LOGPROB, BWD_SUPPORT_LOGPROB, BWD_SUPPORT_KL = range(4)
 MAX_K = 1024
 
@@ -37,6 +37,7 @@ _SIGS = {
     "lmh_workspace_size": (c_size_t, [ctypes.POINTER(lmh_shape), c_int]),
     "lmh_loss_fwd": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 14 + [c_size_t, _P]),
     "lmh_loss_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 10 + [c_size_t, _P]),
+    "lmh_loss_fwd_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 15 + [c_size_t, _P]),
     "lmh_logprob": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6 + [c_size_t, _P]),
     "lmh_support_logprob": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6 + [c_size_t, _P]),
     "lmh_support_kl": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 9 + [c_size_t, _P]),

@@ -89,7 +89,8 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   p.K = p.cands ? (s->K > 0 ? s->K : 1) : 1;
   p.renorm = p.cands && (s->flags & LMH_F_SUPPORT_RENORM);
   const bool fwd_fused = fused && (entry == LMH_ENTRY_LOSS_FWD || entry == LMH_ENTRY_VP_PARTIALS ||
-                                   entry == LMH_ENTRY_SUPPORT_KL);
+                                   entry == LMH_ENTRY_SUPPORT_KL ||
+                                   entry == LMH_ENTRY_LOSS_FWD_BWD);
   p.gbuf = !p.renorm && (bwd || fwd_fused);
   p.acc = p.gbuf && dw_without_acc && p.nchunks > 1;
   const bool stats = !bwd && entry != LMH_ENTRY_VP_COMBINE;
@@ -109,7 +110,8 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   p.o_pm = partials ? take(cT * 4) : 0;
   p.o_ps = partials ? take(cT * 4) : 0;
   p.o_pi = partials ? take(cT * 4) : 0;
-  const bool coef = bwd || (fwd_fused && entry == LMH_ENTRY_SUPPORT_KL);
+  const bool coef = bwd || (fwd_fused && (entry == LMH_ENTRY_SUPPORT_KL ||
+                                          entry == LMH_ENTRY_LOSS_FWD_BWD));
   p.o_alpha = coef ? take(N * 4) : 0;
   p.o_beta = coef ? take(N * p.K * 4) : 0;
   p.o_lloc = (vp_bwd || entry == LMH_ENTRY_VP_PARTIALS) ? take(N * 4) : 0;
@@ -600,36 +602,53 @@ lmh_status empty_call(const Plan& P, float* mean_out, int32_t* nvalid_out, lmh_b
 // ============================================================================ C ABI
 
 extern "C" size_t lmh_workspace_size(const lmh_shape* shape, int entry) {
-  if (!shape_ok(shape) || entry < LMH_ENTRY_LOSS_FWD || entry > LMH_ENTRY_VP_BWD) return 0;
+  if (!shape_ok(shape) || entry < LMH_ENTRY_LOSS_FWD || entry > LMH_ENTRY_LOSS_FWD_BWD) return 0;
   if ((entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL) &&
       (shape->K < 1 || shape->K > LMH_MAX_K))
     return 0;
   const bool fused = (entry == LMH_ENTRY_LOSS_FWD || entry == LMH_ENTRY_VP_PARTIALS ||
-                      entry == LMH_ENTRY_SUPPORT_KL) &&
+                      entry == LMH_ENTRY_SUPPORT_KL || entry == LMH_ENTRY_LOSS_FWD_BWD) &&
                      (shape->flags & LMH_F_FUSED_BWD);
   const bool want_acc = !(shape->flags & LMH_F_DW_ACC_GIVEN);
   return make_plan(shape, entry, fused, want_acc).total;
 }
 
-extern "C" lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,
-                                   const int32_t* labels, float* loss_rows, float* lse,
-                                   float* logprob, int32_t* argmax, float* loss_mean,
-                                   int32_t* n_valid, const int32_t* n_valid_given, lmh_bf16* dH,
-                                   lmh_bf16* dW, float* dW_acc, void* workspace,
-                                   size_t workspace_bytes, void* stream) {
+// The CE forward, and with dH / dW its fused backward. weighted: the backward is that of
+// L = sum_i w_i l_i for the objective `mode` (loss or log-prob rows), with the row weights and
+// target coefficients from bwd_coef_kernel; otherwise of the mean (or summed) loss.
+static lmh_status loss_fwd_impl(const lmh_shape* shape, bool weighted, int mode,
+                                const float* grad, const lmh_bf16* H, const lmh_bf16* W,
+                                const int32_t* labels, float* loss_rows, float* lse,
+                                float* logprob, int32_t* argmax, float* loss_mean,
+                                int32_t* n_valid, const int32_t* n_valid_given, lmh_bf16* dH,
+                                lmh_bf16* dW, float* dW_acc, void* workspace,
+                                size_t workspace_bytes, void* stream) {
   if (!shape_ok(shape)) return LMH_ERR_INVALID_ARG;
   const bool fused = dH || dW || dW_acc;
-  const Plan P = make_plan(shape, LMH_ENTRY_LOSS_FWD, fused, dW && !dW_acc);
+  const Plan P = make_plan(shape, weighted ? LMH_ENTRY_LOSS_FWD_BWD : LMH_ENTRY_LOSS_FWD, fused,
+                           dW && !dW_acc);
   int dev, sms;
   LMH_TRY(common_checks(shape, H, W, workspace, workspace_bytes, P.total, &dev, &sms));
   if (P.N > 0 && (!labels || !loss_rows || !lse)) return LMH_ERR_INVALID_ARG;
   if (!aligned16(dH) || !aligned16(dW) || !aligned16(dW_acc)) return LMH_ERR_ALIGNMENT;
+  if (weighted && (shape->flags & LMH_F_GRAD_SCALAR) && !grad) return LMH_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
   LMH_TRY(clear_header(ws, st));
   if (P.N == 0) return empty_call(P, loss_mean, n_valid, dW, dW_acc, st);
   LMH_TRY(count_labels(P, labels, ws, st));
   const int mean = (shape->flags & LMH_F_MEAN) ? 1 : 0;
+  float* alpha = nullptr;
+  float* beta = nullptr;
+  if (fused && weighted) {
+    alpha = ws.at<float>(P.o_alpha);
+    beta = ws.at<float>(P.o_beta);
+    ProfScope ps(KID_BWD_COEF, st);
+    bwd_coef_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
+        mode, P.N, 1, static_cast<int>(P.V), labels, grad, nullptr, nullptr, nullptr, P.temp,
+        mean, (shape->flags & LMH_F_GRAD_SCALAR) ? 1 : 0, ws.h, alpha, beta, n_valid_given);
+  }
+  LMH_TRY(last_launch());
   Targets tg{};
   tg.labels = labels;
   tg.K = 1;
@@ -642,7 +661,7 @@ extern "C" lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, co
       LMH_TRY((run_stats<kLabel, false>(P, dev, sms, H, W, tg, r0, rows, ws, st)));
     }
     LMH_TRY(run_finalize(P, 0, r0, rows, labels, lse, loss_rows, logprob, argmax, fused ? 1 : 0,
-                         mean, n_valid_given, ws, st));
+                         mean, n_valid_given, ws, st, alpha));
     if (fused) {
       __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
       const int64_t nv = P.Vp / 8;
@@ -659,7 +678,7 @@ extern "C" lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, co
         ProfScope ps(KID_FIX_LABELS, st);
         fix_labels_kernel<<<static_cast<unsigned>(cdiv(rows, 256)), 256, 0, st>>>(
             rows, r0, static_cast<int>(P.V), P.Vp, labels, ws.at<float>(P.o_zt), lse, mean,
-            n_valid_given, ws.h, P.temp, G);
+            n_valid_given, ws.h, P.temp, G, alpha, beta);
       }
       LMH_TRY(last_launch());
       LMH_TRY(run_backward_gemms(P, dev, sms, H, W, r0, rows, static_cast<int>(ci), dH, dW,
@@ -675,6 +694,30 @@ extern "C" lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, co
       cudaMemcpyAsync(n_valid, &ws.h->n_valid, 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return LMH_ERR_CUDA;
   return LMH_OK;
+}
+
+extern "C" lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,
+                                   const int32_t* labels, float* loss_rows, float* lse,
+                                   float* logprob, int32_t* argmax, float* loss_mean,
+                                   int32_t* n_valid, const int32_t* n_valid_given, lmh_bf16* dH,
+                                   lmh_bf16* dW, float* dW_acc, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return loss_fwd_impl(shape, false, LMH_BWD_CE, nullptr, H, W, labels, loss_rows, lse, logprob,
+                       argmax, loss_mean, n_valid, n_valid_given, dH, dW, dW_acc, workspace,
+                       workspace_bytes, stream);
+}
+
+extern "C" lmh_status lmh_loss_fwd_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,
+                                       const lmh_bf16* W, const int32_t* labels,
+                                       const float* grad, float* loss_rows, float* lse,
+                                       float* logprob, int32_t* argmax, float* loss_mean,
+                                       int32_t* n_valid, const int32_t* n_valid_given,
+                                       lmh_bf16* dH, lmh_bf16* dW, float* dW_acc,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (mode != LMH_BWD_CE && mode != LMH_BWD_LOGPROB) return LMH_ERR_INVALID_ARG;
+  return loss_fwd_impl(shape, true, mode, grad, H, W, labels, loss_rows, lse, logprob, argmax,
+                       loss_mean, n_valid, n_valid_given, dH, dW, dW_acc, workspace,
+                       workspace_bytes, stream);
 }
 
 extern "C" lmh_status lmh_logprob(const lmh_shape* shape, const lmh_bf16* H, const lmh_bf16* W,

@@ -232,19 +232,23 @@ __global__ void __launch_bounds__(kGbuildThreads)
   }
 }
 
-// Label column of each valid row: G = alpha exp(z_y - lse) - alpha, from the fp32 logit.
+// Label column of each valid row: G = alpha exp(z_y - lse) - beta, from the fp32 logit, with
+// alpha = beta = the mean / sum weight of the row over tau_i, or alpha_i, beta_i given.
 __global__ void fix_labels_kernel(int rows, long long row0, int V, long long ldp,
                                   const int32_t* __restrict__ labels,
                                   const float* __restrict__ zt, const float* __restrict__ lse,
                                   int mean, const int32_t* n_given, const WsHeader* h,
-                                  Temperature temp, __nv_bfloat16* __restrict__ P) {
+                                  Temperature temp, __nv_bfloat16* __restrict__ P,
+                                  const float* __restrict__ alpha = nullptr,
+                                  const float* __restrict__ beta = nullptr) {
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= rows) return;
   const long long g = row0 + r;
   const int y = labels[g];
   if (y < 0 || y >= V) return;
-  const float a = row_weight(true, mean, n_given, h) * inv_temperature(temp, g);
-  const float v = a * fast_exp2(fmaf(zt[g], kLog2e, -lse[g] * kLog2e)) - a;
+  const float a = alpha ? alpha[g] : row_weight(true, mean, n_given, h) * inv_temperature(temp, g);
+  const float b = beta ? beta[g] : a;
+  const float v = a * fast_exp2(fmaf(zt[g], kLog2e, -lse[g] * kLog2e)) - b;
   P[r * ldp + y] = __float2bfloat16_rn(v);
 }
 
@@ -329,7 +333,7 @@ __global__ void bwd_coef_kernel(int mode, long long N, int K, int V,
                                 const int32_t* __restrict__ rank,
                                 const int32_t* __restrict__ nuniq, Temperature temp, int mean,
                                 int scalar, WsHeader* h, float* __restrict__ alpha,
-                                float* __restrict__ beta) {
+                                float* __restrict__ beta, const int32_t* n_given = nullptr) {
   const int lane = threadIdx.x & 31;
   const long long i = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5);
   if (i >= N) return;
@@ -337,7 +341,7 @@ __global__ void bwd_coef_kernel(int mode, long long N, int K, int V,
   if (lane == 0 && temp.rows && !temperature_ok(temp.rows[i])) atomicOr(&h->err, kErrTemperature);
   float unit = 1.f;  // weight of a row term when no per-term grad is given
   if (mean) {
-    const long long cnt = (mode <= 1) ? h->n_valid : N;
+    const long long cnt = n_given ? *n_given : (mode <= 1) ? h->n_valid : N;
     unit = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
   }
   if (scalar) {

@@ -28,7 +28,7 @@ def test_invalid_shapes_size_zero():
     assert ws(10, 64, 0) == 0
     assert ws(10, 64, 100, K=0, entry=L.ENTRY_SUPPORT_KL) == 0
     assert ws(10, 64, 100, K=L.MAX_K + 1, entry=L.ENTRY_SUPPORT_LOGPROB) == 0
-    assert ws(10, 64, 100, entry=8) == 0
+    assert ws(10, 64, 100, entry=9) == 0
     assert ws(10, 64, 100, entry=-1) == 0
 
 
@@ -125,3 +125,11 @@ def test_binding_rejects_tensors_smaller_than_the_shape():
                               torch.zeros(4, 8), f, workspace=ws)
     with pytest.raises(ValueError, match="records has"):
         L.lmh_vp_combine(shape, 3, torch.zeros(2, 4, 4), y, f, f, workspace=ws)
+
+
+def test_weighted_fused_size_adds_row_coefficients():
+    # lmh_loss_fwd_bwd's plan: the fused forward's plus alpha [N] and beta [N] fp32
+    f = ws(1000, 64, 5000, chunk=1000, flags=L.F_FUSED_BWD | L.F_DW_ACC_GIVEN)
+    w = ws(1000, 64, 5000, chunk=1000, flags=L.F_FUSED_BWD | L.F_DW_ACC_GIVEN,
+           entry=L.ENTRY_LOSS_FWD_BWD)
+    assert w - f == 2 * 4096

@@ -545,3 +545,45 @@ def test_support_kl_fused_sum_caller_accumulator_and_renorm_refused():
     check_grad(out["dH"], ref["dH"], "dH")
     with pytest.raises(L.LmhError, match="INVALID_ARG"):
         L.support_kl(x["H"], x["W"], x["ids"], x["ref_logp"], grads=True, renorm=True)
+
+
+@pytest.mark.parametrize("mode", [L.BWD_CE, L.BWD_LOGPROB])
+@pytest.mark.parametrize("chunk", [0, 100])
+def test_weighted_fused_objective(mode, chunk):
+    # a policy-gradient-like objective: per-row weights known before the forward
+    N, d, V = 300, 192, 2000
+    x, xc = device_inputs(_wl(N, d, V, 7))
+    g = torch.linspace(-1.5, 1.0, N, dtype=torch.float32)
+    out = L.loss_fwd_bwd(mode, x["H"], x["W"], x["labels"], g.cuda(), chunk_rows=chunk)
+    torch.cuda.synchronize()
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    f = O.ce_forward(xc["H"], xc["W"], xc["labels"])
+    check_rows(out["loss_rows"], f["loss_rows"], what="loss_rows")
+    check_rows(out["lse"], f["lse"], what="lse")
+    ref = O.backward(mode, xc["H"], xc["W"], xc["labels"], g.numpy())
+    check_grad(out["dH"], ref["dH"], "dH")
+    check_grad(out["dW"], ref["dW"], "dW")
+    fwd = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=chunk)
+    assert torch.equal(fwd["lse"], out["lse"]) and torch.equal(fwd["loss_rows"], out["loss_rows"])
+    b = L.loss_bwd(mode, x["H"], x["W"], x["labels"], out["lse"], g.cuda(), chunk_rows=chunk)
+    check_grad(out["dH"], b["dH"], "dH fused vs standalone")
+    check_grad(out["dW"], b["dW"], "dW fused vs standalone")
+
+
+def test_weighted_fused_scalar_mean_count_and_temperature():
+    N, d, V = 260, 128, 1500
+    x, xc = device_inputs(_wl(N, d, V, 11))
+    t_dev, t_ref = _temps("rows", N)
+    n = torch.tensor([77], dtype=torch.int32, device="cuda")
+    g = torch.tensor([2.5], dtype=torch.float32, device="cuda")
+    out = L.loss_fwd_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], g, mean=True, scalar_grad=True,
+                         n_valid_given=n, temperature=t_dev, chunk_rows=128)
+    valid = xc["labels"].numpy() >= 0
+    w = np.where(valid, 2.5 / 77, 0.0)
+    ref = O.backward(O.BWD_CE, xc["H"], xc["W"], xc["labels"], w, tau=t_ref)
+    check_grad(out["dH"], ref["dH"], "dH")
+    check_grad(out["dW"], ref["dW"], "dW")
+    # without weights and with the mean: the same bits as lmh_loss_fwd's fused path
+    a = L.loss_fwd_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], None, mean=True, chunk_rows=128)
+    b = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=128, grads=True)
+    assert torch.equal(a["dH"], b["dH"]) and torch.equal(a["dW"], b["dW"])
