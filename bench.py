@@ -55,6 +55,8 @@ def parse_args():
                     help="rows per chunk (the memory budget); 0: the workload's own plan")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="--impl reference: total oracle time the timed and warm-up steps share")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -232,7 +234,7 @@ def oracle_sample(wl, target_s: float, entry="fused_ce"):
 def run_reference(args, wl, n_gpus):
     """The oracle as it stands, on the host cores, steps of a bounded sample."""
     run, what = oracle_runner(wl, args.entry)
-    budget = 150.0 / max(1, args.steps + args.warmup)       # seconds per step
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)       # seconds per step
     n = _rows_for(run, budget, 4, 20)
     for _ in range(args.warmup):
         run(n)

@@ -52,3 +52,27 @@ def test_single_rank_helpers():
     import bench
     assert bench.reduce_max(3.5, 1) == 3.5
     assert bench.job_tflops(1e12, 1, 1.0) == pytest.approx(1000.0)
+
+
+@pytest.mark.parametrize("entry", ["fused_ce", "ce_separate"])
+def test_reference_arm_json_line(entry):
+    # bench.py --impl reference: the oracle on the host cores, one JSON line with the keys the
+    # reference arm reports (no GPU needed)
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    wl = "tiny"
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", wl,
+                        "--entry", entry, "--steps", "1", "--warmup", "1",
+                        "--ref-seconds", "4"],
+                       capture_output=True, text=True, timeout=600, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["impl"] == "reference" and line["value"] > 0 and line["dtype"] == "f64"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["entry"] == entry
