@@ -248,6 +248,23 @@ LMH_API lmh_status lmh_support_kl(const lmh_shape* shape, const lmh_bf16* H, con
                           size_t workspace_bytes, void* stream);
 
 /*
+ * Row scatter of the shards' dH contributions (instead of dH_part, see lmh_vp_loss_bwd): the
+ * N rows form R consecutive slices (the first N % R hold one row more; slice j: rows
+ * [a_j, a_{j+1})), and rank j reduces slice j. recv is a DEVICE array of R pointers; recv[j]
+ * is rank j's receive buffer, [R][a_{j+1} - a_j][d] fp32, and this rank's rows land at slot
+ * `rank`. recv[j] may point into another GPU's memory (a peer mapping over NVLink, e.g.
+ * symmetric memory): the dH GEMM's epilogue writes each fp32 row there with ordinary stores
+ * while the GEMM runs, so the exchange needs no separate collective. The caller orders it:
+ * every rank's call must finish before rank j reduces its buffer (e.g. a barrier on the
+ * stream), and rank j then calls lmh_vp_reduce_rows_to.
+ */
+typedef struct lmh_vp_dest {
+  float* const* recv; /* [R] device array of receive buffers */
+  int32_t R;
+  int32_t rank;       /* this rank, 0 <= rank < R */
+} lmh_vp_dest;
+
+/*
  * Vocabulary-parallel cross entropy. The pages run the head at tensor-parallel size 1 only
  * (miles-ext-kernels PR #14, lm_head op commit: the validate hook's startup checks). These
  * entries split the same definitions over R ranks that each hold a contiguous row range
@@ -300,15 +317,17 @@ LMH_API lmh_status lmh_vp_combine(const lmh_shape* shape, int R, const float* re
  * lmh_vp_loss_bwd: the shard's part of lmh_loss_bwd (mode LMH_BWD_CE or LMH_BWD_LOGPROB; grad
  * nullable as there, with the count over the full vocabulary). lse [N] is the combined one.
  * dH_part [N, d] fp32 out (nullable): sum over the shard's columns of G_iv W_v, to be summed
- * over the ranks. dW_shard [V_r, d] bf16 out and dW_acc_shard [V_r, d] fp32 in/out (nullable,
- * as dW and dW_acc of lmh_loss_bwd). Workspace: lmh_workspace_size(shard, LMH_ENTRY_VP_BWD)
+ * over the ranks; or, with dest (then dH_part must be null), the same rows scattered to the
+ * ranks that reduce them. dW_shard [V_r, d] bf16 out and dW_acc_shard [V_r, d] fp32 in/out
+ * (nullable, as dW and dW_acc of lmh_loss_bwd). Workspace: lmh_workspace_size(shard, LMH_ENTRY_VP_BWD)
  * (with LMH_F_DW_ACC_GIVEN in shard->flags if dW_acc_shard is passed).
  */
 LMH_API lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t v0,
                                    int64_t V_total, const lmh_bf16* H, const lmh_bf16* W_shard,
                                    const int32_t* labels, const float* lse, const float* grad,
                                    float* dH_part, lmh_bf16* dW_shard, float* dW_acc_shard,
-                                   void* workspace, size_t workspace_bytes, void* stream);
+                                   const lmh_vp_dest* dest, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /*
  * lmh_vp_fused_bwd: the shard's backward of the summed loss (or of the mean over the valid
@@ -316,14 +335,15 @@ LMH_API lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t v0,
  * fused path does on one device: G = alpha_i exp(m_t - lse_i) p~ minus alpha_i at the label,
  * with the combined lse. Three GEMMs per step instead of the four of partials + lmh_vp_loss_bwd.
  * Call it with the same shard, flags and workspace as that lmh_vp_partials call, after it and
- * before the workspace is reused. n_valid_given (nullable) as in lmh_loss_fwd. Outputs as
- * lmh_vp_loss_bwd.
+ * before the workspace is reused. n_valid_given (nullable) as in lmh_loss_fwd. Outputs (and
+ * dest) as lmh_vp_loss_bwd.
  */
 LMH_API lmh_status lmh_vp_fused_bwd(const lmh_shape* shard, int64_t v0, int64_t V_total,
                                     const lmh_bf16* H, const lmh_bf16* W_shard,
                                     const int32_t* labels, const float* lse,
                                     const int32_t* n_valid_given, float* dH_part,
-                                    lmh_bf16* dW_shard, float* dW_acc_shard, void* workspace,
+                                    lmh_bf16* dW_shard, float* dW_acc_shard,
+                                    const lmh_vp_dest* dest, void* workspace,
                                     size_t workspace_bytes, void* stream);
 
 /*
@@ -333,6 +353,16 @@ LMH_API lmh_status lmh_vp_fused_bwd(const lmh_shape* shard, int64_t v0, int64_t 
  */
 LMH_API lmh_status lmh_vp_reduce_rows(int R, int64_t rows, int64_t d, const float* parts,
                                       lmh_bf16* out, void* stream);
+
+/*
+ * lmh_vp_reduce_rows_to: the same sum, stored into n_out outputs at row row_offset: outs is a
+ * DEVICE array of n_out pointers to [*, d] bf16 buffers, which may be other GPUs' memory (each
+ * rank's full dH, so that rank j's reduced slice reaches every rank with ordinary stores).
+ * parts 16-byte aligned; every outs[k] + row_offset * d 8-byte aligned.
+ */
+LMH_API lmh_status lmh_vp_reduce_rows_to(int R, int64_t rows, int64_t d, const float* parts,
+                                         lmh_bf16* const* outs, int n_out, int64_t row_offset,
+                                         void* stream);
 
 /*
  * lmh_support_kl_fwd_bwd — lmh_support_kl plus the backward of the mean KL (LMH_F_MEAN:

@@ -20,7 +20,7 @@ from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEV
                    DEVERR_NONFINITE, DEVERR_TEMPERATURE, DEVERR_TIMEOUT, ENTRY_LOGPROB, ENTRY_LOSS_BWD,
                    ENTRY_LOSS_FWD, ENTRY_SUPPORT_KL, ENTRY_SUPPORT_LOGPROB, ENTRY_VP_BWD,
                    ENTRY_LOSS_FWD_BWD, ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN,
-                   F_GRAD_SCALAR,
+                   F_GRAD_SCALAR, lmh_vp_dest,
                    F_FUSED_BWD, F_MEAN, F_SUPPORT_RENORM, IGNORE_INDEX, MAX_K, STATUS_NAMES, lib, lmh_shape)
 
 __all__ = [
@@ -33,7 +33,7 @@ __all__ = [
     "ENTRY_LOGPROB", "ENTRY_SUPPORT_LOGPROB", "ENTRY_SUPPORT_KL", "DEVERR_LABEL_RANGE",
     "DEVERR_TIMEOUT", "DEVERR_NONFINITE", "DEVERR_TEMPERATURE", "MAX_K",
     "lmh_vp_partials", "lmh_vp_combine", "lmh_vp_loss_bwd", "lmh_vp_fused_bwd",
-    "lmh_vp_reduce_rows",
+    "lmh_vp_reduce_rows", "lmh_vp_reduce_rows_to",
     "ENTRY_VP_PARTIALS", "ENTRY_VP_COMBINE", "ENTRY_VP_BWD", "F_GRAD_SCALAR",
     "ENTRY_LOSS_FWD_BWD", "lmh_loss_fwd_bwd", "loss_fwd_bwd",
 ]
@@ -234,8 +234,19 @@ def lmh_vp_combine(shape, R, records, labels, loss_rows, lse, logprob=None, argm
     _ok("lmh_vp_combine", st)
 
 
+def _dest(dest):
+    """(recv pointer table: an int64 CUDA tensor of R device addresses, R, rank) -> struct."""
+    if dest is None:
+        return None
+    table, R, rank = dest
+    if table.dtype != torch.int64 or table.numel() < int(R):
+        raise ValueError("the receive-buffer table must hold R int64 device addresses")
+    return ctypes.byref(lmh_vp_dest(_p(table, None, "recv table"), int(R), int(rank)))
+
+
 def lmh_vp_loss_bwd(shard, mode, v0, V_total, H, W_shard, labels, lse, grad=None, dH_part=None,
-                    dW_shard=None, dW_acc_shard=None, *, workspace, stream=None) -> None:
+                    dW_shard=None, dW_acc_shard=None, dest=None, *, workspace,
+                    stream=None) -> None:
     N, d, Vr = shard.N, shard.d, shard.V
     _fits(H=(H, N * d), W_shard=(W_shard, Vr * d), labels=(labels, N), lse=(lse, N),
           grad=(grad, 1 if shard.flags & F_GRAD_SCALAR else N), dH_part=(dH_part, N * d),
@@ -245,12 +256,13 @@ def lmh_vp_loss_bwd(shard, mode, v0, V_total, H, W_shard, labels, lse, grad=None
                                _p(labels, _i32, "labels"), _p(lse, _f32, "lse"),
                                _p(grad, _f32, "grad"), _p(dH_part, _f32, "dH_part"),
                                _p(dW_shard, _bf, "dW_shard"), _p(dW_acc_shard, _f32, "dW_acc_shard"),
-                               _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
+                               _dest(dest), _p(workspace, _u8, "workspace"), workspace.numel(),
+                               _s(stream))
     _ok("lmh_vp_loss_bwd", st)
 
 
 def lmh_vp_fused_bwd(shard, v0, V_total, H, W_shard, labels, lse, n_valid_given=None,
-                     dH_part=None, dW_shard=None, dW_acc_shard=None, *, workspace,
+                     dH_part=None, dW_shard=None, dW_acc_shard=None, dest=None, *, workspace,
                      stream=None) -> None:
     N, d, Vr = shard.N, shard.d, shard.V
     _fits(H=(H, N * d), W_shard=(W_shard, Vr * d), labels=(labels, N), lse=(lse, N),
@@ -260,7 +272,7 @@ def lmh_vp_fused_bwd(shard, v0, V_total, H, W_shard, labels, lse, n_valid_given=
                                 _p(W_shard, _bf, "W_shard"), _p(labels, _i32, "labels"),
                                 _p(lse, _f32, "lse"), _p(n_valid_given, _i32, "n_valid_given"),
                                 _p(dH_part, _f32, "dH_part"), _p(dW_shard, _bf, "dW_shard"),
-                                _p(dW_acc_shard, _f32, "dW_acc_shard"),
+                                _p(dW_acc_shard, _f32, "dW_acc_shard"), _dest(dest),
                                 _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
     _ok("lmh_vp_fused_bwd", st)
 
@@ -272,6 +284,18 @@ def lmh_vp_reduce_rows(parts, out, stream=None) -> None:
     st = lib().lmh_vp_reduce_rows(int(R), int(rows), int(d), _p(parts, _f32, "parts"),
                                   _p(out, _bf, "out"), _s(stream))
     _ok("lmh_vp_reduce_rows", st)
+
+
+def lmh_vp_reduce_rows_to(parts, outs, n_out, row_offset, stream=None) -> None:
+    """parts [R, rows, d] fp32 summed in ascending R into rows row_offset.. of every output;
+    outs: an int64 CUDA tensor of n_out device addresses of [*, d] bf16 buffers."""
+    R, rows, d = parts.shape
+    if outs.dtype != torch.int64 or outs.numel() < int(n_out):
+        raise ValueError("outs must hold n_out int64 device addresses")
+    st = lib().lmh_vp_reduce_rows_to(int(R), int(rows), int(d), _p(parts, _f32, "parts"),
+                                     _p(outs, None, "outs"), int(n_out), int(row_offset),
+                                     _s(stream))
+    _ok("lmh_vp_reduce_rows_to", st)
 
 
 def lmh_read_errors(workspace: torch.Tensor, stream=None) -> int:

@@ -32,6 +32,10 @@ class lmh_shape(ctypes.Structure):
                 ("row_temperature", c_void_p)]
 
 
+class lmh_vp_dest(ctypes.Structure):
+    _fields_ = [("recv", c_void_p), ("R", ctypes.c_int32), ("rank", ctypes.c_int32)]
+
+
 _P = c_void_p
 _SIGS = {
     "lmh_workspace_size": (c_size_t, [ctypes.POINTER(lmh_shape), c_int]),
@@ -44,10 +48,11 @@ _SIGS = {
     "lmh_vp_partials": (c_int, [ctypes.POINTER(lmh_shape), c_int64, c_int64] + [_P] * 5
                         + [c_size_t, _P]),
     "lmh_vp_combine": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 10 + [c_size_t, _P]),
-    "lmh_vp_loss_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int, c_int64, c_int64] + [_P] * 9
-                        + [c_size_t, _P]),
-    "lmh_vp_fused_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int64, c_int64] + [_P] * 9
-                         + [c_size_t, _P]),
+    "lmh_vp_loss_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int, c_int64, c_int64] + [_P] * 8
+                        + [ctypes.POINTER(lmh_vp_dest), _P, c_size_t, _P]),
+    "lmh_vp_fused_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int64, c_int64] + [_P] * 8
+                         + [ctypes.POINTER(lmh_vp_dest), _P, c_size_t, _P]),
+    "lmh_vp_reduce_rows_to": (c_int, [c_int, c_int64, c_int64, _P, _P, c_int, c_int64, _P]),
     "lmh_vp_reduce_rows": (c_int, [c_int, c_int64, c_int64, _P, _P, _P]),
     "lmh_support_kl_fwd_bwd": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 12 + [c_size_t, _P]),
     "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),

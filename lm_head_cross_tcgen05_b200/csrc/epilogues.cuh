@@ -295,10 +295,38 @@ struct EpiGrad {
   }
 };
 
+// ------------------------------------------------------------------ row scatter
+// Where the fp32 rows of a vocabulary shard's dH contribution go when each is written straight
+// to the rank that reduces it: the N rows form R consecutive slices (the first N % R hold one
+// row more), slice j belongs to rank j, and rank j's receive buffer dest[j] is [R][rows_j][d]
+// fp32 with this rank's rows at slot `rank`. dest[j] may be another GPU's memory (a peer
+// pointer): the epilogue reaches it with ordinary stores, tile by tile, while the GEMM runs.
+struct RowScatter {
+  float* const* dest = nullptr;  // [R] receive buffers (a device array), or null: no scatter
+  long long N = 0;
+  long long row0 = 0;            // global index of the chunk's first row
+  int R = 1;
+  int rank = 0;
+  __device__ __forceinline__ float* row(long long g, int d) const {
+    const long long base = N / R, extra = N % R, big = extra * (base + 1);
+    long long j, start, rows;
+    if (g < big) {
+      j = g / (base + 1);
+      start = j * (base + 1);
+      rows = base + 1;
+    } else {  // base >= 1 here: g >= big only when some slice holds base rows
+      j = extra + (g - big) / base;
+      start = big + (j - extra) * base;
+      rows = base;
+    }
+    return dest[j] + (static_cast<long long>(rank) * rows + (g - start)) * d;
+  }
+};
+
 // ------------------------------------------------------------------ dH = G W
 // ctx.tmC maps this chunk's rows of dH ([rows, d] at row r0). With K (= V) split, each unit
 // writes its fp32 partial to part[split][row][col] instead; a fixed-order reduction over the
-// splits then produces dH.
+// splits then produces dH. With a row scatter each fp32 row goes to its reducing rank.
 struct EpiDH {
   static constexpr int kId = 5;        // gemm_dH
   static constexpr int kAMajorMN = 0;  // G chunk [rows, V], K-major
@@ -306,7 +334,8 @@ struct EpiDH {
   struct Params {
     int rows;
     int d;
-    float* part;  // [splits, rows, d] fp32, or null when K is not split
+    float* part;    // [splits, rows, d] fp32, or null when K is not split
+    RowScatter sc;  // with sc.dest: fp32 rows to their reducing ranks instead (one split)
   };
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
                                               int rit, EpiCtx& ctx) {
@@ -320,10 +349,12 @@ struct EpiDH {
       float a[32], b[32];
       tmem_ld32(taddr + sb * 64, a);
       tmem_ld32(taddr + sb * 64 + 32, b);
-      if (p.part) {
+      if (p.sc.dest || p.part) {
         if (row < p.rows) {
           float4* o = reinterpret_cast<float4*>(
-              p.part + (static_cast<long long>(ctx.split) * p.rows + row) * p.d + col0);
+              (p.sc.dest ? p.sc.row(p.sc.row0 + row, p.d)
+                         : p.part + (static_cast<long long>(ctx.split) * p.rows + row) * p.d) +
+              col0);
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const float* v = u < 8 ? a : b;

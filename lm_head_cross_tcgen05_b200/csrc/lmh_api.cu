@@ -440,9 +440,22 @@ lmh_status cast_dw(const Plan& P, const float* acc, lmh_bf16* dW, cudaStream_t s
 lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H,
                               const lmh_bf16* W, int64_t r0, int rows, int chunk_idx,
                               lmh_bf16* dH, lmh_bf16* dW, float* dW_acc, const Ws& ws,
-                              cudaStream_t st, float* dH_f32 = nullptr) {
+                              cudaStream_t st, float* dH_f32 = nullptr,
+                              const RowScatter* scatter = nullptr) {
   const __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
-  if (dH_f32) {
+  if (scatter) {  // each fp32 row straight to the rank that reduces it
+    CUtensorMap ta, tb;
+    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BK))
+      return LMH_ERR_CUDA;
+    EpiDH::Params ep;
+    ep.rows = rows;
+    ep.d = static_cast<int>(P.d);
+    ep.part = nullptr;
+    ep.sc = *scatter;
+    ep.sc.row0 = r0;
+    LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, ta, rows, P.d, P.V, kOrderDH, &ws.h->err, ep,
+                               st, 1));
+  } else if (dH_f32) {
     CUtensorMap ta, tb;
     if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BK))
       return LMH_ERR_CUDA;
@@ -975,6 +988,19 @@ extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_b
 // ============================================================================ vocab-parallel
 namespace {
 
+// The receive buffers of a row scatter: R ranks, this one among them, N rows split over R.
+lmh_status vp_dest_ok(const lmh_vp_dest* dest, const float* dH_part, int64_t N,
+                      RowScatter* sc) {
+  if (!dest) return LMH_OK;
+  if (dH_part || !dest->recv || dest->R < 1 || dest->rank < 0 || dest->rank >= dest->R)
+    return LMH_ERR_INVALID_ARG;
+  sc->dest = dest->recv;
+  sc->R = dest->R;
+  sc->rank = dest->rank;
+  sc->N = N;
+  return LMH_OK;
+}
+
 lmh_status vp_args_ok(const lmh_shape* shard, int64_t v0, int64_t V_total) {
   if (!shape_ok(shard) || v0 < 0 || V_total <= 0 || V_total > 0x7fffffffLL ||
       v0 + shard->V > V_total)
@@ -1083,9 +1109,12 @@ extern "C" lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t 
                                       int64_t V_total, const lmh_bf16* H,
                                       const lmh_bf16* W_shard, const int32_t* labels,
                                       const float* lse, const float* grad, float* dH_part,
-                                      lmh_bf16* dW_shard, float* dW_acc_shard, void* workspace,
+                                      lmh_bf16* dW_shard, float* dW_acc_shard,
+                                      const lmh_vp_dest* dest, void* workspace,
                                       size_t workspace_bytes, void* stream) {
   LMH_TRY(vp_args_ok(shard, v0, V_total));
+  RowScatter sc;
+  LMH_TRY(vp_dest_ok(dest, dH_part, shard->N, &sc));
   if (mode != LMH_BWD_CE && mode != LMH_BWD_LOGPROB) return LMH_ERR_INVALID_ARG;
   lmh_shape sh = *shard;
   sh.flags &= ~LMH_F_SUPPORT_RENORM;
@@ -1101,7 +1130,7 @@ extern "C" lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t 
   const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
   LMH_TRY(clear_header(ws, st));
   if (P.N == 0) return empty_call(P, nullptr, nullptr, dW_shard, dW_acc_shard, st);
-  if (!dH_part && !dW_shard && !dW_acc_shard) return LMH_OK;
+  if (!dH_part && !dest && !dW_shard && !dW_acc_shard) return LMH_OK;
   LMH_TRY(count_labels_total(P, labels, V_total, ws, st));
   LMH_TRY(vp_local_labels(P, labels, v0, ws, st));
   float* alpha = ws.at<float>(P.o_alpha);
@@ -1132,7 +1161,8 @@ extern "C" lmh_status lmh_vp_loss_bwd(const lmh_shape* shard, int mode, int64_t 
     LMH_TRY(launch_gemm<EpiGrad<kLabel>>(dev, sms, ta, tb, tc, rows, P.V, P.d, kOrderLogits,
                                          &ws.h->err, ep, st));
     LMH_TRY(run_backward_gemms(P, dev, sms, H, W_shard, r0, rows, static_cast<int>(ci), nullptr,
-                               dW_shard, dW_acc_shard, ws, st, dH_part));
+                               dW_shard, dW_acc_shard, ws, st, dH_part,
+                               dest ? &sc : nullptr));
   }
   return LMH_OK;
 }
@@ -1141,10 +1171,13 @@ extern "C" lmh_status lmh_vp_fused_bwd(const lmh_shape* shard, int64_t v0, int64
                                        const lmh_bf16* H, const lmh_bf16* W_shard,
                                        const int32_t* labels, const float* lse,
                                        const int32_t* n_valid_given, float* dH_part,
-                                       lmh_bf16* dW_shard, float* dW_acc_shard, void* workspace,
+                                       lmh_bf16* dW_shard, float* dW_acc_shard,
+                                       const lmh_vp_dest* dest, void* workspace,
                                        size_t workspace_bytes, void* stream) {
   LMH_TRY(vp_args_ok(shard, v0, V_total));
   if (!(shard->flags & LMH_F_FUSED_BWD)) return LMH_ERR_INVALID_ARG;
+  RowScatter sc;
+  LMH_TRY(vp_dest_ok(dest, dH_part, shard->N, &sc));
   const Plan P = make_plan(shard, LMH_ENTRY_VP_PARTIALS, true, false);
   int dev, sms;
   LMH_TRY(common_checks(shard, H, W_shard, workspace, workspace_bytes, P.total, &dev, &sms));
@@ -1156,7 +1189,7 @@ extern "C" lmh_status lmh_vp_fused_bwd(const lmh_shape* shard, int64_t v0, int64
   const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
   LMH_TRY(clear_header(ws, st));
   if (P.N == 0) return empty_call(P, nullptr, nullptr, dW_shard, dW_acc_shard, st);
-  if (!dH_part && !dW_shard && !dW_acc_shard) return LMH_OK;
+  if (!dH_part && !dest && !dW_shard && !dW_acc_shard) return LMH_OK;
   const int mean = (shard->flags & LMH_F_MEAN) ? 1 : 0;
   const int rows = static_cast<int>(P.N);
   LMH_TRY(count_labels_total(P, labels, V_total, ws, st));
@@ -1189,7 +1222,7 @@ extern "C" lmh_status lmh_vp_fused_bwd(const lmh_shape* shard, int64_t v0, int64
   }
   LMH_TRY(last_launch());
   return run_backward_gemms(P, dev, sms, H, W_shard, 0, rows, 0, nullptr, dW_shard,
-                            dW_acc_shard, ws, st, dH_part);
+                            dW_acc_shard, ws, st, dH_part, dest ? &sc : nullptr);
 }
 
 extern "C" lmh_status lmh_vp_reduce_rows(int R, int64_t rows, int64_t d, const float* parts,
@@ -1206,6 +1239,26 @@ extern "C" lmh_status lmh_vp_reduce_rows(int R, int64_t rows, int64_t d, const f
   ProfScope ps(KID_VP_REDUCE, st);
   vp_reduce_rows_kernel<<<static_cast<unsigned>(blocks < 8192 ? blocks : 8192), 256, 0, st>>>(
       R, n4, reinterpret_cast<const float4*>(parts), reinterpret_cast<__nv_bfloat16*>(out));
+  return last_launch();
+}
+
+extern "C" lmh_status lmh_vp_reduce_rows_to(int R, int64_t rows, int64_t d, const float* parts,
+                                            lmh_bf16* const* outs, int n_out, int64_t row_offset,
+                                            void* stream) {
+  if (R < 1 || rows < 0 || d <= 0 || (d % 64) != 0 || n_out < 1 || row_offset < 0)
+    return LMH_ERR_INVALID_ARG;
+  if (rows == 0) return LMH_OK;
+  if (!parts || !outs) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(parts)) return LMH_ERR_ALIGNMENT;
+  int dev, sms;
+  LMH_TRY(current_device(&dev, &sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t n4 = rows * d / 4;
+  const int64_t blocks = cdiv(n4, 256);
+  ProfScope ps(KID_VP_REDUCE, st);
+  vp_reduce_rows_to_kernel<<<static_cast<unsigned>(blocks < 8192 ? blocks : 8192), 256, 0, st>>>(
+      R, n4, reinterpret_cast<const float4*>(parts),
+      reinterpret_cast<__nv_bfloat16* const*>(outs), n_out, row_offset * d / 4);
   return last_launch();
 }
 

@@ -142,4 +142,24 @@ __global__ void vp_reduce_rows_kernel(int R, long long n4, const float4* __restr
   }
 }
 
+// The same sum, stored to n_out copies of the output (the full dH of every rank, other GPUs'
+// memory through peer pointers), at an offset of off4 groups of 4 elements.
+__global__ void vp_reduce_rows_to_kernel(int R, long long n4, const float4* __restrict__ parts,
+                                         __nv_bfloat16* const* __restrict__ outs, int n_out,
+                                         long long off4) {
+  for (long long j = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; j < n4;
+       j += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float4 a = __ldcs(parts + j);
+    for (int r = 1; r < R; ++r) {
+      const float4 b = __ldcs(parts + static_cast<long long>(r) * n4 + j);
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    const uint2 v = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+    for (int k = 0; k < n_out; ++k) reinterpret_cast<uint2*>(outs[k])[off4 + j] = v;
+  }
+}
+
 }  // namespace lmh

@@ -20,7 +20,14 @@ backward
     all-gather returns the bf16 slices to every rank.
 
 With a fixed R every result is bitwise reproducible: no floating-point value is reduced by a
-collective, only moved. The compute steps run in the library's CUDA kernels through
+collective, only moved.
+
+``p2p=True`` fuses the dH exchange into the kernels instead of NCCL: the receive buffers and
+every rank's dH live in symmetric memory (peer-mapped over NVLink); the dH GEMM's epilogue
+writes each fp32 row straight into the receive buffer of the rank that reduces it while the
+GEMM runs, and ``lmh_vp_reduce_rows_to`` stores each reduced bf16 slice into every rank's dH.
+Two stream-ordered barriers of the symmetric memory order the steps. The same fixed order of
+additions gives the same bits as the NCCL path. The compute steps run in the library's CUDA kernels through
 ``CudaOps``; ``VocabParallelCE`` takes any object with the same four methods, which is how its
 exchange logic is tested on CPU ranks.
 """
@@ -33,7 +40,8 @@ import torch.distributed as dist
 
 from . import (BWD_CE, ENTRY_VP_BWD, ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN,
                F_FUSED_BWD, F_MEAN, lmh_vp_combine, lmh_vp_fused_bwd, lmh_vp_loss_bwd,
-               lmh_vp_partials, lmh_vp_reduce_rows, make_shape, workspace)
+               lmh_vp_partials, lmh_vp_reduce_rows, lmh_vp_reduce_rows_to, make_shape,
+               workspace)
 
 __all__ = ["shard_plan", "row_slices", "CudaOps", "VocabParallelCE"]
 
@@ -85,15 +93,18 @@ class CudaOps:
         return rec, (shard, ws)
 
     def fused_backward(self, state, H, W_shard, labels, lse, v0, V_total, n_valid_given=None,
-                       dW_acc=None, want_dW=True):
+                       dW_acc=None, want_dW=True, dest=None):
         shard, ws = state
         N, d = H.shape
-        dH_part = torch.empty(N, d, dtype=torch.float32, device=H.device)
+        dH_part = None if dest else torch.empty(N, d, dtype=torch.float32, device=H.device)
         dW = (torch.empty(W_shard.shape[0], d, dtype=torch.bfloat16, device=H.device)
               if want_dW else None)
         lmh_vp_fused_bwd(shard, v0, V_total, H, W_shard, labels, lse, n_valid_given, dH_part,
-                         dW, dW_acc, workspace=ws)
+                         dW, dW_acc, dest, workspace=ws)
         return dH_part, dW
+
+    def reduce_rows_to(self, parts, out_table, n_out, row_offset):
+        lmh_vp_reduce_rows_to(parts, out_table, n_out, row_offset)
 
     def combine(self, records, labels, V_total, d, n_valid_given=None):
         R, N, _ = records.shape
@@ -112,16 +123,18 @@ class CudaOps:
         return out
 
     def backward(self, mode, H, W_shard, labels, lse, grad, v0, V_total, chunk_rows=0,
-                 mean=True, temperature=None, dW_acc=None, want_dW=True):
+                 mean=True, temperature=None, dW_acc=None, want_dW=True, dest=None):
+        """(dH_part, dW); with dest = (receive-buffer table, R, rank) the dH rows are scattered
+        to the reducing ranks instead and dH_part is None."""
         N, d = H.shape
         Vr = W_shard.shape[0]
         flags = (F_MEAN if mean else 0) | (F_DW_ACC_GIVEN if dW_acc is not None else 0)
         shard = make_shape(N, d, Vr, 0, chunk_rows, flags, temperature)
         ws = workspace(shard, ENTRY_VP_BWD, H.device)
-        dH_part = torch.empty(N, d, dtype=torch.float32, device=H.device)
+        dH_part = None if dest else torch.empty(N, d, dtype=torch.float32, device=H.device)
         dW = torch.empty(Vr, d, dtype=torch.bfloat16, device=H.device) if want_dW else None
         lmh_vp_loss_bwd(shard, mode, v0, V_total, H, W_shard, labels, lse, grad, dH_part, dW,
-                        dW_acc, workspace=ws)
+                        dW_acc, dest, workspace=ws)
         return dH_part, dW
 
     def reduce_rows(self, parts):
@@ -138,7 +151,7 @@ class VocabParallelCE:
     initialised process group it runs as the only rank (R = 1, no collective)."""
 
     def __init__(self, V_total: int, group=None, chunk_rows: int = 0, mean: bool = True,
-                 temperature=None, ops=None):
+                 temperature=None, ops=None, p2p: bool = False):
         self.group = group
         self.distributed = dist.is_available() and dist.is_initialized()
         self.R = dist.get_world_size(group) if self.distributed else 1
@@ -149,6 +162,8 @@ class VocabParallelCE:
         self.mean = mean
         self.temperature = temperature
         self.ops = ops if ops is not None else CudaOps()
+        self.p2p = p2p and self.R > 1   # one rank has nothing to exchange
+        self._sym = None
 
     def _check_shard(self, W_shard):
         if W_shard.shape[0] != self.v1 - self.v0:
@@ -180,9 +195,18 @@ class VocabParallelCE:
         rec, state = self.ops.partials_fused(H, W_shard, labels, self.v0, self.V_total,
                                              self.mean, self.temperature)
         out = self._combine(rec, labels, H.shape[1], n_valid_given)
-        dH_part, dW = self.ops.fused_backward(state, H, W_shard, labels, out["lse"], self.v0,
-                                              self.V_total, n_valid_given, dW_acc, want_dW)
-        out["dH"] = self._sum_rows(dH_part)
+        if self.p2p:
+            sym = self._symmetric(H.shape[0], H.shape[1], H.device)
+            sym["recv_h"].barrier(channel=0)  # no rank still reads its last receive buffer
+            _, dW = self.ops.fused_backward(state, H, W_shard, labels, out["lse"], self.v0,
+                                            self.V_total, n_valid_given, dW_acc, want_dW,
+                                            dest=(sym["recv_tab"], self.R, self.rank))
+            out["dH"] = self._reduce_p2p(sym)
+        else:
+            dH_part, dW = self.ops.fused_backward(state, H, W_shard, labels, out["lse"],
+                                                  self.v0, self.V_total, n_valid_given, dW_acc,
+                                                  want_dW)
+            out["dH"] = self._sum_rows(dH_part)
         out["dW"] = dW
         return out
 
@@ -191,10 +215,51 @@ class VocabParallelCE:
         """dH [N, d] (the same on every rank) and this rank's dW shard [v1 - v0, d]."""
         self._check_shard(W_shard)
         N, d = H.shape
+        if self.p2p:
+            sym = self._symmetric(N, d, H.device)
+            sym["recv_h"].barrier(channel=0)
+            _, dW = self.ops.backward(mode, H, W_shard, labels, lse, grad, self.v0,
+                                      self.V_total, self.chunk_rows, self.mean,
+                                      self.temperature, dW_acc, want_dW,
+                                      dest=(sym["recv_tab"], self.R, self.rank))
+            return dict(dH=self._reduce_p2p(sym), dW=dW)
         dH_part, dW = self.ops.backward(mode, H, W_shard, labels, lse, grad, self.v0,
                                         self.V_total, self.chunk_rows, self.mean,
                                         self.temperature, dW_acc, want_dW)
         return dict(dH=self._sum_rows(dH_part), dW=dW)
+
+    def _symmetric(self, N, d, device):
+        """The receive buffer ([R][rows_j][d] fp32 within R * max_rows * d) and the full bf16
+        dH of every rank in symmetric memory, with the tables of the R ranks' addresses."""
+        if self._sym is not None and self._sym["key"] == (N, d):
+            return self._sym
+        import torch.distributed._symmetric_memory as symm_mem
+        group = self.group if self.group is not None else dist.group.WORLD
+        sizes = [b - a for a, b in row_slices(N, self.R)]
+        n_recv = self.R * max(sizes) * d
+        recv = symm_mem.empty(n_recv, dtype=torch.float32, device=device)
+        recv_h = symm_mem.rendezvous(recv, group)
+        dH = symm_mem.empty(N * d, dtype=torch.bfloat16, device=device)
+        dH_h = symm_mem.rendezvous(dH, group)
+
+        def table(h, n, dtype):
+            return torch.tensor([h.get_buffer(r, (n,), dtype).data_ptr() for r in range(self.R)],
+                                dtype=torch.int64, device=device)
+        self._sym = dict(key=(N, d), sizes=sizes, recv=recv, recv_h=recv_h, dH=dH, dH_h=dH_h,
+                         recv_tab=table(recv_h, n_recv, torch.float32),
+                         dH_tab=table(dH_h, N * d, torch.bfloat16))
+        return self._sym
+
+    def _reduce_p2p(self, sym):
+        """After every rank's rows landed: reduce this rank's slice into every rank's dH."""
+        sizes = sym["sizes"]
+        mine, start = sizes[self.rank], sum(sizes[:self.rank])
+        d = sym["dH"].numel() // sum(sizes)
+        sym["recv_h"].barrier(channel=1)      # every rank's dH rows are in the receive buffers
+        parts = sym["recv"][: self.R * mine * d].view(self.R, mine, d)
+        self.ops.reduce_rows_to(parts, sym["dH_tab"], self.R, start)
+        sym["dH_h"].barrier(channel=0)        # every rank's slice is in every dH
+        return sym["dH"].view(-1, d).clone()
 
     def _sum_rows(self, part: torch.Tensor) -> torch.Tensor:
         """sum over ranks of part [N, d], added in ascending rank order, on every rank."""

@@ -95,8 +95,15 @@ def test_vocab_parallel_host_errors_without_gpu():
     # shard past the vocabulary, negative offset, empty vocabulary: refused before any CUDA call
     assert lib.lmh_vp_partials(ctypes.byref(shard), 50, 120, *P, 0, None) == 1
     assert lib.lmh_vp_partials(ctypes.byref(shard), -1, 120, *P, 0, None) == 1
-    assert lib.lmh_vp_loss_bwd(ctypes.byref(shard), 0, 0, 0, *([None] * 9), 0, None) == 1
-    assert lib.lmh_vp_loss_bwd(ctypes.byref(shard), 2, 0, 100, *([None] * 9), 0, None) == 1
+    assert lib.lmh_vp_loss_bwd(ctypes.byref(shard), 0, 0, 0, *([None] * 9), None, 0,
+                               None) == 1
+    assert lib.lmh_vp_loss_bwd(ctypes.byref(shard), 2, 0, 100, *([None] * 9), None, 0,
+                               None) == 1
+    # a receive table with an out-of-range rank, and one alongside dH_part: refused
+    bad = _abi.lmh_vp_dest(ctypes.c_void_p(256), 2, 2)
+    assert lib.lmh_vp_loss_bwd(ctypes.byref(shard), 0, 0, 100, *([None] * 8),
+                               ctypes.byref(bad), None, 0, None) == 1
+    assert lib.lmh_vp_reduce_rows_to(2, 4, 64, None, None, 0, 0, None) == 1   # no output
     assert lib.lmh_vp_combine(ctypes.byref(shard), 0, *([None] * 10), 0, None) == 1
     assert lib.lmh_vp_reduce_rows(2, 4, 96, None, None, None) == 1     # d not a multiple of 64
     assert lib.lmh_vp_reduce_rows(0, 4, 64, None, None, None) == 1
@@ -133,3 +140,15 @@ def test_weighted_fused_size_adds_row_coefficients():
     w = ws(1000, 64, 5000, chunk=1000, flags=L.F_FUSED_BWD | L.F_DW_ACC_GIVEN,
            entry=L.ENTRY_LOSS_FWD_BWD)
     assert w - f == 2 * 4096
+
+
+def test_ctypes_signatures_match_header_parameter_counts():
+    # every declaration in include/lmh.h and the binding's ctypes signature agree on the
+    # number of parameters (a drifted count would shift every pointer after it)
+    import re
+    src = open(_abi.HEADER).read()
+    decls = re.findall(r"LMH_API\s+[\w\s\*]*?\b(lmh_\w+)\s*\(([^;]*?)\);", src, flags=re.S)
+    assert len(decls) == len(_abi.header_symbols())
+    for name, params in decls:
+        n = 0 if params.strip() in ("", "void") else len(params.split(","))
+        assert n == len(_abi._SIGS[name][1]), name

@@ -219,3 +219,71 @@ def test_vocab_parallel_class_on_one_rank():
     ref = O.ce_fused(xc["H"], xc["W"], xc["labels"])
     check_ce_fused(dict(f, dH=b["dH"], dW=b["dW"]), ref)
     check_ce_fused(fb, ref)
+
+
+def _scatter_buffers(N, d, R):
+    """Stand-ins for the ranks' symmetric buffers on this one GPU: R receive buffers (NaN, so
+    a row never written shows) and R full dH outputs, with their address tables."""
+    from lm_head_cross_tcgen05_b200.vocab_parallel import row_slices
+    sizes = [b - a for a, b in row_slices(N, R)]
+    recv = [torch.full((R * max(sizes) * d,), float("nan"), device="cuda") for _ in range(R)]
+    outs = [torch.zeros(N, d, dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    rt = torch.tensor([t.data_ptr() for t in recv], dtype=torch.int64, device="cuda")
+    ot = torch.tensor([t.data_ptr() for t in outs], dtype=torch.int64, device="cuda")
+    return sizes, recv, outs, rt, ot
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("N,d,V,R", [
+    (300, 192, 1000, 2),
+    (129, 128, 4100, 3),       # ragged row slices (43 each)
+    (64, 256, 2048, 8),
+    (5, 64, 900, 8),           # fewer rows than ranks: three ranks reduce nothing
+])
+def test_row_scatter_exchange_matches_collective_path(fused, N, d, V, R):
+    # the dH GEMM epilogue writes every fp32 row into its reducing rank's buffer (local buffers
+    # stand in for peer memory); each rank's reduce stores its bf16 slice into every dH:
+    # the same bits as the gathered, rank-ordered sum
+    x, xc = device_inputs(_wl(N, d, V, 3 if N > 10 else 0))
+    ref = (_emulate_fused if fused else _emulate)(x, V, R)
+    H, W, y = x["H"], x["W"], x["labels"]
+    ops = CudaOps()
+    plan = shard_plan(V, R)
+    sizes, recv, outs, rt, ot = _scatter_buffers(N, d, R)
+    if fused:
+        recs, states = zip(*[ops.partials_fused(H, W[a:b], y, a, V) for a, b in plan])
+    else:
+        recs = [ops.partials(H, W[a:b], y, a, V) for a, b in plan]
+    f = ops.combine(torch.stack(list(recs)), y, V, d)
+    dWs = []
+    for r, (a, b) in enumerate(plan):
+        if fused:
+            part, dw = ops.fused_backward(states[r], H, W[a:b], y, f["lse"], a, V,
+                                          dest=(rt, R, r))
+        else:
+            part, dw = ops.backward(L.BWD_CE, H, W[a:b], y, f["lse"], None, a, V,
+                                    dest=(rt, R, r))
+        assert part is None
+        dWs.append(dw)
+    for j in range(R):
+        parts = recv[j][: R * sizes[j] * d].view(R, sizes[j], d)
+        L.lmh_vp_reduce_rows_to(parts, ot, R, sum(sizes[:j]))
+    torch.cuda.synchronize()
+    for k in range(R):
+        assert torch.equal(outs[k], ref["dH"]), k
+    assert torch.equal(torch.cat(dWs), ref["dW"])
+    check_grad(outs[0], O.ce_fused(xc["H"], xc["W"], xc["labels"])["dH"], "dH")
+
+
+def test_row_scatter_argument_checks():
+    N, d, V = 40, 64, 600
+    x, _ = device_inputs(_wl(N, d, V, 0))
+    shard = L.make_shape(N, d, 300, 0, 0, L.F_MEAN)
+    ws = L.workspace(shard, L.ENTRY_VP_BWD, "cuda")
+    lse = torch.zeros(N, dtype=torch.float32, device="cuda")
+    _, recv, _, rt, _ = _scatter_buffers(N, d, 2)
+    part = torch.empty(N, d, dtype=torch.float32, device="cuda")
+    for dest, dh in [((rt, 2, 2), None), ((rt, 2, -1), None), ((rt, 2, 0), part)]:
+        with pytest.raises(L.LmhError, match="INVALID_ARG"):
+            L.lmh_vp_loss_bwd(shard, L.BWD_CE, 0, V, x["H"], x["W"][:300], x["labels"], lse,
+                              None, dh, None, None, dest, workspace=ws)

@@ -40,7 +40,7 @@ class OracleOps:
                     n_valid=torch.tensor([int(valid.sum())]))
 
     def backward(self, mode, H, W_shard, labels, lse, grad, v0, V_total, chunk_rows=0,
-                 mean=True, temperature=None, dW_acc=None, want_dW=True):
+                 mean=True, temperature=None, dW_acc=None, want_dW=True, dest=None):
         z = O.logits(H, W_shard, temperature)
         N, Vr = z.shape
         y = O.as_i64(labels)
@@ -64,7 +64,7 @@ class OracleOps:
             dict(mean=mean, temperature=temperature)
 
     def fused_backward(self, state, H, W_shard, labels, lse, v0, V_total, n_valid_given=None,
-                       dW_acc=None, want_dW=True):
+                       dW_acc=None, want_dW=True, dest=None):
         grad = None
         if n_valid_given is not None:
             n = int(n_valid_given)
