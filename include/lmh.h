@@ -386,6 +386,15 @@ LMH_API lmh_status lmh_support_kl_fwd_bwd(const lmh_shape* shape, const lmh_bf16
                                           size_t workspace_bytes, void* stream);
 
 /*
+ * lmh_scale_bf16 — x = bf16(x * g[0]) in place over n elements (n a multiple of 4, x 8-byte
+ * aligned; g one float in device memory; rounding to nearest even, so g = 1 changes no bit).
+ * Not part of the method: it lets a training framework apply the upstream gradient g of a
+ * summed or averaged loss to the dH and dW that a one-pass entry (lmh_loss_fwd with dH/dW,
+ * lmh_support_kl_fwd_bwd) computed for g = 1, with no host synchronisation.
+ */
+LMH_API lmh_status lmh_scale_bf16(lmh_bf16* x, int64_t n, const float* g, void* stream);
+
+/*
  * lmh_read_errors — synchronises `stream`, then copies the device error word of the last
  * call that used `workspace` into *errors (host). Each entry clears the word when it starts.
  */

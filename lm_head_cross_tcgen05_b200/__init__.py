@@ -33,7 +33,7 @@ __all__ = [
     "ENTRY_LOGPROB", "ENTRY_SUPPORT_LOGPROB", "ENTRY_SUPPORT_KL", "DEVERR_LABEL_RANGE",
     "DEVERR_TIMEOUT", "DEVERR_NONFINITE", "DEVERR_TEMPERATURE", "MAX_K",
     "lmh_vp_partials", "lmh_vp_combine", "lmh_vp_loss_bwd", "lmh_vp_fused_bwd",
-    "lmh_vp_reduce_rows", "lmh_vp_reduce_rows_to",
+    "lmh_vp_reduce_rows", "lmh_vp_reduce_rows_to", "lmh_scale_bf16",
     "ENTRY_VP_PARTIALS", "ENTRY_VP_COMBINE", "ENTRY_VP_BWD", "F_GRAD_SCALAR",
     "ENTRY_LOSS_FWD_BWD", "lmh_loss_fwd_bwd", "loss_fwd_bwd",
 ]
@@ -296,6 +296,13 @@ def lmh_vp_reduce_rows_to(parts, outs, n_out, row_offset, stream=None) -> None:
                                      _p(outs, None, "outs"), int(n_out), int(row_offset),
                                      _s(stream))
     _ok("lmh_vp_reduce_rows_to", st)
+
+
+def lmh_scale_bf16(x, g, stream=None) -> None:
+    """x *= g[0] in place (x bf16 with a multiple of 4 elements; g a one-element device fp32)."""
+    _fits(g=(g, 1))
+    st = lib().lmh_scale_bf16(_p(x, _bf, "x"), int(x.numel()), _p(g, _f32, "g"), _s(stream))
+    _ok("lmh_scale_bf16", st)
 
 
 def lmh_read_errors(workspace: torch.Tensor, stream=None) -> int:

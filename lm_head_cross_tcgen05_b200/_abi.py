@@ -55,6 +55,7 @@ _SIGS = {
     "lmh_vp_reduce_rows_to": (c_int, [c_int, c_int64, c_int64, _P, _P, c_int, c_int64, _P]),
     "lmh_vp_reduce_rows": (c_int, [c_int, c_int64, c_int64, _P, _P, _P]),
     "lmh_support_kl_fwd_bwd": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 12 + [c_size_t, _P]),
+    "lmh_scale_bf16": (c_int, [_P, c_int64, _P, _P]),
     "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),
     "lmh_logprob_noalloc": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6),
     "lmh_selftest_wait_timeout": (c_int, [_P, c_uint32, _P]),

@@ -4,21 +4,27 @@
 The pages' training integration exposes the head as an autograd function whose entry point
 returns per-row log-probabilities (miles-ext-kernels PR #14, lm_head op commit: ``log_probs``,
 its backward run by the same package as the forward). These functions do the same with this
-library: the forward runs a forward entry and keeps the per-row lse; the backward runs
-``lmh_loss_bwd`` with the upstream gradient, recomputing the logits chunk by chunk. The
-upstream gradient of a reduced loss stays on the device (``LMH_F_GRAD_SCALAR``), so no call
-synchronises the host. All arithmetic runs in the library's kernels.
+library, in one of two ways:
 
-For a step whose loss is final (gradient 1), ``loss_fwd(..., grads=True)`` does forward and
-backward in one pass and saves one of the four GEMMs; these functions suit graphs where the
-head's output feeds further computation.
+* per-row outputs (``log_probs``, ``cross_entropy(reduction="none")``, ``support_log_probs``,
+  ``support_kl(reduction="none")``): the upstream gradient is a row vector known only in the
+  backward, so the forward keeps lse and the backward runs ``lmh_loss_bwd``, recomputing the
+  logits chunk by chunk (four GEMMs per step);
+* reduced losses (``cross_entropy`` with "mean" or "sum", ``support_kl`` with "mean"): the
+  gradient is the one for g = 1 times the scalar upstream g, so the forward already runs the
+  one-pass entry (``lmh_loss_fwd`` with dH / dW, ``lmh_support_kl_fwd_bwd``: three GEMMs) and
+  keeps dH and dW, and the backward scales them by g on the device (``lmh_scale_bf16``; g = 1
+  changes no bit). They hold dH and dW from the forward to the backward, like activations.
+
+No call synchronises the host, and all arithmetic runs in the library's kernels.
 """
 from __future__ import annotations
 
 import torch
 
-from . import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, logprob, loss_bwd,
-               loss_fwd, support_kl as _support_kl, support_logprob as _support_logprob)
+from . import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, lmh_scale_bf16,
+               logprob, loss_bwd, loss_fwd, support_kl as _support_kl,
+               support_logprob as _support_logprob)
 
 __all__ = ["log_probs", "cross_entropy", "support_log_probs", "support_kl"]
 
@@ -52,26 +58,42 @@ def log_probs(H, W, labels, *, chunk_rows: int = 0, temperature=None) -> torch.T
     return _LogProbs.apply(H, W, labels, chunk_rows, temperature)
 
 
+def _scaled(ctx, g):
+    """The one-pass gradients of the forward, times the scalar upstream gradient g."""
+    g = g.reshape(1).contiguous().float()
+    out = []
+    for t in (ctx.dH, ctx.dW):
+        if t is not None:
+            lmh_scale_bf16(t, g)
+        out.append(t)
+    ctx.dH = ctx.dW = None
+    return out
+
+
 class _CrossEntropy(torch.autograd.Function):
     @staticmethod
     def forward(ctx, H, W, labels, reduction, chunk_rows, temperature):
         one = None
         if reduction == "sum":  # the entry's mean divides by a given count: give it 1
             one = torch.ones(1, dtype=torch.int32, device=H.device)
-        out = loss_fwd(H, W, labels, chunk_rows=chunk_rows, n_valid_given=one,
-                       temperature=temperature)
         ctx.chunk_rows, ctx.temperature, ctx.reduction = chunk_rows, temperature, reduction
-        ctx.save_for_backward(H, W, out["lse"], labels)
-        return out["loss_rows"] if reduction == "none" else out["loss_mean"].view(())
+        fused = reduction != "none" and (ctx.needs_input_grad[0] or ctx.needs_input_grad[1])
+        out = loss_fwd(H, W, labels, chunk_rows=chunk_rows, n_valid_given=one,
+                       temperature=temperature, grads=fused, mean=reduction == "mean",
+                       want_dH=ctx.needs_input_grad[0], want_dW=ctx.needs_input_grad[1])
+        ctx.dH, ctx.dW = (out.get("dH"), out.get("dW")) if fused else (None, None)
+        if not fused:
+            ctx.save_for_backward(H, W, out["lse"], labels)
+        if reduction == "none":
+            return out["loss_rows"]
+        return out["loss_mean"].view(())
 
     @staticmethod
     def backward(ctx, g):
-        labels = ctx.saved_tensors[3]
         if ctx.reduction == "none":
-            dH, dW = _grads(ctx, BWD_CE, labels, g)
+            dH, dW = _grads(ctx, BWD_CE, ctx.saved_tensors[3], g)
         else:
-            dH, dW = _grads(ctx, BWD_CE, labels, g.reshape(1), mean=ctx.reduction == "mean",
-                            scalar=True)
+            dH, dW = _scaled(ctx, g)
         return dH, dW, None, None, None, None
 
 
@@ -110,15 +132,25 @@ def support_log_probs(H, W, ids, *, chunk_rows: int = 0, temperature=None,
 class _SupportKL(torch.autograd.Function):
     @staticmethod
     def forward(ctx, H, W, ids, ref_logp, reduction, chunk_rows, temperature, renorm):
-        out = _support_kl(H, W, ids, ref_logp, chunk_rows=chunk_rows, temperature=temperature,
-                          renorm=renorm)
         ctx.chunk_rows, ctx.temperature, ctx.renorm = chunk_rows, temperature, renorm
         ctx.reduction = reduction
-        ctx.save_for_backward(H, W, out["lse"], ids, ref_logp)
+        # the one-pass entry covers the full-vocabulary reading; the renormalised one's
+        # backward is a sparse gather / scatter with no logits GEMM to save
+        fused = (reduction == "mean" and not renorm
+                 and (ctx.needs_input_grad[0] or ctx.needs_input_grad[1]))
+        out = _support_kl(H, W, ids, ref_logp, chunk_rows=chunk_rows, temperature=temperature,
+                          renorm=renorm, grads=fused)
+        ctx.dH = out.get("dH") if fused and ctx.needs_input_grad[0] else None
+        ctx.dW = out.get("dW") if fused and ctx.needs_input_grad[1] else None
+        if not fused:
+            ctx.save_for_backward(H, W, out["lse"], ids, ref_logp)
         return out["kl_rows"] if reduction == "none" else out["kl_mean"].view(())
 
     @staticmethod
     def backward(ctx, g):
+        if ctx.reduction != "none" and (ctx.dH is not None or ctx.dW is not None):
+            dH, dW = _scaled(ctx, g)
+            return dH, dW, None, None, None, None, None, None
         ids, ref = ctx.saved_tensors[3], ctx.saved_tensors[4]
         if ctx.reduction == "none":
             dH, dW = _grads(ctx, BWD_SUPPORT_KL, ids, g, ref, renorm=ctx.renorm)

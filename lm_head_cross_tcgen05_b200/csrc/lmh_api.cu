@@ -174,14 +174,14 @@ enum KernelId {
   KID_GEMM_DH, KID_GEMM_DW, KID_FINALIZE, KID_GBUILD, KID_FIX_LABELS, KID_MEAN,
   KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_SUPPORT_DOTS, KID_SUPPORT_LSE,
   KID_SUPPORT_DH, KID_SUPPORT_DW, KID_SPLIT_SUM, KID_VP_LABELS, KID_VP_FINALIZE,
-  KID_VP_COMBINE, KID_VP_REDUCE, KID_VP_SCALE, KID_FIX_CANDS, KID_COUNT
+  KID_VP_COMBINE, KID_VP_REDUCE, KID_VP_SCALE, KID_FIX_CANDS, KID_SCALE, KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "count_labels", "prep_cands", "gemm_logits_stats", "gemm_logits_stats_store",
     "gemm_logits_grad", "gemm_dH", "gemm_dW", "row_finalize", "gbuild", "fix_labels",
     "mean", "support_out", "bwd_coef", "cast_bf16", "support_dots", "support_lse",
     "support_grad_dh", "support_dw", "split_sum", "vp_local_labels", "vp_finalize",
-    "vp_combine", "vp_reduce_rows", "vp_scale", "fix_cands"};
+    "vp_combine", "vp_reduce_rows", "vp_scale", "fix_cands", "scale_bf16"};
 
 struct ProfRec {
   int id;
@@ -1259,6 +1259,22 @@ extern "C" lmh_status lmh_vp_reduce_rows_to(int R, int64_t rows, int64_t d, cons
   vp_reduce_rows_to_kernel<<<static_cast<unsigned>(blocks < 8192 ? blocks : 8192), 256, 0, st>>>(
       R, n4, reinterpret_cast<const float4*>(parts),
       reinterpret_cast<__nv_bfloat16* const*>(outs), n_out, row_offset * d / 4);
+  return last_launch();
+}
+
+extern "C" lmh_status lmh_scale_bf16(lmh_bf16* x, int64_t n, const float* g, void* stream) {
+  if (n < 0 || (n % 4) != 0) return LMH_ERR_INVALID_ARG;
+  if (n == 0) return LMH_OK;
+  if (!x || !g) return LMH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 7u) != 0 || (reinterpret_cast<uintptr_t>(g) & 3u) != 0)
+    return LMH_ERR_ALIGNMENT;
+  int dev, sms;
+  LMH_TRY(current_device(&dev, &sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t blocks = cdiv(n / 4, 256);
+  ProfScope ps(KID_SCALE, st);
+  scale_bf16_kernel<<<static_cast<unsigned>(blocks < 8192 ? blocks : 8192), 256, 0, st>>>(
+      n / 4, g, reinterpret_cast<__nv_bfloat16*>(x));
   return last_launch();
 }
 

@@ -425,4 +425,19 @@ __global__ void cast_bf16_kernel(const float* __restrict__ src, long long n4,
   }
 }
 
+// ---------------------------------------------------------------------------- gradient scale
+// x = bf16(x * g[0]) in place over n4 groups of 4 elements (round to nearest even; g = 1
+// leaves every bit unchanged).
+__global__ void scale_bf16_kernel(long long n4, const float* __restrict__ g,
+                                  __nv_bfloat16* __restrict__ x) {
+  const float s = *g;
+  uint2* x4 = reinterpret_cast<uint2*>(x);
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint2 w = x4[i];
+    const float2 a = unpack_bf16x2(w.x), b = unpack_bf16x2(w.y);
+    x4[i] = make_uint2(pack_bf16x2(a.x * s, a.y * s), pack_bf16x2(b.x * s, b.y * s));
+  }
+}
+
 }  // namespace lmh

@@ -95,3 +95,22 @@ def test_scalar_grad_requires_a_pointer():
     with pytest.raises(L.LmhError):
         L.lmh_loss_bwd(shape, L.BWD_CE, x["H"], x["W"], x["labels"], lse, None, None, dH,
                        workspace=ws)
+
+
+def test_reduced_cross_entropy_uses_the_one_pass_gradient():
+    # loss.backward() with g = 1 returns exactly lmh_loss_fwd's fused dH / dW (the scale by
+    # g = 1 changes no bit), and the step launches no recomputing logits GEMM
+    from tests.test_parity_gpu import _kernels_launched
+    x, _ = device_inputs(ragged(150, 128, 1800, n_ignored=4, seed=4250))
+    H, W = _leaf(x)
+    res = {}
+
+    def step():
+        loss = A.cross_entropy(H, W, x["labels"], chunk_rows=64)
+        loss.backward()
+        res["loss"] = loss
+    names = _kernels_launched(step)
+    assert "gemm_logits_grad" not in names and names.count("scale_bf16") == 2
+    ref = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=64, grads=True)
+    assert torch.equal(H.grad, ref["dH"]) and torch.equal(W.grad, ref["dW"])
+    assert torch.equal(res["loss"].detach().view(1), ref["loss_mean"])
