@@ -91,6 +91,9 @@ typedef enum lmh_status {
 #define LMH_ENTRY_VP_COMBINE 6
 #define LMH_ENTRY_VP_BWD 7
 #define LMH_ENTRY_LOSS_FWD_BWD 8
+#define LMH_ENTRY_VP_SUPPORT_PARTIALS 9
+#define LMH_ENTRY_VP_SUPPORT_COMBINE 10
+#define LMH_ENTRY_VP_SUPPORT_BWD 11
 
 /* objectives of lmh_loss_bwd */
 #define LMH_BWD_CE 0              /* L = sum_i g_i loss_i                                */
@@ -345,6 +348,38 @@ LMH_API lmh_status lmh_vp_fused_bwd(const lmh_shape* shard, int64_t v0, int64_t 
                                     lmh_bf16* dW_shard, float* dW_acc_shard,
                                     const lmh_vp_dest* dest, void* workspace,
                                     size_t workspace_bytes, void* stream);
+
+/*
+ * Vocabulary-parallel support entries (the split of lmh_support_logprob / lmh_support_kl and
+ * of lmh_loss_bwd's support objectives; full-vocabulary reading only, LMH_F_SUPPORT_RENORM is
+ * refused). shape->K candidates per row; ids [N, K] are the global candidate ids.
+ * lmh_vp_support_partials: records [N, K + 1] fp32 out: { lse_r as for lmh_vp_partials; for
+ *   each slot k the logit of c_ik if it lies in the shard, else -inf }. Workspace:
+ *   lmh_workspace_size(shard, LMH_ENTRY_VP_SUPPORT_PARTIALS).
+ * lmh_vp_support_combine: shape->V = V_total; records [R, N, K + 1] in rank order. Outputs as
+ *   lmh_support_kl: lp [N, K] (nullable), lse [N], kl_rows [N] and kl_mean [1] (nullable; they
+ *   need ref_logp [N, K]). Candidate ids >= V_total set LMH_DEVERR_LABEL_RANGE and count as
+ *   padding. Workspace: lmh_workspace_size(shape, LMH_ENTRY_VP_SUPPORT_COMBINE).
+ * lmh_vp_support_bwd: mode LMH_BWD_SUPPORT_LOGPROB or LMH_BWD_SUPPORT_KL, grad / ref_logp /
+ *   flags as lmh_loss_bwd, lse the combined one; outputs and dest as lmh_vp_loss_bwd. G is
+ *   formed on the shard's columns with alpha over all of a row's valid candidates and beta at
+ *   the shard's own. Workspace: lmh_workspace_size(shard, LMH_ENTRY_VP_SUPPORT_BWD).
+ */
+LMH_API lmh_status lmh_vp_support_partials(const lmh_shape* shard, int64_t v0, int64_t V_total,
+                                           const lmh_bf16* H, const lmh_bf16* W_shard,
+                                           const int32_t* ids, float* records, void* workspace,
+                                           size_t workspace_bytes, void* stream);
+LMH_API lmh_status lmh_vp_support_combine(const lmh_shape* shape, int R, const float* records,
+                                          const int32_t* ids, const float* ref_logp, float* lp,
+                                          float* lse, float* kl_rows, float* kl_mean,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+LMH_API lmh_status lmh_vp_support_bwd(const lmh_shape* shard, int mode, int64_t v0,
+                                      int64_t V_total, const lmh_bf16* H,
+                                      const lmh_bf16* W_shard, const int32_t* ids,
+                                      const float* lse, const float* grad, const float* ref_logp,
+                                      float* dH_part, lmh_bf16* dW_shard, float* dW_acc_shard,
+                                      const lmh_vp_dest* dest, void* workspace,
+                                      size_t workspace_bytes, void* stream);
 
 /*
  * lmh_vp_reduce_rows: out[j] = bf16(sum_{r = 0..R-1} parts[r, j]) over rows x d elements, the

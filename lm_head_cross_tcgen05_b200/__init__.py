@@ -19,7 +19,9 @@ import torch
 from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEVERR_LABEL_RANGE,
                    DEVERR_NONFINITE, DEVERR_TEMPERATURE, DEVERR_TIMEOUT, ENTRY_LOGPROB, ENTRY_LOSS_BWD,
                    ENTRY_LOSS_FWD, ENTRY_SUPPORT_KL, ENTRY_SUPPORT_LOGPROB, ENTRY_VP_BWD,
-                   ENTRY_LOSS_FWD_BWD, ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN,
+                   ENTRY_LOSS_FWD_BWD, ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS,
+                   ENTRY_VP_SUPPORT_BWD, ENTRY_VP_SUPPORT_COMBINE, ENTRY_VP_SUPPORT_PARTIALS,
+                   F_DW_ACC_GIVEN,
                    F_GRAD_SCALAR, lmh_vp_dest,
                    F_FUSED_BWD, F_MEAN, F_SUPPORT_RENORM, IGNORE_INDEX, MAX_K, STATUS_NAMES, lib, lmh_shape)
 
@@ -36,6 +38,8 @@ __all__ = [
     "lmh_vp_reduce_rows", "lmh_vp_reduce_rows_to", "lmh_scale_bf16",
     "ENTRY_VP_PARTIALS", "ENTRY_VP_COMBINE", "ENTRY_VP_BWD", "F_GRAD_SCALAR",
     "ENTRY_LOSS_FWD_BWD", "lmh_loss_fwd_bwd", "loss_fwd_bwd",
+    "ENTRY_VP_SUPPORT_PARTIALS", "ENTRY_VP_SUPPORT_COMBINE", "ENTRY_VP_SUPPORT_BWD",
+    "lmh_vp_support_partials", "lmh_vp_support_combine", "lmh_vp_support_bwd",
 ]
 
 lib()  # load now: a missing library is an import error, never a silent fallback
@@ -275,6 +279,51 @@ def lmh_vp_fused_bwd(shard, v0, V_total, H, W_shard, labels, lse, n_valid_given=
                                 _p(dW_acc_shard, _f32, "dW_acc_shard"), _dest(dest),
                                 _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
     _ok("lmh_vp_fused_bwd", st)
+
+
+def lmh_vp_support_partials(shard, v0, V_total, H, W_shard, ids, records, *, workspace,
+                            stream=None) -> None:
+    N, d, K = shard.N, shard.d, shard.K
+    _fits(H=(H, N * d), W_shard=(W_shard, shard.V * d), ids=(ids, N * K),
+          records=(records, N * (K + 1)))
+    st = lib().lmh_vp_support_partials(ctypes.byref(shard), int(v0), int(V_total),
+                                       _p(H, _bf, "H"), _p(W_shard, _bf, "W_shard"),
+                                       _p(ids, _i32, "ids"), _p(records, _f32, "records"),
+                                       _p(workspace, _u8, "workspace"), workspace.numel(),
+                                       _s(stream))
+    _ok("lmh_vp_support_partials", st)
+
+
+def lmh_vp_support_combine(shape, R, records, ids, ref_logp, lp, lse, kl_rows=None,
+                           kl_mean=None, *, workspace, stream=None) -> None:
+    N, K = shape.N, shape.K
+    _fits(records=(records, int(R) * N * (K + 1)), ids=(ids, N * K), ref_logp=(ref_logp, N * K),
+          lp=(lp, N * K), lse=(lse, N), kl_rows=(kl_rows, N), kl_mean=(kl_mean, 1))
+    st = lib().lmh_vp_support_combine(ctypes.byref(shape), int(R), _p(records, _f32, "records"),
+                                      _p(ids, _i32, "ids"), _p(ref_logp, _f32, "ref_logp"),
+                                      _p(lp, _f32, "lp"), _p(lse, _f32, "lse"),
+                                      _p(kl_rows, _f32, "kl_rows"), _p(kl_mean, _f32, "kl_mean"),
+                                      _p(workspace, _u8, "workspace"), workspace.numel(),
+                                      _s(stream))
+    _ok("lmh_vp_support_combine", st)
+
+
+def lmh_vp_support_bwd(shard, mode, v0, V_total, H, W_shard, ids, lse, grad=None, ref_logp=None,
+                       dH_part=None, dW_shard=None, dW_acc_shard=None, dest=None, *, workspace,
+                       stream=None) -> None:
+    N, d, Vr, K = shard.N, shard.d, shard.V, shard.K
+    g = 1 if shard.flags & F_GRAD_SCALAR else (N * K if int(mode) == BWD_SUPPORT_LOGPROB else N)
+    _fits(H=(H, N * d), W_shard=(W_shard, Vr * d), ids=(ids, N * K), lse=(lse, N),
+          grad=(grad, g), ref_logp=(ref_logp, N * K), dH_part=(dH_part, N * d),
+          dW_shard=(dW_shard, Vr * d), dW_acc_shard=(dW_acc_shard, Vr * d))
+    st = lib().lmh_vp_support_bwd(ctypes.byref(shard), int(mode), int(v0), int(V_total),
+                                  _p(H, _bf, "H"), _p(W_shard, _bf, "W_shard"),
+                                  _p(ids, _i32, "ids"), _p(lse, _f32, "lse"),
+                                  _p(grad, _f32, "grad"), _p(ref_logp, _f32, "ref_logp"),
+                                  _p(dH_part, _f32, "dH_part"), _p(dW_shard, _bf, "dW_shard"),
+                                  _p(dW_acc_shard, _f32, "dW_acc_shard"), _dest(dest),
+                                  _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
+    _ok("lmh_vp_support_bwd", st)
 
 
 def lmh_vp_reduce_rows(parts, out, stream=None) -> None:

@@ -22,6 +22,7 @@ DEVERR_LABEL_RANGE, DEVERR_TIMEOUT, DEVERR_NONFINITE, DEVERR_TEMPERATURE = 0x1, 
 F_MEAN, F_FUSED_BWD, F_DW_ACC_GIVEN, F_SUPPORT_RENORM, F_GRAD_SCALAR = 0x1, 0x2, 0x4, 0x8, 0x10
 ENTRY_LOSS_FWD, ENTRY_LOSS_BWD, ENTRY_LOGPROB, ENTRY_SUPPORT_LOGPROB, ENTRY_SUPPORT_KL = range(5)
 ENTRY_VP_PARTIALS, ENTRY_VP_COMBINE, ENTRY_VP_BWD, ENTRY_LOSS_FWD_BWD = 5, 6, 7, 8
+ENTRY_VP_SUPPORT_PARTIALS, ENTRY_VP_SUPPORT_COMBINE, ENTRY_VP_SUPPORT_BWD = 9, 10, 11
 BWD_CE, BWD_LOGPROB, BWD_SUPPORT_LOGPROB, BWD_SUPPORT_KL = range(4)
 MAX_K = 1024
 
@@ -53,6 +54,12 @@ _SIGS = {
     "lmh_vp_fused_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int64, c_int64] + [_P] * 8
                          + [ctypes.POINTER(lmh_vp_dest), _P, c_size_t, _P]),
     "lmh_vp_reduce_rows_to": (c_int, [c_int, c_int64, c_int64, _P, _P, c_int, c_int64, _P]),
+    "lmh_vp_support_partials": (c_int, [ctypes.POINTER(lmh_shape), c_int64, c_int64] + [_P] * 5
+                                + [c_size_t, _P]),
+    "lmh_vp_support_combine": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 8
+                               + [c_size_t, _P]),
+    "lmh_vp_support_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int, c_int64, c_int64] + [_P] * 9
+                           + [ctypes.POINTER(lmh_vp_dest), _P, c_size_t, _P]),
     "lmh_vp_reduce_rows": (c_int, [c_int, c_int64, c_int64, _P, _P, _P]),
     "lmh_support_kl_fwd_bwd": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 12 + [c_size_t, _P]),
     "lmh_scale_bf16": (c_int, [_P, c_int64, _P, _P]),

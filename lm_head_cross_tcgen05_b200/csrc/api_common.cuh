@@ -68,10 +68,11 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   const int64_t c = s->chunk_rows > 0 ? s->chunk_rows : kDefaultChunk;
   p.c = p.N > 0 ? (c < p.N ? c : p.N) : 0;
   p.nchunks = p.N > 0 ? cdiv(p.N, p.c) : 0;
-  const bool vp_bwd = entry == LMH_ENTRY_VP_BWD;
+  const bool vp_sup = entry == LMH_ENTRY_VP_SUPPORT_PARTIALS || entry == LMH_ENTRY_VP_SUPPORT_BWD;
+  const bool vp_bwd = entry == LMH_ENTRY_VP_BWD || entry == LMH_ENTRY_VP_SUPPORT_BWD;
   const bool bwd = entry == LMH_ENTRY_LOSS_BWD || vp_bwd;
   p.cands = (entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL ||
-             entry == LMH_ENTRY_LOSS_BWD);
+             entry == LMH_ENTRY_LOSS_BWD || vp_sup);
   p.K = p.cands ? (s->K > 0 ? s->K : 1) : 1;
   p.renorm = p.cands && (s->flags & LMH_F_SUPPORT_RENORM);
   const bool fwd_fused = fused && (entry == LMH_ENTRY_LOSS_FWD || entry == LMH_ENTRY_VP_PARTIALS ||
@@ -79,7 +80,8 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
                                    entry == LMH_ENTRY_LOSS_FWD_BWD);
   p.gbuf = !p.renorm && (bwd || fwd_fused);
   p.acc = p.gbuf && dw_without_acc && p.nchunks > 1;
-  const bool stats = !bwd && entry != LMH_ENTRY_VP_COMBINE;
+  const bool stats = !bwd && entry != LMH_ENTRY_VP_COMBINE &&
+                     entry != LMH_ENTRY_VP_SUPPORT_COMBINE;
   const bool partials = stats && !p.renorm;
   size_t o = sizeof(WsHeader);
   auto take = [&](size_t bytes) {
@@ -100,10 +102,11 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
                                           entry == LMH_ENTRY_LOSS_FWD_BWD));
   p.o_alpha = coef ? take(N * 4) : 0;
   p.o_beta = coef ? take(N * p.K * 4) : 0;
-  p.o_lloc = (vp_bwd || entry == LMH_ENTRY_VP_PARTIALS) ? take(N * 4) : 0;
+  // shard-local labels [N], or shard-local candidate ids [N, K]
+  p.o_lloc = (vp_bwd || entry == LMH_ENTRY_VP_PARTIALS || vp_sup) ? take(N * p.K * 4) : 0;
   p.o_gbuf = p.gbuf ? take(static_cast<size_t>(p.c) * p.Vp * 2) : 0;
   p.o_acc = p.acc ? take(static_cast<size_t>(p.V) * p.d * 4) : 0;
-  const bool vp = vp_bwd || entry == LMH_ENTRY_VP_PARTIALS;  // dH leaves in fp32, unsplit
+  const bool vp = vp_bwd || entry == LMH_ENTRY_VP_PARTIALS || vp_sup;  // dH in fp32, unsplit
   if (p.gbuf && p.nchunks > 0 && !vp) {  // the largest split-K partial of any chunk
     const int64_t last = p.N - (p.nchunks - 1) * p.c;
     const int64_t a = dh_splits(p.c, p.d, p.V) > 1 ? dh_splits(p.c, p.d, p.V) * p.c : 0;

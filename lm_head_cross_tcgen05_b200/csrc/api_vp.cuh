@@ -242,6 +242,160 @@ extern "C" lmh_status lmh_vp_fused_bwd(const lmh_shape* shard, int64_t v0, int64
                             dW_acc_shard, ws, st, dH_part, dest ? &sc : nullptr);
 }
 
+// ---------------------------------------------------------------- support entries
+namespace {
+
+// Shard-local candidate ids: c - v0 inside [v0, v0 + Vr), else -1 (padding here).
+lmh_status vp_local_ids(const Plan& P, const int32_t* ids, int64_t v0, const Ws& ws,
+                        cudaStream_t st) {
+  const int64_t n = P.N * P.K;
+  const int64_t blocks = cdiv(n, 256);
+  ProfScope ps(KID_VP_LABELS, st);
+  vp_local_labels_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(
+      n, ids, v0, P.V, ws.at<int32_t>(P.o_lloc));
+  return last_launch();
+}
+
+bool vp_support_shape_ok(const lmh_shape* s) {
+  return s->K >= 1 && s->K <= LMH_MAX_K && !(s->flags & LMH_F_SUPPORT_RENORM);
+}
+
+}  // namespace
+
+extern "C" lmh_status lmh_vp_support_partials(const lmh_shape* shard, int64_t v0,
+                                              int64_t V_total, const lmh_bf16* H,
+                                              const lmh_bf16* W_shard, const int32_t* ids,
+                                              float* records, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  LMH_TRY(vp_args_ok(shard, v0, V_total));
+  if (!vp_support_shape_ok(shard)) return LMH_ERR_INVALID_ARG;
+  const Plan P = make_plan(shard, LMH_ENTRY_VP_SUPPORT_PARTIALS, false, false);
+  int dev, sms;
+  LMH_TRY(common_checks(shard, H, W_shard, workspace, workspace_bytes, P.total, &dev, &sms));
+  if (P.N > 0 && (!ids || !records)) return LMH_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return LMH_OK;
+  LMH_TRY(vp_local_ids(P, ids, v0, ws, st));
+  LMH_TRY(prep_cands(P, ws.at<int32_t>(P.o_lloc), ws, st));
+  Targets tg{};
+  tg.sorted = ws.at<int32_t>(P.o_sorted);
+  tg.nuniq = ws.at<int32_t>(P.o_nuniq);
+  tg.K = static_cast<int>(P.K);
+  for (int64_t ci = 0; ci < P.nchunks; ++ci) {
+    const int64_t r0 = ci * P.c;
+    const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
+    LMH_TRY((run_stats<kCands, false>(P, dev, sms, H, W_shard, tg, r0, rows, ws, st)));
+    ProfScope ps(KID_VP_FINALIZE, st);
+    vp_support_finalize_kernel<<<static_cast<unsigned>(cdiv(rows, 8)), 256, 0, st>>>(
+        rows, r0, static_cast<int>(P.T), static_cast<int>(P.K), ws.at<float>(P.o_pm),
+        ws.at<float>(P.o_ps), ws.at<int32_t>(P.o_rank), ws.at<float>(P.o_zt), P.temp, ws.h,
+        records);
+    LMH_TRY(last_launch());
+  }
+  return LMH_OK;
+}
+
+extern "C" lmh_status lmh_vp_support_combine(const lmh_shape* shape, int R,
+                                             const float* records, const int32_t* ids,
+                                             const float* ref_logp, float* lp, float* lse,
+                                             float* kl_rows, float* kl_mean, void* workspace,
+                                             size_t workspace_bytes, void* stream) {
+  if (!shape_ok(shape) || R < 1 || shape->K < 1 || shape->K > LMH_MAX_K)
+    return LMH_ERR_INVALID_ARG;
+  const Plan P = make_plan(shape, LMH_ENTRY_VP_SUPPORT_COMBINE, false, false);
+  if (!workspace) return LMH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return LMH_ERR_ALIGNMENT;
+  if (workspace_bytes < P.total) return LMH_ERR_WORKSPACE_TOO_SMALL;
+  if (P.N > 0 && (!records || !ids || !lse)) return LMH_ERR_INVALID_ARG;
+  if ((kl_rows || kl_mean) && !ref_logp) return LMH_ERR_INVALID_ARG;
+  if (kl_mean && !kl_rows) return LMH_ERR_INVALID_ARG;
+  int dev, sms;
+  LMH_TRY(current_device(&dev, &sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return empty_call(P, kl_mean, nullptr, nullptr, nullptr, st);
+  {
+    ProfScope ps(KID_VP_COMBINE, st);
+    vp_support_combine_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
+        P.N, R, static_cast<int>(shape->K), static_cast<int>(P.V), records, ids,
+        kl_rows ? ref_logp : nullptr, lp, lse, kl_rows, ws.h);
+  }
+  LMH_TRY(last_launch());
+  if (kl_mean) {
+    ProfScope ps(KID_MEAN, st);
+    mean_kernel<<<1, 1024, 0, st>>>(kl_rows, P.N, 0, nullptr, ws.h, kl_mean);
+    LMH_TRY(last_launch());
+  }
+  return LMH_OK;
+}
+
+extern "C" lmh_status lmh_vp_support_bwd(const lmh_shape* shard, int mode, int64_t v0,
+                                         int64_t V_total, const lmh_bf16* H,
+                                         const lmh_bf16* W_shard, const int32_t* ids,
+                                         const float* lse, const float* grad,
+                                         const float* ref_logp, float* dH_part,
+                                         lmh_bf16* dW_shard, float* dW_acc_shard,
+                                         const lmh_vp_dest* dest, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  LMH_TRY(vp_args_ok(shard, v0, V_total));
+  if (!vp_support_shape_ok(shard)) return LMH_ERR_INVALID_ARG;
+  if (mode != LMH_BWD_SUPPORT_LOGPROB && mode != LMH_BWD_SUPPORT_KL) return LMH_ERR_INVALID_ARG;
+  RowScatter sc;
+  LMH_TRY(vp_dest_ok(dest, dH_part, shard->N, &sc));
+  const Plan P = make_plan(shard, LMH_ENTRY_VP_SUPPORT_BWD, true, dW_shard && !dW_acc_shard);
+  int dev, sms;
+  LMH_TRY(common_checks(shard, H, W_shard, workspace, workspace_bytes, P.total, &dev, &sms));
+  if (P.N > 0 && (!ids || !lse)) return LMH_ERR_INVALID_ARG;
+  if (mode == LMH_BWD_SUPPORT_KL && P.N > 0 && !ref_logp) return LMH_ERR_INVALID_ARG;
+  if ((shard->flags & LMH_F_GRAD_SCALAR) && !grad) return LMH_ERR_INVALID_ARG;
+  if (!aligned16(dH_part) || !aligned16(dW_shard) || !aligned16(dW_acc_shard))
+    return LMH_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
+  LMH_TRY(clear_header(ws, st));
+  if (P.N == 0) return empty_call(P, nullptr, nullptr, dW_shard, dW_acc_shard, st);
+  if (!dH_part && !dest && !dW_shard && !dW_acc_shard) return LMH_OK;
+  LMH_TRY(vp_local_ids(P, ids, v0, ws, st));
+  LMH_TRY(prep_cands(P, ws.at<int32_t>(P.o_lloc), ws, st));
+  const int K = static_cast<int>(P.K);
+  float* alpha = ws.at<float>(P.o_alpha);
+  float* beta = ws.at<float>(P.o_beta);
+  {
+    // beta over this shard's candidates; alpha over every valid candidate of the vocabulary
+    ProfScope ps(KID_BWD_COEF, st);
+    bwd_coef_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
+        mode, P.N, K, static_cast<int>(P.V), ws.at<int32_t>(P.o_lloc), grad, ref_logp,
+        ws.at<int32_t>(P.o_rank), ws.at<int32_t>(P.o_nuniq), P.temp,
+        (shard->flags & LMH_F_MEAN) ? 1 : 0, (shard->flags & LMH_F_GRAD_SCALAR) ? 1 : 0, ws.h,
+        alpha, beta, nullptr, ids, static_cast<int>(V_total));
+  }
+  LMH_TRY(last_launch());
+  Targets tg{};
+  tg.sorted = ws.at<int32_t>(P.o_sorted);
+  tg.nuniq = ws.at<int32_t>(P.o_nuniq);
+  tg.K = K;
+  for (int64_t ci = 0; ci < P.nchunks; ++ci) {
+    const int64_t r0 = ci * P.c;
+    const int rows = static_cast<int>(P.N - r0 < P.c ? P.N - r0 : P.c);
+    CUtensorMap ta, tb, tc;
+    if (!tmap_2d(&ta, H + r0 * P.d, P.d, rows, P.d, BM) ||
+        !tmap_2d(&tb, W_shard, P.d, P.V, P.d, BNH) ||
+        !tmap_out(&tc, ws.at<__nv_bfloat16>(P.o_gbuf), P.Vp, rows, P.Vp))
+      return LMH_ERR_CUDA;
+    EpiGrad<kCands>::Params ep{rows, r0, static_cast<int>(P.V), P.Vp, tg, lse, alpha, beta,
+                               P.temp};
+    LMH_TRY(launch_gemm<EpiGrad<kCands>>(dev, sms, ta, tb, tc, rows, P.V, P.d, kOrderLogits,
+                                         &ws.h->err, ep, st));
+    LMH_TRY(run_backward_gemms(P, dev, sms, H, W_shard, r0, rows, static_cast<int>(ci), nullptr,
+                               dW_shard, dW_acc_shard, ws, st, dH_part,
+                               dest ? &sc : nullptr));
+  }
+  return LMH_OK;
+}
+
 extern "C" lmh_status lmh_vp_reduce_rows(int R, int64_t rows, int64_t d, const float* parts,
                                          lmh_bf16* out, void* stream) {
   if (R < 1 || rows < 0 || d <= 0 || (d % 64) != 0) return LMH_ERR_INVALID_ARG;

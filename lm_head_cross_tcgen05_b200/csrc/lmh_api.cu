@@ -24,8 +24,10 @@ using namespace lmh;
 // ============================================================================ C ABI
 
 extern "C" size_t lmh_workspace_size(const lmh_shape* shape, int entry) {
-  if (!shape_ok(shape) || entry < LMH_ENTRY_LOSS_FWD || entry > LMH_ENTRY_LOSS_FWD_BWD) return 0;
-  if ((entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL) &&
+  if (!shape_ok(shape) || entry < LMH_ENTRY_LOSS_FWD || entry > LMH_ENTRY_VP_SUPPORT_BWD) return 0;
+  if ((entry == LMH_ENTRY_SUPPORT_LOGPROB || entry == LMH_ENTRY_SUPPORT_KL ||
+       entry == LMH_ENTRY_VP_SUPPORT_PARTIALS || entry == LMH_ENTRY_VP_SUPPORT_COMBINE ||
+       entry == LMH_ENTRY_VP_SUPPORT_BWD) &&
       (shape->K < 1 || shape->K > LMH_MAX_K))
     return 0;
   const bool fused = (entry == LMH_ENTRY_LOSS_FWD || entry == LMH_ENTRY_VP_PARTIALS ||

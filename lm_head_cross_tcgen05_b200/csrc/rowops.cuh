@@ -326,14 +326,17 @@ __global__ void support_out_kernel(long long N, int K, const int32_t* __restrict
 // G = alpha P - sum beta e_t for the four objectives; one warp per row.
 // Without `grad` every row term has the weight 1, or 1 / count with `mean` (count: the valid
 // rows of the labels for CE / LOGPROB, N for the support objectives); with `scalar` grad[0]
-// multiplies that weight instead of grad holding one weight per term.
+// multiplies that weight instead of grad holding one weight per term. beta covers the
+// candidates of `rank` (this vocabulary or shard); alpha all valid ones (see alpha_ids).
 __global__ void bwd_coef_kernel(int mode, long long N, int K, int V,
                                 const int32_t* __restrict__ targets,
                                 const float* __restrict__ grad, const float* __restrict__ ref,
                                 const int32_t* __restrict__ rank,
                                 const int32_t* __restrict__ nuniq, Temperature temp, int mean,
                                 int scalar, WsHeader* h, float* __restrict__ alpha,
-                                float* __restrict__ beta, const int32_t* n_given = nullptr) {
+                                float* __restrict__ beta, const int32_t* n_given = nullptr,
+                                const int32_t* __restrict__ alpha_ids = nullptr,
+                                int alpha_V = 0) {
   const int lane = threadIdx.x & 31;
   const long long i = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5);
   if (i >= N) return;
@@ -364,7 +367,11 @@ __global__ void bwd_coef_kernel(int mode, long long N, int K, int V,
   const float gi = (mode == 3) ? (grad ? grad[i] : unit) * it : 0.f;
   float sum = 0.f;
   for (int k = lane; k < K; k += 32) {
-    if (rank[i * K + k] < 0) continue;
+    // alpha sums every valid candidate: of this vocabulary (rank >= 0), or, for one shard of a
+    // split vocabulary, of the whole one (alpha_ids: the global ids, valid below alpha_V)
+    const bool counted = alpha_ids ? (alpha_ids[i * K + k] >= 0 && alpha_ids[i * K + k] < alpha_V)
+                                   : rank[i * K + k] >= 0;
+    if (!counted) continue;
     sum += (mode == 2) ? (grad ? grad[i * K + k] : unit) * it : gi * expf(ref[i * K + k]);
   }
   sum = warp_sum(sum);

@@ -104,6 +104,87 @@ __global__ void vp_combine_kernel(long long N, int R, int V, const float4* __res
   }
 }
 
+// ---------------------------------------------------------------------------- support entries
+// Record of row i on rank r for the support entries (K + 1 floats): [0] lse_r as above, then
+// for every slot k the logit of candidate c_ik if it lies in the shard, else -inf.
+// One warp per row of a chunk; sorted / rank describe the shard-local candidates.
+__global__ void vp_support_finalize_kernel(int rows, long long row0, int T, int K,
+                                           const float* __restrict__ part_m,
+                                           const float* __restrict__ part_s,
+                                           const int32_t* __restrict__ rank,
+                                           const float* __restrict__ zt, Temperature temp,
+                                           WsHeader* h, float* __restrict__ rec) {
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const long long grow = row0 + row;
+  const float* pm = part_m + static_cast<long long>(row) * T;
+  const float* ps = part_s + static_cast<long long>(row) * T;
+  float M = -__int_as_float(0x7f800000);
+  for (int t = lane; t < T; t += 32) M = fmaxf(M, pm[t]);
+  M = warp_max(M);
+  const float moff = -M * kLog2e;
+  float S = 0.f;
+  for (int t = lane; t < T; t += 32) S += ps[t] * fast_exp2(fmaf(pm[t], kLog2e, moff));
+  S = warp_sum(S);
+  float* out = rec + grow * (K + 1);
+  if (lane == 0) {
+    const float l = M + logf(S);
+    if (!isfinite(l)) atomicOr(&h->err, kErrNonFinite);
+    if (temp.rows && !temperature_ok(temp.rows[grow])) atomicOr(&h->err, kErrTemperature);
+    out[0] = l;
+  }
+  for (int k = lane; k < K; k += 32) {
+    const int r = rank[grow * K + k];
+    out[1 + k] = r >= 0 ? zt[grow * K + r] : -__int_as_float(0x7f800000);
+  }
+}
+
+// One warp per row: the R support records (rank order) of the row into lse (as for the CE
+// records), lp_ik = z_ik - lse_i with z_ik the one finite candidate logit over the ranks (0 for
+// padding ids < 0; ids >= V flagged and treated as padding), and with ref the KL term
+// sum_k exp(r_ik) (r_ik - lp_ik) over the valid slots.
+__global__ void vp_support_combine_kernel(long long N, int R, int K, int V,
+                                          const float* __restrict__ rec,
+                                          const int32_t* __restrict__ ids,
+                                          const float* __restrict__ ref, float* __restrict__ lp,
+                                          float* __restrict__ lse, float* __restrict__ kl,
+                                          WsHeader* h) {
+  const int lane = threadIdx.x & 31;
+  const long long i = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (i >= N) return;
+  const long long rs = N * (K + 1);  // one rank's records
+  float l = 0.f;
+  if (lane == 0) {
+    float m = -__int_as_float(0x7f800000);
+    for (int r = 0; r < R; ++r) m = fmaxf(m, rec[r * rs + i * (K + 1)]);
+    const float moff = -m * kLog2e;
+    float s = 0.f;
+    for (int r = 0; r < R; ++r) s += fast_exp2(fmaf(rec[r * rs + i * (K + 1)], kLog2e, moff));
+    l = m + logf(s);
+    lse[i] = l;
+    if (!isfinite(l)) atomicOr(&h->err, kErrNonFinite);
+  }
+  l = __shfl_sync(0xffffffffu, l, 0);
+  float acc = 0.f;
+  for (int k = lane; k < K; k += 32) {
+    const int id = ids[i * K + k];
+    if (id >= V) atomicOr(&h->err, kErrLabelRange);
+    const bool valid = id >= 0 && id < V;
+    float z = -__int_as_float(0x7f800000);
+    for (int r = 0; r < R; ++r) z = fmaxf(z, rec[r * rs + i * (K + 1) + 1 + k]);
+    if (valid && !isfinite(z)) atomicOr(&h->err, kErrNonFinite);
+    const float v = valid ? z - l : 0.f;
+    if (lp) lp[i * K + k] = v;
+    if (ref && valid) {
+      const float rr = ref[i * K + k];
+      acc += expf(rr) * (rr - v);
+    }
+  }
+  acc = warp_sum(acc);
+  if (kl && lane == 0) kl[i] = acc;
+}
+
 // Fused backward of a shard, one warp per row: the tile factors that turn the stored
 // p~ = exp(z - m_t) into the softmax gradient with the combined lse,
 //   s_t = alpha_i exp(m_t - lse_i),  alpha_i = weight of row i / tau_i,

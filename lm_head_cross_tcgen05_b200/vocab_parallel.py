@@ -38,12 +38,14 @@ from typing import List, Optional, Tuple
 import torch
 import torch.distributed as dist
 
-from . import (BWD_CE, ENTRY_VP_BWD, ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS, F_DW_ACC_GIVEN,
-               F_FUSED_BWD, F_MEAN, lmh_vp_combine, lmh_vp_fused_bwd, lmh_vp_loss_bwd,
-               lmh_vp_partials, lmh_vp_reduce_rows, lmh_vp_reduce_rows_to, make_shape,
-               workspace)
+from . import (BWD_CE, BWD_SUPPORT_KL, ENTRY_VP_BWD, ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS,
+               ENTRY_VP_SUPPORT_BWD, ENTRY_VP_SUPPORT_COMBINE, ENTRY_VP_SUPPORT_PARTIALS,
+               F_DW_ACC_GIVEN, F_FUSED_BWD, F_GRAD_SCALAR, F_MEAN, lmh_vp_combine,
+               lmh_vp_fused_bwd, lmh_vp_loss_bwd, lmh_vp_partials, lmh_vp_reduce_rows,
+               lmh_vp_reduce_rows_to, lmh_vp_support_bwd, lmh_vp_support_combine,
+               lmh_vp_support_partials, make_shape, workspace)
 
-__all__ = ["shard_plan", "row_slices", "CudaOps", "VocabParallelCE"]
+__all__ = ["shard_plan", "row_slices", "CudaOps", "VocabParallelCE", "VocabParallelSupport"]
 
 
 def shard_plan(V: int, R: int) -> List[Tuple[int, int]]:
@@ -143,12 +145,52 @@ class CudaOps:
         lmh_vp_reduce_rows(parts, out)
         return out
 
+    # support entries: records [N, K + 1] (lse_r, then the candidates' logits or -inf)
+    def support_partials(self, H, W_shard, ids, v0, V_total, chunk_rows=0, temperature=None):
+        N, d = H.shape
+        K = ids.shape[1]
+        shard = make_shape(N, d, W_shard.shape[0], K, chunk_rows, 0, temperature)
+        ws = workspace(shard, ENTRY_VP_SUPPORT_PARTIALS, H.device)
+        rec = torch.empty(N, K + 1, dtype=torch.float32, device=H.device)
+        lmh_vp_support_partials(shard, v0, V_total, H, W_shard, ids, rec, workspace=ws)
+        return rec
 
-class VocabParallelCE:
-    """Cross entropy (and the per-row log-prob objective) with W split over the ranks of
-    ``group``. Every rank calls ``forward`` and ``backward`` with its own shard
-    ``W[v0:v1]`` (``self.v0``, ``self.v1``) and the same H, labels and options. Without an
-    initialised process group it runs as the only rank (R = 1, no collective)."""
+    def support_combine(self, records, ids, ref_logp, V_total, d):
+        R, N, _ = records.shape
+        K = ids.shape[1]
+        shape = make_shape(N, d, V_total, K, 0, 0)
+        ws = workspace(shape, ENTRY_VP_SUPPORT_COMBINE, records.device)
+        f32, dev = torch.float32, records.device
+        out = dict(lp=torch.empty(N, K, dtype=f32, device=dev),
+                   lse=torch.empty(N, dtype=f32, device=dev))
+        if ref_logp is not None:
+            out["kl_rows"] = torch.empty(N, dtype=f32, device=dev)
+            out["kl_mean"] = torch.empty(1, dtype=f32, device=dev)
+        lmh_vp_support_combine(shape, R, records, ids, ref_logp, out["lp"], out["lse"],
+                               out.get("kl_rows"), out.get("kl_mean"), workspace=ws)
+        return out
+
+    def support_backward(self, mode, H, W_shard, ids, lse, grad, ref_logp, v0, V_total,
+                         chunk_rows=0, mean=True, temperature=None, dW_acc=None, want_dW=True,
+                         dest=None, scalar_grad=False):
+        N, d = H.shape
+        Vr, K = W_shard.shape[0], ids.shape[1]
+        flags = ((F_MEAN if mean else 0) | (F_DW_ACC_GIVEN if dW_acc is not None else 0)
+                 | (F_GRAD_SCALAR if scalar_grad else 0))
+        shard = make_shape(N, d, Vr, K, chunk_rows, flags, temperature)
+        ws = workspace(shard, ENTRY_VP_SUPPORT_BWD, H.device)
+        dH_part = None if dest else torch.empty(N, d, dtype=torch.float32, device=H.device)
+        dW = torch.empty(Vr, d, dtype=torch.bfloat16, device=H.device) if want_dW else None
+        lmh_vp_support_bwd(shard, mode, v0, V_total, H, W_shard, ids, lse, grad, ref_logp,
+                           dH_part, dW, dW_acc, dest, workspace=ws)
+        return dH_part, dW
+
+
+class _VocabParallel:
+    """The shard plan of ``group``'s ranks and the exchange steps every vocabulary-parallel
+    objective shares: gathering per-row records, and summing the ranks' dH contributions in
+    a fixed order (collectives, or peer-memory stores with ``p2p``). Without an initialised
+    process group it runs as the only rank (R = 1, no collective)."""
 
     def __init__(self, V_total: int, group=None, chunk_rows: int = 0, mean: bool = True,
                  temperature=None, ops=None, p2p: bool = False):
@@ -170,63 +212,25 @@ class VocabParallelCE:
             raise ValueError(f"rank {self.rank} holds rows [{self.v0}, {self.v1}) of W, "
                              f"got {W_shard.shape[0]} rows")
 
-    def _combine(self, rec, labels, d, n_valid_given):
-        N = rec.shape[0]
+    def _gather(self, rec):
+        """[N, w] records of this rank -> [R, N, w] of all ranks in rank order."""
+        N, w = rec.shape
         if self.R == 1:
-            every = rec.reshape(-1)
-        else:
-            every = torch.empty(self.R * N * 4, dtype=rec.dtype, device=rec.device)
-            dist.all_gather_into_tensor(every, rec.reshape(-1).contiguous(), group=self.group)
-        return self.ops.combine(every.view(self.R, N, 4), labels, self.V_total, d, n_valid_given)
+            return rec.view(1, N, w)
+        every = torch.empty(self.R * N * w, dtype=rec.dtype, device=rec.device)
+        dist.all_gather_into_tensor(every, rec.reshape(-1).contiguous(), group=self.group)
+        return every.view(self.R, N, w)
 
-    def forward(self, H, W_shard, labels, n_valid_given=None) -> dict:
-        """loss_rows, lse, logprob, argmax, loss_mean, n_valid: the same on every rank."""
-        self._check_shard(W_shard)
-        rec = self.ops.partials(H, W_shard, labels, self.v0, self.V_total, self.chunk_rows,
-                                self.temperature)
-        return self._combine(rec, labels, H.shape[1], n_valid_given)
-
-    def forward_backward(self, H, W_shard, labels, n_valid_given=None,
-                         dW_acc: Optional[torch.Tensor] = None, want_dW: bool = True) -> dict:
-        """forward() plus dH and this rank's dW of the loss (mean or sum), in one pass: the
-        backward reuses the forward's softmax numerators instead of recomputing the logits.
-        All rows form one chunk (chunk_rows is not used)."""
-        self._check_shard(W_shard)
-        rec, state = self.ops.partials_fused(H, W_shard, labels, self.v0, self.V_total,
-                                             self.mean, self.temperature)
-        out = self._combine(rec, labels, H.shape[1], n_valid_given)
+    def _dH(self, run, N, d, device):
+        """dH summed over the ranks from run(dest) -> (dH_part or None, dW): collectives, or
+        with p2p the rows scattered straight to their reducing ranks."""
         if self.p2p:
-            sym = self._symmetric(H.shape[0], H.shape[1], H.device)
-            sym["recv_h"].barrier(channel=0)  # no rank still reads its last receive buffer
-            _, dW = self.ops.fused_backward(state, H, W_shard, labels, out["lse"], self.v0,
-                                            self.V_total, n_valid_given, dW_acc, want_dW,
-                                            dest=(sym["recv_tab"], self.R, self.rank))
-            out["dH"] = self._reduce_p2p(sym)
-        else:
-            dH_part, dW = self.ops.fused_backward(state, H, W_shard, labels, out["lse"],
-                                                  self.v0, self.V_total, n_valid_given, dW_acc,
-                                                  want_dW)
-            out["dH"] = self._sum_rows(dH_part)
-        out["dW"] = dW
-        return out
-
-    def backward(self, H, W_shard, labels, lse, grad=None, mode: int = BWD_CE,
-                 dW_acc: Optional[torch.Tensor] = None, want_dW: bool = True) -> dict:
-        """dH [N, d] (the same on every rank) and this rank's dW shard [v1 - v0, d]."""
-        self._check_shard(W_shard)
-        N, d = H.shape
-        if self.p2p:
-            sym = self._symmetric(N, d, H.device)
-            sym["recv_h"].barrier(channel=0)
-            _, dW = self.ops.backward(mode, H, W_shard, labels, lse, grad, self.v0,
-                                      self.V_total, self.chunk_rows, self.mean,
-                                      self.temperature, dW_acc, want_dW,
-                                      dest=(sym["recv_tab"], self.R, self.rank))
-            return dict(dH=self._reduce_p2p(sym), dW=dW)
-        dH_part, dW = self.ops.backward(mode, H, W_shard, labels, lse, grad, self.v0,
-                                        self.V_total, self.chunk_rows, self.mean,
-                                        self.temperature, dW_acc, want_dW)
-        return dict(dH=self._sum_rows(dH_part), dW=dW)
+            sym = self._symmetric(N, d, device)
+            sym["recv_h"].barrier(channel=0)   # no rank still reads its last receive buffer
+            _, dW = run((sym["recv_tab"], self.R, self.rank))
+            return self._reduce_p2p(sym), dW
+        dH_part, dW = run(None)
+        return self._sum_rows(dH_part), dW
 
     def _symmetric(self, N, d, device):
         """The receive buffer ([R][rows_j][d] fp32 within R * max_rows * d) and the full bf16
@@ -286,3 +290,74 @@ class VocabParallelCE:
         if all(n == top for n in sizes):
             return every
         return torch.cat([every[j * top: j * top + sizes[j]] for j in range(self.R)])
+
+
+class VocabParallelCE(_VocabParallel):
+    """Cross entropy (and the per-row log-prob objective) with W split over the ranks of
+    ``group``. Every rank calls ``forward`` and ``backward`` (or ``forward_backward``) with its
+    own shard ``W[v0:v1]`` (``self.v0``, ``self.v1``) and the same H, labels and options."""
+
+    def forward(self, H, W_shard, labels, n_valid_given=None) -> dict:
+        """loss_rows, lse, logprob, argmax, loss_mean, n_valid: the same on every rank."""
+        self._check_shard(W_shard)
+        rec = self.ops.partials(H, W_shard, labels, self.v0, self.V_total, self.chunk_rows,
+                                self.temperature)
+        return self.ops.combine(self._gather(rec), labels, self.V_total, H.shape[1],
+                                n_valid_given)
+
+    def forward_backward(self, H, W_shard, labels, n_valid_given=None,
+                         dW_acc: Optional[torch.Tensor] = None, want_dW: bool = True) -> dict:
+        """forward() plus dH and this rank's dW of the loss (mean or sum), in one pass: the
+        backward reuses the forward's softmax numerators instead of recomputing the logits.
+        All rows form one chunk (chunk_rows is not used)."""
+        self._check_shard(W_shard)
+        N, d = H.shape
+        rec, state = self.ops.partials_fused(H, W_shard, labels, self.v0, self.V_total,
+                                             self.mean, self.temperature)
+        out = self.ops.combine(self._gather(rec), labels, self.V_total, d, n_valid_given)
+        out["dH"], out["dW"] = self._dH(
+            lambda dest: self.ops.fused_backward(state, H, W_shard, labels, out["lse"], self.v0,
+                                                 self.V_total, n_valid_given, dW_acc, want_dW,
+                                                 dest=dest), N, d, H.device)
+        return out
+
+    def backward(self, H, W_shard, labels, lse, grad=None, mode: int = BWD_CE,
+                 dW_acc: Optional[torch.Tensor] = None, want_dW: bool = True) -> dict:
+        """dH [N, d] (the same on every rank) and this rank's dW shard [v1 - v0, d]."""
+        self._check_shard(W_shard)
+        N, d = H.shape
+        dH, dW = self._dH(
+            lambda dest: self.ops.backward(mode, H, W_shard, labels, lse, grad, self.v0,
+                                           self.V_total, self.chunk_rows, self.mean,
+                                           self.temperature, dW_acc, want_dW, dest=dest),
+            N, d, H.device)
+        return dict(dH=dH, dW=dW)
+
+
+class VocabParallelSupport(_VocabParallel):
+    """The support-set entries with W split over the ranks: log-probs at K candidate ids per
+    row (full-vocabulary normaliser) and the KL against reference log-probs, and the backward of
+    sum_ik g_ik lp_ik (BWD_SUPPORT_LOGPROB) or of the (mean) KL (BWD_SUPPORT_KL). Each rank
+    reports its lse and the logits of the candidates in its shard (K + 1 floats per row)."""
+
+    def forward(self, H, W_shard, ids, ref_logp=None) -> dict:
+        """lp [N, K], lse [N] (and kl_rows, kl_mean with ref_logp): the same on every rank."""
+        self._check_shard(W_shard)
+        rec = self.ops.support_partials(H, W_shard, ids, self.v0, self.V_total, self.chunk_rows,
+                                        self.temperature)
+        return self.ops.support_combine(self._gather(rec), ids, ref_logp, self.V_total,
+                                        H.shape[1])
+
+    def backward(self, H, W_shard, ids, lse, mode: int = BWD_SUPPORT_KL, grad=None,
+                 ref_logp=None, dW_acc: Optional[torch.Tensor] = None,
+                 want_dW: bool = True, scalar_grad: bool = False) -> dict:
+        """dH [N, d] (the same on every rank) and this rank's dW shard."""
+        self._check_shard(W_shard)
+        N, d = H.shape
+        dH, dW = self._dH(
+            lambda dest: self.ops.support_backward(mode, H, W_shard, ids, lse, grad, ref_logp,
+                                                   self.v0, self.V_total, self.chunk_rows,
+                                                   self.mean, self.temperature, dW_acc, want_dW,
+                                                   dest=dest, scalar_grad=scalar_grad),
+            N, d, H.device)
+        return dict(dH=dH, dW=dW)

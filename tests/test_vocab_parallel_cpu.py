@@ -106,3 +106,51 @@ def test_vocab_parallel_exchange_gloo(world, case):
         assert r["nvalid"] and r["argmax"]
         assert r["dH"] < 1e-9 and r["dW"] < 1e-9
     assert len({r["dH_digest"] for r in res}) == 1   # every rank holds the same dH
+
+
+def _support_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from lm_head_cross_tcgen05_b200.vocab_parallel import VocabParallelSupport
+        from oracle import lmh_oracle as O
+        from tests.vp_oracle_ops import OracleOps
+        from workloads import make_inputs, ragged
+        N, d, V, K = 24, 64, 900, 6
+        x = make_inputs(ragged(N, d, V, seed=91, K=K), device="cpu")
+        H, W, ids, ref = x["H"], x["W"], x["ids"].clone(), x["ref_logp"]
+        ids[0, -1] = -1                       # padding
+        ids[1, 1] = ids[1, 0]                 # a repeated id
+        vp = VocabParallelSupport(V, ops=OracleOps())
+        Ws = W[vp.v0:vp.v1]
+        f = vp.forward(H, Ws, ids, ref)
+        b = vp.backward(H, Ws, ids, f["lse"], mode=O.BWD_SUPPORT_KL, ref_logp=ref)
+        g = np.linspace(-1, 1, N * K).reshape(N, K)
+        b2 = vp.backward(H, Ws, ids, f["lse"], mode=O.BWD_SUPPORT_LOGPROB,
+                         grad=torch.from_numpy(g))
+        rk = O.support_kl(H, W, ids, ref)
+        rb = O.backward(O.BWD_SUPPORT_KL, H, W, ids, np.full(N, 1.0 / N), ref)
+        rb2 = O.backward(O.BWD_SUPPORT_LOGPROB, H, W, ids, g)
+        err = lambda a, r: np.abs(a.numpy() - r).max() / max(np.abs(r).max(), 1e-300)
+        q.put(dict(rank=rank, lp=err(f["lp"], rk["lp"]), lse=err(f["lse"], rk["lse"]),
+                   kl=err(f["kl_rows"], rk["kl_rows"]),
+                   dH=err(b["dH"], rb["dH"]), dW=err(b["dW"], rb["dW"][vp.v0:vp.v1]),
+                   dH2=err(b2["dH"], rb2["dH"]), dW2=err(b2["dW"], rb2["dW"][vp.v0:vp.v1])))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_vocab_parallel_support_exchange_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_support_worker, args=(r, 3, port, q)) for r in range(3)]
+    for p in ps:
+        p.start()
+    res = [q.get(timeout=180) for _ in ps]
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in res:
+        for k in ("lp", "lse", "kl", "dH", "dW", "dH2", "dW2"):
+            assert r[k] < 1e-9, (r["rank"], k, r[k])

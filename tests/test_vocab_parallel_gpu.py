@@ -287,3 +287,65 @@ def test_row_scatter_argument_checks():
         with pytest.raises(L.LmhError, match="INVALID_ARG"):
             L.lmh_vp_loss_bwd(shard, L.BWD_CE, 0, V, x["H"], x["W"][:300], x["labels"], lse,
                               None, dh, None, None, dest, workspace=ws)
+
+
+def _emulate_support(x, ids, V, R, mode, grad=None, ref=None, tau=None, chunk=0):
+    H, W = x["H"], x["W"]
+    d = H.shape[1]
+    ops = CudaOps()
+    plan = shard_plan(V, R)
+    recs = [ops.support_partials(H, W[a:b], ids, a, V, chunk, tau) for a, b in plan]
+    f = ops.support_combine(torch.stack(recs), ids, ref, V, d)
+    parts, dWs = zip(*[ops.support_backward(mode, H, W[a:b], ids, f["lse"], grad, ref, a, V,
+                                            chunk, True, tau) for a, b in plan])
+    f["dH"] = ops.reduce_rows(torch.stack(list(parts)))
+    f["dW"] = torch.cat(dWs)
+    torch.cuda.synchronize()
+    return f
+
+
+@pytest.mark.parametrize("N,d,V,K,R,chunk,tau", [
+    (150, 128, 2500, 16, 2, 0, None),
+    (96, 256, 5000, 8, 3, 40, "scalar"),    # three row chunks, a temperature
+    (64, 128, 2048, 64, 8, 0, None),        # 8 shards of 256: most candidates off-shard
+])
+def test_vocab_parallel_support_matches_oracle(N, d, V, K, R, chunk, tau):
+    x, xc = device_inputs(ragged(N, d, V, seed=5000 + N, K=K))
+    ids = x["ids"].clone()
+    ids[0, -1] = -1                  # padding
+    ids[1, 1] = ids[1, 0]            # a repeated id counts once per slot
+    ids[2, 0] = V + 3                # out of range: padding (and flagged)
+    ids_c = ids.cpu()
+    t_dev, t_ref = (0.75, 0.75) if tau else (None, None)
+    out = _emulate_support(x, ids, V, R, L.BWD_SUPPORT_KL, ref=x["ref_logp"], tau=t_dev,
+                           chunk=chunk)
+    rk = O.support_kl(xc["H"], xc["W"], ids_c, xc["ref_logp"], tau=t_ref)
+    check_rows(out["lp"], rk["lp"], what="lp")
+    check_rows(out["lse"], rk["lse"], what="lse")
+    check_rows(out["kl_rows"], rk["kl_rows"], what="kl_rows")
+    check_rows(out["kl_mean"], np.array([rk["kl_mean"]]), what="kl_mean")
+    ref = O.backward(O.BWD_SUPPORT_KL, xc["H"], xc["W"], ids_c, np.full(N, 1.0 / N),
+                     xc["ref_logp"], tau=t_ref)
+    check_grad(out["dH"], ref["dH"], "dH KL")
+    check_grad(out["dW"], ref["dW"], "dW KL")
+    again = _emulate_support(x, ids, V, R, L.BWD_SUPPORT_KL, ref=x["ref_logp"], tau=t_dev,
+                             chunk=chunk)
+    assert torch.equal(again["dH"], out["dH"]) and torch.equal(again["lp"], out["lp"])
+    gam = torch.linspace(-1.0, 1.0, N * K, dtype=torch.float32).view(N, K)
+    lpo = _emulate_support(x, ids, V, R, L.BWD_SUPPORT_LOGPROB, grad=gam.cuda(), tau=t_dev,
+                           chunk=chunk)
+    ref2 = O.backward(O.BWD_SUPPORT_LOGPROB, xc["H"], xc["W"], ids_c, gam.numpy(), tau=t_ref)
+    check_grad(lpo["dH"], ref2["dH"], "dH support log-prob")
+    check_grad(lpo["dW"], ref2["dW"], "dW support log-prob")
+    one = L.support_logprob(x["H"], x["W"], ids, chunk_rows=chunk, temperature=t_dev)
+    assert (one["lse"] - out["lse"]).abs().max().item() < 1e-4
+
+
+def test_vocab_parallel_support_refuses_renorm():
+    N, d, V, K = 16, 64, 600, 4
+    x, _ = device_inputs(ragged(N, d, V, seed=5100, K=K))
+    shard = L.make_shape(N, d, 300, K, 0, L.F_SUPPORT_RENORM)
+    ws = L.workspace(L.make_shape(N, d, 300, K), L.ENTRY_VP_SUPPORT_PARTIALS, "cuda")
+    rec = torch.empty(N, K + 1, dtype=torch.float32, device="cuda")
+    with pytest.raises(L.LmhError, match="INVALID_ARG"):
+        L.lmh_vp_support_partials(shard, 0, V, x["H"], x["W"][:300], x["ids"], rec, workspace=ws)

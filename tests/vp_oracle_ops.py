@@ -72,6 +72,56 @@ class OracleOps:
         return self.backward(0, H, W_shard, labels, lse, grad, v0, V_total, 0, state["mean"],
                              state["temperature"], dW_acc, want_dW)
 
+    # support entries
+    def support_partials(self, H, W_shard, ids, v0, V_total, chunk_rows=0, temperature=None):
+        z = O.logits(H, W_shard, temperature)
+        c = O.as_i64(ids)
+        loc = c - v0
+        inside = (loc >= 0) & (loc < z.shape[1])
+        zc = np.where(inside, z[np.arange(z.shape[0])[:, None], np.clip(loc, 0, z.shape[1] - 1)],
+                      -np.inf)
+        return _t(np.concatenate([O.logsumexp_rows(z)[:, None], zc], axis=1))
+
+    def support_combine(self, records, ids, ref_logp, V_total, d):
+        r = records.numpy()
+        lse = np.logaddexp.reduce(r[:, :, 0], axis=0)
+        z = r[:, :, 1:].max(axis=0)
+        c = O.as_i64(ids)
+        ok = (c >= 0) & (c < V_total)
+        lp = np.where(ok, z - lse[:, None], 0.0)
+        out = dict(lp=_t(lp), lse=_t(lse))
+        if ref_logp is not None:
+            rr = O.as_f64(ref_logp).reshape(c.shape)
+            kl = np.where(ok, np.exp(rr) * (rr - lp), 0.0).sum(axis=1)
+            out.update(kl_rows=_t(kl), kl_mean=_t([kl.sum() / len(kl)]))
+        return out
+
+    def support_backward(self, mode, H, W_shard, ids, lse, grad, ref_logp, v0, V_total,
+                         chunk_rows=0, mean=True, temperature=None, dW_acc=None, want_dW=True,
+                         dest=None, scalar_grad=False):
+        z = O.logits(H, W_shard, temperature)
+        N, Vr = z.shape
+        c = O.as_i64(ids)
+        K = c.shape[1]
+        ok = (c >= 0) & (c < V_total)
+        unit = (1.0 / N if N else 0.0) if mean else 1.0
+        if mode == 2:   # sum_ik g_ik lp_ik
+            g = np.full((N, K), unit) if grad is None else O.as_f64(grad).reshape(N, K)
+            w = -g
+        else:           # sum_i g_i KL_i
+            g = np.full(N, unit) if grad is None else O.as_f64(grad).reshape(N)
+            w = g[:, None] * np.exp(O.as_f64(ref_logp).reshape(N, K))
+        w = np.where(ok, w, 0.0)
+        P = np.exp(z - O.as_f64(lse)[:, None])
+        G = w.sum(axis=1)[:, None] * P
+        loc = c - v0
+        hit = ok & (loc >= 0) & (loc < Vr)
+        for i, k in zip(*np.nonzero(hit)):
+            G[i, loc[i, k]] -= w[i, k]
+        G = G / O.tau_rows(temperature, N)[:, None]
+        dH, dW = O.lm_head_backward(H, W_shard, G)
+        return _t(dH), (_t(dW) if want_dW else None)
+
     def reduce_rows(self, parts):
         out = parts[0].clone()
         for r in range(1, parts.shape[0]):
