@@ -413,6 +413,22 @@ LMH_API lmh_status lmh_vp_reduce_rows_to(int R, int64_t rows, int64_t d, const f
  *   LMH_F_SUPPORT_RENORM is refused (LMH_ERR_INVALID_ARG): that reading's backward is the
  *   sparse path of lmh_loss_bwd, which has no logits GEMM to save.
  */
+/*
+ * lmh_support_fwd_bwd — the general one-pass support entry: the forward of lmh_support_kl
+ * (mode LMH_BWD_SUPPORT_KL; ref_logp and kl_rows required) or of lmh_support_logprob (mode
+ * LMH_BWD_SUPPORT_LOGPROB; kl outputs and ref_logp unused), plus the backward of
+ * L = sum_i g_i KL_i or L = sum_ik g_ik lp_ik with weights known before the call: grad [N]
+ * (KL) or [N, K] (log-probs), one shared grad[0] with LMH_F_GRAD_SCALAR, or 1 with grad NULL;
+ * each times 1 / N with LMH_F_MEAN. Workspace and outputs as lmh_support_kl_fwd_bwd, which is
+ * this entry with mode LMH_BWD_SUPPORT_KL and grad NULL.
+ */
+LMH_API lmh_status lmh_support_fwd_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,
+                                       const lmh_bf16* W, const int32_t* ids,
+                                       const float* ref_logp, const float* grad, float* kl_rows,
+                                       float* kl_mean, float* lp, float* lse, lmh_bf16* dH,
+                                       lmh_bf16* dW, float* dW_acc, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
 LMH_API lmh_status lmh_support_kl_fwd_bwd(const lmh_shape* shape, const lmh_bf16* H,
                                           const lmh_bf16* W, const int32_t* ids,
                                           const float* ref_logp, float* kl_rows, float* kl_mean,

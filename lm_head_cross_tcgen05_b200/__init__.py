@@ -28,6 +28,7 @@ from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEV
 __all__ = [
     "lmh_shape", "make_shape", "lmh_workspace_size", "lmh_loss_fwd", "lmh_loss_bwd",
     "lmh_logprob", "lmh_support_logprob", "lmh_support_kl", "lmh_support_kl_fwd_bwd",
+    "lmh_support_fwd_bwd", "support_fwd_bwd",
     "lmh_read_errors", "LmhError",
     "loss_fwd", "loss_bwd", "logprob", "support_logprob", "support_kl", "workspace",
     "IGNORE_INDEX", "BWD_CE", "BWD_LOGPROB", "BWD_SUPPORT_LOGPROB", "BWD_SUPPORT_KL",
@@ -207,6 +208,50 @@ def lmh_support_kl_fwd_bwd(shape, H, W, ids, ref_logp, kl_rows, kl_mean=None, lp
         _p(dH, _bf, "dH"), _p(dW, _bf, "dW"), _p(dW_acc, _f32, "dW_acc"),
         _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
     _ok("lmh_support_kl_fwd_bwd", st)
+
+
+def lmh_support_fwd_bwd(shape, mode, H, W, ids, ref_logp, grad, kl_rows=None, kl_mean=None,
+                        lp=None, lse=None, dH=None, dW=None, dW_acc=None, *, workspace,
+                        stream=None) -> None:
+    N, d, V, K = shape.N, shape.d, shape.V, shape.K
+    g = 1 if shape.flags & F_GRAD_SCALAR else (N * K if int(mode) == BWD_SUPPORT_LOGPROB else N)
+    _fits(H=(H, N * d), W=(W, V * d), ids=(ids, N * K), ref_logp=(ref_logp, N * K),
+          grad=(grad, g), kl_rows=(kl_rows, N), kl_mean=(kl_mean, 1), lp=(lp, N * K),
+          lse=(lse, N), dH=(dH, N * d), dW=(dW, V * d), dW_acc=(dW_acc, V * d))
+    st = lib().lmh_support_fwd_bwd(
+        ctypes.byref(shape), int(mode), _p(H, _bf, "H"), _p(W, _bf, "W"), _p(ids, _i32, "ids"),
+        _p(ref_logp, _f32, "ref_logp"), _p(grad, _f32, "grad"), _p(kl_rows, _f32, "kl_rows"),
+        _p(kl_mean, _f32, "kl_mean"), _p(lp, _f32, "lp"), _p(lse, _f32, "lse"),
+        _p(dH, _bf, "dH"), _p(dW, _bf, "dW"), _p(dW_acc, _f32, "dW_acc"),
+        _p(workspace, _u8, "workspace"), workspace.numel(), _s(stream))
+    _ok("lmh_support_fwd_bwd", st)
+
+
+def support_fwd_bwd(mode: int, H, W, ids, grad=None, ref_logp=None, *, chunk_rows: int = 0,
+                    mean: bool = False, scalar_grad: bool = False, dW_acc=None,
+                    temperature=None, ws=None, stream=None) -> dict:
+    """The support forward (lp, lse; kl_rows, kl_mean for BWD_SUPPORT_KL) plus dH, dW of
+    sum_i g_i KL_i or sum_ik g_ik lp_ik in one pass, the weights known before the call."""
+    N, d = H.shape
+    V, K = W.shape[0], ids.shape[1]
+    dev = H.device
+    flags = (F_FUSED_BWD | (F_MEAN if mean else 0) | (F_GRAD_SCALAR if scalar_grad else 0)
+             | (F_DW_ACC_GIVEN if dW_acc is not None else 0))
+    shape = make_shape(N, d, V, K, chunk_rows, flags, temperature)
+    kl = int(mode) == BWD_SUPPORT_KL
+    out = dict(lp=torch.empty(N, K, dtype=_f32, device=dev),
+               lse=torch.empty(N, dtype=_f32, device=dev),
+               dH=torch.empty(N, d, dtype=_bf, device=dev),
+               dW=torch.empty(V, d, dtype=_bf, device=dev))
+    if kl:
+        out["kl_rows"] = torch.empty(N, dtype=_f32, device=dev)
+        out["kl_mean"] = torch.empty(1, dtype=_f32, device=dev)
+    ws = workspace(shape, ENTRY_SUPPORT_KL, dev) if ws is None else ws
+    lmh_support_fwd_bwd(shape, mode, H, W, ids, ref_logp, grad, out.get("kl_rows"),
+                        out.get("kl_mean"), out["lp"], out["lse"], out["dH"], out["dW"], dW_acc,
+                        workspace=ws, stream=stream)
+    out["workspace"] = ws
+    return out
 
 
 def lmh_vp_partials(shard, v0, V_total, H, W_shard, labels, records, *, workspace,

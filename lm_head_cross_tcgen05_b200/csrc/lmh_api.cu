@@ -241,20 +241,24 @@ extern "C" lmh_status lmh_support_kl(const lmh_shape* shape, const lmh_bf16* H,
                      workspace, workspace_bytes, stream);
 }
 
-extern "C" lmh_status lmh_support_kl_fwd_bwd(const lmh_shape* shape, const lmh_bf16* H,
-                                             const lmh_bf16* W, const int32_t* ids,
-                                             const float* ref_logp, float* kl_rows,
-                                             float* kl_mean, float* lp, float* lse,
-                                             lmh_bf16* dH, lmh_bf16* dW, float* dW_acc,
-                                             void* workspace, size_t workspace_bytes,
-                                             void* stream) {
+extern "C" lmh_status lmh_support_fwd_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,
+                                          const lmh_bf16* W, const int32_t* ids,
+                                          const float* ref_logp, const float* grad,
+                                          float* kl_rows, float* kl_mean, float* lp, float* lse,
+                                          lmh_bf16* dH, lmh_bf16* dW, float* dW_acc,
+                                          void* workspace, size_t workspace_bytes,
+                                          void* stream) {
   if (!shape_ok(shape) || shape->K < 1 || shape->K > LMH_MAX_K) return LMH_ERR_INVALID_ARG;
   if (shape->flags & LMH_F_SUPPORT_RENORM) return LMH_ERR_INVALID_ARG;  // sparse path: two calls
+  if (mode != LMH_BWD_SUPPORT_LOGPROB && mode != LMH_BWD_SUPPORT_KL) return LMH_ERR_INVALID_ARG;
+  const bool kl = mode == LMH_BWD_SUPPORT_KL;
   const bool grads = dH || dW || dW_acc;
   const Plan P = make_plan(shape, LMH_ENTRY_SUPPORT_KL, grads, dW && !dW_acc);
   int dev, sms;
   LMH_TRY(common_checks(shape, H, W, workspace, workspace_bytes, P.total, &dev, &sms));
-  if (P.N > 0 && (!ids || !lse || !ref_logp || !kl_rows)) return LMH_ERR_INVALID_ARG;
+  if (P.N > 0 && (!ids || !lse)) return LMH_ERR_INVALID_ARG;
+  if (kl && P.N > 0 && (!ref_logp || !kl_rows)) return LMH_ERR_INVALID_ARG;
+  if ((shape->flags & LMH_F_GRAD_SCALAR) && !grad) return LMH_ERR_INVALID_ARG;
   if (!aligned16(dH) || !aligned16(dW) || !aligned16(dW_acc)) return LMH_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
@@ -265,13 +269,14 @@ extern "C" lmh_status lmh_support_kl_fwd_bwd(const lmh_shape* shape, const lmh_b
   float* alpha = grads ? ws.at<float>(P.o_alpha) : nullptr;
   float* beta = grads ? ws.at<float>(P.o_beta) : nullptr;
   if (grads) {
-    // the KL's coefficients depend on the reference log-probs only, not on lse: alpha_i =
-    // g_i sum_k exp(r_ik), beta_ic = g_i sum_{k: c_ik = c} exp(r_ik), g_i = 1 / N or 1
+    // the coefficients depend on the weights (and the reference log-probs) only, not on lse:
+    // KL: alpha_i = g_i sum_k exp(r_ik), beta_ic = g_i sum_{k: c_ik = c} exp(r_ik);
+    // log-probs: alpha_i = -sum_k g_ik, beta_ic = -sum_{k: c_ik = c} g_ik
     ProfScope ps(KID_BWD_COEF, st);
     bwd_coef_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
-        LMH_BWD_SUPPORT_KL, P.N, K, static_cast<int>(P.V), ids, nullptr, ref_logp,
-        ws.at<int32_t>(P.o_rank), ws.at<int32_t>(P.o_nuniq), P.temp,
-        (shape->flags & LMH_F_MEAN) ? 1 : 0, 0, ws.h, alpha, beta);
+        mode, P.N, K, static_cast<int>(P.V), ids, grad, ref_logp, ws.at<int32_t>(P.o_rank),
+        ws.at<int32_t>(P.o_nuniq), P.temp, (shape->flags & LMH_F_MEAN) ? 1 : 0,
+        (shape->flags & LMH_F_GRAD_SCALAR) ? 1 : 0, ws.h, alpha, beta);
   }
   LMH_TRY(last_launch());
   Targets tg{};
@@ -314,15 +319,29 @@ extern "C" lmh_status lmh_support_kl_fwd_bwd(const lmh_shape* shape, const lmh_b
   {
     ProfScope ps(KID_SUPPORT_OUT, st);
     support_out_kernel<<<static_cast<unsigned>(cdiv(P.N, 8)), 256, 0, st>>>(
-        P.N, K, ws.at<int32_t>(P.o_rank), ws.at<float>(P.o_zt), lse, ref_logp, lp, kl_rows);
+        P.N, K, ws.at<int32_t>(P.o_rank), ws.at<float>(P.o_zt), lse, kl ? ref_logp : nullptr,
+        lp, kl ? kl_rows : nullptr);
   }
   LMH_TRY(last_launch());
-  if (kl_mean) {
+  if (kl && kl_mean) {
     ProfScope ps(KID_MEAN, st);
     mean_kernel<<<1, 1024, 0, st>>>(kl_rows, P.N, 0, nullptr, ws.h, kl_mean);
     LMH_TRY(last_launch());
   }
   return LMH_OK;
+}
+
+extern "C" lmh_status lmh_support_kl_fwd_bwd(const lmh_shape* shape, const lmh_bf16* H,
+                                             const lmh_bf16* W, const int32_t* ids,
+                                             const float* ref_logp, float* kl_rows,
+                                             float* kl_mean, float* lp, float* lse,
+                                             lmh_bf16* dH, lmh_bf16* dW, float* dW_acc,
+                                             void* workspace, size_t workspace_bytes,
+                                             void* stream) {
+  if (shape && (shape->flags & LMH_F_GRAD_SCALAR)) return LMH_ERR_INVALID_ARG;  // no grad here
+  return lmh_support_fwd_bwd(shape, LMH_BWD_SUPPORT_KL, H, W, ids, ref_logp, nullptr, kl_rows,
+                             kl_mean, lp, lse, dH, dW, dW_acc, workspace, workspace_bytes,
+                             stream);
 }
 
 extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,

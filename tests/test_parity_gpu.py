@@ -587,3 +587,30 @@ def test_weighted_fused_scalar_mean_count_and_temperature():
     a = L.loss_fwd_bwd(L.BWD_CE, x["H"], x["W"], x["labels"], None, mean=True, chunk_rows=128)
     b = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=128, grads=True)
     assert torch.equal(a["dH"], b["dH"]) and torch.equal(a["dW"], b["dW"])
+
+
+@pytest.mark.parametrize("mode", [L.BWD_SUPPORT_LOGPROB, L.BWD_SUPPORT_KL])
+def test_support_fwd_bwd_weighted(mode):
+    N, d, V, K = 120, 128, 3000, 12
+    x, xc = device_inputs(ragged(N, d, V, seed=5200, K=K))
+    kl = mode == L.BWD_SUPPORT_KL
+    shape_g = (N,) if kl else (N, K)
+    g = torch.linspace(-1.0, 2.0, int(np.prod(shape_g)), dtype=torch.float32).view(shape_g)
+    ref_lp = x["ref_logp"] if kl else None
+    out = L.support_fwd_bwd(mode, x["H"], x["W"], x["ids"], g.cuda(), ref_lp, chunk_rows=50)
+    torch.cuda.synchronize()
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    if kl:
+        rf = O.support_kl(xc["H"], xc["W"], xc["ids"], xc["ref_logp"])
+        check_rows(out["kl_rows"], rf["kl_rows"], what="kl_rows")
+    else:
+        rf = O.support_logprob(xc["H"], xc["W"], xc["ids"])
+    check_rows(out["lp"], rf["lp"], what="lp")
+    check_rows(out["lse"], rf["lse"], what="lse")
+    ref = O.backward(mode, xc["H"], xc["W"], xc["ids"], g.numpy(),
+                     xc["ref_logp"] if kl else None)
+    check_grad(out["dH"], ref["dH"], "dH")
+    check_grad(out["dW"], ref["dW"], "dW")
+    b = L.loss_bwd(mode, x["H"], x["W"], x["ids"], out["lse"], g.cuda(), ref_lp, chunk_rows=50)
+    check_grad(out["dH"], b["dH"], "dH one pass vs standalone")
+    check_grad(out["dW"], b["dW"], "dW one pass vs standalone")
