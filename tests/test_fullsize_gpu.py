@@ -187,6 +187,27 @@ def test_support_workload_sampled_rows():
                     ref[rows].cpu())
     check_grad(b["dH"][rows], rb["dH"], "dH rows (KL)")
     check_dw_properties(b["dW"])
+    # the one-pass entry bench.py times for this workload: same forward bits, same gradients
+    f = L.support_kl(x["H"], x["W"], ids, ref, chunk_rows=wl.N, grads=True)
+    assert torch.equal(f["kl_rows"], kl["kl_rows"]) and torch.equal(f["lse"], kl["lse"])
+    check_grad(f["dH"][rows], rb["dH"], "dH rows (KL, one pass)")
+    check_grad(f["dH"], b["dH"], "dH one pass vs two calls")
+    check_grad(f["dW"], b["dW"], "dW one pass vs two calls")
+    check_dw_properties(f["dW"])
+
+
+def test_large_vocab_vocabulary_parallel_step(large_vocab):
+    # bench.py's vocab_parallel step at one rank (the full workload): the records' combine
+    # gives the one-device lse to fp32 rounding and the same argmax; gradients agree
+    from lm_head_cross_tcgen05_b200.vocab_parallel import VocabParallelCE
+    wl, x, out = large_vocab
+    vp = VocabParallelCE(wl.V, chunk_rows=wl.N)
+    f = vp.forward_backward(x["H"], x["W"], x["labels"])
+    torch.cuda.synchronize()
+    assert (f["lse"] - out["lse"]).abs().max().item() < 1e-4
+    assert torch.equal(f["argmax"], out["argmax"])
+    check_grad(f["dH"], f64(out["dH"]), "dH vocabulary-parallel vs one device")
+    check_grad(f["dW"], f64(out["dW"]), "dW vocabulary-parallel vs one device")
 
 
 def test_many_chunks_and_large_row_indices():
