@@ -43,14 +43,17 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_vocab")
     ap.add_argument("--entry", choices=["fused_ce", "ce_separate", "support_kl",
-                                        "support_kl_separate", "vocab_parallel"],
+                                        "support_kl_separate", "vocab_parallel",
+                                        "data_parallel"],
                     default="fused_ce",
                     help="fused_ce: lmh_loss_fwd with dH/dW (the headline step); ce_separate: "
                          "lmh_loss_fwd then lmh_loss_bwd (recomputed logits); support_kl: "
                          "lmh_support_kl_fwd_bwd (the mean KL's forward and backward in one "
                          "pass); support_kl_separate: lmh_support_kl then lmh_loss_bwd; "
                          "vocab_parallel: one "
-                         "CE problem with W split over the GPUs (strong scaling)")
+                         "CE problem with W split over the GPUs (strong scaling); "
+                         "data_parallel: each GPU's own rows, the global mean and the dW sum "
+                         "over the GPUs in rank order (weak scaling)")
     ap.add_argument("--chunk-rows", type=int, default=0,
                     help="rows per chunk (the memory budget); 0: the workload's own plan")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -86,7 +89,9 @@ ENTRY_TEXT = {"fused_ce": "fused CE forward+backward",
               "support_kl_separate": "support-set KL forward (K candidates), then its backward "
                                      "with recomputed logits",
               "vocab_parallel": "vocabulary-parallel fused CE forward+backward (W split over "
-                                "the GPUs)"}
+                                "the GPUs)",
+              "data_parallel": "row data-parallel fused CE forward+backward (global mean, dW "
+                               "summed over the GPUs in rank order)"}
 
 
 def workload_config(wl, chunk_rows, n_gpus, entry="fused_ce"):
@@ -95,7 +100,9 @@ def workload_config(wl, chunk_rows, n_gpus, entry="fused_ce"):
                         f"{wl.labels} labels, {wl.num_ignored} ignored rows, bf16 H/W",
             "entry": entry,
             "N": wl.N, "d": wl.d, "V": wl.V, "chunk_rows": chunk_rows,
-            "parallelism": (f"vocab-parallel over {n_gpus}" if vp else f"replicas x{n_gpus}"),
+            "parallelism": (f"vocab-parallel over {n_gpus}" if vp else
+                            f"data-parallel over {n_gpus}" if entry == "data_parallel" else
+                            f"replicas x{n_gpus}"),
             "rows_per_gpu": wl.N, "total_rows": wl.N if vp else wl.N * n_gpus,
             "l2": "inputs larger than L2 (W alone is %.2f GB)" % (wl.V * wl.d * 2 / 1e9)}
 
@@ -340,6 +347,16 @@ def main():
 
         def step(b=batch):
             f = vp.forward_backward(b["H"], W_shard, b["labels"])   # fused: 3 GEMMs per shard
+            out["loss_mean"].copy_(f["loss_mean"])
+            out["n_valid"].copy_(f["n_valid"])
+    elif args.entry == "data_parallel":
+        from lm_head_cross_tcgen05_b200.data_parallel import DataParallelCE
+        dp = DataParallelCE(chunk_rows=chunk)          # the default group when world > 1
+
+        def step(b=batch):
+            # fused step on this rank's rows with the global count, then the rank-ordered
+            # sums of the mean's shares and of the fp32 dW
+            f = dp.forward_backward(b["H"], W, b["labels"])
             out["loss_mean"].copy_(f["loss_mean"])
             out["n_valid"].copy_(f["n_valid"])
     else:

@@ -80,6 +80,7 @@ typedef enum lmh_status {
 #define LMH_F_DW_ACC_GIVEN 0x4u /* sizing only: the caller passes an fp32 dW_acc       */
 #define LMH_F_SUPPORT_RENORM 0x8u /* support entries: renormalise over the candidates   */
 #define LMH_F_GRAD_SCALAR 0x10u   /* backward: grad is one float shared by every term    */
+#define LMH_F_DW_ACC_STORE 0x20u  /* dW_acc receives this call's dW instead of adding it */
 
 /* entries, for lmh_workspace_size */
 #define LMH_ENTRY_LOSS_FWD 0
@@ -151,6 +152,9 @@ LMH_API size_t lmh_workspace_size(const lmh_shape* shape, int entry);
  *     sum_i loss_i (not set), reusing the forward's softmax instead of recomputing logits.
  *     dW_acc, if given, is incremented by this call's dW in chunk order (zero it first for
  *     a fresh gradient) and dW, if given, receives its round-to-nearest-even bf16 cast.
+ *     With LMH_F_DW_ACC_STORE in shape->flags the first chunk overwrites dW_acc instead (no
+ *     zeroing needed; a call without rows zeroes it), so dW_acc holds exactly this call's
+ *     fp32 dW. The flag applies wherever dW_acc is taken.
  *     Each increment is one IEEE fp32 add per element and chunk, rounded to nearest even.
  *     Without dW_acc and with one chunk, dW is the bf16 cast of the fp32 tile sums.
  */
@@ -175,6 +179,7 @@ LMH_API lmh_status lmh_loss_fwd(const lmh_shape* shape, const lmh_bf16* H, const
  *   LMH_BWD_SUPPORT_KL:      targets = ids [N, K]; grad [N] = dL/dKL_i; ref_logp [N, K];
  *                            alpha_i = g_i sum_k exp(r_ik), beta_ik = g_i exp(r_ik).
  * Candidate ids < 0 are padding and are skipped. lse [N] is the forward's output.
+ * A given grad is taken as is (LMH_F_MEAN does not scale it).
  * grad may be NULL: every row term then has the weight 1, or 1 / count with LMH_F_MEAN in
  * shape->flags (count: the valid rows of the labels for CE / LOGPROB, N for the support
  * objectives), taken on the device without a host synchronisation. With LMH_F_GRAD_SCALAR,
@@ -192,9 +197,10 @@ LMH_API lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_bf16
  * before the call: L = sum_i w_i loss_i (mode LMH_BWD_CE) or L = sum_i w_i logprob_i (mode
  * LMH_BWD_LOGPROB), e.g. a policy-gradient loss whose per-row weights (advantages) are fixed
  * before the forward (FlashInfer PR #8059, description: "the CE and policy losses"). The
- * weights are those of lmh_loss_bwd: w_i = grad[i]; one shared grad[0] with
- * LMH_F_GRAD_SCALAR; 1 with grad NULL; each times 1 / count with LMH_F_MEAN, the count
- * being *n_valid_given if given, else the valid rows. Ignored rows get 0. The forward outputs
+ * weights are those of lmh_loss_bwd: w_i = grad[i], taken as given (LMH_F_MEAN does not
+ * scale per-row weights); or one shared grad[0] with LMH_F_GRAD_SCALAR, or 1 with grad NULL,
+ * these two times 1 / count with LMH_F_MEAN, the count being *n_valid_given if given, else
+ * the valid rows. Ignored rows get 0. The forward outputs
  * are those of lmh_loss_fwd (loss_mean is always the mean loss); dH, dW, dW_acc as there.
  * The softmax is reused as in lmh_loss_fwd's fused path: three GEMMs per chunk.
  * Workspace: lmh_workspace_size(shape, LMH_ENTRY_LOSS_FWD_BWD) with LMH_F_FUSED_BWD.
@@ -418,9 +424,9 @@ LMH_API lmh_status lmh_vp_reduce_rows_to(int R, int64_t rows, int64_t d, const f
  * (mode LMH_BWD_SUPPORT_KL; ref_logp and kl_rows required) or of lmh_support_logprob (mode
  * LMH_BWD_SUPPORT_LOGPROB; kl outputs and ref_logp unused), plus the backward of
  * L = sum_i g_i KL_i or L = sum_ik g_ik lp_ik with weights known before the call: grad [N]
- * (KL) or [N, K] (log-probs), one shared grad[0] with LMH_F_GRAD_SCALAR, or 1 with grad NULL;
- * each times 1 / N with LMH_F_MEAN. Workspace and outputs as lmh_support_kl_fwd_bwd, which is
- * this entry with mode LMH_BWD_SUPPORT_KL and grad NULL.
+ * (KL) or [N, K] (log-probs), taken as given; or one shared grad[0] with LMH_F_GRAD_SCALAR,
+ * or 1 with grad NULL, these two times 1 / N with LMH_F_MEAN. Workspace and outputs as
+ * lmh_support_kl_fwd_bwd, which is this entry with mode LMH_BWD_SUPPORT_KL and grad NULL.
  */
 LMH_API lmh_status lmh_support_fwd_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,
                                        const lmh_bf16* W, const int32_t* ids,
@@ -435,6 +441,35 @@ LMH_API lmh_status lmh_support_kl_fwd_bwd(const lmh_shape* shape, const lmh_bf16
                                           float* lp, float* lse, lmh_bf16* dH, lmh_bf16* dW,
                                           float* dW_acc, void* workspace,
                                           size_t workspace_bytes, void* stream);
+
+/*
+ * Row data-parallel steps. Every rank holds all of W and its own rows of the batch; the mean
+ * loss divides by the valid rows of all ranks, and dW is the sum of the ranks' dW. The pages'
+ * ops sum a weight gradient over the rows of one call and leave its reduction across ranks
+ * to the caller (miles-ext-kernels PR #14, gated RMSNorm commit notes). These two entries
+ * let the caller make that reduction reproducible, with the arithmetic in this library:
+ *   1. lmh_count_valid on every rank; the caller sums the counts over the ranks (an integer
+ *      all-reduce, exact in any order).
+ *   2. lmh_loss_fwd or lmh_loss_fwd_bwd on every rank with LMH_F_MEAN, n_valid_given = that
+ *      sum, dW = NULL and an fp32 dW_acc with LMH_F_DW_ACC_STORE: loss_mean is then the rank's
+ *      share of the global mean, dH its own rows' gradient, dW_acc its fp32 dW.
+ *   3. The caller gathers the R shares of the mean and adds them in rank order
+ *      (lmh_reduce_ranks_f32), and sums the fp32 dW in rank order by row slices with
+ *      lmh_vp_reduce_rows (each rank reduces the rows of its slice from every rank; the bf16
+ *      slices are then gathered), as for the vocabulary-parallel dH.
+ * With a fixed rank count and batch split every output is bitwise reproducible; against one
+ * device on the concatenated batch the values agree to fp32 rounding.
+ *
+ * lmh_count_valid: *n_valid = the number of rows with 0 <= labels[i] < V (int32 device out).
+ *   labels [N] int32 device. No workspace; labels >= V are not flagged here (the loss entries
+ *   flag them). N = 0 writes 0.
+ * lmh_reduce_ranks_f32: out[i] = sum_{r = 0..R-1} parts[r * n + i] in ascending r, fp32
+ *   (round to nearest even). parts [R, n] and out [n] fp32 device, 4-byte aligned; any n.
+ */
+LMH_API lmh_status lmh_count_valid(int64_t N, int64_t V, const int32_t* labels,
+                                   int32_t* n_valid, void* stream);
+LMH_API lmh_status lmh_reduce_ranks_f32(int R, int64_t n, const float* parts, float* out,
+                                        void* stream);
 
 /*
  * lmh_scale_bf16 — x = bf16(x * g[0]) in place over n elements (n a multiple of 4, x 8-byte

@@ -21,7 +21,7 @@ from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEV
                    ENTRY_LOSS_FWD, ENTRY_SUPPORT_KL, ENTRY_SUPPORT_LOGPROB, ENTRY_VP_BWD,
                    ENTRY_LOSS_FWD_BWD, ENTRY_VP_COMBINE, ENTRY_VP_PARTIALS,
                    ENTRY_VP_SUPPORT_BWD, ENTRY_VP_SUPPORT_COMBINE, ENTRY_VP_SUPPORT_PARTIALS,
-                   F_DW_ACC_GIVEN,
+                   F_DW_ACC_GIVEN, F_DW_ACC_STORE,
                    F_GRAD_SCALAR, lmh_vp_dest,
                    F_FUSED_BWD, F_MEAN, F_SUPPORT_RENORM, IGNORE_INDEX, MAX_K, STATUS_NAMES, lib, lmh_shape)
 
@@ -41,6 +41,7 @@ __all__ = [
     "ENTRY_LOSS_FWD_BWD", "lmh_loss_fwd_bwd", "loss_fwd_bwd",
     "ENTRY_VP_SUPPORT_PARTIALS", "ENTRY_VP_SUPPORT_COMBINE", "ENTRY_VP_SUPPORT_BWD",
     "lmh_vp_support_partials", "lmh_vp_support_combine", "lmh_vp_support_bwd",
+    "F_DW_ACC_STORE", "lmh_count_valid", "lmh_reduce_ranks_f32",
 ]
 
 lib()  # load now: a missing library is an import error, never a silent fallback
@@ -390,6 +391,23 @@ def lmh_vp_reduce_rows_to(parts, outs, n_out, row_offset, stream=None) -> None:
                                      _p(outs, None, "outs"), int(n_out), int(row_offset),
                                      _s(stream))
     _ok("lmh_vp_reduce_rows_to", st)
+
+
+def lmh_count_valid(labels, V, n_valid, stream=None) -> None:
+    """n_valid[0] = the rows with 0 <= label < V (int32, on the device)."""
+    _fits(n_valid=(n_valid, 1))
+    st = lib().lmh_count_valid(int(labels.numel()), int(V), _p(labels, _i32, "labels"),
+                               _p(n_valid, _i32, "n_valid"), _s(stream))
+    _ok("lmh_count_valid", st)
+
+
+def lmh_reduce_ranks_f32(parts, out, stream=None) -> None:
+    """parts [R, n] fp32 -> out [n] fp32, summed in ascending R."""
+    R, n = parts.shape
+    _fits(out=(out, n))
+    st = lib().lmh_reduce_ranks_f32(int(R), int(n), _p(parts, _f32, "parts"),
+                                    _p(out, _f32, "out"), _s(stream))
+    _ok("lmh_reduce_ranks_f32", st)
 
 
 def lmh_scale_bf16(x, g, stream=None) -> None:

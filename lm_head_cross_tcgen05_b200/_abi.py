@@ -20,6 +20,7 @@ STATUS_NAMES = {0: "LMH_OK", 1: "LMH_ERR_INVALID_ARG", 2: "LMH_ERR_UNSUPPORTED_D
 IGNORE_INDEX = -100
 DEVERR_LABEL_RANGE, DEVERR_TIMEOUT, DEVERR_NONFINITE, DEVERR_TEMPERATURE = 0x1, 0x2, 0x4, 0x8
 F_MEAN, F_FUSED_BWD, F_DW_ACC_GIVEN, F_SUPPORT_RENORM, F_GRAD_SCALAR = 0x1, 0x2, 0x4, 0x8, 0x10
+F_DW_ACC_STORE = 0x20
 ENTRY_LOSS_FWD, ENTRY_LOSS_BWD, ENTRY_LOGPROB, ENTRY_SUPPORT_LOGPROB, ENTRY_SUPPORT_KL = range(5)
 ENTRY_VP_PARTIALS, ENTRY_VP_COMBINE, ENTRY_VP_BWD, ENTRY_LOSS_FWD_BWD = 5, 6, 7, 8
 ENTRY_VP_SUPPORT_PARTIALS, ENTRY_VP_SUPPORT_COMBINE, ENTRY_VP_SUPPORT_BWD = 9, 10, 11
@@ -65,6 +66,8 @@ _SIGS = {
     "lmh_support_fwd_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 13
                             + [c_size_t, _P]),
     "lmh_scale_bf16": (c_int, [_P, c_int64, _P, _P]),
+    "lmh_count_valid": (c_int, [c_int64, c_int64, _P, _P, _P]),
+    "lmh_reduce_ranks_f32": (c_int, [c_int, c_int64, _P, _P, _P]),
     "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),
     "lmh_logprob_noalloc": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6),
     "lmh_selftest_wait_timeout": (c_int, [_P, c_uint32, _P]),

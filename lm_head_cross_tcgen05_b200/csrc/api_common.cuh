@@ -19,6 +19,7 @@ struct Plan {
   bool cands;   // per-row candidate lists (support entries, candidate backward)
   bool gbuf;    // chunk softmax / gradient buffer
   bool acc;     // internal fp32 dW accumulator
+  bool acc_store;  // the caller's dW_acc is overwritten by the first chunk, not added to
   bool renorm;  // support entries renormalised over the candidate set (sparse path)
   size_t o_zt, o_sorted, o_nuniq, o_rank, o_pm, o_ps, o_pi, o_alpha, o_beta, o_gbuf, o_acc;
   size_t o_gu, o_cnt, o_off, o_fill, o_prow, o_pslot;  // sparse backward
@@ -80,6 +81,7 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
                                    entry == LMH_ENTRY_LOSS_FWD_BWD);
   p.gbuf = !p.renorm && (bwd || fwd_fused);
   p.acc = p.gbuf && dw_without_acc && p.nchunks > 1;
+  p.acc_store = (s->flags & LMH_F_DW_ACC_STORE) != 0;
   const bool stats = !bwd && entry != LMH_ENTRY_VP_COMBINE &&
                      entry != LMH_ENTRY_VP_SUPPORT_COMBINE;
   const bool partials = stats && !p.renorm;
@@ -163,14 +165,16 @@ enum KernelId {
   KID_GEMM_DH, KID_GEMM_DW, KID_FINALIZE, KID_GBUILD, KID_FIX_LABELS, KID_MEAN,
   KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_SUPPORT_DOTS, KID_SUPPORT_LSE,
   KID_SUPPORT_DH, KID_SUPPORT_DW, KID_SPLIT_SUM, KID_VP_LABELS, KID_VP_FINALIZE,
-  KID_VP_COMBINE, KID_VP_REDUCE, KID_VP_SCALE, KID_FIX_CANDS, KID_SCALE, KID_COUNT
+  KID_VP_COMBINE, KID_VP_REDUCE, KID_VP_SCALE, KID_FIX_CANDS, KID_SCALE, KID_COUNT_VALID,
+  KID_REDUCE_RANKS, KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "count_labels", "prep_cands", "gemm_logits_stats", "gemm_logits_stats_store",
     "gemm_logits_grad", "gemm_dH", "gemm_dW", "row_finalize", "gbuild", "fix_labels",
     "mean", "support_out", "bwd_coef", "cast_bf16", "support_dots", "support_lse",
     "support_grad_dh", "support_dw", "split_sum", "vp_local_labels", "vp_finalize",
-    "vp_combine", "vp_reduce_rows", "vp_scale", "fix_cands", "scale_bf16"};
+    "vp_combine", "vp_reduce_rows", "vp_scale", "fix_cands", "scale_bf16", "count_valid",
+    "reduce_ranks"};
 
 struct ProfRec {
   int id;
@@ -481,14 +485,15 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
       return LMH_ERR_CUDA;
     // Internal accumulator (several chunks, no caller dW_acc): store, add, ..., and the last
     // chunk adds and casts in its epilogue without writing the sum back. Caller's dW_acc:
-    // add in every chunk, then cast it. One chunk without dW_acc: bf16 tile sums directly.
+    // add in every chunk (the first stores with LMH_F_DW_ACC_STORE), then cast it. One chunk
+    // without dW_acc: bf16 tile sums directly.
     const bool last = chunk_idx == P.nchunks - 1;
     float* acc = dW_acc ? dW_acc : (P.acc ? ws.at<float>(P.o_acc) : nullptr);
     EpiDW::Params ep;
     ep.V = static_cast<int>(P.V);
     ep.d = static_cast<int>(P.d);
     if (!acc) ep.acc_mode = 0;
-    else if (dW_acc) ep.acc_mode = 2;
+    else if (dW_acc) ep.acc_mode = (P.acc_store && chunk_idx == 0) ? 1 : 2;
     else ep.acc_mode = chunk_idx == 0 ? 1 : (last ? 3 : 2);
     CUtensorMap td;  // mode 3: the accumulator, read by the epilogue
     bool ok;
@@ -582,15 +587,19 @@ lmh_status sparse_backward(const Plan& P, const lmh_bf16* H, const lmh_bf16* W, 
   support_dw_kernel<<<static_cast<unsigned>(vblocks), 256, 0, st>>>(
       V, K, d, reinterpret_cast<const __nv_bfloat16*>(H), ws.at<int32_t>(P.o_off),
       ws.at<int32_t>(P.o_prow), ws.at<int32_t>(P.o_pslot), ws.at<float>(P.o_gu), dW_acc,
-      dW_acc ? 2 : 0, reinterpret_cast<__nv_bfloat16*>(dW));
+      dW_acc ? (P.acc_store ? 1 : 2) : 0, reinterpret_cast<__nv_bfloat16*>(dW));
   return last_launch();
 }
 
-// Outputs of a call without rows: zero counts / means, dW = cast of the given accumulator.
+// Outputs of a call without rows: zero counts / means, dW = cast of the given accumulator
+// (zeroed first with LMH_F_DW_ACC_STORE: the call's dW is zero).
 lmh_status empty_call(const Plan& P, float* mean_out, int32_t* nvalid_out, lmh_bf16* dW,
                       float* dW_acc, cudaStream_t st) {
   if (mean_out && cudaMemsetAsync(mean_out, 0, 4, st) != cudaSuccess) return LMH_ERR_CUDA;
   if (nvalid_out && cudaMemsetAsync(nvalid_out, 0, 4, st) != cudaSuccess) return LMH_ERR_CUDA;
+  if (dW_acc && P.acc_store &&
+      cudaMemsetAsync(dW_acc, 0, static_cast<size_t>(P.V) * P.d * 4, st) != cudaSuccess)
+    return LMH_ERR_CUDA;
   if (dW) {
     const int64_t n = P.V * P.d;
     if (dW_acc) return cast_dw(P, dW_acc, dW, st);

@@ -417,6 +417,43 @@ extern "C" lmh_status lmh_loss_bwd(const lmh_shape* shape, int mode, const lmh_b
 
 #include "api_vp.cuh"
 
+extern "C" lmh_status lmh_count_valid(int64_t N, int64_t V, const int32_t* labels,
+                                      int32_t* n_valid, void* stream) {
+  if (N < 0 || V <= 0 || V > 0x7fffffffLL || !n_valid) return LMH_ERR_INVALID_ARG;
+  if (N > 0 && !labels) return LMH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(labels) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(n_valid) & 3u) != 0)
+    return LMH_ERR_ALIGNMENT;
+  int dev, sms;
+  LMH_TRY(current_device(&dev, &sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(n_valid, 0, 4, st) != cudaSuccess) return LMH_ERR_CUDA;
+  if (N == 0) return LMH_OK;
+  const int64_t blocks = cdiv(N, 256);
+  ProfScope ps(KID_COUNT_VALID, st);
+  count_valid_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 256, 0, st>>>(
+      labels, N, static_cast<int>(V), n_valid);
+  return last_launch();
+}
+
+extern "C" lmh_status lmh_reduce_ranks_f32(int R, int64_t n, const float* parts, float* out,
+                                           void* stream) {
+  if (R < 1 || n < 0) return LMH_ERR_INVALID_ARG;
+  if (n == 0) return LMH_OK;
+  if (!parts || !out) return LMH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(parts) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(out) & 3u) != 0)
+    return LMH_ERR_ALIGNMENT;
+  int dev, sms;
+  LMH_TRY(current_device(&dev, &sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t blocks = cdiv(n, 256);
+  ProfScope ps(KID_REDUCE_RANKS, st);
+  reduce_ranks_kernel<<<static_cast<unsigned>(blocks < 8192 ? blocks : 8192), 256, 0, st>>>(
+      R, n, parts, out);
+  return last_launch();
+}
+
 extern "C" lmh_status lmh_scale_bf16(lmh_bf16* x, int64_t n, const float* g, void* stream) {
   if (n < 0 || (n % 4) != 0) return LMH_ERR_INVALID_ARG;
   if (n == 0) return LMH_OK;

@@ -66,6 +66,30 @@ __global__ void count_labels_kernel(const int32_t* __restrict__ labels, long lon
   }
 }
 
+// Rows with 0 <= label < V, added into *out (zeroed before the launch).
+__global__ void count_valid_kernel(const int32_t* __restrict__ labels, long long N, int V,
+                                   int32_t* out) {
+  int cnt = 0;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < N;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int y = labels[i];
+    cnt += (y >= 0 && y < V) ? 1 : 0;
+  }
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if ((threadIdx.x & 31) == 0 && cnt) atomicAdd(out, cnt);  // integer: exact in any order
+}
+
+// out[i] = sum over r = 0..R-1 of parts[r * n + i], added in ascending r.
+__global__ void reduce_ranks_kernel(int R, long long n, const float* __restrict__ parts,
+                                    float* __restrict__ out) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float a = parts[i];
+    for (int r = 1; r < R; ++r) a += parts[static_cast<long long>(r) * n + i];
+    out[i] = a;
+  }
+}
+
 // ---------------------------------------------------------------------------- candidates
 // One block per row (grid-stride), blockDim >= K. For row i: the distinct valid ids in
 // ascending order (sorted[i, 0..nuniq)), and for every slot k the sorted index of its id

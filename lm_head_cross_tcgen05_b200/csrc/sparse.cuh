@@ -194,7 +194,7 @@ __global__ void support_sort_buckets_kernel(int V, const int32_t* __restrict__ o
 }
 
 // dW_v = sum over the bucket of v (rows ascending) of gu[i, u] H_i; one block per id,
-// threads over d. acc_mode as for the dense dW: 0 the sum is dW, 2 acc += sum.
+// threads over d. acc_mode as for the dense dW: 0 the sum is dW, 1 acc = sum, 2 acc += sum.
 __global__ void support_dw_kernel(int V, int K, int d, const __nv_bfloat16* __restrict__ H,
                                   const int32_t* __restrict__ off,
                                   const int32_t* __restrict__ pair_row,
@@ -212,7 +212,9 @@ __global__ void support_dw_kernel(int V, int K, int d, const __nv_bfloat16* __re
         s0 = fmaf(g, hv.x, s0);
         s1 = fmaf(g, hv.y, s1);
       }
-      if (acc_mode == 2) {
+      if (acc_mode == 1) {
+        *reinterpret_cast<float2*>(acc + v * d + j) = make_float2(s0, s1);
+      } else if (acc_mode == 2) {
         float2* a2 = reinterpret_cast<float2*>(acc + v * d + j);
         float2 a = *a2;
         a.x += s0;

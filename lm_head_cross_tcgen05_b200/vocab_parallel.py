@@ -44,6 +44,7 @@ from . import (BWD_CE, BWD_SUPPORT_KL, ENTRY_VP_BWD, ENTRY_VP_COMBINE, ENTRY_VP_
                lmh_vp_fused_bwd, lmh_vp_loss_bwd, lmh_vp_partials, lmh_vp_reduce_rows,
                lmh_vp_reduce_rows_to, lmh_vp_support_bwd, lmh_vp_support_combine,
                lmh_vp_support_partials, make_shape, workspace)
+from ._ranks import RankGroup, row_slices
 
 __all__ = ["shard_plan", "row_slices", "CudaOps", "VocabParallelCE", "VocabParallelSupport"]
 
@@ -60,17 +61,6 @@ def shard_plan(V: int, R: int) -> List[Tuple[int, int]]:
         if (R - 1) * tiled < V:  # every range keeps at least one word
             per = tiled
     return [(min(r * per, V), min((r + 1) * per, V)) for r in range(R)]
-
-
-def row_slices(N: int, R: int) -> List[Tuple[int, int]]:
-    """The rows [a, b) whose dH rank j reduces: N split as evenly as possible, in order."""
-    base, extra = divmod(N, R)
-    out, a = [], 0
-    for j in range(R):
-        b = a + base + (1 if j < extra else 0)
-        out.append((a, b))
-        a = b
-    return out
 
 
 class CudaOps:
@@ -186,7 +176,7 @@ class CudaOps:
         return dH_part, dW
 
 
-class _VocabParallel:
+class _VocabParallel(RankGroup):
     """The shard plan of ``group``'s ranks and the exchange steps every vocabulary-parallel
     objective shares: gathering per-row records, and summing the ranks' dH contributions in
     a fixed order (collectives, or peer-memory stores with ``p2p``). Without an initialised
@@ -194,16 +184,12 @@ class _VocabParallel:
 
     def __init__(self, V_total: int, group=None, chunk_rows: int = 0, mean: bool = True,
                  temperature=None, ops=None, p2p: bool = False):
-        self.group = group
-        self.distributed = dist.is_available() and dist.is_initialized()
-        self.R = dist.get_world_size(group) if self.distributed else 1
-        self.rank = dist.get_rank(group) if self.distributed else 0
+        super().__init__(group, ops if ops is not None else CudaOps())
         self.V_total = int(V_total)
         self.v0, self.v1 = shard_plan(self.V_total, self.R)[self.rank]
         self.chunk_rows = chunk_rows
         self.mean = mean
         self.temperature = temperature
-        self.ops = ops if ops is not None else CudaOps()
         self.p2p = p2p and self.R > 1   # one rank has nothing to exchange
         self._sym = None
 
@@ -211,15 +197,6 @@ class _VocabParallel:
         if W_shard.shape[0] != self.v1 - self.v0:
             raise ValueError(f"rank {self.rank} holds rows [{self.v0}, {self.v1}) of W, "
                              f"got {W_shard.shape[0]} rows")
-
-    def _gather(self, rec):
-        """[N, w] records of this rank -> [R, N, w] of all ranks in rank order."""
-        N, w = rec.shape
-        if self.R == 1:
-            return rec.view(1, N, w)
-        every = torch.empty(self.R * N * w, dtype=rec.dtype, device=rec.device)
-        dist.all_gather_into_tensor(every, rec.reshape(-1).contiguous(), group=self.group)
-        return every.view(self.R, N, w)
 
     def _dH(self, run, N, d, device):
         """dH summed over the ranks from run(dest) -> (dH_part or None, dW): collectives, or
@@ -264,32 +241,6 @@ class _VocabParallel:
         self.ops.reduce_rows_to(parts, sym["dH_tab"], self.R, start)
         sym["dH_h"].barrier(channel=0)        # every rank's slice is in every dH
         return sym["dH"].view(-1, d).clone()
-
-    def _sum_rows(self, part: torch.Tensor) -> torch.Tensor:
-        """sum over ranks of part [N, d], added in ascending rank order, on every rank."""
-        N, d = part.shape
-        if self.R == 1:
-            return self.ops.reduce_rows(part.view(1, N, d))
-        sl = row_slices(N, self.R)
-        sizes = [b - a for a, b in sl]
-        mine = sizes[self.rank]
-        recv = torch.empty(self.R * mine, d, dtype=part.dtype, device=part.device)
-        dist.all_to_all_single(recv, part.contiguous(), output_split_sizes=[mine] * self.R,
-                               input_split_sizes=sizes, group=self.group)
-        red = self.ops.reduce_rows(recv.view(self.R, mine, d))
-        top = max(sizes)
-        if top == 0:
-            return red
-        if mine == top:
-            pad = red
-        else:  # slices differ by one row at most: gather equal blocks, drop the padding
-            pad = torch.zeros(top, d, dtype=red.dtype, device=red.device)
-            pad[:mine] = red
-        every = torch.empty(self.R * top, d, dtype=red.dtype, device=red.device)
-        dist.all_gather_into_tensor(every, pad.contiguous(), group=self.group)
-        if all(n == top for n in sizes):
-            return every
-        return torch.cat([every[j * top: j * top + sizes[j]] for j in range(self.R)])
 
 
 class VocabParallelCE(_VocabParallel):

@@ -152,3 +152,27 @@ def test_ctypes_signatures_match_header_parameter_counts():
     for name, params in decls:
         n = 0 if params.strip() in ("", "void") else len(params.split(","))
         assert n == len(_abi._SIGS[name][1]), name
+
+
+def test_data_parallel_host_errors_without_gpu():
+    lib = _abi.lib()
+    # refused before any CUDA call: negative rows, empty vocabulary, no output, no labels
+    assert lib.lmh_count_valid(-1, 100, None, None, None) == 1
+    assert lib.lmh_count_valid(4, 0, None, ctypes.c_void_p(256), None) == 1
+    assert lib.lmh_count_valid(4, 100, ctypes.c_void_p(256), None, None) == 1
+    assert lib.lmh_count_valid(4, 100, None, ctypes.c_void_p(256), None) == 1
+    assert lib.lmh_count_valid(4, 100, ctypes.c_void_p(258), ctypes.c_void_p(256), None) == 4
+    assert lib.lmh_reduce_ranks_f32(0, 4, None, None, None) == 1
+    assert lib.lmh_reduce_ranks_f32(2, -1, None, None, None) == 1
+    assert lib.lmh_reduce_ranks_f32(2, 0, None, None, None) == 0     # nothing to do
+    assert lib.lmh_reduce_ranks_f32(2, 4, ctypes.c_void_p(256), None, None) == 1
+    assert lib.lmh_reduce_ranks_f32(2, 4, ctypes.c_void_p(256), ctypes.c_void_p(6), None) == 4
+
+
+def test_dw_store_flag_is_sizing_neutral():
+    # LMH_F_DW_ACC_STORE changes what the call writes into the caller's accumulator, not the
+    # workspace it needs
+    for entry in (L.ENTRY_LOSS_FWD, L.ENTRY_LOSS_FWD_BWD, L.ENTRY_LOSS_BWD):
+        base = L.F_FUSED_BWD | L.F_DW_ACC_GIVEN
+        assert ws(3000, 64, 5000, chunk=1000, flags=base, entry=entry) == \
+            ws(3000, 64, 5000, chunk=1000, flags=base | L.F_DW_ACC_STORE, entry=entry)
