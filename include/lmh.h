@@ -468,6 +468,30 @@ LMH_API lmh_status lmh_support_kl_fwd_bwd(const lmh_shape* shape, const lmh_bf16
  */
 LMH_API lmh_status lmh_count_valid(int64_t N, int64_t V, const int32_t* labels,
                                    int32_t* n_valid, void* stream);
+
+/*
+ * lmh_dp_loss_fwd_bwd — step 2 above with the dW exchange fused into the dW GEMM: instead of
+ * writing the rank's fp32 dW locally for a collective to move, the GEMM's epilogue stores
+ * each fp32 row (0 + tile sum) straight into the receive buffer of the rank that reduces it,
+ * while the GEMM runs (ordinary stores; the buffers may be other GPUs' memory through peer
+ * mappings). The vocabulary rows are split as evenly as possible into R slices in order;
+ * rank j reduces slice j, and its buffer dW_dest->recv[j] is [R][rows_j][d] fp32 with slot r
+ * for rank r (16-byte aligned). A rank without rows zeroes its slots. The caller orders the
+ * steps: every rank's call has finished before rank j adds its R slots in rank order with
+ * lmh_vp_reduce_rows_to (which can store the bf16 slice into every rank's dW). The additions
+ * are those of the collective route, so the bits are the same.
+ *   Arguments as lmh_loss_fwd_bwd (mode LMH_BWD_CE or LMH_BWD_LOGPROB; grad NULL for the
+ *   plain mean or summed CE), without n_valid, dW and dW_acc. One chunk only:
+ *   shape->chunk_rows >= N (LMH_ERR_INVALID_ARG otherwise). Workspace:
+ *   lmh_workspace_size(shape, LMH_ENTRY_LOSS_FWD_BWD) with LMH_F_FUSED_BWD.
+ */
+LMH_API lmh_status lmh_dp_loss_fwd_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,
+                                       const lmh_bf16* W, const int32_t* labels,
+                                       const float* grad, float* loss_rows, float* lse,
+                                       float* logprob, int32_t* argmax, float* loss_mean,
+                                       const int32_t* n_valid_given, lmh_bf16* dH,
+                                       const lmh_vp_dest* dW_dest, void* workspace,
+                                       size_t workspace_bytes, void* stream);
 LMH_API lmh_status lmh_reduce_ranks_f32(int R, int64_t n, const float* parts, float* out,
                                         void* stream);
 

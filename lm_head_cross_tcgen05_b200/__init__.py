@@ -41,7 +41,7 @@ __all__ = [
     "ENTRY_LOSS_FWD_BWD", "lmh_loss_fwd_bwd", "loss_fwd_bwd",
     "ENTRY_VP_SUPPORT_PARTIALS", "ENTRY_VP_SUPPORT_COMBINE", "ENTRY_VP_SUPPORT_BWD",
     "lmh_vp_support_partials", "lmh_vp_support_combine", "lmh_vp_support_bwd",
-    "F_DW_ACC_STORE", "lmh_count_valid", "lmh_reduce_ranks_f32",
+    "F_DW_ACC_STORE", "lmh_count_valid", "lmh_reduce_ranks_f32", "lmh_dp_loss_fwd_bwd",
 ]
 
 lib()  # load now: a missing library is an import error, never a silent fallback
@@ -399,6 +399,25 @@ def lmh_count_valid(labels, V, n_valid, stream=None) -> None:
     st = lib().lmh_count_valid(int(labels.numel()), int(V), _p(labels, _i32, "labels"),
                                _p(n_valid, _i32, "n_valid"), _s(stream))
     _ok("lmh_count_valid", st)
+
+
+def lmh_dp_loss_fwd_bwd(shape, mode, H, W, labels, grad, loss_rows, lse, logprob=None,
+                        argmax=None, loss_mean=None, n_valid_given=None, dH=None, dest=None, *,
+                        workspace, stream=None) -> None:
+    """dest: (int64 CUDA tensor of the R receive-buffer addresses, R, rank)."""
+    N, d, V = shape.N, shape.d, shape.V
+    _fits(H=(H, N * d), W=(W, V * d), labels=(labels, N),
+          grad=(grad, 1 if shape.flags & F_GRAD_SCALAR else N), loss_rows=(loss_rows, N),
+          lse=(lse, N), logprob=(logprob, N), argmax=(argmax, N), loss_mean=(loss_mean, 1),
+          n_valid_given=(n_valid_given, 1), dH=(dH, N * d))
+    st = lib().lmh_dp_loss_fwd_bwd(
+        ctypes.byref(shape), int(mode), _p(H, _bf, "H"), _p(W, _bf, "W"),
+        _p(labels, _i32, "labels"), _p(grad, _f32, "grad"), _p(loss_rows, _f32, "loss_rows"),
+        _p(lse, _f32, "lse"), _p(logprob, _f32, "logprob"), _p(argmax, _i32, "argmax"),
+        _p(loss_mean, _f32, "loss_mean"), _p(n_valid_given, _i32, "n_valid_given"),
+        _p(dH, _bf, "dH"), _dest(dest), _p(workspace, _u8, "workspace"), workspace.numel(),
+        _s(stream))
+    _ok("lmh_dp_loss_fwd_bwd", st)
 
 
 def lmh_reduce_ranks_f32(parts, out, stream=None) -> None:

@@ -67,6 +67,8 @@ _SIGS = {
                             + [c_size_t, _P]),
     "lmh_scale_bf16": (c_int, [_P, c_int64, _P, _P]),
     "lmh_count_valid": (c_int, [c_int64, c_int64, _P, _P, _P]),
+    "lmh_dp_loss_fwd_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 11
+                            + [ctypes.POINTER(lmh_vp_dest), _P, c_size_t, _P]),
     "lmh_reduce_ranks_f32": (c_int, [c_int, c_int64, _P, _P, _P]),
     "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),
     "lmh_logprob_noalloc": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6),

@@ -30,6 +30,7 @@ class RankGroup:
         self.R = dist.get_world_size(group) if self.distributed else 1
         self.rank = dist.get_rank(group) if self.distributed else 0
         self.ops = ops
+        self._sym = None
 
     def _gather(self, rec):
         """[N, w] records of this rank -> [R, N, w] of all ranks in rank order."""
@@ -75,3 +76,39 @@ class RankGroup:
         if all(n == top for n in sizes):
             return every
         return torch.cat([every[j * top: j * top + sizes[j]] for j in range(self.R)])
+
+    # ------------------------------------------------------------- peer-memory exchange
+    def _symmetric(self, rows, d, device):
+        """For a sum over the ranks of [rows, d] fp32 parts, in symmetric memory (peer-mapped
+        over NVLink): the receive buffer of this rank ([R][rows_j][d] fp32 within
+        R * max_j rows_j * d) and the full bf16 [rows, d] output of every rank, with the
+        device tables of the R ranks' addresses of both."""
+        if self._sym is not None and self._sym["key"] == (rows, d):
+            return self._sym
+        import torch.distributed._symmetric_memory as symm_mem
+        group = self.group if self.group is not None else dist.group.WORLD
+        sizes = [b - a for a, b in row_slices(rows, self.R)]
+        n_recv = self.R * max(sizes) * d
+        recv = symm_mem.empty(n_recv, dtype=torch.float32, device=device)
+        recv_h = symm_mem.rendezvous(recv, group)
+        out = symm_mem.empty(rows * d, dtype=torch.bfloat16, device=device)
+        out_h = symm_mem.rendezvous(out, group)
+
+        def table(h, n, dtype):
+            return torch.tensor([h.get_buffer(r, (n,), dtype).data_ptr() for r in range(self.R)],
+                                dtype=torch.int64, device=device)
+        self._sym = dict(key=(rows, d), sizes=sizes, recv=recv, recv_h=recv_h, out=out,
+                         out_h=out_h, recv_tab=table(recv_h, n_recv, torch.float32),
+                         out_tab=table(out_h, rows * d, torch.bfloat16))
+        return self._sym
+
+    def _reduce_p2p(self, sym):
+        """After every rank's rows landed: reduce this rank's slice into every rank's output."""
+        sizes = sym["sizes"]
+        mine, start = sizes[self.rank], sum(sizes[:self.rank])
+        d = sym["key"][1]
+        sym["recv_h"].barrier(channel=1)      # every rank's rows are in the receive buffers
+        parts = sym["recv"][: self.R * mine * d].view(self.R, mine, d)
+        self.ops.reduce_rows_to(parts, sym["out_tab"], self.R, start)
+        sym["out_h"].barrier(channel=0)       # every rank's slice is in every output
+        return sym["out"].view(-1, d).clone()

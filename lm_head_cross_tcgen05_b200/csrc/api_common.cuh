@@ -166,7 +166,7 @@ enum KernelId {
   KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_SUPPORT_DOTS, KID_SUPPORT_LSE,
   KID_SUPPORT_DH, KID_SUPPORT_DW, KID_SPLIT_SUM, KID_VP_LABELS, KID_VP_FINALIZE,
   KID_VP_COMBINE, KID_VP_REDUCE, KID_VP_SCALE, KID_FIX_CANDS, KID_SCALE, KID_COUNT_VALID,
-  KID_REDUCE_RANKS, KID_COUNT
+  KID_REDUCE_RANKS, KID_ZERO_SLOTS, KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "count_labels", "prep_cands", "gemm_logits_stats", "gemm_logits_stats_store",
@@ -174,7 +174,7 @@ const char* const kKernelNames[KID_COUNT] = {
     "mean", "support_out", "bwd_coef", "cast_bf16", "support_dots", "support_lse",
     "support_grad_dh", "support_dw", "split_sum", "vp_local_labels", "vp_finalize",
     "vp_combine", "vp_reduce_rows", "vp_scale", "fix_cands", "scale_bf16", "count_valid",
-    "reduce_ranks"};
+    "reduce_ranks", "zero_slots"};
 
 struct ProfRec {
   int id;
@@ -434,7 +434,8 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
                               const lmh_bf16* W, int64_t r0, int rows, int chunk_idx,
                               lmh_bf16* dH, lmh_bf16* dW, float* dW_acc, const Ws& ws,
                               cudaStream_t st, float* dH_f32 = nullptr,
-                              const RowScatter* scatter = nullptr) {
+                              const RowScatter* scatter = nullptr,
+                              const RowScatter* dw_scatter = nullptr) {
   const __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
   if (scatter) {  // each fp32 row straight to the rank that reduces it
     CUtensorMap ta, tb;
@@ -479,7 +480,7 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
       LMH_TRY(last_launch());
     }
   }
-  if (dW || dW_acc) {
+  if (dW || dW_acc || dw_scatter) {
     CUtensorMap ta, tb, tc;
     if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BK) || !tmap_2d(&tb, H + r0 * P.d, P.d, rows, P.d, BK))
       return LMH_ERR_CUDA;
@@ -492,12 +493,22 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
     EpiDW::Params ep;
     ep.V = static_cast<int>(P.V);
     ep.d = static_cast<int>(P.d);
-    if (!acc) ep.acc_mode = 0;
-    else if (dW_acc) ep.acc_mode = (P.acc_store && chunk_idx == 0) ? 1 : 2;
-    else ep.acc_mode = chunk_idx == 0 ? 1 : (last ? 3 : 2);
+    if (dw_scatter) {  // one chunk: fp32 rows to the reducing ranks (no output map)
+      ep.acc_mode = 4;
+      ep.sc = *dw_scatter;
+    } else if (!acc) {
+      ep.acc_mode = 0;
+    } else if (dW_acc) {
+      ep.acc_mode = (P.acc_store && chunk_idx == 0) ? 1 : 2;
+    } else {
+      ep.acc_mode = chunk_idx == 0 ? 1 : (last ? 3 : 2);
+    }
     CUtensorMap td;  // mode 3: the accumulator, read by the epilogue
     bool ok;
-    if (ep.acc_mode == 0) {
+    if (ep.acc_mode == 4) {
+      tc = ta;
+      ok = true;
+    } else if (ep.acc_mode == 0) {
       ok = tmap_out(&tc, dW, P.d, P.V, P.d);
     } else if (ep.acc_mode == 3) {
       ok = tmap_out(&tc, dW, P.d, P.V, P.d) && tmap_acc(&td, acc, P.d, P.V, P.d);

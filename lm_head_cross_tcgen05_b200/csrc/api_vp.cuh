@@ -396,6 +396,24 @@ extern "C" lmh_status lmh_vp_support_bwd(const lmh_shape* shard, int mode, int64
   return LMH_OK;
 }
 
+// Row data-parallel one-pass step whose dW GEMM stores each fp32 row of the rank's dW into the
+// receive buffer of the rank that reduces that vocabulary row (the row scatter over V).
+extern "C" lmh_status lmh_dp_loss_fwd_bwd(const lmh_shape* shape, int mode, const lmh_bf16* H,
+                                          const lmh_bf16* W, const int32_t* labels,
+                                          const float* grad, float* loss_rows, float* lse,
+                                          float* logprob, int32_t* argmax, float* loss_mean,
+                                          const int32_t* n_valid_given, lmh_bf16* dH,
+                                          const lmh_vp_dest* dW_dest, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+  if (!shape_ok(shape) || !dW_dest) return LMH_ERR_INVALID_ARG;
+  if (mode != LMH_BWD_CE && mode != LMH_BWD_LOGPROB) return LMH_ERR_INVALID_ARG;
+  RowScatter sc;
+  LMH_TRY(vp_dest_ok(dW_dest, nullptr, shape->V, &sc));
+  return loss_fwd_impl(shape, true, mode, grad, H, W, labels, loss_rows, lse, logprob, argmax,
+                       loss_mean, nullptr, n_valid_given, dH, nullptr, nullptr, workspace,
+                       workspace_bytes, stream, &sc);
+}
+
 extern "C" lmh_status lmh_vp_reduce_rows(int R, int64_t rows, int64_t d, const float* parts,
                                          lmh_bf16* out, void* stream) {
   if (R < 1 || rows < 0 || d <= 0 || (d % 64) != 0) return LMH_ERR_INVALID_ARG;

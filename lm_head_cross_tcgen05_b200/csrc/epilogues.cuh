@@ -376,6 +376,8 @@ struct EpiDH {
 // acc_mode 3: dW = bf16(acc + sum) (last chunk of an internal accumulator, which is not
 //             written back): the accumulator block is loaded by TMA into the warp's staging
 //             buffers, added in registers, and the bf16 result stored through ctx.tmC.
+// acc_mode 4: 0 + sum in fp32, each row stored straight into the receive buffer of the rank
+//             that reduces it (p.sc: row data-parallel dW over peer memory; one chunk).
 // In modes 1 and 2 ctx.tmC maps the fp32 accumulator [V, d]; in mode 3 ctx.tmD does (fp32,
 // box 32 x 32 rows, 128-byte swizzle) and ctx.tmC maps bf16 dW. Every
 // element has one owner tile per launch and the launches of a call run in chunk order, so the
@@ -392,6 +394,7 @@ struct EpiDW {
     int V;
     int d;
     int acc_mode;
+    RowScatter sc;  // acc_mode 4: the receive buffers of the R ranks, N = V
   };
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
                                               int rit, EpiCtx& ctx) {
@@ -407,6 +410,18 @@ struct EpiDW {
       tmem_ld32(taddr + sb * 64 + 32, b);
       if (p.acc_mode == 0) {
         stage_store_64(ctx, a, b, col0, wrow, wv);
+      } else if (p.acc_mode == 4) {
+        const int row = mb * BM + rit;
+        if (row < p.V) {
+          float4* o = reinterpret_cast<float4*>(p.sc.row(row, p.d) + col0);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float* v = u < 8 ? a : b;
+            const int q = (u & 7) * 4;
+            __stcs(o + u, make_float4(__fadd_rn(0.f, v[q]), __fadd_rn(0.f, v[q + 1]),
+                                      __fadd_rn(0.f, v[q + 2]), __fadd_rn(0.f, v[q + 3])));
+          }
+        }
       } else if (p.acc_mode == 3) {
         if (!wv) continue;  // warp-uniform: nothing of this block exists
         add_loaded_64(ctx, col0, wrow, a, b);

@@ -46,9 +46,10 @@ static lmh_status loss_fwd_impl(const lmh_shape* shape, bool weighted, int mode,
                                 float* logprob, int32_t* argmax, float* loss_mean,
                                 int32_t* n_valid, const int32_t* n_valid_given, lmh_bf16* dH,
                                 lmh_bf16* dW, float* dW_acc, void* workspace,
-                                size_t workspace_bytes, void* stream) {
+                                size_t workspace_bytes, void* stream,
+                                const RowScatter* dw_scatter = nullptr) {
   if (!shape_ok(shape)) return LMH_ERR_INVALID_ARG;
-  const bool fused = dH || dW || dW_acc;
+  const bool fused = dH || dW || dW_acc || dw_scatter;
   const Plan P = make_plan(shape, weighted ? LMH_ENTRY_LOSS_FWD_BWD : LMH_ENTRY_LOSS_FWD, fused,
                            dW && !dW_acc);
   int dev, sms;
@@ -56,9 +57,18 @@ static lmh_status loss_fwd_impl(const lmh_shape* shape, bool weighted, int mode,
   if (P.N > 0 && (!labels || !loss_rows || !lse)) return LMH_ERR_INVALID_ARG;
   if (!aligned16(dH) || !aligned16(dW) || !aligned16(dW_acc)) return LMH_ERR_ALIGNMENT;
   if (weighted && (shape->flags & LMH_F_GRAD_SCALAR) && !grad) return LMH_ERR_INVALID_ARG;
+  if (dw_scatter && (dW || dW_acc || P.nchunks > 1)) return LMH_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ws ws{static_cast<uint8_t*>(workspace), static_cast<WsHeader*>(workspace)};
   LMH_TRY(clear_header(ws, st));
+  if (P.N == 0 && dw_scatter) {  // this rank's slots of every receive buffer are zero
+    const int64_t n4 = P.V * P.d / 4;
+    const int64_t blocks = cdiv(n4, 256);
+    ProfScope ps(KID_ZERO_SLOTS, st);
+    zero_slots_kernel<<<static_cast<unsigned>(blocks < 8192 ? blocks : 8192), 256, 0, st>>>(
+        *dw_scatter, P.V, static_cast<int>(P.d));
+    LMH_TRY(last_launch());
+  }
   if (P.N == 0) return empty_call(P, loss_mean, n_valid, dW, dW_acc, st);
   LMH_TRY(count_labels(P, labels, ws, st));
   const int mean = (shape->flags & LMH_F_MEAN) ? 1 : 0;
@@ -106,7 +116,7 @@ static lmh_status loss_fwd_impl(const lmh_shape* shape, bool weighted, int mode,
       }
       LMH_TRY(last_launch());
       LMH_TRY(run_backward_gemms(P, dev, sms, H, W, r0, rows, static_cast<int>(ci), dH, dW,
-                                 dW_acc, ws, st));
+                                 dW_acc, ws, st, nullptr, nullptr, dw_scatter));
     }
   }
   if (loss_mean) {

@@ -12,6 +12,7 @@
 // z is the tempered logit (z / tau_i) when a temperature is given.
 #pragma once
 
+#include "epilogues.cuh"
 #include "rowops.cuh"
 
 namespace lmh {
@@ -220,6 +221,17 @@ __global__ void vp_reduce_rows_kernel(int R, long long n4, const float4* __restr
       a.w += b.w;
     }
     __stcs(o + j, make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w)));
+  }
+}
+
+// A rank without rows still owns one slot of rows in every receive buffer of a row scatter
+// (its fp32 contribution to each slice): zero them, V x d elements in float4 groups.
+__global__ void zero_slots_kernel(RowScatter sc, long long V, int d) {
+  const long long q = d / 4;  // float4 groups per row
+  for (long long j = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; j < V * q;
+       j += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long v = j / q;
+    reinterpret_cast<float4*>(sc.row(v, d))[j - v * q] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 

@@ -19,9 +19,16 @@ in a fixed order, so the result is bitwise reproducible for a given rank count a
    slice j from every rank, ``lmh_vp_reduce_rows`` adds them, and an all-gather returns the
    bf16 slices to every rank.
 
+With ``p2p=True`` the dW exchange runs over peer memory instead of NCCL: the receive buffers
+and every rank's dW live in symmetric memory (peer-mapped over NVLink), the dW GEMM's epilogue
+stores each fp32 row straight into the receive buffer of the rank that reduces it while the
+GEMM runs (``lmh_dp_loss_fwd_bwd``), and ``lmh_vp_reduce_rows_to`` stores each reduced bf16
+slice into every rank's dW. The additions are the same, so the bits are the same; all rows of
+a rank then form one chunk.
+
 Against one device on the concatenated batch the values agree to fp32 rounding (the dW sum and
 the mean are grouped by rank). The compute steps run in the library's CUDA kernels through
-``CudaOps``; ``DataParallelCE`` takes any object with the same four methods, which is how its
+``CudaOps``; ``DataParallelCE`` takes any object with the same methods, which is how its
 exchange logic is tested on CPU ranks.
 """
 from __future__ import annotations
@@ -29,9 +36,9 @@ from __future__ import annotations
 import torch
 
 from . import (BWD_CE, ENTRY_LOSS_FWD, ENTRY_LOSS_FWD_BWD, F_DW_ACC_GIVEN, F_DW_ACC_STORE,
-               F_FUSED_BWD, F_GRAD_SCALAR, F_MEAN, lmh_count_valid, lmh_loss_fwd,
-               lmh_loss_fwd_bwd, lmh_reduce_ranks_f32, lmh_vp_reduce_rows, make_shape,
-               workspace)
+               F_FUSED_BWD, F_GRAD_SCALAR, F_MEAN, lmh_count_valid, lmh_dp_loss_fwd_bwd,
+               lmh_loss_fwd, lmh_loss_fwd_bwd, lmh_reduce_ranks_f32, lmh_vp_reduce_rows,
+               lmh_vp_reduce_rows_to, make_shape, workspace)
 from ._ranks import RankGroup
 
 __all__ = ["CudaOps", "DataParallelCE"]
@@ -83,6 +90,32 @@ class CudaOps:
         out["workspace"] = ws
         return out
 
+    def fused_scatter(self, H, W, labels, n_given, dest, *, mode=BWD_CE, grad=None,
+                      mean=True, scalar_grad=False, temperature=None, want_dH=True):
+        """fused() whose dW GEMM stores the rank's fp32 dW rows into the reducing ranks'
+        receive buffers (dest = (address table, R, rank)); all rows form one chunk."""
+        N, d = H.shape
+        V = W.shape[0]
+        dev = H.device
+        flags = F_FUSED_BWD | (F_MEAN if mean else 0) | (F_GRAD_SCALAR if scalar_grad else 0)
+        shape = make_shape(N, d, V, 0, max(N, 1), flags, temperature)
+        f32 = torch.float32
+        out = dict(loss_rows=torch.empty(N, dtype=f32, device=dev),
+                   lse=torch.empty(N, dtype=f32, device=dev),
+                   logprob=torch.empty(N, dtype=f32, device=dev),
+                   argmax=torch.empty(N, dtype=torch.int32, device=dev),
+                   loss_mean=torch.empty(1, dtype=f32, device=dev),
+                   dH=torch.empty(N, d, dtype=torch.bfloat16, device=dev) if want_dH else None)
+        ws = workspace(shape, ENTRY_LOSS_FWD_BWD, dev)
+        lmh_dp_loss_fwd_bwd(shape, mode, H, W, labels, grad, out["loss_rows"], out["lse"],
+                            out["logprob"], out["argmax"], out["loss_mean"], n_given, out["dH"],
+                            dest, workspace=ws)
+        out["workspace"] = ws
+        return out
+
+    def reduce_rows_to(self, parts, out_table, n_out, row_offset):
+        lmh_vp_reduce_rows_to(parts, out_table, n_out, row_offset)
+
     def sum_ranks(self, parts):
         out = torch.empty(parts.shape[1], dtype=torch.float32, device=parts.device)
         lmh_reduce_ranks_f32(parts, out)
@@ -108,11 +141,12 @@ class DataParallelCE(RankGroup):
     before the step, for callers whose per-row weights depend on it."""
 
     def __init__(self, group=None, chunk_rows: int = 0, mean: bool = True, temperature=None,
-                 ops=None):
+                 ops=None, p2p: bool = False):
         super().__init__(group, ops if ops is not None else CudaOps())
         self.chunk_rows = chunk_rows
         self.mean = mean
         self.temperature = temperature
+        self.p2p = p2p and self.R > 1   # one rank has nothing to exchange
 
     def count(self, labels, V: int):
         """The valid rows (0 <= label < V) of all ranks: a one-element int32 device tensor."""
@@ -123,15 +157,27 @@ class DataParallelCE(RankGroup):
         """loss_rows, lse, logprob, argmax, dH: this rank's rows; loss_mean, n_valid and dW
         [V, d] bf16: the same on every rank."""
         n = self.count(labels, W.shape[0])
-        # one rank has nothing to add: its bf16 dW comes straight from the GEMM's fp32 tile
-        # sums, the bits the rank-ordered sum of one fp32 part would give
-        out = self.ops.fused(H, W, labels, n, mode=mode, grad=grad, weighted=grad is not None,
-                             mean=self.mean, scalar_grad=scalar_grad,
-                             chunk_rows=self.chunk_rows, temperature=self.temperature,
-                             want_dH=want_dH, bf16_dW=self.R == 1)
+        if self.p2p:
+            V, d = W.shape
+            sym = self._symmetric(V, d, H.device)   # receive buffers for V rows, dW outputs
+            sym["recv_h"].barrier(channel=0)        # no rank still reads its last buffer
+            out = self.ops.fused_scatter(H, W, labels, n, (sym["recv_tab"], self.R, self.rank),
+                                         mode=mode, grad=grad, mean=self.mean,
+                                         scalar_grad=scalar_grad,
+                                         temperature=self.temperature, want_dH=want_dH)
+            out["dW"] = self._reduce_p2p(sym)
+        else:
+            # one rank has nothing to add: its bf16 dW comes straight from the GEMM's fp32
+            # tile sums, the bits the rank-ordered sum of one fp32 part would give
+            out = self.ops.fused(H, W, labels, n, mode=mode, grad=grad,
+                                 weighted=grad is not None, mean=self.mean,
+                                 scalar_grad=scalar_grad, chunk_rows=self.chunk_rows,
+                                 temperature=self.temperature, want_dH=want_dH,
+                                 bf16_dW=self.R == 1)
+            if self.R > 1:
+                out["dW"] = self._sum_rows(out.pop("dW_part"))
         if self.R > 1:
             shares = self._gather(out["loss_mean"].reshape(1, 1)).reshape(self.R, 1)
             out["loss_mean"] = self.ops.sum_ranks(shares)
-            out["dW"] = self._sum_rows(out.pop("dW_part"))
         out["n_valid"] = n
         return out

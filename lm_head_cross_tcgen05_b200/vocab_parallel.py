@@ -191,7 +191,6 @@ class _VocabParallel(RankGroup):
         self.mean = mean
         self.temperature = temperature
         self.p2p = p2p and self.R > 1   # one rank has nothing to exchange
-        self._sym = None
 
     def _check_shard(self, W_shard):
         if W_shard.shape[0] != self.v1 - self.v0:
@@ -202,45 +201,12 @@ class _VocabParallel(RankGroup):
         """dH summed over the ranks from run(dest) -> (dH_part or None, dW): collectives, or
         with p2p the rows scattered straight to their reducing ranks."""
         if self.p2p:
-            sym = self._symmetric(N, d, device)
+            sym = self._symmetric(N, d, device)   # receive buffers for N rows, dH outputs
             sym["recv_h"].barrier(channel=0)   # no rank still reads its last receive buffer
             _, dW = run((sym["recv_tab"], self.R, self.rank))
             return self._reduce_p2p(sym), dW
         dH_part, dW = run(None)
         return self._sum_rows(dH_part), dW
-
-    def _symmetric(self, N, d, device):
-        """The receive buffer ([R][rows_j][d] fp32 within R * max_rows * d) and the full bf16
-        dH of every rank in symmetric memory, with the tables of the R ranks' addresses."""
-        if self._sym is not None and self._sym["key"] == (N, d):
-            return self._sym
-        import torch.distributed._symmetric_memory as symm_mem
-        group = self.group if self.group is not None else dist.group.WORLD
-        sizes = [b - a for a, b in row_slices(N, self.R)]
-        n_recv = self.R * max(sizes) * d
-        recv = symm_mem.empty(n_recv, dtype=torch.float32, device=device)
-        recv_h = symm_mem.rendezvous(recv, group)
-        dH = symm_mem.empty(N * d, dtype=torch.bfloat16, device=device)
-        dH_h = symm_mem.rendezvous(dH, group)
-
-        def table(h, n, dtype):
-            return torch.tensor([h.get_buffer(r, (n,), dtype).data_ptr() for r in range(self.R)],
-                                dtype=torch.int64, device=device)
-        self._sym = dict(key=(N, d), sizes=sizes, recv=recv, recv_h=recv_h, dH=dH, dH_h=dH_h,
-                         recv_tab=table(recv_h, n_recv, torch.float32),
-                         dH_tab=table(dH_h, N * d, torch.bfloat16))
-        return self._sym
-
-    def _reduce_p2p(self, sym):
-        """After every rank's rows landed: reduce this rank's slice into every rank's dH."""
-        sizes = sym["sizes"]
-        mine, start = sizes[self.rank], sum(sizes[:self.rank])
-        d = sym["dH"].numel() // sum(sizes)
-        sym["recv_h"].barrier(channel=1)      # every rank's dH rows are in the receive buffers
-        parts = sym["recv"][: self.R * mine * d].view(self.R, mine, d)
-        self.ops.reduce_rows_to(parts, sym["dH_tab"], self.R, start)
-        sym["dH_h"].barrier(channel=0)        # every rank's slice is in every dH
-        return sym["dH"].view(-1, d).clone()
 
 
 class VocabParallelCE(_VocabParallel):

@@ -167,6 +167,14 @@ def test_data_parallel_host_errors_without_gpu():
     assert lib.lmh_reduce_ranks_f32(2, 0, None, None, None) == 0     # nothing to do
     assert lib.lmh_reduce_ranks_f32(2, 4, ctypes.c_void_p(256), None, None) == 1
     assert lib.lmh_reduce_ranks_f32(2, 4, ctypes.c_void_p(256), ctypes.c_void_p(6), None) == 4
+    # the row-scattering step: no destination, a rank outside the group, a support mode
+    sh = L.make_shape(4, 64, 100, 0, 4, L.F_FUSED_BWD)
+    P = [None] * 11
+    assert lib.lmh_dp_loss_fwd_bwd(ctypes.byref(sh), 0, *P, None, None, 0, None) == 1
+    bad = _abi.lmh_vp_dest(ctypes.c_void_p(256), 2, 2)
+    assert lib.lmh_dp_loss_fwd_bwd(ctypes.byref(sh), 0, *P, ctypes.byref(bad), None, 0, None) == 1
+    ok = _abi.lmh_vp_dest(ctypes.c_void_p(256), 2, 1)
+    assert lib.lmh_dp_loss_fwd_bwd(ctypes.byref(sh), 2, *P, ctypes.byref(ok), None, 0, None) == 1
 
 
 def test_dw_store_flag_is_sizing_neutral():

@@ -174,6 +174,48 @@ def test_dw_acc_store_flag_overwrites(chunk):
         assert torch.equal(zero, junk), (mode, renorm)
 
 
+@pytest.mark.parametrize("split,d,V", [
+    ((150, 150), 192, 1000),
+    ((300, 0, 129, 71), 256, 2048),            # a rank without rows zeroes its slots
+    ((37,) * 8, 64, 3000),
+    ((40, 21, 7), 128, 70000),
+])
+def test_dw_row_scatter_matches_collective_path(split, d, V):
+    # the dW GEMM storing fp32 rows into the reducing ranks' receive buffers (stand-ins on
+    # this GPU, NaN so a row never written shows), then each slice reduced into every rank's
+    # dW: the collective path's bits
+    from lm_head_cross_tcgen05_b200._ranks import row_slices
+    N, R = sum(split), len(split)
+    x, _ = device_inputs(ragged(N, d, V, n_ignored=3, seed=4500 + N + V))
+    ref = _emulate(x, split)
+    H, W, y = x["H"], x["W"], x["labels"]
+    sizes = [b - a for a, b in row_slices(V, R)]
+    recv = [torch.full((R * max(sizes) * d,), float("nan"), device="cuda") for _ in range(R)]
+    outs = [torch.zeros(V, d, dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    rt = torch.tensor([t.data_ptr() for t in recv], dtype=torch.int64, device="cuda")
+    ot = torch.tensor([t.data_ptr() for t in outs], dtype=torch.int64, device="cuda")
+    ops = CudaOps()
+    got = [ops.fused_scatter(H[a:b], W, y[a:b], ref["n_valid"], (rt, R, r))
+           for r, (a, b) in enumerate(_bounds(split))]
+    start = 0
+    for j in range(R):
+        ops.reduce_rows_to(recv[j][: R * sizes[j] * d].view(R, sizes[j], d), ot, R, start)
+        start += sizes[j]
+    torch.cuda.synchronize()
+    for k in range(R):
+        assert torch.equal(outs[k], ref["dW"]), k
+    assert torch.equal(torch.cat([g["dH"] for g in got]), ref["dH"])
+    assert torch.equal(torch.cat([g["lse"] for g in got]), ref["lse"])
+    assert torch.equal(ops.sum_ranks(torch.stack([g["loss_mean"] for g in got])),
+                       ref["loss_mean"])
+    # the scatter runs the rank's rows as one chunk
+    sh = L.make_shape(N, d, V, 0, N // 2, L.F_FUSED_BWD | L.F_MEAN)
+    with pytest.raises(L.LmhError):
+        L.lmh_dp_loss_fwd_bwd(sh, L.BWD_CE, H, W, y, None, torch.empty(N, device="cuda"),
+                              torch.empty(N, device="cuda"), dest=(rt, R, 0),
+                              workspace=L.workspace(sh, L.ENTRY_LOSS_FWD_BWD, "cuda"))
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
