@@ -210,6 +210,39 @@ def test_large_vocab_vocabulary_parallel_step(large_vocab):
     check_grad(f["dW"], f64(out["dW"]), "dW vocabulary-parallel vs one device")
 
 
+def test_large_vocab_data_parallel_two_ranks(large_vocab):
+    # the large_vocab batch split over two data-parallel ranks on this GPU, through both dW
+    # exchanges: per-row results are the one-device bits, the dW sums agree with the
+    # one-device dW, and the row scatter from the dW GEMM gives the collective route's bits
+    from lm_head_cross_tcgen05_b200._ranks import row_slices
+    from lm_head_cross_tcgen05_b200.data_parallel import CudaOps
+    wl, x, out = large_vocab
+    H, W, y = x["H"], x["W"], x["labels"]
+    V, d = W.shape
+    bounds = [(0, 5000), (5000, wl.N)]
+    ops = CudaOps()
+    n = (ops.count_valid(y[:5000], V) + ops.count_valid(y[5000:], V)).to(torch.int32)
+    parts = [ops.fused(H[a:b], W, y[a:b], n, chunk_rows=b - a) for a, b in bounds]
+    for k in ("loss_rows", "lse", "argmax"):
+        assert torch.equal(torch.cat([p[k] for p in parts]), out[k]), k
+    dW = ops.reduce_rows(torch.stack([p.pop("dW_part") for p in parts]))
+    check_grad(torch.cat([p["dH"] for p in parts]), f64(out["dH"]), "dH two ranks")
+    check_grad(dW, f64(out["dW"]), "dW two ranks vs one device")
+    check_dw_properties(dW)
+    sizes = [b - a for a, b in row_slices(V, 2)]
+    recv = [torch.full((2 * max(sizes) * d,), float("nan"), device="cuda") for _ in range(2)]
+    outs = [torch.zeros(V, d, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    rt = torch.tensor([t.data_ptr() for t in recv], dtype=torch.int64, device="cuda")
+    ot = torch.tensor([t.data_ptr() for t in outs], dtype=torch.int64, device="cuda")
+    for r, (a, b) in enumerate(bounds):
+        g = ops.fused_scatter(H[a:b], W, y[a:b], n, (rt, 2, r))
+        assert torch.equal(g["dH"], parts[r]["dH"])
+    ops.reduce_rows_to(recv[0][: 2 * sizes[0] * d].view(2, sizes[0], d), ot, 2, 0)
+    ops.reduce_rows_to(recv[1][: 2 * sizes[1] * d].view(2, sizes[1], d), ot, 2, sizes[0])
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], dW) and torch.equal(outs[1], dW)
+
+
 def test_many_chunks_and_large_row_indices():
     # 131149 rows in 33 default-size chunks (32 x 4096 + 77): the dW accumulator is stored,
     # added 31 times and finally added and cast in the epilogue; row indices pass 2^17 and
