@@ -1,8 +1,8 @@
-"""The exchange steps the multi-rank drivers share. Each one only moves data between the ranks
-of a torch.distributed group; the additions that combine the moved values run in the library's
-kernels (through the driver's ``ops``), always in ascending rank order, so no floating-point
-value is reduced inside a collective and the results are bitwise reproducible for a given
-rank count."""
+"""The exchange steps the multi-rank classes (VocabParallelCE, VocabParallelSupport,
+DataParallelCE) share. Each one only moves data between the ranks of a torch.distributed
+group; the additions that combine the moved values run in the library's kernels (through the
+class's ``ops``), always in ascending rank order, so no floating-point value is reduced inside
+a collective and the results are bitwise reproducible for a given rank count."""
 from __future__ import annotations
 
 import torch

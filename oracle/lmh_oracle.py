@@ -19,7 +19,7 @@ The method reaches these results exactly up to rounding order, so each function 
 plain definition, with library matmuls as steps. Chunking only reorders rounding and has no
 place here; ``chunk_plan`` states the row partition the library walks, for host-side tests.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * "candidate-restricted log-probabilities" are full-vocabulary log-probs evaluated at the
   candidate ids: lp_ik = z_i,c_ik - lse_i.
