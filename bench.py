@@ -216,7 +216,7 @@ def _timed(fn, n):
     return time.perf_counter() - t
 
 
-def _rows_for(fn, target_s, n0, n1, cap=1024):
+def _rows_for(fn, target_s, n0, n1, cap=2048):
     """Rows that take about target_s seconds, from t(n) = a + b n at two calibration sizes
     (a is the per-call fp64 widening of W, b the per-row work)."""
     t0, t1 = _timed(fn, n0), _timed(fn, n1)
