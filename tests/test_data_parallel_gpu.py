@@ -174,20 +174,25 @@ def test_dw_acc_store_flag_overwrites(chunk):
         assert torch.equal(zero, junk), (mode, renorm)
 
 
-@pytest.mark.parametrize("split,d,V", [
-    ((150, 150), 192, 1000),
-    ((300, 0, 129, 71), 256, 2048),            # a rank without rows zeroes its slots
-    ((37,) * 8, 64, 3000),
-    ((40, 21, 7), 128, 70000),
+@pytest.mark.parametrize("split,d,V,weighted", [
+    ((150, 150), 192, 1000, False),
+    ((300, 0, 129, 71), 256, 2048, False),     # a rank without rows zeroes its slots
+    ((37,) * 8, 64, 3000, False),
+    ((40, 21, 7), 128, 70000, False),
+    ((90, 45, 121), 128, 5000, True),          # weighted log-prob objective, temperature
 ])
-def test_dw_row_scatter_matches_collective_path(split, d, V):
+def test_dw_row_scatter_matches_collective_path(split, d, V, weighted):
     # the dW GEMM storing fp32 rows into the reducing ranks' receive buffers (stand-ins on
     # this GPU, NaN so a row never written shows), then each slice reduced into every rank's
     # dW: the collective path's bits
     from lm_head_cross_tcgen05_b200._ranks import row_slices
     N, R = sum(split), len(split)
     x, _ = device_inputs(ragged(N, d, V, n_ignored=3, seed=4500 + N + V))
-    ref = _emulate(x, split)
+    kw = {}
+    if weighted:
+        kw = dict(mode=L.BWD_LOGPROB, tau=0.8,
+                  grad=torch.linspace(-1.0, 2.0, N, device="cuda").contiguous())
+    ref = _emulate(x, split, **kw)
     H, W, y = x["H"], x["W"], x["labels"]
     sizes = [b - a for a, b in row_slices(V, R)]
     recv = [torch.full((R * max(sizes) * d,), float("nan"), device="cuda") for _ in range(R)]
@@ -195,7 +200,9 @@ def test_dw_row_scatter_matches_collective_path(split, d, V):
     rt = torch.tensor([t.data_ptr() for t in recv], dtype=torch.int64, device="cuda")
     ot = torch.tensor([t.data_ptr() for t in outs], dtype=torch.int64, device="cuda")
     ops = CudaOps()
-    got = [ops.fused_scatter(H[a:b], W, y[a:b], ref["n_valid"], (rt, R, r))
+    got = [ops.fused_scatter(H[a:b], W, y[a:b], ref["n_valid"], (rt, R, r),
+                             mode=kw.get("mode", L.BWD_CE), temperature=kw.get("tau"),
+                             grad=kw["grad"][a:b].contiguous() if weighted else None)
            for r, (a, b) in enumerate(_bounds(split))]
     start = 0
     for j in range(R):
