@@ -80,3 +80,45 @@ def test_data_parallel_exchange_gloo(world, case):
         assert r["nvalid"] and r["argmax"], r
         assert r["dH"] < 1e-9 and r["dW"] < 1e-9, r
     assert len({r["dW_digest"] for r in res}) == 1   # every rank holds the same dW
+
+
+def _absent_rank_worker(rank, world, port, q):
+    import datetime
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=3))
+    try:
+        if rank == 1:            # leaves between steps: never joins the step's collectives
+            time.sleep(10)
+            q.put(dict(rank=rank))
+            return
+        from lm_head_cross_tcgen05_b200.data_parallel import DataParallelCE
+        from tests.dp_oracle_ops import DataParallelOracleOps
+        from workloads import make_inputs, ragged
+        x = make_inputs(ragged(8, 64, 300, seed=5), device="cpu")
+        dp = DataParallelCE(ops=DataParallelOracleOps())
+        t0 = time.monotonic()
+        try:
+            dp.forward_backward(x["H"], x["W"], x["labels"])
+            q.put(dict(rank=rank, error=None))
+        except Exception as e:   # the group's timeout ends the first collective
+            q.put(dict(rank=rank, error=type(e).__name__, after=time.monotonic() - t0))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_absent_rank_ends_the_step_with_an_error():
+    # a rank that never joins: the others' first exchange (the global count) fails after the
+    # process group's timeout instead of waiting for ever
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_absent_rank_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    res = sorted((q.get(timeout=120) for _ in ps), key=lambda r: r["rank"])
+    for p in ps:
+        p.join(timeout=60)
+    assert res[0]["error"] is not None, res
+    assert res[0]["after"] < 9.0, res
