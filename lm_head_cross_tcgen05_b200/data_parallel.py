@@ -138,7 +138,9 @@ class DataParallelCE(RankGroup):
     of ``lmh_loss_fwd_bwd``: sum_i w_i l_i over all ranks' rows, with w_i = this rank's
     ``grad[i]`` taken as given, or with ``scalar_grad`` one upstream gradient g for every
     row (divided by the global count with mean=True). ``count`` gives the global count
-    before the step, for callers whose per-row weights depend on it."""
+    before the step, for callers whose per-row weights depend on it. With ``p2p`` (and more
+    than one rank) dW is exchanged over peer memory and each rank's rows form one chunk
+    (``chunk_rows`` is not used)."""
 
     def __init__(self, group=None, chunk_rows: int = 0, mean: bool = True, temperature=None,
                  ops=None, p2p: bool = False):
