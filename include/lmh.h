@@ -541,6 +541,36 @@ LMH_API lmh_status lmh_logprob_noalloc(const lmh_shape* shape, const lmh_bf16* H
                                        float* lse, void* stream);
 
 /*
+ * lmh_peer_barrier — a stream-ordered barrier of R ranks through peer memory, with a bounded
+ * wait. Not part of the method: it orders the peer-memory exchanges of the multi-rank steps
+ * (the RowScatter of lmh_vp_loss_bwd / lmh_vp_fused_bwd / lmh_dp_loss_fwd_bwd writes into
+ * another rank's receive buffer, and that rank may reduce the buffer only after every rank's
+ * stores have landed; lmh_vp_reduce_rows_to writes into every rank's output, which the
+ * owners may read only after every rank's reduce).
+ *   signals: DEVICE array of R pointers, 8-byte aligned. signals[j] is rank j's signal array
+ *     of R uint32 words, which may live in another GPU's memory (a peer mapping over NVLink,
+ *     e.g. symmetric memory). Zero every rank's array once, and make sure every rank has done
+ *     so (e.g. a host-side collective), before the first barrier.
+ *   epoch: the barrier's number, 1, 2, 3, ... in the same sequence on every rank (0 is
+ *     invalid). Words are compared modulo 2^32.
+ *   The kernel makes this rank's earlier writes on `stream` (peer stores included) visible
+ *   system-wide, stores `epoch` into word `rank` of every rank's array, then waits until
+ *   every word of signals[rank] has reached `epoch`. Later work on `stream` sees what the
+ *   other ranks wrote before their signals.
+ *   timeout_ms (1..60000): the wait gives up after this long, sets LMH_DEVERR_TIMEOUT in the
+ *     workspace's error word and returns; the context stays usable. The word is never cleared
+ *     here: read it with lmh_read_errors (which synchronises the stream) before trusting the
+ *     exchange that the barrier ordered, and clear it before the next use.
+ *   workspace: at least 256 bytes, 256-byte aligned (only its error word is used).
+ *   R in 1..1024, 0 <= rank < R. LMH_ERR_INVALID_ARG / LMH_ERR_ALIGNMENT before any launch.
+ * Never run two ranks of one barrier as separate launches on the same GPU: nothing makes them
+ * run at the same time, so they would wait out the time-out on each other.
+ */
+LMH_API lmh_status lmh_peer_barrier(void* workspace, uint32_t* const* signals, int32_t R,
+                                    int32_t rank, uint32_t epoch, uint32_t timeout_ms,
+                                    void* stream);
+
+/*
  * lmh_selftest_wait_timeout — failure-path self-test (not part of the method). Enqueues one
  * thread that waits, with the bounded wait every kernel of this library uses, on an mbarrier
  * that nothing arrives on. The wait gives up after timeout_ms (1..5000) and sets

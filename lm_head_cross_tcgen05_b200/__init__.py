@@ -42,6 +42,7 @@ __all__ = [
     "ENTRY_VP_SUPPORT_PARTIALS", "ENTRY_VP_SUPPORT_COMBINE", "ENTRY_VP_SUPPORT_BWD",
     "lmh_vp_support_partials", "lmh_vp_support_combine", "lmh_vp_support_bwd",
     "F_DW_ACC_STORE", "lmh_count_valid", "lmh_reduce_ranks_f32", "lmh_dp_loss_fwd_bwd",
+    "lmh_peer_barrier",
 ]
 
 lib()  # load now: a missing library is an import error, never a silent fallback
@@ -434,6 +435,18 @@ def lmh_scale_bf16(x, g, stream=None) -> None:
     _fits(g=(g, 1))
     st = lib().lmh_scale_bf16(_p(x, _bf, "x"), int(x.numel()), _p(g, _f32, "g"), _s(stream))
     _ok("lmh_scale_bf16", st)
+
+
+def lmh_peer_barrier(workspace, signals, R: int, rank: int, epoch: int,
+                     timeout_ms: int = 4000, stream=None) -> None:
+    """Barrier number ``epoch`` of R ranks through peer memory: signals is an int64 CUDA
+    tensor [R] of the ranks' signal-array addresses (each R uint32 words, zeroed before the
+    first barrier); a time-out sets LMH_DEVERR_TIMEOUT in the workspace's error word."""
+    _fits(signals=(signals, R))
+    st = lib().lmh_peer_barrier(_p(workspace, _u8, "workspace"),
+                                _p(signals, torch.int64, "signals"), int(R), int(rank),
+                                int(epoch), int(timeout_ms), _s(stream))
+    _ok("lmh_peer_barrier", st)
 
 
 def lmh_read_errors(workspace: torch.Tensor, stream=None) -> int:

@@ -72,6 +72,7 @@ _SIGS = {
     "lmh_reduce_ranks_f32": (c_int, [c_int, c_int64, _P, _P, _P]),
     "lmh_read_errors": (c_int, [_P, ctypes.POINTER(c_uint32), _P]),
     "lmh_logprob_noalloc": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 6),
+    "lmh_peer_barrier": (c_int, [_P, _P, ctypes.c_int32, ctypes.c_int32, c_uint32, c_uint32, _P]),
     "lmh_selftest_wait_timeout": (c_int, [_P, c_uint32, _P]),
     "lmh_profile_enable": (c_int, [c_int]),
     "lmh_profile_read": (c_int, [c_int, ctypes.POINTER(ctypes.c_int32),

@@ -166,7 +166,7 @@ enum KernelId {
   KID_SUPPORT_OUT, KID_BWD_COEF, KID_CAST, KID_SUPPORT_DOTS, KID_SUPPORT_LSE,
   KID_SUPPORT_DH, KID_SUPPORT_DW, KID_SPLIT_SUM, KID_VP_LABELS, KID_VP_FINALIZE,
   KID_VP_COMBINE, KID_VP_REDUCE, KID_VP_SCALE, KID_FIX_CANDS, KID_SCALE, KID_COUNT_VALID,
-  KID_REDUCE_RANKS, KID_ZERO_SLOTS, KID_COUNT
+  KID_REDUCE_RANKS, KID_ZERO_SLOTS, KID_PEER_BARRIER, KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "count_labels", "prep_cands", "gemm_logits_stats", "gemm_logits_stats_store",
@@ -174,7 +174,7 @@ const char* const kKernelNames[KID_COUNT] = {
     "mean", "support_out", "bwd_coef", "cast_bf16", "support_dots", "support_lse",
     "support_grad_dh", "support_dw", "split_sum", "vp_local_labels", "vp_finalize",
     "vp_combine", "vp_reduce_rows", "vp_scale", "fix_cands", "scale_bf16", "count_valid",
-    "reduce_ranks", "zero_slots"};
+    "reduce_ranks", "zero_slots", "peer_barrier"};
 
 struct ProfRec {
   int id;

@@ -450,3 +450,26 @@ extern "C" lmh_status lmh_vp_reduce_rows_to(int R, int64_t rows, int64_t d, cons
       reinterpret_cast<__nv_bfloat16* const*>(outs), n_out, row_offset * d / 4);
   return last_launch();
 }
+
+// The barrier that orders the peer-memory exchanges (peer.cuh). The error word is the
+// workspace header's; this entry never clears it, so a time-out stays recorded until the
+// caller reads and clears it.
+extern "C" lmh_status lmh_peer_barrier(void* workspace, uint32_t* const* signals, int32_t R,
+                                       int32_t rank, uint32_t epoch, uint32_t timeout_ms,
+                                       void* stream) {
+  if (!workspace || !signals || R < 1 || R > 1024 || rank < 0 || rank >= R || epoch == 0 ||
+      timeout_ms < 1 || timeout_ms > 60000)
+    return LMH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 ||
+      (reinterpret_cast<uintptr_t>(signals) & 7u) != 0)
+    return LMH_ERR_ALIGNMENT;
+  int dev, sms;
+  LMH_TRY(current_device(&dev, &sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned threads = static_cast<unsigned>((R + 31) / 32 * 32);
+  ProfScope ps(KID_PEER_BARRIER, st);
+  peer_barrier_kernel<<<1, threads, 0, st>>>(signals, R, rank, epoch,
+                                             uint64_t(timeout_ms) * 1000000ull,
+                                             &static_cast<WsHeader*>(workspace)->err);
+  return last_launch();
+}

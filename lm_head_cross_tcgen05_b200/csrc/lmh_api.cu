@@ -16,6 +16,7 @@
 #include "rowops.cuh"
 #include "sparse.cuh"
 #include "vp.cuh"
+#include "peer.cuh"
 
 using namespace lmh;
 

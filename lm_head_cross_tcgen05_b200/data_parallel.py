@@ -23,8 +23,11 @@ With ``p2p=True`` the dW exchange runs over peer memory instead of NCCL: the rec
 and every rank's dW live in symmetric memory (peer-mapped over NVLink), the dW GEMM's epilogue
 stores each fp32 row straight into the receive buffer of the rank that reduces it while the
 GEMM runs (``lmh_dp_loss_fwd_bwd``), and ``lmh_vp_reduce_rows_to`` stores each reduced bf16
-slice into every rank's dW. The additions are the same, so the bits are the same; all rows of
-a rank then form one chunk.
+slice into every rank's dW. The library's bounded peer-memory barrier (``lmh_peer_barrier``)
+orders the steps, and each step first checks on the host that the previous step's barriers
+did not time out. The additions are the same, so the bits are the same. All rows of a rank
+then form one chunk, so the workspace holds the softmax buffer of all of them
+(rows x round_up(V, 8) x 2 bytes); ``chunk_rows`` cannot be combined with ``p2p``.
 
 Against one device on the concatenated batch the values agree to fp32 rounding (the dW sum and
 the mean are grouped by rank). The compute steps run in the library's CUDA kernels through
@@ -139,8 +142,8 @@ class DataParallelCE(RankGroup):
     ``grad[i]`` taken as given, or with ``scalar_grad`` one upstream gradient g for every
     row (divided by the global count with mean=True). ``count`` gives the global count
     before the step, for callers whose per-row weights depend on it. With ``p2p`` (and more
-    than one rank) dW is exchanged over peer memory and each rank's rows form one chunk
-    (``chunk_rows`` is not used)."""
+    than one rank) dW is exchanged over peer memory and each rank's rows form one chunk, so
+    ``chunk_rows`` must stay 0 (a ValueError otherwise)."""
 
     def __init__(self, group=None, chunk_rows: int = 0, mean: bool = True, temperature=None,
                  ops=None, p2p: bool = False):
@@ -149,6 +152,9 @@ class DataParallelCE(RankGroup):
         self.mean = mean
         self.temperature = temperature
         self.p2p = p2p and self.R > 1   # one rank has nothing to exchange
+        if self.p2p and chunk_rows:
+            raise ValueError("p2p runs each rank's rows as one chunk: chunk_rows cannot be set "
+                             "(the workspace holds rows x round_up(V, 8) x 2 bytes of softmax)")
 
     def count(self, labels, V: int):
         """The valid rows (0 <= label < V) of all ranks: a one-element int32 device tensor."""
@@ -161,8 +167,7 @@ class DataParallelCE(RankGroup):
         n = self.count(labels, W.shape[0])
         if self.p2p:
             V, d = W.shape
-            sym = self._symmetric(V, d, H.device)   # receive buffers for V rows, dW outputs
-            sym["recv_h"].barrier(channel=0)        # no rank still reads its last buffer
+            sym = self._open_p2p(V, d, H.device)
             out = self.ops.fused_scatter(H, W, labels, n, (sym["recv_tab"], self.R, self.rank),
                                          mode=mode, grad=grad, mean=self.mean,
                                          scalar_grad=scalar_grad,

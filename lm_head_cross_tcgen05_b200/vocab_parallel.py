@@ -26,7 +26,9 @@ collective, only moved.
 every rank's dH live in symmetric memory (peer-mapped over NVLink); the dH GEMM's epilogue
 writes each fp32 row straight into the receive buffer of the rank that reduces it while the
 GEMM runs, and ``lmh_vp_reduce_rows_to`` stores each reduced bf16 slice into every rank's dH.
-Two stream-ordered barriers of the symmetric memory order the steps. The same fixed order of
+Stream-ordered barriers of the library (``lmh_peer_barrier``: signal words in symmetric memory,
+a bounded wait that records a time-out instead of spinning) order the steps; the next step
+reads that record on the host first and raises if a barrier gave up. The same fixed order of
 additions gives the same bits as the NCCL path. The compute steps run in the library's CUDA kernels through
 ``CudaOps``; ``VocabParallelCE`` takes any object with the same four methods, which is how its
 exchange logic is tested on CPU ranks.
@@ -201,8 +203,7 @@ class _VocabParallel(RankGroup):
         """dH summed over the ranks from run(dest) -> (dH_part or None, dW): collectives, or
         with p2p the rows scattered straight to their reducing ranks."""
         if self.p2p:
-            sym = self._symmetric(N, d, device)   # receive buffers for N rows, dH outputs
-            sym["recv_h"].barrier(channel=0)   # no rank still reads its last receive buffer
+            sym = self._open_p2p(N, d, device)
             _, dW = run((sym["recv_tab"], self.R, self.rank))
             return self._reduce_p2p(sym), dW
         dH_part, dW = run(None)

@@ -184,3 +184,19 @@ def test_dw_store_flag_is_sizing_neutral():
         base = L.F_FUSED_BWD | L.F_DW_ACC_GIVEN
         assert ws(3000, 64, 5000, chunk=1000, flags=base, entry=entry) == \
             ws(3000, 64, 5000, chunk=1000, flags=base | L.F_DW_ACC_STORE, entry=entry)
+
+
+def test_peer_barrier_host_errors_without_gpu():
+    lib = _abi.lib()
+    ws, tab = ctypes.c_void_p(256), ctypes.c_void_p(512)
+    assert lib.lmh_peer_barrier(None, tab, 2, 0, 1, 100, None) == 1
+    assert lib.lmh_peer_barrier(ws, None, 2, 0, 1, 100, None) == 1
+    assert lib.lmh_peer_barrier(ws, tab, 0, 0, 1, 100, None) == 1      # no rank
+    assert lib.lmh_peer_barrier(ws, tab, 1025, 0, 1, 100, None) == 1   # more than one block
+    assert lib.lmh_peer_barrier(ws, tab, 2, 2, 1, 100, None) == 1      # rank outside 0..R-1
+    assert lib.lmh_peer_barrier(ws, tab, 2, -1, 1, 100, None) == 1
+    assert lib.lmh_peer_barrier(ws, tab, 2, 0, 0, 100, None) == 1      # epoch 0
+    assert lib.lmh_peer_barrier(ws, tab, 2, 0, 1, 0, None) == 1        # unbounded wait
+    assert lib.lmh_peer_barrier(ws, tab, 2, 0, 1, 60001, None) == 1
+    assert lib.lmh_peer_barrier(ctypes.c_void_p(264), tab, 2, 0, 1, 100, None) == 4
+    assert lib.lmh_peer_barrier(ws, ctypes.c_void_p(516), 2, 0, 1, 100, None) == 4
