@@ -133,16 +133,54 @@ def job_tflops(flops_per_rank_step: float, world: int, ms_per_step: float) -> fl
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU during the timed region: NVML read
+    every 10 ms on a thread (nvidia-smi's 100 ms floor gives too few samples for a region of
+    about a second), else nvidia-smi -lms 100. Reads only; no setting is changed."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
              "clocks_event_reasons.sw_power_cap")
     NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    # NVML clock-event reason bits of the four names above
+    NVML_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                 "sw_power_cap": 0x4}
 
-    def __init__(self, gpu_id: str):
+    def __init__(self, gpu_id: str, period_s: float = 0.01):
         self.gpu_id = gpu_id
+        self.period_s = period_s
         self.proc = None
+        self.thread = None
+        self.samples = []
+
+    def _nvml_handle(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            if self.gpu_id.startswith("GPU-"):
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu_id))
+        except Exception:
+            return None, None
 
     def start(self):
+        import threading
+        nv, h = self._nvml_handle()
+        if h is not None:
+            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or getattr(
+                nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.stop_flag = threading.Event()
+
+            def loop():
+                while not self.stop_flag.is_set():
+                    try:
+                        self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                             nv.nvmlDeviceGetPowerUsage(h) / 1e3, int(reasons(h))))
+                    except Exception:
+                        pass
+                    self.stop_flag.wait(self.period_s)
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.QUERY}",
@@ -152,6 +190,20 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            if not self.samples:
+                return None
+            sm = [c for c, _, _ in self.samples]
+            bits = 0
+            for _, _, b in self.samples:
+                bits |= b
+            reasons = sorted(n for n, b in self.NVML_BITS.items() if bits & b)
+            return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz,
+                    "reasons": reasons, "samples": len(sm), "source": "nvml, every 10 ms",
+                    "sm_mhz_p10_p90": [sorted(sm)[len(sm) // 10], sorted(sm)[(9 * len(sm)) // 10]],
+                    "power_w_median": statistics.median(p for _, p, _ in self.samples)}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -176,7 +228,25 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi, every 100 ms"}
+
+
+# bf16 dense tensor throughput of one SM per clock (4096 multiply-adds)
+BF16_FLOP_PER_SM_CLK = 8192
+
+
+def tensor_peak_at(sm_mhz: float, sms: int) -> float:
+    """TFLOP/s the tensor pipes can do at this SM clock: SMs x 8192 flop/clk x clock."""
+    return sms * BF16_FLOP_PER_SM_CLK * sm_mhz * 1e6 / 1e12
+
+
+def pick_peak(peaks: dict, timed_s: float) -> tuple:
+    """The bf16 peak a kernel timed in this region is held to: the burst figure for a region
+    of a few seconds at most (the power cap has not pulled the clock down to its sustained
+    level), the sustained one for longer regions."""
+    if timed_s <= 3.0:
+        return peaks["bf16_tflops"], "burst"
+    return peaks["bf16_tflops_sustained"], "sustained"
 
 
 def gpu_id_for_smi(torch, dev) -> str:
@@ -288,6 +358,7 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     if world > 1:
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
 
@@ -392,7 +463,8 @@ def main():
 
     sampler = ClockSampler(gpu_id_for_smi(torch, local))
     sampler.start()
-    time.sleep(0.3)
+    if sampler.thread is None:
+        time.sleep(0.3)          # nvidia-smi needs a moment before its first sample
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     lib().lmh_profile_enable(1)
     barrier()
@@ -432,11 +504,19 @@ def main():
         hbm_bytes = {"gbuild": 4.0 * chunk * ((V + 7) // 8 * 8)}
         if dom.startswith("gemm"):
             ach = gemm_flops / (kernels[dom]["avg_ms"] / 1e3) / 1e12
-            pk = peaks["bf16_tflops_sustained"]
+            pk, kind = pick_peak(peaks, ms_total / 1e3)
             roofline = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": pk,
                         "unit": "TFLOP/s", "frac": ach / pk,
-                        "peak_kind": f"bf16 dense, sustained, of {peak_src}",
+                        "peak_kind": f"bf16 dense, {kind} (timed region {ms_total / 1e3:.2f} s), "
+                                     f"of {peak_src}",
+                        "frac_of_sustained": ach / peaks["bf16_tflops_sustained"],
                         "algorithmic_per_launch": gemm_flops}
+            if clocks:
+                at = tensor_peak_at(clocks["sm_mhz"], sms)
+                roofline["at_sampled_clock"] = {
+                    "sm_mhz": clocks["sm_mhz"], "sms": sms, "tensor_peak": at,
+                    "frac": ach / at,
+                    "how": "achieved / (SMs x 8192 bf16 flop/clk x median sampled SM clock)"}
         else:
             b = hbm_bytes.get(dom, 0.0)
             ach = b / (kernels[dom]["avg_ms"] / 1e3) / 1e9
@@ -526,6 +606,8 @@ def main():
                 "config": workload_config(wl, chunk, world, args.entry),
                 "peak_frac": {"of_burst": value / world / peaks["bf16_tflops"],
                               "of_sustained": value / world / peaks["bf16_tflops_sustained"],
+                              "of_sampled_clock": (value / world / tensor_peak_at(
+                                  clocks["sm_mhz"], sms) if clocks else None),
                               "peaks": peak_src},
                 "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
                 "gpu_launches": n_rec, "kernels": kernels, "clocks": clocks}

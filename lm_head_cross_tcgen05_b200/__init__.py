@@ -231,9 +231,11 @@ def lmh_support_fwd_bwd(shape, mode, H, W, ids, ref_logp, grad, kl_rows=None, kl
 
 def support_fwd_bwd(mode: int, H, W, ids, grad=None, ref_logp=None, *, chunk_rows: int = 0,
                     mean: bool = False, scalar_grad: bool = False, dW_acc=None,
-                    temperature=None, ws=None, stream=None) -> dict:
+                    temperature=None, want_dH: bool = True, want_dW: bool = True, ws=None,
+                    stream=None) -> dict:
     """The support forward (lp, lse; kl_rows, kl_mean for BWD_SUPPORT_KL) plus dH, dW of
-    sum_i g_i KL_i or sum_ik g_ik lp_ik in one pass, the weights known before the call."""
+    sum_i g_i KL_i or sum_ik g_ik lp_ik in one pass, the weights known before the call.
+    want_dH / want_dW False leaves that gradient out (its GEMM is skipped)."""
     N, d = H.shape
     V, K = W.shape[0], ids.shape[1]
     dev = H.device
@@ -243,8 +245,8 @@ def support_fwd_bwd(mode: int, H, W, ids, grad=None, ref_logp=None, *, chunk_row
     kl = int(mode) == BWD_SUPPORT_KL
     out = dict(lp=torch.empty(N, K, dtype=_f32, device=dev),
                lse=torch.empty(N, dtype=_f32, device=dev),
-               dH=torch.empty(N, d, dtype=_bf, device=dev),
-               dW=torch.empty(V, d, dtype=_bf, device=dev))
+               dH=torch.empty(N, d, dtype=_bf, device=dev) if want_dH else None,
+               dW=torch.empty(V, d, dtype=_bf, device=dev) if want_dW else None)
     if kl:
         out["kl_rows"] = torch.empty(N, dtype=_f32, device=dev)
         out["kl_mean"] = torch.empty(1, dtype=_f32, device=dev)
@@ -495,10 +497,12 @@ def loss_fwd(H, W, labels, *, chunk_rows: int = 0, mean: bool = True, grads: boo
 
 def loss_fwd_bwd(mode: int, H, W, labels, grad=None, *, chunk_rows: int = 0,
                  mean: bool = False, scalar_grad: bool = False, dW_acc=None,
-                 n_valid_given=None, temperature=None, ws=None, stream=None) -> dict:
+                 n_valid_given=None, temperature=None, want_dH: bool = True,
+                 want_dW: bool = True, ws=None, stream=None) -> dict:
     """Forward outputs plus dH, dW of L = sum_i w_i l_i (l = loss for BWD_CE, log-prob for
     BWD_LOGPROB; w from grad as in loss_bwd) in one pass: the fused path for objectives whose
-    row weights are known before the forward, such as policy-gradient losses."""
+    row weights are known before the forward, such as policy-gradient losses. want_dH /
+    want_dW False: that gradient is not computed (its GEMM is skipped; a frozen input)."""
     N, d = H.shape
     V = W.shape[0]
     dev = H.device
@@ -511,8 +515,8 @@ def loss_fwd_bwd(mode: int, H, W, labels, grad=None, *, chunk_rows: int = 0,
                argmax=torch.empty(N, dtype=_i32, device=dev),
                loss_mean=torch.empty(1, dtype=_f32, device=dev),
                n_valid=torch.empty(1, dtype=_i32, device=dev),
-               dH=torch.empty(N, d, dtype=_bf, device=dev),
-               dW=torch.empty(V, d, dtype=_bf, device=dev))
+               dH=torch.empty(N, d, dtype=_bf, device=dev) if want_dH else None,
+               dW=torch.empty(V, d, dtype=_bf, device=dev) if want_dW else None)
     ws = workspace(shape, ENTRY_LOSS_FWD_BWD, dev) if ws is None else ws
     lmh_loss_fwd_bwd(shape, mode, H, W, labels, grad, out["loss_rows"], out["lse"],
                      out["logprob"], out["argmax"], out["loss_mean"], out["n_valid"],
@@ -573,9 +577,10 @@ def support_logprob(H, W, ids, *, chunk_rows: int = 0, temperature=None, renorm:
 
 def support_kl(H, W, ids, ref_logp, *, chunk_rows: int = 0, temperature=None,
                renorm: bool = False, grads: bool = False, mean: bool = True, dW_acc=None,
-               ws=None, stream=None) -> dict:
+               want_dH: bool = True, want_dW: bool = True, ws=None, stream=None) -> dict:
     """KL(ref || model) over the candidates (kl_rows, kl_mean, lp, lse). grads=True: also dH
-    and dW of the mean (or summed) KL in the same pass (lmh_support_kl_fwd_bwd)."""
+    and dW of the mean (or summed) KL in the same pass (lmh_support_kl_fwd_bwd); want_dH /
+    want_dW False leaves that gradient out."""
     N, d = H.shape
     V, K = W.shape[0], ids.shape[1]
     flags = (F_SUPPORT_RENORM if renorm else 0) | (F_FUSED_BWD | (F_MEAN if mean else 0)
@@ -589,8 +594,8 @@ def support_kl(H, W, ids, ref_logp, *, chunk_rows: int = 0, temperature=None,
                lse=torch.empty(N, dtype=_f32, device=dev))
     ws = workspace(shape, ENTRY_SUPPORT_KL, dev) if ws is None else ws
     if grads:
-        out["dH"] = torch.empty(N, d, dtype=_bf, device=dev)
-        out["dW"] = torch.empty(V, d, dtype=_bf, device=dev)
+        out["dH"] = torch.empty(N, d, dtype=_bf, device=dev) if want_dH else None
+        out["dW"] = torch.empty(V, d, dtype=_bf, device=dev) if want_dW else None
         lmh_support_kl_fwd_bwd(shape, H, W, ids, ref_logp, out["kl_rows"], out["kl_mean"],
                                out["lp"], out["lse"], out["dH"], out["dW"], dW_acc,
                                workspace=ws, stream=stream)

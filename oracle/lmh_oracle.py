@@ -142,8 +142,8 @@ def grad_logits(mode: int, z: np.ndarray, lse: np.ndarray, targets, grad, ref_lo
     """
     N, V = z.shape
     P = softmax_from(z, lse)
-    G = np.zeros_like(z)
     if mode in (BWD_CE, BWD_LOGPROB):
+        G = np.zeros_like(z)
         y = as_i64(targets)
         g = as_f64(grad).reshape(N)
         sign = 1.0 if mode == BWD_CE else -1.0
@@ -152,28 +152,24 @@ def grad_logits(mode: int, z: np.ndarray, lse: np.ndarray, targets, grad, ref_lo
                 G[i] = sign * g[i] * P[i]
                 G[i, y[i]] -= sign * g[i]
         return G
+    # Support objectives: each valid slot (i, k) adds w_ik (e_{c_ik} - P_i) to row i, with
+    # w = g for the log-probs and w = -g_i exp(r_ik) for the KL. The P_i parts of a row are
+    # one multiple of P_i (the sum of its slots' w), the one-hot parts a scatter-add of the
+    # slots' w at their ids (repeated ids add once per slot).
     ids = as_i64(targets)
     K = ids.shape[1]
+    ok = (ids >= 0) & (ids < V)
     if mode == BWD_SUPPORT_LOGPROB:
-        gam = as_f64(grad).reshape(N, K)
-        for i in range(N):
-            for k in range(K):
-                c = ids[i, k]
-                if 0 <= c < V:
-                    G[i] -= gam[i, k] * P[i]
-                    G[i, c] += gam[i, k]
-        return G
-    if mode == BWD_SUPPORT_KL:
-        g = as_f64(grad).reshape(N)
-        p = np.exp(as_f64(ref_logp).reshape(N, K))
-        for i in range(N):
-            for k in range(K):
-                c = ids[i, k]
-                if 0 <= c < V:
-                    G[i] += g[i] * p[i, k] * P[i]
-                    G[i, c] -= g[i] * p[i, k]
-        return G
-    raise ValueError(f"unknown backward mode {mode}")
+        w = as_f64(grad).reshape(N, K)
+    elif mode == BWD_SUPPORT_KL:
+        w = -as_f64(grad).reshape(N)[:, None] * np.exp(as_f64(ref_logp).reshape(N, K))
+    else:
+        raise ValueError(f"unknown backward mode {mode}")
+    w = np.where(ok, w, 0.0)
+    G = -w.sum(axis=1)[:, None] * P
+    rr, kk = np.nonzero(ok)
+    np.add.at(G, (rr, ids[rr, kk]), w[rr, kk])
+    return G
 
 
 def lm_head_backward(H, W, G: np.ndarray):
