@@ -56,6 +56,10 @@ def parse_args():
                          "over the GPUs in rank order (weak scaling)")
     ap.add_argument("--chunk-rows", type=int, default=0,
                     help="rows per chunk (the memory budget); 0: the workload's own plan")
+    ap.add_argument("--vocab", type=int, default=0,
+                    help="override the workload's V (a smaller case for profiler captures; the "
+                         "line's config then names the changed shape)")
+    ap.add_argument("--rows", type=int, default=0, help="override the workload's N (as --vocab)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
@@ -342,6 +346,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     from workloads import WORKLOADS, make_inputs
     wl = WORKLOADS[args.workload]
+    if args.vocab or args.rows:
+        wl = wl.scaled(V=args.vocab or wl.V, N=args.rows or wl.N,
+                       name=f"{wl.name}[N={args.rows or wl.N},V={args.vocab or wl.V}]")
 
     if args.impl == "reference":
         if rank == 0:

@@ -53,7 +53,47 @@ def check_grad(got, ref, what: str = "grad"):
     g, r = f64(got), f64(ref)
     assert g.shape == r.shape, (what, g.shape, r.shape)
     assert np.all(np.isfinite(g)), f"{what}: non-finite values"
-    m = grad_metrics(g, r)
+    return assert_grad_metrics(grad_metrics(g, r), what)
+
+
+class GradStats:
+    """check_grad over an array compared one block at a time, for arrays too large to hold
+    twice in fp64 (a full-size dW): the same maximum errors, norms and inner product,
+    accumulated over the blocks, then the same gates."""
+
+    def __init__(self, what: str):
+        self.what = what
+        self.maxerr = self.maxref = 0.0
+        self.dot = self.gg = self.rr = self.dd = 0.0
+
+    def add(self, got, ref):
+        g, r = f64(got), f64(ref)
+        assert g.shape == r.shape, (self.what, g.shape, r.shape)
+        assert np.all(np.isfinite(g)), f"{self.what}: non-finite values"
+        if not r.size:
+            return
+        d = g - r
+        self.maxerr = max(self.maxerr, float(np.max(np.abs(d))))
+        self.maxref = max(self.maxref, float(np.max(np.abs(r))))
+        gv, rv, dv = g.ravel(), r.ravel(), d.ravel()
+        self.dot += float(np.dot(gv, rv))
+        self.gg += float(np.dot(gv, gv))
+        self.rr += float(np.dot(rv, rv))
+        self.dd += float(np.dot(dv, dv))
+
+    def check(self):
+        nr, ng = self.rr ** 0.5, self.gg ** 0.5
+        if nr == 0.0 and ng == 0.0:
+            cos, rel = 1.0, 0.0
+        elif nr == 0.0 or ng == 0.0:
+            cos, rel = 0.0, float("inf")
+        else:
+            cos, rel = self.dot / (ng * nr), self.dd ** 0.5 / nr
+        return assert_grad_metrics(dict(maxerr=self.maxerr, maxref=self.maxref, cos=cos,
+                                        rel_rms=rel), self.what)
+
+
+def assert_grad_metrics(m: dict, what: str):
     if m["maxref"] == 0.0:
         assert m["maxerr"] == 0.0, f"{what}: reference is zero, got max {m['maxerr']:.3e}"
         return m

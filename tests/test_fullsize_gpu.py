@@ -1,16 +1,15 @@
 """Parity at the full sizes of the four large workloads, in the launch configuration bench.py
-uses (one chunk of all rows for large_vocab, 2048-row chunks for budgeted).
+uses (one chunk of all rows for large_vocab and support, 2048-row chunks into a caller-owned
+fp32 accumulator for budgeted).
 
-Per-row outputs (loss, lse, logprob, argmax, dH rows, support lp / KL rows) are compared with
-the fp64 oracle on sampled rows, which it computes one by one. dW depends on every row's
-log-sum-exp, so at full N it is checked through properties that hold at any size (columns
-sum to zero, fused forward+backward == recompute backward, one chunk == many chunks within
-tolerance, bitwise repeats), and element by element against the oracle at full V and d on a
-128-row slice. ``LMH_FULL_ORACLE=1`` adds the complete fp64 dW of the large-vocab workload
-(row-blocked; minutes of CPU time)."""
+Every output of those steps is compared with the fp64 oracle element by element: per-row
+outputs for all rows, dH for all rows and dW in full. The oracle runs over 1024-row blocks
+(its logits, softmax gradient and both contractions per block, dW summed over the blocks in
+fp64), and the gradient gates are accumulated block by block (``GradStats``), so a full-size
+dW never needs two fp64 copies. That is about 3.3e13, 9.8e13 and 4.1e13 fp64 flops for the
+three workloads: minutes of host CPU. Properties that hold at any size (columns of dW summing
+to zero, bitwise repeats, one chunk against many) are checked as well."""
 from __future__ import annotations
-
-import os
 
 import numpy as np
 import pytest
@@ -18,6 +17,7 @@ import torch
 
 import lm_head_cross_tcgen05_b200 as L
 from tests.gpu_common import O, check_argmax, check_grad, check_rows, digest, f64
+from tests.parity import GradStats
 from workloads import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -120,20 +120,70 @@ def test_full_vocab_and_hidden_dw_slice():
     check_rows(out["lse"], ref["lse"], what="lse")
 
 
-@pytest.mark.skipif(os.environ.get("LMH_FULL_ORACLE") != "1", reason="minutes of fp64 CPU work")
-def test_large_vocab_full_fp64_dw(large_vocab):
+BLOCK = 1024
+
+
+def full_oracle(x, out, kind, n_valid=None, acc=None):
+    """Every row's outputs, all of dH and all of dW (and acc, a caller's fp32 accumulator)
+    against the fp64 oracle, over blocks of BLOCK rows. kind "ce": the mean cross entropy
+    over n_valid rows (loss_rows, lse, logprob, argmax, loss_mean); "support_kl": the mean KL
+    over all rows (kl_rows, kl_mean, lp, lse)."""
+    Hc = x["H"].cpu()
+    W64 = O.as_f64(x["W"].cpu())
+    N, d = Hc.shape
+    V = W64.shape[0]
+    got = {k: v.cpu() for k, v in out.items()
+           if isinstance(v, torch.Tensor) and k not in ("workspace", "dW")}
+    dW = np.zeros((V, d))
+    sH = GradStats("dH (all rows)")
+    total = 0.0
+    for r0 in range(0, N, BLOCK):
+        r1 = min(N, r0 + BLOCK)
+        Hb = O.as_f64(Hc[r0:r1])
+        if kind == "ce":
+            y = x["labels"][r0:r1].cpu()
+            f = O.ce_forward(Hb, W64, y)
+            for k in ("loss_rows", "lse", "logprob"):
+                check_rows(got[k][r0:r1], f[k], what=f"{k} rows {r0}..{r1}")
+            check_argmax(got["argmax"][r0:r1], f["z"])
+            total += float(f["loss_rows"].sum())
+            g = np.where(O.valid_rows(y, V)[0], 1.0 / n_valid, 0.0)
+            G = O.grad_logits(O.BWD_CE, f["z"], f["lse"], y, g)
+        else:
+            ids, ref = x["ids"][r0:r1].cpu(), x["ref_logp"][r0:r1].cpu()
+            f = O.support_kl(Hb, W64, ids, ref)
+            for k in ("kl_rows", "lp", "lse"):
+                check_rows(got[k][r0:r1], f[k], what=f"{k} rows {r0}..{r1}")
+            total += float(f["kl_rows"].sum())
+            G = O.grad_logits(O.BWD_SUPPORT_KL, f["z"], f["lse"], ids, np.full(r1 - r0, 1.0 / N),
+                              ref)
+        del f
+        dHb, dWb = O.lm_head_backward(Hb, W64, G)
+        del G
+        sH.add(got["dH"][r0:r1], dHb)
+        dW += dWb
+        del dWb
+    sH.check()
+    mean = "loss_mean" if kind == "ce" else "kl_mean"
+    check_rows(got[mean], np.array([total / (n_valid if kind == "ce" else N)]), what=mean)
+    sW, sA = GradStats("dW (full)"), GradStats("fp32 dW accumulator (full)")
+    dW_got = out["dW"].cpu()
+    acc_got = acc.cpu() if acc is not None else None
+    for v0 in range(0, V, 8192):
+        sW.add(dW_got[v0:v0 + 8192], dW[v0:v0 + 8192])
+        if acc_got is not None:
+            sA.add(acc_got[v0:v0 + 8192], dW[v0:v0 + 8192])
+    sW.check()
+    if acc_got is not None:
+        sA.check()
+
+
+def test_large_vocab_full_oracle(large_vocab):
+    """The headline step (8192 x 128256 x 4096, one chunk): every output against the oracle."""
     wl, x, out = large_vocab
-    Hc, Wc, yc = x["H"].cpu(), x["W"].cpu(), x["labels"].cpu()
-    n = int(((yc >= 0) & (yc < wl.V)).sum())
-    dW = np.zeros((wl.V, wl.d))
-    for r0 in range(0, wl.N, 512):
-        r1 = min(wl.N, r0 + 512)
-        z = O.logits(Hc[r0:r1], Wc)
-        lse = O.logsumexp_rows(z)
-        g = np.where(yc[r0:r1].numpy() >= 0, 1.0 / n, 0.0)
-        G = O.grad_logits(O.BWD_CE, z, lse, yc[r0:r1], g)
-        dW += G.T @ O.as_f64(Hc[r0:r1])
-    check_grad(out["dW"], dW, "dW full")
+    n = int(O.valid_rows(x["labels"].cpu(), wl.V)[0].sum())
+    assert int(out["n_valid"].item()) == n
+    full_oracle(x, out, "ce", n_valid=n)
 
 
 def test_small_workload_full_oracle():
@@ -151,6 +201,9 @@ def test_small_workload_full_oracle():
 
 
 def test_budgeted_workload_chunked_with_caller_accumulator():
+    """16384 x 151936 x 5120 in 8 chunks of 2048 rows, dW accumulated in chunk order into a
+    caller-owned fp32 buffer: every output, the accumulator and the log-prob entry against
+    the oracle."""
     wl, x = dev_inputs("budgeted")
     shape = L.make_shape(wl.N, wl.d, wl.V, 0, wl.chunk_rows,
                          L.F_MEAN | L.F_FUSED_BWD | L.F_DW_ACC_GIVEN)
@@ -158,12 +211,16 @@ def test_budgeted_workload_chunked_with_caller_accumulator():
     acc = torch.zeros(wl.V, wl.d, dtype=torch.float32, device="cuda")
     out = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=wl.chunk_rows, grads=True,
                      dW_acc=acc)
+    torch.cuda.synchronize()
+    assert L.lmh_read_errors(out["workspace"]) == 0
     assert torch.equal(out["dW"], acc.to(torch.bfloat16))
     check_dw_properties(out["dW"])
     y = x["labels"]
-    check_sampled_ce(out, x, sample_rows(y, seed=3), wl.N)
     lp = L.logprob(x["H"], x["W"], y, chunk_rows=wl.chunk_rows)
     assert torch.equal(lp["logprob"], out["logprob"]) and torch.equal(lp["lse"], out["lse"])
+    n = int(O.valid_rows(y.cpu(), wl.V)[0].sum())
+    assert int(out["n_valid"].item()) == n == wl.N
+    full_oracle(x, out, "ce", n_valid=n, acc=acc)
 
 
 def test_support_workload_sampled_rows():
@@ -264,3 +321,15 @@ def test_many_chunks_and_large_row_indices():
     check_grad(out["dW"], ref["dW"], "dW")
     again = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
     assert torch.equal(again["dW"], out["dW"]) and torch.equal(again["dH"], out["dH"])
+
+
+def test_support_workload_one_pass_full_oracle():
+    """The support step bench.py times (8192 x 151936 x 4096, K = 64, the mean KL's forward
+    and backward in one pass): every output against the oracle."""
+    wl, x = dev_inputs("support")
+    out = L.support_kl(x["H"], x["W"], x["ids"], x["ref_logp"], chunk_rows=wl.N, grads=True)
+    torch.cuda.synchronize()
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    lp = L.support_logprob(x["H"], x["W"], x["ids"], chunk_rows=wl.N)
+    assert torch.equal(lp["lp"], out["lp"]) and torch.equal(lp["lse"], out["lse"])
+    full_oracle(x, out, "support_kl")
