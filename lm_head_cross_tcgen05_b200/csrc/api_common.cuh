@@ -273,6 +273,7 @@ bool tmap_acc(CUtensorMap* m, const float* base, uint64_t inner, uint64_t outer,
 struct GemmOrder {
   int group_m;  // pair-row tiles per group (rows fastest inside a group)
   int hint_a, hint_b;
+  int group_n = 0;  // > 0: column tiles per group instead (columns fastest inside a group)
 };
 
 template <class Epi>
@@ -307,6 +308,7 @@ lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap
   g.k_blocks = static_cast<int>(cdiv(K, BK));
   g.k_splits = k_splits;
   g.group_m = order.group_m < 1 ? g.m_tiles : (order.group_m < g.m_tiles ? order.group_m : g.m_tiles);
+  g.group_n = order.group_n < 1 ? 0 : (order.group_n < g.n_tiles ? order.group_n : g.n_tiles);
   g.hint_a = order.hint_a;
   g.hint_b = order.hint_b;
   g.err = err;

@@ -7,7 +7,8 @@
 // CTAs. Per SM this halves the B operand traffic of a 128 x 256 single-CTA tile.
 //
 // Persistent schedule: grid = 2 x (number of co-resident pairs); pair p walks the work units
-// p, p + pairs, ... of a fixed, grouped order (group_m row tiles at a time, rows fastest). A
+// p, p + pairs, ... of a fixed, grouped order (group_m row tiles at a time, rows fastest; or
+// group_n column tiles at a time, columns fastest). A
 // work unit is an output tile, or a tile and one of k_splits consecutive K ranges when a
 // launch has too few tiles to fill the GPU (its epilogue then writes an fp32 partial).
 // Every output tile is owned by one pair and its K loop runs in ascending order, so the fp32
@@ -79,6 +80,7 @@ struct GemmGrid {
   int k_blocks;  // ceil(K / BK)
   int k_splits;  // K split into this many consecutive ranges (work units = tiles x splits)
   int group_m;   // tile order: group_m row tiles at a time, rows fastest within a group
+  int group_n;   // > 0: group_n column tiles at a time instead, columns fastest within a group
   int hint_a;    // L2 eviction priority of A's loads (L2Hint)
   int hint_b;    // L2 eviction priority of B's loads
   uint32_t* err; // device error word
@@ -90,13 +92,23 @@ __device__ __forceinline__ void unit_coords(const GemmGrid& g, int u, int& mb, i
   const int tiles = g.m_tiles * g.n_tiles;
   split = u / tiles;
   int t = u - split * tiles;
-  const int per_group = g.group_m * g.n_tiles;
-  const int grp = t / per_group;
-  const int rem = t - grp * per_group;
-  const int m0 = grp * g.group_m;
-  const int gm = min(g.group_m, g.m_tiles - m0);
-  mb = m0 + rem % gm;
-  nb = rem / gm;
+  if (g.group_n > 0) {
+    const int per_group = g.group_n * g.m_tiles;
+    const int grp = t / per_group;
+    const int rem = t - grp * per_group;
+    const int n0 = grp * g.group_n;
+    const int gn = min(g.group_n, g.n_tiles - n0);
+    nb = n0 + rem % gn;
+    mb = rem / gn;
+  } else {
+    const int per_group = g.group_m * g.n_tiles;
+    const int grp = t / per_group;
+    const int rem = t - grp * per_group;
+    const int m0 = grp * g.group_m;
+    const int gm = min(g.group_m, g.m_tiles - m0);
+    mb = m0 + rem % gm;
+    nb = rem / gm;
+  }
   kb0 = static_cast<int>(static_cast<long long>(g.k_blocks) * split / g.k_splits);
   kb1 = static_cast<int>(static_cast<long long>(g.k_blocks) * (split + 1) / g.k_splits);
 }
