@@ -273,7 +273,6 @@ bool tmap_acc(CUtensorMap* m, const float* base, uint64_t inner, uint64_t outer,
 struct GemmOrder {
   int group_m;  // pair-row tiles per group (rows fastest inside a group)
   int hint_a, hint_b;
-  int group_n = 0;  // > 0: column tiles per group instead (columns fastest inside a group)
 };
 
 template <class Epi>
@@ -286,13 +285,13 @@ lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap
   const uint64_t bit = 1ull << dev;
   if (!(attr_done.load() & bit)) {
     if (cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GEMM_SMEM_BYTES) != cudaSuccess)
+                             Pipe<Epi>::SMEM_BYTES) != cudaSuccess)
       return LMH_ERR_CUDA;
     // how many CTA pairs can be resident at once (one CTA per SM)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(sms / 2 * 2));
     cfg.blockDim = dim3(GEMM_THREADS);
-    cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+    cfg.dynamicSmemBytes = Pipe<Epi>::SMEM_BYTES;
     int nclusters = 0;
     if (cudaOccupancyMaxActiveClusters(&nclusters, gemm_tc_kernel<Epi>, &cfg) != cudaSuccess ||
         nclusters < 1) {
@@ -305,10 +304,9 @@ lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap
   GemmGrid g;
   g.m_tiles = static_cast<int>(cdiv(M, PM));
   g.n_tiles = static_cast<int>(cdiv(Ncols, BN));
-  g.k_blocks = static_cast<int>(cdiv(K, BK));
+  g.k_blocks = static_cast<int>(cdiv(K, Pipe<Epi>::BK));
   g.k_splits = k_splits;
   g.group_m = order.group_m < 1 ? g.m_tiles : (order.group_m < g.m_tiles ? order.group_m : g.m_tiles);
-  g.group_n = order.group_n < 1 ? 0 : (order.group_n < g.n_tiles ? order.group_n : g.n_tiles);
   g.hint_a = order.hint_a;
   g.hint_b = order.hint_b;
   g.err = err;
@@ -317,8 +315,8 @@ lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap
   const int64_t pairs_max = pairs_cache[dev].load();
   const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
   ProfScope ps(Epi::kId, st);
-  gemm_tc_kernel<Epi><<<2 * pairs, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(a, b, c, d ? *d : c,
-                                                                        g, ep);
+  gemm_tc_kernel<Epi><<<2 * pairs, GEMM_THREADS, Pipe<Epi>::SMEM_BYTES, st>>>(
+      a, b, c, d ? *d : c, g, ep);
   return cudaGetLastError() == cudaSuccess ? LMH_OK : LMH_ERR_CUDA;
 }
 
@@ -329,6 +327,11 @@ constexpr GemmOrder kOrderLogits{16, kL2Normal, kL2Normal};
 // dH: two 256-row tiles at a time across all hidden tiles (13.8 GB of DRAM reads per launch
 // at the headline size, against 19.7 GB for groups of eight and 22.7 GB for rows fastest)
 constexpr GemmOrder kOrderDH{2, kL2Normal, kL2Normal};
+// dH split over vocabulary ranges (a chunk with few row tiles): every row tile of the chunk
+// in one group, so a wave spans all rows and a few hidden tiles of one range and each slice
+// of W is read by one wave (2048 x 5120 x 151936 in 4 ranges: 5.2-5.5 GB of DRAM reads per
+// launch instead of 7.2-7.5 GB for groups of two)
+constexpr GemmOrder kOrderDHSplit{0, kL2Normal, kL2Normal};
 // dW: one 256-word vocabulary tile across all hidden tiles (each G tile is read once while
 // its 16 hidden tiles run side by side; keeping H at evict-last priority measured worse)
 constexpr GemmOrder kOrderDW{1, kL2Normal, kL2Normal};
@@ -430,6 +433,37 @@ lmh_status cast_dw(const Plan& P, const float* acc, lmh_bf16* dW, cudaStream_t s
   return last_launch();
 }
 
+// One chunk's dW GEMM in accumulate mode acc_mode (EpiDW); its tensor maps use the
+// instantiation's K per stage.
+template <class Epi>
+lmh_status run_dw(const Plan& P, int dev, int sms, const __nv_bfloat16* G, const lmh_bf16* H,
+                  int64_t r0, int rows, int acc_mode, float* acc, lmh_bf16* dW,
+                  const RowScatter* dw_scatter, const Ws& ws, cudaStream_t st) {
+  CUtensorMap ta, tb, tc, td;  // td: mode 3 reads the accumulator through it
+  if (!tmap_2d(&ta, G, P.V, rows, P.Vp, Pipe<Epi>::BK) ||
+      !tmap_2d(&tb, H + r0 * P.d, P.d, rows, P.d, Pipe<Epi>::BK))
+    return LMH_ERR_CUDA;
+  typename Epi::Params ep;
+  ep.V = static_cast<int>(P.V);
+  ep.d = static_cast<int>(P.d);
+  ep.acc_mode = acc_mode;
+  if (acc_mode == 4) ep.sc = *dw_scatter;
+  bool ok;
+  if (acc_mode == 4) {
+    tc = ta;
+    ok = true;
+  } else if (acc_mode == 0) {
+    ok = tmap_out(&tc, dW, P.d, P.V, P.d);
+  } else if (acc_mode == 3) {
+    ok = tmap_out(&tc, dW, P.d, P.V, P.d) && tmap_acc(&td, acc, P.d, P.V, P.d);
+  } else {
+    ok = tmap_acc(&tc, acc, P.d, P.V, P.d);
+  }
+  if (!ok) return LMH_ERR_CUDA;
+  return launch_gemm<Epi>(dev, sms, ta, tb, tc, P.V, P.d, rows, kOrderDW, &ws.h->err, ep, st, 1,
+                          acc_mode == 3 ? &td : nullptr);
+}
+
 // dH = G W and dW (+)= G^T H_c for one chunk whose G sits in the workspace buffer.
 // With dH_f32 (vocabulary-parallel shards) dH's rows go to it in fp32 instead, unsplit.
 lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H,
@@ -441,7 +475,7 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
   const __nv_bfloat16* G = ws.at<__nv_bfloat16>(P.o_gbuf);
   if (scatter) {  // each fp32 row straight to the rank that reduces it
     CUtensorMap ta, tb;
-    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BK))
+    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, Pipe<EpiDH>::BK))
       return LMH_ERR_CUDA;
     EpiDH::Params ep;
     ep.rows = rows;
@@ -453,7 +487,7 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
                                st, 1));
   } else if (dH_f32) {
     CUtensorMap ta, tb;
-    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BK))
+    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, Pipe<EpiDH>::BK))
       return LMH_ERR_CUDA;
     EpiDH::Params ep;
     ep.rows = rows;
@@ -463,7 +497,7 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
                                st, 1));
   } else if (dH) {
     CUtensorMap ta, tb, tc;
-    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, BK) ||
+    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, Pipe<EpiDH>::BK) ||
         !tmap_out(&tc, dH + r0 * P.d, P.d, rows, P.d))
       return LMH_ERR_CUDA;
     EpiDH::Params ep;
@@ -471,8 +505,8 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
     ep.d = static_cast<int>(P.d);
     const int sp = dh_splits(rows, P.d, P.V);
     ep.part = sp > 1 ? ws.at<float>(P.o_dhpart) : nullptr;
-    LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, tc, rows, P.d, P.V, kOrderDH, &ws.h->err, ep,
-                               st, sp));
+    LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, tc, rows, P.d, P.V,
+                               sp > 1 ? kOrderDHSplit : kOrderDH, &ws.h->err, ep, st, sp));
     if (sp > 1) {
       ProfScope ps(KID_SPLIT_SUM, st);
       const int64_t blocks = cdiv(static_cast<int64_t>(rows) * P.d / 2, 256);
@@ -483,43 +517,23 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
     }
   }
   if (dW || dW_acc || dw_scatter) {
-    CUtensorMap ta, tb, tc;
-    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BK) || !tmap_2d(&tb, H + r0 * P.d, P.d, rows, P.d, BK))
-      return LMH_ERR_CUDA;
     // Internal accumulator (several chunks, no caller dW_acc): store, add, ..., and the last
     // chunk adds and casts in its epilogue without writing the sum back. Caller's dW_acc:
     // add in every chunk (the first stores with LMH_F_DW_ACC_STORE), then cast it. One chunk
     // without dW_acc: bf16 tile sums directly.
     const bool last = chunk_idx == P.nchunks - 1;
     float* acc = dW_acc ? dW_acc : (P.acc ? ws.at<float>(P.o_acc) : nullptr);
-    EpiDW::Params ep;
-    ep.V = static_cast<int>(P.V);
-    ep.d = static_cast<int>(P.d);
+    int acc_mode;
     if (dw_scatter) {  // one chunk: fp32 rows to the reducing ranks (no output map)
-      ep.acc_mode = 4;
-      ep.sc = *dw_scatter;
+      acc_mode = 4;
     } else if (!acc) {
-      ep.acc_mode = 0;
+      acc_mode = 0;
     } else if (dW_acc) {
-      ep.acc_mode = (P.acc_store && chunk_idx == 0) ? 1 : 2;
+      acc_mode = (P.acc_store && chunk_idx == 0) ? 1 : 2;
     } else {
-      ep.acc_mode = chunk_idx == 0 ? 1 : (last ? 3 : 2);
+      acc_mode = chunk_idx == 0 ? 1 : (last ? 3 : 2);
     }
-    CUtensorMap td;  // mode 3: the accumulator, read by the epilogue
-    bool ok;
-    if (ep.acc_mode == 4) {
-      tc = ta;
-      ok = true;
-    } else if (ep.acc_mode == 0) {
-      ok = tmap_out(&tc, dW, P.d, P.V, P.d);
-    } else if (ep.acc_mode == 3) {
-      ok = tmap_out(&tc, dW, P.d, P.V, P.d) && tmap_acc(&td, acc, P.d, P.V, P.d);
-    } else {
-      ok = tmap_acc(&tc, acc, P.d, P.V, P.d);
-    }
-    if (!ok) return LMH_ERR_CUDA;
-    LMH_TRY(launch_gemm<EpiDW>(dev, sms, ta, tb, tc, P.V, P.d, rows, kOrderDW, &ws.h->err, ep,
-                               st, 1, ep.acc_mode == 3 ? &td : nullptr));
+    LMH_TRY(run_dw<EpiDW>(P, dev, sms, G, H, r0, rows, acc_mode, acc, dW, dw_scatter, ws, st));
     if (dW_acc && dW && last) LMH_TRY(cast_dw(P, acc, dW, st));
   }
   return LMH_OK;

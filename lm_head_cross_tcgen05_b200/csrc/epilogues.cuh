@@ -114,13 +114,22 @@ __device__ __forceinline__ void stage_store_64(EpiCtx& c, const float (&a)[32],
   ++c.nstore;
 }
 
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read_le() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
 // The fp32 counterpart: the warp's 32 rows x 32 columns (v of each thread's row, 128 bytes)
-// go through one staging buffer to a TMA store, or with `reduce` to a TMA add into the
-// destination, at (x, y) of ctx.tmC (fp32, box 32 columns x 32 rows, 128-byte swizzle).
+// go through one of its NBUF staging buffers (in turn) to a TMA store, or with `reduce` to a
+// TMA add into the destination, at (x, y) of ctx.tmC (fp32, box 32 columns x 32 rows, 128-byte
+// swizzle). A buffer is reused once the operation issued from it NBUF calls earlier has read
+// it, so NBUF operations can be in flight per warp.
+template <int NBUF>
 __device__ __forceinline__ void stage_f32_32(EpiCtx& c, const float (&v)[32], int x, int y,
                                              bool do_op, bool reduce) {
-  const uint32_t buf = c.stage + (c.nstore & 1u) * EPI_BUF_BYTES;
-  if (c.lane == 0) bulk_wait_read_le1();
+  const uint32_t buf = c.stage + (c.nstore % NBUF) * EPI_BUF_BYTES;
+  if (c.lane == 0) bulk_wait_read_le<NBUF - 1>();
   __syncwarp();
   const uint32_t row = buf + static_cast<uint32_t>(c.lane) * 128u;
   const uint32_t sw = static_cast<uint32_t>(c.lane & 7);
@@ -150,7 +159,7 @@ __device__ __forceinline__ void stage_f32_32(EpiCtx& c, const float (&v)[32], in
 // which the fused backward rescales into the softmax gradient. Columns >= V are masked.
 // ctx.tmC (kStoreP): the chunk's [rows, ldp] bf16 buffer.
 template <int TK, bool kStoreP>
-struct EpiStats {
+struct EpiStats : PipeDefault {
   static constexpr int kId = kStoreP ? 3 : 2;  // gemm_logits_stats(_store)
   static constexpr int kAMajorMN = 0;          // H chunk [rows, d], K-major
   static constexpr int kBMajorMN = 0;          // W [V, d], K-major
@@ -242,7 +251,7 @@ struct EpiStats {
 // Backward epilogue with recomputed logits: G = alpha_i exp(z - lse_i) - beta at the row's
 // targets, written in bf16 to the chunk's G buffer (zero past column V; ctx.tmC maps it).
 template <int TK>
-struct EpiGrad {
+struct EpiGrad : PipeDefault {
   static constexpr int kId = 4;  // gemm_logits_grad
   static constexpr int kAMajorMN = 0;
   static constexpr int kBMajorMN = 0;
@@ -327,7 +336,7 @@ struct RowScatter {
 // ctx.tmC maps this chunk's rows of dH ([rows, d] at row r0). With K (= V) split, each unit
 // writes its fp32 partial to part[split][row][col] instead; a fixed-order reduction over the
 // splits then produces dH. With a row scatter each fp32 row goes to its reducing rank.
-struct EpiDH {
+struct EpiDH : PipeDefault {
   static constexpr int kId = 5;        // gemm_dH
   static constexpr int kAMajorMN = 0;  // G chunk [rows, V], K-major
   static constexpr int kBMajorMN = 1;  // W [V, d] read as [K = V, N = d], N contiguous
@@ -386,7 +395,13 @@ struct EpiDH {
 // as a zeroed caller-owned one. The accumulator is never read by 16-byte register loads that
 // wait on DRAM one row at a time: writes are staged stores and L2 reduce-adds, and the one
 // read (mode 3) is a TMA block load.
-struct EpiDW {
+// kBK_, kStages_, kEpiBufs_: the pipeline shape (Pipe). Trading ring depth for more staging
+// buffers (more reduce-adds in flight per warp) made the accumulate modes slower, not faster
+// (96 x 3 stages with 5 buffers, 64 x 5 with 4, 64 x 4 with 6: 2.94 -> 3.27 ms per 2048-row
+// chunk at 16384 x 5120 x 151936), so every mode runs the default shape.
+template <int kBK_, int kStages_, int kEpiBufs_>
+struct EpiDWT {
+  static constexpr int kBK = kBK_, kStages = kStages_, kEpiBufs = kEpiBufs_;
   static constexpr int kId = 6;        // gemm_dW
   static constexpr int kAMajorMN = 1;  // G^T: G chunk [rows, V] read as [K = rows, M = V]
   static constexpr int kBMajorMN = 1;  // H chunk [rows, d] read as [K = rows, N = d]
@@ -434,8 +449,8 @@ struct EpiDW {
             b[j] = __fadd_rn(0.f, b[j]);
           }
         }
-        stage_f32_32(ctx, a, col0, wrow, wv, p.acc_mode == 2);
-        stage_f32_32(ctx, b, col0 + 32, wrow, wv, p.acc_mode == 2);
+        stage_f32_32<kEpiBufs>(ctx, a, col0, wrow, wv, p.acc_mode == 2);
+        stage_f32_32<kEpiBufs>(ctx, b, col0 + 32, wrow, wv, p.acc_mode == 2);
       }
     }
   }
@@ -473,5 +488,6 @@ struct EpiDW {
     __syncwarp();  // every lane has read both buffers before the bf16 staging reuses one
   }
 };
+using EpiDW = EpiDWT<PipeDefault::kBK, PipeDefault::kStages, PipeDefault::kEpiBufs>;
 
 }  // namespace lmh

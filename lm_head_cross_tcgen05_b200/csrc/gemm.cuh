@@ -7,8 +7,7 @@
 // CTAs. Per SM this halves the B operand traffic of a 128 x 256 single-CTA tile.
 //
 // Persistent schedule: grid = 2 x (number of co-resident pairs); pair p walks the work units
-// p, p + pairs, ... of a fixed, grouped order (group_m row tiles at a time, rows fastest; or
-// group_n column tiles at a time, columns fastest). A
+// p, p + pairs, ... of a fixed, grouped order (group_m row tiles at a time, rows fastest). A
 // work unit is an output tile, or a tile and one of k_splits consecutive K ranges when a
 // launch has too few tiles to fill the GPU (its epilogue then writes an fp32 partial).
 // Every output tile is owned by one pair and its K loop runs in ascending order, so the fp32
@@ -40,22 +39,40 @@ constexpr int BM = 128;   // accumulator rows per CTA (half of a pair tile)
 constexpr int PM = 256;   // rows per pair tile
 constexpr int BN = 256;   // columns per tile
 constexpr int BNH = 128;  // B rows staged per CTA
-// K per pipeline stage: 128, i.e. 8 MMAs per barrier round trip. Each round trip (wait for
-// the stage, commit its release) costs the tensor pipe a roughly fixed bubble, so the deeper
-// stage runs about 18 % more MMAs per clock than a 64-deep one; 3 stages of 64 KiB per CTA.
-constexpr int BK = 128;
-constexpr int KSUB = BK / 64;                // 128-byte-wide K sub-tiles of a K-major stage
-constexpr int STAGES = 3;
-constexpr int A_STAGE_BYTES = BM * BK * 2;
-constexpr int B_STAGE_BYTES = BNH * BK * 2;
-constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int A_SUB_BYTES = BM * 128;        // one K-major sub-tile of A (rows x 64 K)
 constexpr int B_SUB_BYTES = BNH * 128;
-constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x BK (K) box
 constexpr int GEMM_THREADS = 192;
-constexpr int EPI_BUF_BYTES = 32 * 128;                      // 32 rows x 64 bf16, 128B-swizzled
-constexpr int EPI_STAGE_BYTES = 4 * 2 * EPI_BUF_BYTES;       // two buffers per epilogue warp
-constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + 1024;  // + align slack
+constexpr int EPI_BUF_BYTES = 32 * 128;      // 32 rows x 64 bf16 (or 32 fp32), 128B-swizzled
+constexpr int kMaxDynSmem = 232448;          // 227 KiB per CTA on sm_100
+
+// Pipeline shape of a GEMM instantiation, taken from its epilogue: K per stage (kBK), ring
+// depth (kStages) and staging buffers per epilogue warp (kEpiBufs). The default is K = 128 per
+// stage, i.e. 8 MMAs per barrier round trip: each round trip (wait for the stage, commit its
+// release) costs the tensor pipe a roughly fixed bubble, so the deeper stage runs about 18 %
+// more MMAs per clock than a 64-deep one; 3 stages of 64 KiB per CTA, two 4 KiB staging buffers
+// per epilogue warp. An epilogue whose stores must wait on DRAM (the dW accumulation) can trade
+// ring depth for staging.
+struct PipeDefault {
+  static constexpr int kBK = 128, kStages = 3, kEpiBufs = 2;
+};
+
+template <class Epi>
+struct Pipe {
+  static constexpr int BK = Epi::kBK;
+  static constexpr int STAGES = Epi::kStages;
+  static constexpr int EPI_BUFS = Epi::kEpiBufs;
+  static constexpr int KSUB = BK / 64;                // 128-byte-wide K sub-tiles (K-major)
+  static constexpr int A_STAGE_BYTES = BM * BK * 2;
+  static constexpr int B_STAGE_BYTES = BNH * BK * 2;
+  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+  static constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x BK (K) box
+  static constexpr int EPI_STAGE_BYTES = 4 * EPI_BUFS * EPI_BUF_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + 1024;  // + align
+  static_assert(BK % 16 == 0 && STAGES >= 2 && EPI_BUFS >= 2 && EPI_BUFS <= 8, "pipeline shape");
+  static_assert((Epi::kAMajorMN && Epi::kBMajorMN) || BK % 64 == 0,
+                "a K-major operand is staged in 64-wide K boxes");
+  static_assert(SMEM_BYTES + 256 <= kMaxDynSmem, "shared memory per CTA");
+};
 
 // What an epilogue warp needs to stage bf16 output through shared memory and store it with
 // TMA: the output tensor map (bf16, box 64 columns x 32 rows, 128-byte swizzle), its two
@@ -77,10 +94,9 @@ constexpr uint32_t TMEM_COLS = 512;
 struct GemmGrid {
   int m_tiles;   // pair tiles along M (256 rows each)
   int n_tiles;   // tiles along N (256 columns each)
-  int k_blocks;  // ceil(K / BK)
+  int k_blocks;  // ceil(K / Pipe<Epi>::BK)
   int k_splits;  // K split into this many consecutive ranges (work units = tiles x splits)
   int group_m;   // tile order: group_m row tiles at a time, rows fastest within a group
-  int group_n;   // > 0: group_n column tiles at a time instead, columns fastest within a group
   int hint_a;    // L2 eviction priority of A's loads (L2Hint)
   int hint_b;    // L2 eviction priority of B's loads
   uint32_t* err; // device error word
@@ -92,23 +108,13 @@ __device__ __forceinline__ void unit_coords(const GemmGrid& g, int u, int& mb, i
   const int tiles = g.m_tiles * g.n_tiles;
   split = u / tiles;
   int t = u - split * tiles;
-  if (g.group_n > 0) {
-    const int per_group = g.group_n * g.m_tiles;
-    const int grp = t / per_group;
-    const int rem = t - grp * per_group;
-    const int n0 = grp * g.group_n;
-    const int gn = min(g.group_n, g.n_tiles - n0);
-    nb = n0 + rem % gn;
-    mb = rem / gn;
-  } else {
-    const int per_group = g.group_m * g.n_tiles;
-    const int grp = t / per_group;
-    const int rem = t - grp * per_group;
-    const int m0 = grp * g.group_m;
-    const int gm = min(g.group_m, g.m_tiles - m0);
-    mb = m0 + rem % gm;
-    nb = rem / gm;
-  }
+  const int per_group = g.group_m * g.n_tiles;
+  const int grp = t / per_group;
+  const int rem = t - grp * per_group;
+  const int m0 = grp * g.group_m;
+  const int gm = min(g.group_m, g.m_tiles - m0);
+  mb = m0 + rem % gm;
+  nb = rem / gm;
   kb0 = static_cast<int>(static_cast<long long>(g.k_blocks) * split / g.k_splits);
   kb1 = static_cast<int>(static_cast<long long>(g.k_blocks) * (split + 1) / g.k_splits);
 }
@@ -120,6 +126,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                    const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmD, const GemmGrid g,
                    const typename Epi::Params ep) {
+  using P = Pipe<Epi>;
+  constexpr int BK = P::BK, STAGES = P::STAGES, STAGE_BYTES = P::STAGE_BYTES;
+  constexpr int A_STAGE_BYTES = P::A_STAGE_BYTES, MN_BLOCK_BYTES = P::MN_BLOCK_BYTES;
+  constexpr int KSUB = P::KSUB;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];   // rank 0: operands of a stage landed
   __shared__ __align__(8) uint64_t empty_bar[STAGES];  // both: the stage was read by the MMAs
@@ -262,7 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // the TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
-    EpiCtx ctx{&tmC, &tmD, smem_base + STAGES * STAGE_BYTES + (warp - 2) * 2 * EPI_BUF_BYTES, lane,
+    EpiCtx ctx{&tmC, &tmD, smem_base + STAGES * STAGE_BYTES + (warp - 2) * P::EPI_BUFS * EPI_BUF_BYTES, lane,
                q * 32, 0u, 0, smem_u32(&epi_bar[warp - 2]), 0u, g.err};
     if (lane == 0) tma_prefetch_desc(&tmC);
     int it = 0;

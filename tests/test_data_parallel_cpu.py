@@ -122,3 +122,39 @@ def test_absent_rank_ends_the_step_with_an_error():
         p.join(timeout=60)
     assert res[0]["error"] is not None, res
     assert res[0]["after"] < 9.0, res
+
+
+def _p2p_chunk_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from lm_head_cross_tcgen05_b200.data_parallel import DataParallelCE
+        from tests.dp_oracle_ops import DataParallelOracleOps
+        try:
+            DataParallelCE(ops=DataParallelOracleOps(), p2p=True, chunk_rows=128)
+            refused = None
+        except ValueError as e:
+            refused = str(e)
+        ok = DataParallelCE(ops=DataParallelOracleOps(), p2p=True)   # one chunk: accepted
+        q.put(dict(rank=rank, refused=refused, p2p=ok.p2p))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_memory_exchange_refuses_a_chunk_plan():
+    # the peer-memory dW exchange runs each rank's rows as one chunk: a chunk_rows budget
+    # cannot be honoured, so it is refused instead of ignored (two gloo ranks: p2p is only
+    # active with more than one rank)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_p2p_chunk_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    res = [q.get(timeout=120) for _ in ps]
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in res:
+        assert r["refused"] and "chunk_rows" in r["refused"], r
+        assert r["p2p"] is True
