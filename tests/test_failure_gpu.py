@@ -90,6 +90,24 @@ def test_peer_barrier_passes_once_every_rank_signalled(epoch, peer_word):
     assert all(sig[j][0].item() == e32 for j in range(R))
 
 
+def test_peer_barrier_more_ranks_than_a_warp():
+    # 40 ranks: a two-warp block; rank 17's barrier with every other word preset passes, and
+    # with one word (rank 33's) missing it times out
+    R, rank, epoch = 40, 17, 5
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    sig, tab = _signals(R)
+    sig[rank].fill_(epoch)
+    assert _barrier(ws, tab, R, rank, epoch, 2000) == 0
+    torch.cuda.synchronize()
+    assert L.lmh_read_errors(ws) == 0
+    assert all(sig[j][rank].item() == epoch for j in range(R))
+    sig[rank].fill_(epoch + 1)
+    sig[rank][33] = epoch                          # rank 33 is one barrier behind
+    assert _barrier(ws, tab, R, rank, epoch + 1, 150) == 0
+    torch.cuda.synchronize()
+    assert L.lmh_read_errors(ws) == L.DEVERR_TIMEOUT
+
+
 def test_peer_barrier_one_rank_and_argument_checks():
     ws = torch.zeros(512, dtype=torch.uint8, device="cuda")
     sig, tab = _signals(1)
