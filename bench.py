@@ -383,9 +383,14 @@ def main():
     H, W, y = x["H"], x["W"], x["labels"]
     N, d, V = wl.N, wl.d, wl.V
     chunk = args.chunk_rows or wl.chunk_rows or N
-    shape = L.make_shape(N, d, V, 0, chunk, L.F_MEAN | L.F_FUSED_BWD)
-    ws = L.workspace(shape, L.ENTRY_LOSS_FWD, dev)
     f32, i32, bf = torch.float32, torch.int32, torch.bfloat16
+    # several chunks: the fp32 dW accumulator is the caller's (the workspace holds one chunk's
+    # softmax buffer, within the memory budget); the first chunk stores into it, so no step
+    # needs a zeroing pass
+    dW_acc = (torch.empty(V, d, dtype=f32, device=dev) if chunk < N else None)
+    acc_flags = L.F_DW_ACC_GIVEN | L.F_DW_ACC_STORE if dW_acc is not None else 0
+    shape = L.make_shape(N, d, V, 0, chunk, L.F_MEAN | L.F_FUSED_BWD | acc_flags)
+    ws = L.workspace(shape, L.ENTRY_LOSS_FWD, dev)
     out = dict(loss_rows=torch.empty(N, dtype=f32, device=dev),
                lse=torch.empty(N, dtype=f32, device=dev),
                logprob=torch.empty(N, dtype=f32, device=dev),
@@ -402,7 +407,7 @@ def main():
         def step(b=batch):
             L.lmh_loss_fwd(shape, b["H"], W, b["labels"], out["loss_rows"], out["lse"], out["logprob"],
                            out["argmax"], out["loss_mean"], out["n_valid"], None, out["dH"],
-                           out["dW"], None, workspace=ws, stream=stream)
+                           out["dW"], dW_acc, workspace=ws, stream=stream)
     elif args.entry == "ce_separate":
         fshape = L.make_shape(N, d, V, 0, chunk, L.F_MEAN)
         fws = L.workspace(fshape, L.ENTRY_LOSS_FWD, dev)
@@ -606,11 +611,16 @@ def main():
                                   f"{t:.1f} s"}
 
     if rank == 0:
+        cfg = workload_config(wl, chunk, world, args.entry)
+        if args.entry == "fused_ce":
+            cfg["workspace_bytes"] = int(ws.numel())
+            cfg["dW_accumulator"] = ("caller-owned fp32 [V, d], stored by the first chunk"
+                                     if dW_acc is not None else "none (one chunk: bf16 dW)")
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "strong" if vp_entry else "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": workload_config(wl, chunk, world, args.entry),
+                "config": cfg,
                 "peak_frac": {"of_burst": value / world / peaks["bf16_tflops"],
                               "of_sustained": value / world / peaks["bf16_tflops_sustained"],
                               "of_sampled_clock": (value / world / tensor_peak_at(

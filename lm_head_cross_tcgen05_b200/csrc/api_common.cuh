@@ -454,14 +454,14 @@ lmh_status run_dw(const Plan& P, int dev, int sms, const __nv_bfloat16* G, const
     ok = true;
   } else if (acc_mode == 0) {
     ok = tmap_out(&tc, dW, P.d, P.V, P.d);
-  } else if (acc_mode == 3) {
+  } else if (acc_mode == 3 || acc_mode == 5) {
     ok = tmap_out(&tc, dW, P.d, P.V, P.d) && tmap_acc(&td, acc, P.d, P.V, P.d);
   } else {
     ok = tmap_acc(&tc, acc, P.d, P.V, P.d);
   }
   if (!ok) return LMH_ERR_CUDA;
   return launch_gemm<Epi>(dev, sms, ta, tb, tc, P.V, P.d, rows, kOrderDW, &ws.h->err, ep, st, 1,
-                          acc_mode == 3 ? &td : nullptr);
+                          (acc_mode == 3 || acc_mode == 5) ? &td : nullptr);
 }
 
 // dH = G W and dW (+)= G^T H_c for one chunk whose G sits in the workspace buffer.
@@ -529,12 +529,15 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
     } else if (!acc) {
       acc_mode = 0;
     } else if (dW_acc) {
-      acc_mode = (P.acc_store && chunk_idx == 0) ? 1 : 2;
+      const bool first_store = P.acc_store && chunk_idx == 0;
+      // the last chunk adds, stores the sum and casts it in one pass, unless it is also the
+      // stored first chunk (then: store, and the cast below)
+      acc_mode = (dW && last && !first_store) ? 5 : (first_store ? 1 : 2);
     } else {
       acc_mode = chunk_idx == 0 ? 1 : (last ? 3 : 2);
     }
     LMH_TRY(run_dw<EpiDW>(P, dev, sms, G, H, r0, rows, acc_mode, acc, dW, dw_scatter, ws, st));
-    if (dW_acc && dW && last) LMH_TRY(cast_dw(P, acc, dW, st));
+    if (dW_acc && dW && last && acc_mode != 5) LMH_TRY(cast_dw(P, acc, dW, st));
   }
   return LMH_OK;
 }

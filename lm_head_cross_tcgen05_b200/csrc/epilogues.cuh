@@ -387,8 +387,11 @@ struct EpiDH : PipeDefault {
 //             buffers, added in registers, and the bf16 result stored through ctx.tmC.
 // acc_mode 4: 0 + sum in fp32, each row stored straight into the receive buffer of the rank
 //             that reduces it (p.sc: row data-parallel dW over peer memory; one chunk).
-// In modes 1 and 2 ctx.tmC maps the fp32 accumulator [V, d]; in mode 3 ctx.tmD does (fp32,
-// box 32 x 32 rows, 128-byte swizzle) and ctx.tmC maps bf16 dW. Every
+// acc_mode 5: as mode 3, and the fp32 sum is also stored back into the accumulator (last
+//             chunk of a caller-owned accumulator that must end up holding the sum): the
+//             bf16 cast of the final accumulator needs no separate pass.
+// In modes 1 and 2 ctx.tmC maps the fp32 accumulator [V, d]; in modes 3 and 5 ctx.tmD does
+// (fp32, box 32 x 32 rows, 128-byte swizzle) and ctx.tmC maps bf16 dW. Every
 // element has one owner tile per launch and the launches of a call run in chunk order, so the
 // accumulation order is fixed. Every add (modes 1 and 3 in registers, mode 2 in the TMA unit)
 // is an IEEE fp32 add rounded to nearest even, so an internal accumulator gives the same bits
@@ -437,9 +440,10 @@ struct EpiDWT {
                                       __fadd_rn(0.f, v[q + 2]), __fadd_rn(0.f, v[q + 3])));
           }
         }
-      } else if (p.acc_mode == 3) {
+      } else if (p.acc_mode == 3 || p.acc_mode == 5) {
         if (!wv) continue;  // warp-uniform: nothing of this block exists
         add_loaded_64(ctx, col0, wrow, a, b);
+        if (p.acc_mode == 5) store_sum_64(ctx, col0, wrow, a, b);
         stage_store_64(ctx, a, b, col0, wrow, true);
       } else {
         if (p.acc_mode == 1) {
@@ -453,6 +457,32 @@ struct EpiDWT {
         stage_f32_32<kEpiBufs>(ctx, b, col0 + 32, wrow, wv, p.acc_mode == 2);
       }
     }
+  }
+  // The warp's 32 x 64 fp32 sums back into the accumulator at (col0, wrow) through both
+  // staging buffers (free after add_loaded_64); returns once the TMA has read them, so the
+  // bf16 store that follows may reuse either buffer. Rows past V are clipped by the map.
+  static __device__ __forceinline__ void store_sum_64(EpiCtx& c, int col0, int wrow,
+                                                      const float (&a)[32], const float (&b)[32]) {
+    const uint32_t b0 = c.stage, b1 = c.stage + EPI_BUF_BYTES;
+    const uint32_t off = static_cast<uint32_t>(c.lane) * 128u;
+    const uint32_t sw = static_cast<uint32_t>(c.lane & 7);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t ch = ((static_cast<uint32_t>(u) ^ sw) << 4) + off;
+      st_shared_v4(b0 + ch, make_uint4(__float_as_uint(a[u * 4 + 0]), __float_as_uint(a[u * 4 + 1]),
+                                       __float_as_uint(a[u * 4 + 2]), __float_as_uint(a[u * 4 + 3])));
+      st_shared_v4(b1 + ch, make_uint4(__float_as_uint(b[u * 4 + 0]), __float_as_uint(b[u * 4 + 1]),
+                                       __float_as_uint(b[u * 4 + 2]), __float_as_uint(b[u * 4 + 3])));
+    }
+    fence_async_smem();
+    __syncwarp();
+    if (c.lane == 0) {
+      tma_store_2d(c.tmD, b0, col0, wrow);
+      tma_store_2d(c.tmD, b1, col0 + 32, wrow);
+      bulk_commit();
+      bulk_wait_read_all();
+    }
+    __syncwarp();
   }
   // a (+)= acc[wrow + lane, col0 .. col0+31], b (+)= acc[.., col0+32 .. col0+63], the 32 x 64
   // fp32 block loaded by TMA into the warp's two staging buffers (zero past V).
