@@ -252,3 +252,34 @@ def test_data_parallel_class_on_one_rank():
     q = ops.fused(x["H"], x["W"], x["labels"], n, bf16_dW=True)
     assert torch.equal(ops.reduce_rows(p["dW_part"][None]), q["dW"])
     assert torch.equal(p["dH"], q["dH"]) and torch.equal(p["loss_mean"], q["loss_mean"])
+
+
+def test_peer_memory_exchange_runs_on_one_rank():
+    # The peer-memory dW exchange end to end on one NCCL rank, with p2p forced on (a single rank
+    # normally skips the exchange): torch symmetric memory for the receive buffer, the dW
+    # outputs and the barrier's signal words; the library's barrier kernel; the dW GEMM's row
+    # scatter; the rank-order reduce into the symmetric output. Two steps, so the second one
+    # checks the first one's barrier record and reuses the buffers. The dW must be the bits of
+    # the one-device fused step (the reduce of one fp32 part is its bf16 cast).
+    import torch.distributed as dist
+    N, d, V = 300, 128, 2100
+    x, xc = device_inputs(ragged(N, d, V, n_ignored=6, seed=4410))
+    one = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        dp = DataParallelCE()
+        dp.p2p = True
+        outs = [dp.forward_backward(x["H"], x["W"], x["labels"]) for _ in range(2)]
+        torch.cuda.synchronize()
+        dp.check_exchange()                        # no barrier gave up
+        assert dp._sym["epoch"] == 6               # three barriers per step
+        dp._sym = None
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    for out in outs:
+        assert torch.equal(out["dW"], one["dW"])
+        assert torch.equal(out["dH"], one["dH"]) and torch.equal(out["lse"], one["lse"])
+        assert torch.equal(out["loss_mean"], one["loss_mean"])
+    check_ce_fused(outs[0], O.ce_fused(xc["H"], xc["W"], xc["labels"]))

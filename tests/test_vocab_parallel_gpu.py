@@ -349,3 +349,30 @@ def test_vocab_parallel_support_refuses_renorm():
     rec = torch.empty(N, K + 1, dtype=torch.float32, device="cuda")
     with pytest.raises(L.LmhError, match="INVALID_ARG"):
         L.lmh_vp_support_partials(shard, 0, V, x["H"], x["W"][:300], x["ids"], rec, workspace=ws)
+
+
+def test_peer_memory_dh_exchange_runs_on_one_rank():
+    # The vocabulary-parallel dH exchange over peer memory on one NCCL rank, p2p forced on:
+    # symmetric buffers, the barrier kernel, the dH GEMM's row scatter and the reduce into the
+    # symmetric output, twice. The results must be the collective path's bits.
+    import torch.distributed as dist
+    N, d, V = 130, 128, 2100
+    x, xc = device_inputs(_wl(N, d, V, 4))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        ref = VocabParallelCE(V).forward_backward(x["H"], x["W"], x["labels"])
+        vp = VocabParallelCE(V)
+        vp.p2p = True
+        outs = [vp.forward_backward(x["H"], x["W"], x["labels"]) for _ in range(2)]
+        torch.cuda.synchronize()
+        vp.check_exchange()
+        assert vp._sym["epoch"] == 6
+        vp._sym = None
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    for out in outs:
+        assert torch.equal(out["dH"], ref["dH"]) and torch.equal(out["dW"], ref["dW"])
+        assert torch.equal(out["lse"], ref["lse"])
+    check_ce_fused(outs[0], O.ce_fused(xc["H"], xc["W"], xc["labels"]))
