@@ -120,36 +120,40 @@ __device__ __forceinline__ void bulk_wait_read_le() {
   asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
-// The fp32 counterpart: the warp's 32 rows x 32 columns (v of each thread's row, 128 bytes)
-// go through one of its NBUF staging buffers (in turn) to a TMA store, or with `reduce` to a
-// TMA add into the destination, at (x, y) of ctx.tmC (fp32, box 32 columns x 32 rows, 128-byte
-// swizzle). A buffer is reused once the operation issued from it NBUF calls earlier has read
-// it, so NBUF operations can be in flight per warp.
-template <int NBUF>
-__device__ __forceinline__ void stage_f32_32(EpiCtx& c, const float (&v)[32], int x, int y,
-                                             bool do_op, bool reduce) {
-  const uint32_t buf = c.stage + (c.nstore % NBUF) * EPI_BUF_BYTES;
-  if (c.lane == 0) bulk_wait_read_le<NBUF - 1>();
+// The fp32 counterpart: the warp's 32 rows x 64 columns of fp32 (a: columns x .. x+31, b:
+// x+32 .. x+63 of each thread's row) go through both of its staging buffers with one proxy
+// fence, then to two TMA stores, or with `reduce` two TMA adds into the destination, at (x, y)
+// and (x + 32, y) of ctx.tmC (fp32, box 32 columns x 32 rows, 128-byte swizzle), committed as
+// one group. The buffers are reused once the previous group has read them. (One fence per
+// 64 columns instead of per 32: 3 % off the accumulating dW GEMM.)
+__device__ __forceinline__ void stage_f32_64(EpiCtx& c, const float (&a)[32], const float (&b)[32],
+                                             int x, int y, bool do_op, bool reduce) {
+  const uint32_t b0 = c.stage, b1 = c.stage + EPI_BUF_BYTES;
+  if (c.lane == 0) bulk_wait_read_le<0>();
   __syncwarp();
-  const uint32_t row = buf + static_cast<uint32_t>(c.lane) * 128u;
+  const uint32_t row = static_cast<uint32_t>(c.lane) * 128u;
   const uint32_t sw = static_cast<uint32_t>(c.lane & 7);
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    uint4 w;
-    w.x = __float_as_uint(v[u * 4 + 0]);
-    w.y = __float_as_uint(v[u * 4 + 1]);
-    w.z = __float_as_uint(v[u * 4 + 2]);
-    w.w = __float_as_uint(v[u * 4 + 3]);
-    st_shared_v4(row + ((static_cast<uint32_t>(u) ^ sw) << 4), w);
+    const uint32_t ch = row + ((static_cast<uint32_t>(u) ^ sw) << 4);
+    st_shared_v4(b0 + ch, make_uint4(__float_as_uint(a[u * 4 + 0]), __float_as_uint(a[u * 4 + 1]),
+                                     __float_as_uint(a[u * 4 + 2]), __float_as_uint(a[u * 4 + 3])));
+    st_shared_v4(b1 + ch, make_uint4(__float_as_uint(b[u * 4 + 0]), __float_as_uint(b[u * 4 + 1]),
+                                     __float_as_uint(b[u * 4 + 2]), __float_as_uint(b[u * 4 + 3])));
   }
   fence_async_smem();
   __syncwarp();
   if (c.lane == 0 && do_op) {
-    if (reduce) tma_reduce_add_2d(c.tmC, buf, x, y);
-    else tma_store_2d(c.tmC, buf, x, y);
+    if (reduce) {
+      tma_reduce_add_2d(c.tmC, b0, x, y);
+      tma_reduce_add_2d(c.tmC, b1, x + 32, y);
+    } else {
+      tma_store_2d(c.tmC, b0, x, y);
+      tma_store_2d(c.tmC, b1, x + 32, y);
+    }
     bulk_commit();
   }
-  ++c.nstore;
+  c.nstore += 2;
 }
 
 // ------------------------------------------------------------------ logits statistics
@@ -453,8 +457,7 @@ struct EpiDWT {
             b[j] = __fadd_rn(0.f, b[j]);
           }
         }
-        stage_f32_32<kEpiBufs>(ctx, a, col0, wrow, wv, p.acc_mode == 2);
-        stage_f32_32<kEpiBufs>(ctx, b, col0 + 32, wrow, wv, p.acc_mode == 2);
+        stage_f32_64(ctx, a, b, col0, wrow, wv, p.acc_mode == 2);
       }
     }
   }
