@@ -159,3 +159,29 @@ def test_no_gradient_at_all_runs_no_backward_gemm():
     assert not any(n in names for n in ("gemm_dH", "gemm_dW", "split_sum", "gbuild"))
     fwd = L.loss_fwd(x["H"], x["W"], x["labels"])
     assert torch.equal(out["lse"], fwd["lse"]) and torch.equal(out["loss_rows"], fwd["loss_rows"])
+
+
+@pytest.mark.parametrize("want", ["dH", "dW"])
+@pytest.mark.parametrize("mode", [L.BWD_SUPPORT_LOGPROB, L.BWD_SUPPORT_KL])
+def test_renormalised_support_backward_frozen(mode, want):
+    # the other reading of the support set (log-probs normalised over each row's candidates):
+    # its backward has no GEMM, dH is a gather of W rows and dW a scatter per vocabulary row,
+    # so a frozen input skips the gather's output or the whole scatter
+    N, d, V, K = 200, 128, 3000, 12
+    x, xc = _inputs(N, d, V, 0, K=K)
+    ids, ref_lp = x["ids"], x["ref_logp"]
+    kl = mode == L.BWD_SUPPORT_KL
+    lse = L.support_logprob(x["H"], x["W"], ids, renorm=True)["lse"]
+    g = (torch.linspace(0.5, 1.5, N, dtype=torch.float32) / N if kl else
+         torch.linspace(-1.0, 2.0, N * K, dtype=torch.float32).view(N, K) / N)
+    args = (mode, x["H"], x["W"], ids, lse, g.cuda(), ref_lp if kl else None)
+    both = L.loss_bwd(*args, renorm=True)
+    only, names = launched(lambda: L.loss_bwd(*args, renorm=True, want_dH=want == "dH",
+                                              want_dW=want == "dW"))
+    ref = O.backward_renorm(mode, xc["H"], xc["W"], xc["ids"], g.numpy(),
+                            xc["ref_logp"] if kl else None)
+    other = "dW" if want == "dH" else "dH"
+    assert only.get(other) is None
+    check_grad(only[want], ref[want], f"{want} only (renormalised)")
+    assert torch.equal(only[want], both[want])
+    assert ("support_dw" in names) == (want == "dW"), names
