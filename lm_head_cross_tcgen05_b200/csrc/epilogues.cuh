@@ -126,21 +126,33 @@ __device__ __forceinline__ void bulk_wait_read_le() {
 // and (x + 32, y) of ctx.tmC (fp32, box 32 columns x 32 rows, 128-byte swizzle), committed as
 // one group. The buffers are reused once the previous group has read them. (One fence per
 // 64 columns instead of per 32: 3 % off the accumulating dW GEMM.)
-__device__ __forceinline__ void stage_f32_64(EpiCtx& c, const float (&a)[32], const float (&b)[32],
-                                             int x, int y, bool do_op, bool reduce) {
+__device__ __forceinline__ uint4 f32x4_bits(const float (&v)[32], int u) {
+  return make_uint4(__float_as_uint(v[u * 4 + 0]), __float_as_uint(v[u * 4 + 1]),
+                    __float_as_uint(v[u * 4 + 2]), __float_as_uint(v[u * 4 + 3]));
+}
+
+// Each thread's 64 fp32 (a: columns 0..31, b: 32..63 of its row) into the warp's two staging
+// buffers, each the 128-byte-swizzled layout of a 32 x 32 fp32 TMA box. The buffers must be
+// free; the caller fences before a TMA operation reads them.
+__device__ __forceinline__ void write_f32_pair(const EpiCtx& c, const float (&a)[32],
+                                               const float (&b)[32]) {
   const uint32_t b0 = c.stage, b1 = c.stage + EPI_BUF_BYTES;
-  if (c.lane == 0) bulk_wait_read_le<0>();
-  __syncwarp();
   const uint32_t row = static_cast<uint32_t>(c.lane) * 128u;
   const uint32_t sw = static_cast<uint32_t>(c.lane & 7);
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const uint32_t ch = row + ((static_cast<uint32_t>(u) ^ sw) << 4);
-    st_shared_v4(b0 + ch, make_uint4(__float_as_uint(a[u * 4 + 0]), __float_as_uint(a[u * 4 + 1]),
-                                     __float_as_uint(a[u * 4 + 2]), __float_as_uint(a[u * 4 + 3])));
-    st_shared_v4(b1 + ch, make_uint4(__float_as_uint(b[u * 4 + 0]), __float_as_uint(b[u * 4 + 1]),
-                                     __float_as_uint(b[u * 4 + 2]), __float_as_uint(b[u * 4 + 3])));
+    st_shared_v4(b0 + ch, f32x4_bits(a, u));
+    st_shared_v4(b1 + ch, f32x4_bits(b, u));
   }
+}
+
+__device__ __forceinline__ void stage_f32_64(EpiCtx& c, const float (&a)[32], const float (&b)[32],
+                                             int x, int y, bool do_op, bool reduce) {
+  const uint32_t b0 = c.stage, b1 = c.stage + EPI_BUF_BYTES;
+  if (c.lane == 0) bulk_wait_read_le<0>();
+  __syncwarp();
+  write_f32_pair(c, a, b);
   fence_async_smem();
   __syncwarp();
   if (c.lane == 0 && do_op) {
@@ -467,16 +479,7 @@ struct EpiDWT {
   static __device__ __forceinline__ void store_sum_64(EpiCtx& c, int col0, int wrow,
                                                       const float (&a)[32], const float (&b)[32]) {
     const uint32_t b0 = c.stage, b1 = c.stage + EPI_BUF_BYTES;
-    const uint32_t off = static_cast<uint32_t>(c.lane) * 128u;
-    const uint32_t sw = static_cast<uint32_t>(c.lane & 7);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const uint32_t ch = ((static_cast<uint32_t>(u) ^ sw) << 4) + off;
-      st_shared_v4(b0 + ch, make_uint4(__float_as_uint(a[u * 4 + 0]), __float_as_uint(a[u * 4 + 1]),
-                                       __float_as_uint(a[u * 4 + 2]), __float_as_uint(a[u * 4 + 3])));
-      st_shared_v4(b1 + ch, make_uint4(__float_as_uint(b[u * 4 + 0]), __float_as_uint(b[u * 4 + 1]),
-                                       __float_as_uint(b[u * 4 + 2]), __float_as_uint(b[u * 4 + 3])));
-    }
+    write_f32_pair(c, a, b);
     fence_async_smem();
     __syncwarp();
     if (c.lane == 0) {

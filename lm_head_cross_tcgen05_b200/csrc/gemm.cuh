@@ -50,8 +50,8 @@ constexpr int kMaxDynSmem = 232448;          // 227 KiB per CTA on sm_100
 // stage, i.e. 8 MMAs per barrier round trip: each round trip (wait for the stage, commit its
 // release) costs the tensor pipe a roughly fixed bubble, so the deeper stage runs about 18 %
 // more MMAs per clock than a 64-deep one; 3 stages of 64 KiB per CTA, two 4 KiB staging buffers
-// per epilogue warp. An epilogue whose stores must wait on DRAM (the dW accumulation) can trade
-// ring depth for staging.
+// per epilogue warp. Every epilogue uses this shape: the alternatives measured (64-deep stages,
+// ring depth traded for staging in the dW accumulation) were slower.
 struct PipeDefault {
   static constexpr int kBK = 128, kStages = 3, kEpiBufs = 2;
 };
@@ -272,8 +272,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // the TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
-    EpiCtx ctx{&tmC, &tmD, smem_base + STAGES * STAGE_BYTES + (warp - 2) * P::EPI_BUFS * EPI_BUF_BYTES, lane,
-               q * 32, 0u, 0, smem_u32(&epi_bar[warp - 2]), 0u, g.err};
+    const uint32_t stage_w =
+        smem_base + STAGES * STAGE_BYTES + (warp - 2) * P::EPI_BUFS * EPI_BUF_BYTES;
+    EpiCtx ctx{&tmC, &tmD, stage_w, lane, q * 32, 0u, 0, smem_u32(&epi_bar[warp - 2]), 0u, g.err};
     if (lane == 0) tma_prefetch_desc(&tmC);
     int it = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++it) {
