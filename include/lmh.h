@@ -30,10 +30,10 @@
  *   error word gets LMH_DEVERR_LABEL_RANGE (no trap; read it with lmh_read_errors).
  * - Rows are processed in chunks of shape->chunk_rows rows (0 selects 4096, the default of
  *   the same commit's --cake-lm-head-chunk-size), in ascending order. The chunk plan changes
- *   the summation order of dW across chunks and, for chunks too small to fill the GPU with
- *   dH tiles (fewer than 384 tiles of 256 x 256), of dH, whose vocabulary sum is then split
- *   into up to 8 ranges added in a fixed order. The forward outputs (loss, lse, log-probs,
- *   argmax, counts) do not depend on it; no output depends on the GPU's SM count.
+ *   the summation order of dW across chunks and, where a chunk's dH tiling splits the
+ *   vocabulary sum into ranges added in a fixed order (lmh_dh_plan), of dH. The forward
+ *   outputs (loss, lse, log-probs, argmax, counts) do not depend on it; no output depends on
+ *   the GPU's SM count.
  * - Return value: LMH_OK, or an error found on the host before anything was enqueued
  *   (invalid argument, misalignment, short workspace, unsupported device), or
  *   LMH_ERR_CUDA when a launch failed. Errors found on the device go to the error word.
@@ -133,6 +133,22 @@ typedef struct lmh_shape {
  * Returns 0 for an invalid shape or entry.
  */
 LMH_API size_t lmh_workspace_size(const lmh_shape* shape, int entry);
+
+/*
+ * lmh_dh_plan — how the dH = G W contraction of one chunk of `rows` rows is tiled (host,
+ * pure; no CUDA call). *wide (host) receives 1 for 256 x 512 CTA-pair tiles, whose two MMAs
+ * per K step share one staged block of G, or 0 for 256 x 256 tiles; *splits (host) the
+ * number of vocabulary ranges whose fp32 partial products are summed in ascending order
+ * (1: no split). The plan reads (rows, d, V) only, never the device, so dH's bits do not
+ * depend on the GPU; a split changes dH's summation order, so two chunk plans whose chunks
+ * get different plans round dH differently. The wide tile with one range gives the bits of
+ * the 256 x 256 tile. Entries that write dH as fp32 rows (the vocabulary-parallel backward,
+ * the row scatters) always use 256 x 256 tiles without a split.
+ * Returns LMH_ERR_INVALID_ARG if rows < 1, d is not a positive multiple of 64, V is not in
+ * 1 .. 2^31 - 1, or an output pointer is null.
+ */
+LMH_API lmh_status lmh_dh_plan(int64_t rows, int64_t d, int64_t V, int32_t* wide,
+                               int32_t* splits);
 
 /*
  * lmh_loss_fwd — cross-entropy forward, optionally fused with its backward.

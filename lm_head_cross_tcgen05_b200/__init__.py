@@ -26,7 +26,7 @@ from ._abi import (BWD_CE, BWD_LOGPROB, BWD_SUPPORT_KL, BWD_SUPPORT_LOGPROB, DEV
                    F_FUSED_BWD, F_MEAN, F_SUPPORT_RENORM, IGNORE_INDEX, MAX_K, STATUS_NAMES, lib, lmh_shape)
 
 __all__ = [
-    "lmh_shape", "make_shape", "lmh_workspace_size", "lmh_loss_fwd", "lmh_loss_bwd",
+    "lmh_shape", "make_shape", "lmh_workspace_size", "lmh_dh_plan", "lmh_loss_fwd", "lmh_loss_bwd",
     "lmh_logprob", "lmh_support_logprob", "lmh_support_kl", "lmh_support_kl_fwd_bwd",
     "lmh_support_fwd_bwd", "support_fwd_bwd",
     "lmh_read_errors", "LmhError",
@@ -106,6 +106,14 @@ _bf, _f32, _i32, _u8 = torch.bfloat16, torch.float32, torch.int32, torch.uint8
 
 def lmh_workspace_size(shape: lmh_shape, entry: int) -> int:
     return int(lib().lmh_workspace_size(ctypes.byref(shape), int(entry)))
+
+
+def lmh_dh_plan(rows: int, d: int, V: int) -> tuple[bool, int]:
+    """(wide 256 x 512 tiles?, vocabulary ranges) of one chunk's dH GEMM."""
+    wide, splits = ctypes.c_int32(), ctypes.c_int32()
+    _ok("lmh_dh_plan",
+        lib().lmh_dh_plan(int(rows), int(d), int(V), ctypes.byref(wide), ctypes.byref(splits)))
+    return bool(wide.value), int(splits.value)
 
 
 def lmh_loss_fwd(shape, H, W, labels, loss_rows, lse, logprob=None, argmax=None, loss_mean=None,

@@ -41,6 +41,7 @@ class lmh_vp_dest(ctypes.Structure):
 _P = c_void_p
 _SIGS = {
     "lmh_workspace_size": (c_size_t, [ctypes.POINTER(lmh_shape), c_int]),
+    "lmh_dh_plan": (c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _P, _P]),
     "lmh_loss_fwd": (c_int, [ctypes.POINTER(lmh_shape)] + [_P] * 14 + [c_size_t, _P]),
     "lmh_loss_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 10 + [c_size_t, _P]),
     "lmh_loss_fwd_bwd": (c_int, [ctypes.POINTER(lmh_shape), c_int] + [_P] * 15 + [c_size_t, _P]),

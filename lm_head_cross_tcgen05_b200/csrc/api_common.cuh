@@ -39,12 +39,12 @@ bool shape_ok(const lmh_shape* s) {
   return true;
 }
 
-// K splits of the dH GEMM of a chunk with `rows` rows. Chunks with too few output tiles to keep
-// every SM busy (fewer than 384 pair tiles) split the vocabulary into up to 8 ranges, aiming at
-// 512 work units. Each split costs a write and a read of an fp32 [rows, d] partial, i.e. 8 / V
-// bytes per flop of the GEMM: a range must span at least 32768 vocabulary rows, which keeps
-// that traffic near 3 % of the GEMM's time (at V = 32000 no split pays). The rule reads the
-// shape only (never the SM count), so the result bits do not depend on the GPU's size.
+// K splits of the narrow (256 x 256) dH GEMM of a chunk with `rows` rows. Chunks with too few
+// output tiles to keep every SM busy (fewer than 384 pair tiles) split the vocabulary into up
+// to 8 ranges, aiming at 512 work units. Each split costs a write and a read of an fp32
+// [rows, d] partial, i.e. 8 / V bytes per flop of the GEMM: a range must span at least 32768
+// vocabulary rows, which keeps that traffic near 3 % of the GEMM's time (at V = 32000 no split
+// pays).
 int dh_splits(int64_t rows, int64_t d, int64_t V) {
   const int64_t tiles = cdiv(rows, PM) * cdiv(d, BN);
   if (tiles >= 384) return 1;
@@ -53,6 +53,38 @@ int dh_splits(int64_t rows, int64_t d, int64_t V) {
   if (sp > 8) sp = 8;
   if (sp > by_v) sp = by_v;
   return sp < 1 ? 1 : static_cast<int>(sp);
+}
+
+// The dH GEMM of a chunk: narrow (256 x 256) or wide (256 x 512) pair tiles, and its K splits.
+// Work is counted in rounds of the 74 CTA pairs of a 148-SM B200 (a wide unit takes two narrow
+// units' time); the wide tile, whose operand traffic is a quarter lower, is taken when its
+// rounds cost less than 0.95 of the narrow tile's (the 0.95: a step measured 5 % faster with a
+// quarter of dH's operand loads left out). Its splits (up to 8, each range at least 32768
+// vocabulary rows) minimise its rounds. The rule reads the shape only, never the device, so
+// the result bits do not depend on the GPU that runs it.
+struct DhPlan {
+  bool wide;
+  int splits;
+};
+constexpr int kPlanPairs = 74;
+DhPlan dh_plan(int64_t rows, int64_t d, int64_t V) {
+  const int sn = dh_splits(rows, d, V);
+  const double narrow = static_cast<double>(cdiv(cdiv(rows, PM) * cdiv(d, BN) * sn, kPlanPairs)) / sn;
+  const int64_t tw = cdiv(rows, PM) * cdiv(d, 2 * BN);
+  int64_t max_sp = V / 32768;
+  if (max_sp > 8) max_sp = 8;
+  if (max_sp < 1) max_sp = 1;
+  int best_sp = 1;
+  double best = 2.0 * cdiv(tw, kPlanPairs);
+  for (int sp = 2; sp <= max_sp; ++sp) {
+    const double t = 2.0 * cdiv(tw * sp, kPlanPairs) / sp;
+    if (t < best) {
+      best = t;
+      best_sp = sp;
+    }
+  }
+  if (best * 0.95 < narrow) return DhPlan{true, best_sp};
+  return DhPlan{false, sn};
 }
 
 // fused: the entry keeps a [c, Vp] bf16 buffer; need_acc: an fp32 [V, d] accumulator.
@@ -111,8 +143,8 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   const bool vp = vp_bwd || entry == LMH_ENTRY_VP_PARTIALS || vp_sup;  // dH in fp32, unsplit
   if (p.gbuf && p.nchunks > 0 && !vp) {  // the largest split-K partial of any chunk
     const int64_t last = p.N - (p.nchunks - 1) * p.c;
-    const int64_t a = dh_splits(p.c, p.d, p.V) > 1 ? dh_splits(p.c, p.d, p.V) * p.c : 0;
-    const int64_t b = dh_splits(last, p.d, p.V) > 1 ? dh_splits(last, p.d, p.V) * last : 0;
+    const int64_t a = dh_plan(p.c, p.d, p.V).splits > 1 ? dh_plan(p.c, p.d, p.V).splits * p.c : 0;
+    const int64_t b = dh_plan(last, p.d, p.V).splits > 1 ? dh_plan(last, p.d, p.V).splits * last : 0;
     const int64_t r = a > b ? a : b;
     p.o_dhpart = r ? take(static_cast<size_t>(r) * p.d * 4) : 0;
   }
@@ -303,7 +335,7 @@ lmh_status launch_gemm(int dev, int sms, const CUtensorMap& a, const CUtensorMap
   }
   GemmGrid g;
   g.m_tiles = static_cast<int>(cdiv(M, PM));
-  g.n_tiles = static_cast<int>(cdiv(Ncols, BN));
+  g.n_tiles = static_cast<int>(cdiv(Ncols, BN * Pipe<Epi>::WIDE));
   g.k_blocks = static_cast<int>(cdiv(K, Pipe<Epi>::BK));
   g.k_splits = k_splits;
   g.group_m = order.group_m < 1 ? g.m_tiles : (order.group_m < g.m_tiles ? order.group_m : g.m_tiles);
@@ -332,6 +364,8 @@ constexpr GemmOrder kOrderDH{2, kL2Normal, kL2Normal};
 // of W is read by one wave (2048 x 5120 x 151936 in 4 ranges: 5.2-5.5 GB of DRAM reads per
 // launch instead of 7.2-7.5 GB for groups of two)
 constexpr GemmOrder kOrderDHSplit{0, kL2Normal, kL2Normal};
+// dH with wide tiles: two 256-row tiles at a time across all 512-column tiles, split-major
+constexpr GemmOrder kOrderDHWide{2, kL2Normal, kL2Normal};
 // dW: one 256-word vocabulary tile across all hidden tiles (each G tile is read once while
 // its 16 hidden tiles run side by side; keeping H at evict-last priority measured worse)
 constexpr GemmOrder kOrderDW{1, kL2Normal, kL2Normal};
@@ -496,17 +530,23 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
     LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, ta, rows, P.d, P.V, kOrderDH, &ws.h->err, ep,
                                st, 1));
   } else if (dH) {
+    const DhPlan dp = dh_plan(rows, P.d, P.V);
+    const int sp = dp.splits;
     CUtensorMap ta, tb, tc;
-    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) || !tmap_2d(&tb, W, P.d, P.V, P.d, Pipe<EpiDH>::BK) ||
+    if (!tmap_2d(&ta, G, P.V, rows, P.Vp, BM) ||
+        !tmap_2d(&tb, W, P.d, P.V, P.d, dp.wide ? Pipe<EpiDHWide>::BK : Pipe<EpiDH>::BK) ||
         !tmap_out(&tc, dH + r0 * P.d, P.d, rows, P.d))
       return LMH_ERR_CUDA;
-    EpiDH::Params ep;
+    EpiDH::Params ep;  // the same parameters for both tile widths
     ep.rows = rows;
     ep.d = static_cast<int>(P.d);
-    const int sp = dh_splits(rows, P.d, P.V);
     ep.part = sp > 1 ? ws.at<float>(P.o_dhpart) : nullptr;
-    LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, tc, rows, P.d, P.V,
-                               sp > 1 ? kOrderDHSplit : kOrderDH, &ws.h->err, ep, st, sp));
+    if (dp.wide)
+      LMH_TRY(launch_gemm<EpiDHWide>(dev, sms, ta, tb, tc, rows, P.d, P.V, kOrderDHWide,
+                                     &ws.h->err, ep, st, sp));
+    else
+      LMH_TRY(launch_gemm<EpiDH>(dev, sms, ta, tb, tc, rows, P.d, P.V,
+                                 sp > 1 ? kOrderDHSplit : kOrderDH, &ws.h->err, ep, st, sp));
     if (sp > 1) {
       ProfScope ps(KID_SPLIT_SUM, st);
       const int64_t blocks = cdiv(static_cast<int64_t>(rows) * P.d / 2, 256);

@@ -352,16 +352,26 @@ struct RowScatter {
 // ctx.tmC maps this chunk's rows of dH ([rows, d] at row r0). With K (= V) split, each unit
 // writes its fp32 partial to part[split][row][col] instead; a fixed-order reduction over the
 // splits then produces dH. With a row scatter each fp32 row goes to its reducing rank.
-struct EpiDH : PipeDefault {
+// kWide_ = 2: 256 x 512 pair tiles. dH's K loop runs over the whole vocabulary (about 1000
+// K blocks per tile at V = 128256), so an epilogue that no longer overlaps the next tile costs
+// under 1 %, while reading each staged block of G for two MMAs cuts a quarter of the operand
+// bytes moved from L2 into shared memory (at 8192 x 128256 x 4096 the step ran 7 % faster:
+// less power, higher clock). K per stage is 128 in 2 stages of 96 KiB: 16 MMAs per barrier
+// round trip (4 stages of 64 measured 3 % slower). The tensor core adds the same K steps in
+// the same order either way, so an unsplit wide tile gives the narrow tile's bits.
+struct DhParams {
+  int rows;
+  int d;
+  float* part;    // [splits, rows, d] fp32, or null when K is not split
+  RowScatter sc;  // with sc.dest: fp32 rows to their reducing ranks instead (one split)
+};
+template <int kWide_, int kBK_, int kStages_>
+struct EpiDHT {
+  static constexpr int kBK = kBK_, kStages = kStages_, kEpiBufs = 2, kWide = kWide_;
   static constexpr int kId = 5;        // gemm_dH
   static constexpr int kAMajorMN = 0;  // G chunk [rows, V], K-major
   static constexpr int kBMajorMN = 1;  // W [V, d] read as [K = V, N = d], N contiguous
-  struct Params {
-    int rows;
-    int d;
-    float* part;    // [splits, rows, d] fp32, or null when K is not split
-    RowScatter sc;  // with sc.dest: fp32 rows to their reducing ranks instead (one split)
-  };
+  using Params = DhParams;
   static __device__ __forceinline__ void tile(const Params& p, int mb, int nb, uint32_t taddr,
                                               int rit, EpiCtx& ctx) {
     const int n0 = nb * BN;
@@ -394,6 +404,9 @@ struct EpiDH : PipeDefault {
   }
 };
 
+using EpiDH = EpiDHT<1, PipeDefault::kBK, PipeDefault::kStages>;
+using EpiDHWide = EpiDHT<2, 128, 2>;
+
 // ------------------------------------------------------------------ dW = G^T H_c
 // acc_mode 0: the tile sum is the whole dW, stored in bf16 (ctx.tmC: bf16 dW [V, d]).
 // acc_mode 1: acc = 0 + sum (first chunk), stored in fp32.
@@ -420,7 +433,7 @@ struct EpiDH : PipeDefault {
 // chunk at 16384 x 5120 x 151936), so every mode runs the default shape.
 template <int kBK_, int kStages_, int kEpiBufs_>
 struct EpiDWT {
-  static constexpr int kBK = kBK_, kStages = kStages_, kEpiBufs = kEpiBufs_;
+  static constexpr int kBK = kBK_, kStages = kStages_, kEpiBufs = kEpiBufs_, kWide = 1;
   static constexpr int kId = 6;        // gemm_dW
   static constexpr int kAMajorMN = 1;  // G^T: G chunk [rows, V] read as [K = rows, M = V]
   static constexpr int kBMajorMN = 1;  // H chunk [rows, d] read as [K = rows, N = d]

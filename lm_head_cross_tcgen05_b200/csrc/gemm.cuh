@@ -20,7 +20,10 @@
 //   warp 1, lane 0  MMA issuer (rank 0 only): tcgen05.mma 256x256x16 into one of two TMEM
 //                   accumulators (2 x 256 fp32 columns = all 512), so the epilogue of tile i
 //                   overlaps the main loop of tile i+1; commits free the smem stage and signal
-//                   the accumulator in both CTAs (multicast commit, no multicast loads).
+//                   the accumulator in both CTAs (multicast commit, no multicast loads). A wide
+//                   instantiation (Pipe::WIDE = 2) has 256 x 512 pair tiles instead: two MMAs
+//                   per K step, one per 256-column half, share the staged A, and the single
+//                   accumulator fills all 512 columns (no overlap with the next tile).
 //   warps 2..5      epilogue (both CTAs): tcgen05.ld of the CTA's accumulator half (warp w
 //                   reads TMEM lanes 32*(w%4) .. +31), then the fused math of `Epi`; releases
 //                   the accumulator with an arrival on the rank-0 CTA's `tmem_empty` barrier.
@@ -51,9 +54,11 @@ constexpr int kMaxDynSmem = 232448;          // 227 KiB per CTA on sm_100
 // release) costs the tensor pipe a roughly fixed bubble, so the deeper stage runs about 18 %
 // more MMAs per clock than a 64-deep one; 3 stages of 64 KiB per CTA, two 4 KiB staging buffers
 // per epilogue warp. Every epilogue uses this shape: the alternatives measured (64-deep stages,
-// ring depth traded for staging in the dW accumulation) were slower.
+// ring depth traded for staging in the dW accumulation) were slower. kWide = 2 makes the pair
+// tile 256 x 512: two MMAs per K step share the A stage, the one accumulator takes all 512 TMEM
+// columns, so the epilogue no longer overlaps the next tile's main loop (see dH's wide tile).
 struct PipeDefault {
-  static constexpr int kBK = 128, kStages = 3, kEpiBufs = 2;
+  static constexpr int kBK = 128, kStages = 3, kEpiBufs = 2, kWide = 1;
 };
 
 template <class Epi>
@@ -61,14 +66,18 @@ struct Pipe {
   static constexpr int BK = Epi::kBK;
   static constexpr int STAGES = Epi::kStages;
   static constexpr int EPI_BUFS = Epi::kEpiBufs;
+  static constexpr int WIDE = Epi::kWide;             // 256-column halves of a pair tile
+  static constexpr int NACC = 2 / WIDE;               // accumulators in the 512 TMEM columns
   static constexpr int KSUB = BK / 64;                // 128-byte-wide K sub-tiles (K-major)
   static constexpr int A_STAGE_BYTES = BM * BK * 2;
-  static constexpr int B_STAGE_BYTES = BNH * BK * 2;
+  static constexpr int B_HALF_BYTES = BNH * BK * 2;   // this CTA's B rows of one half
+  static constexpr int B_STAGE_BYTES = WIDE * B_HALF_BYTES;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
   static constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x BK (K) box
   static constexpr int EPI_STAGE_BYTES = 4 * EPI_BUFS * EPI_BUF_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + 1024;  // + align
   static_assert(BK % 16 == 0 && STAGES >= 2 && EPI_BUFS >= 2 && EPI_BUFS <= 8, "pipeline shape");
+  static_assert(WIDE == 1 || WIDE == 2, "a pair tile is 256 or 512 columns wide");
   static_assert((Epi::kAMajorMN && Epi::kBMajorMN) || BK % 64 == 0,
                 "a K-major operand is staged in 64-wide K boxes");
   static_assert(SMEM_BYTES + 256 <= kMaxDynSmem, "shared memory per CTA");
@@ -93,7 +102,7 @@ constexpr uint32_t TMEM_COLS = 512;
 
 struct GemmGrid {
   int m_tiles;   // pair tiles along M (256 rows each)
-  int n_tiles;   // tiles along N (256 columns each)
+  int n_tiles;   // tiles along N (256 x Pipe<Epi>::WIDE columns each)
   int k_blocks;  // ceil(K / Pipe<Epi>::BK)
   int k_splits;  // K split into this many consecutive ranges (work units = tiles x splits)
   int group_m;   // tile order: group_m row tiles at a time, rows fastest within a group
@@ -130,6 +139,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   constexpr int BK = P::BK, STAGES = P::STAGES, STAGE_BYTES = P::STAGE_BYTES;
   constexpr int A_STAGE_BYTES = P::A_STAGE_BYTES, MN_BLOCK_BYTES = P::MN_BLOCK_BYTES;
   constexpr int KSUB = P::KSUB;
+  constexpr int WIDE = P::WIDE, NACC = P::NACC, B_HALF_BYTES = P::B_HALF_BYTES;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];   // rank 0: operands of a stage landed
   __shared__ __align__(8) uint64_t empty_bar[STAGES];  // both: the stage was read by the MMAs
@@ -180,7 +190,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         int mb, nb, sp, kb0, kb1;
         unit_coords(g, t, mb, nb, sp, kb0, kb1);
         const int arow = mb * PM + static_cast<int>(rank) * BM;    // this CTA's A rows
-        const int brow = nb * BN + static_cast<int>(rank) * BNH;   // this CTA's B rows
+        const int brow = nb * BN * WIDE + static_cast<int>(rank) * BNH;  // its B rows, half 0
         for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
           const uint32_t s = kbg % STAGES;
           const uint32_t ph = (kbg / STAGES) & 1u;
@@ -202,15 +212,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
               tma_load_2d_pair(a_dst + j * MN_BLOCK_BYTES, &tmA, lfull, arow + 64 * j, kb * BK,
                                pol_a);
           }
-          if (!Epi::kBMajorMN) {
 #pragma unroll
-            for (int j = 0; j < KSUB; ++j)
-              tma_load_2d_pair(b_dst + j * B_SUB_BYTES, &tmB, lfull, kb * BK + 64 * j, brow, pol_b);
-          } else {
+          for (int h = 0; h < WIDE; ++h) {  // half h: the pair tile's columns h*256 .. +255
+            const uint32_t bh = b_dst + h * B_HALF_BYTES;
+            if (!Epi::kBMajorMN) {
 #pragma unroll
-            for (int j = 0; j < BNH / 64; ++j)
-              tma_load_2d_pair(b_dst + j * MN_BLOCK_BYTES, &tmB, lfull, brow + 64 * j, kb * BK,
-                               pol_b);
+              for (int j = 0; j < KSUB; ++j)
+                tma_load_2d_pair(bh + j * B_SUB_BYTES, &tmB, lfull, kb * BK + 64 * j,
+                                 brow + h * BN, pol_b);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BNH / 64; ++j)
+                tma_load_2d_pair(bh + j * MN_BLOCK_BYTES, &tmB, lfull, brow + h * BN + 64 * j,
+                                 kb * BK, pol_b);
+            }
           }
         }
       }
@@ -222,8 +237,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       uint32_t kbg = 0;
       int it = 0;
       for (int t = pair; t < num_tiles && !abort_flag; t += npairs, ++it) {
-        const int b = it & 1;
-        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        const int b = it % NACC;
+        const uint32_t use = static_cast<uint32_t>(it / NACC);
         if (!mbar_wait(smem_u32(&tempty_bar[b]), (use & 1u) ^ 1u, g.err)) {
           abort_flag = 1;
           break;
@@ -231,7 +246,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         tc_fence_after();
         int mb, nb, sp, kb0, kb1;
         unit_coords(g, t, mb, nb, sp, kb0, kb1);
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN * WIDE);
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
           const uint32_t s = kbg % STAGES;
@@ -250,11 +265,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                 Epi::kAMajorMN
                     ? make_sw128_desc(a_base + k * 2048, MN_BLOCK_BYTES, 1024)
                     : make_sw128_desc(a_base + (k >> 2) * A_SUB_BYTES + (k & 3) * 32, 16, 1024);
-            const uint64_t bdesc =
-                Epi::kBMajorMN
-                    ? make_sw128_desc(b_base + k * 2048, MN_BLOCK_BYTES, 1024)
-                    : make_sw128_desc(b_base + (k >> 2) * B_SUB_BYTES + (k & 3) * 32, 16, 1024);
-            mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < WIDE; ++h) {  // both halves reuse this A step
+              const uint32_t bh = b_base + h * B_HALF_BYTES;
+              const uint64_t bdesc =
+                  Epi::kBMajorMN
+                      ? make_sw128_desc(bh + k * 2048, MN_BLOCK_BYTES, 1024)
+                      : make_sw128_desc(bh + (k >> 2) * B_SUB_BYTES + (k & 3) * 32, 16, 1024);
+              mma_bf16_pair(d_tmem + h * BN, adesc, bdesc, idesc,
+                            (kb != kb0 || k != 0) ? 1u : 0u);
+            }
           }
           mma_commit_pair(smem_u32(&empty_bar[s]), 0x3);  // both CTAs may refill stage s
         }
@@ -278,8 +298,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     if (lane == 0) tma_prefetch_desc(&tmC);
     int it = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++it) {
-      const int b = it & 1;
-      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      const int b = it % NACC;
+      const uint32_t use = static_cast<uint32_t>(it / NACC);
       bool ok = !abort_flag && mbar_wait(smem_u32(&tfull_bar[b]), use & 1u, g.err);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
@@ -290,9 +310,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       int mb, nb, sp, kb0, kb1;
       unit_coords(g, t, mb, nb, sp, kb0, kb1);
       ctx.split = sp;
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
-      Epi::tile(ep, mb * 2 + static_cast<int>(rank), nb, taddr, row_in_tile, ctx);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(b * BN * WIDE);
+#pragma unroll 1
+      for (int h = 0; h < WIDE; ++h)  // each 256-column half as a tile of its own
+        Epi::tile(ep, mb * 2 + static_cast<int>(rank), nb * WIDE + h, taddr + h * BN,
+                  row_in_tile, ctx);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty_bar[b]), 0));

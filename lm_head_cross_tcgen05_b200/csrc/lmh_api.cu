@@ -38,6 +38,16 @@ extern "C" size_t lmh_workspace_size(const lmh_shape* shape, int entry) {
   return make_plan(shape, entry, fused, want_acc).total;
 }
 
+extern "C" lmh_status lmh_dh_plan(int64_t rows, int64_t d, int64_t V, int32_t* wide,
+                                  int32_t* splits) {
+  if (rows < 1 || d <= 0 || (d % 64) != 0 || V < 1 || V > 0x7fffffffLL || !wide || !splits)
+    return LMH_ERR_INVALID_ARG;
+  const DhPlan p = dh_plan(rows, d, V);
+  *wide = p.wide ? 1 : 0;
+  *splits = p.splits;
+  return LMH_OK;
+}
+
 // The CE forward, and with dH / dW its fused backward. weighted: the backward is that of
 // L = sum_i w_i l_i for the objective `mode` (loss or log-prob rows), with the row weights and
 // target coefficients from bwd_coef_kernel; otherwise of the mean (or summed) loss.

@@ -36,10 +36,33 @@ def test_chunk_buffer_term():
     N, d, V = 8192, 4096, 128256
     base = ws(N, d, V, chunk=N)
     fused = ws(N, d, V, chunk=N, flags=L.F_FUSED_BWD)
-    # the fused forward adds one chunk's bf16 softmax buffer [c, round_up(V, 8)]
-    assert fused - base == pytest.approx(N * 128256 * 2, abs=256)
+    # the fused forward adds one chunk's bf16 softmax buffer [c, round_up(V, 8)] and the fp32
+    # partials [2, c, d] of its dH, whose 256 x 512 tiles split the vocabulary in two ranges
+    # (256 tiles: 4 rounds of 74 CTA pairs unsplit, 3.5 split in two)
+    assert fused - base == pytest.approx(N * 128256 * 2 + 2 * N * d * 4, abs=512)
     # one chunk: no internal dW accumulator
     assert ws(N, d, V, chunk=N, flags=L.F_FUSED_BWD | L.F_DW_ACC_GIVEN) == fused
+
+
+def test_dh_tile_plan():
+    # (rows, d, V) -> (256 x 512 tiles, vocabulary ranges), counted in rounds of 74 CTA pairs
+    assert L.lmh_dh_plan(8192, 4096, 128256) == (True, 2)   # 256 wide tiles: 3.5 rounds split
+    assert L.lmh_dh_plan(8192, 4096, 151936) == (True, 2)   # the support workload's chunk
+    assert L.lmh_dh_plan(2048, 5120, 151936) == (False, 4)  # 160 narrow units x 4: 2.25 rounds
+    assert L.lmh_dh_plan(4096, 2048, 32000) == (True, 1)    # V too short to split
+    assert L.lmh_dh_plan(1000, 4096, 65536) == (True, 2)
+    assert L.lmh_dh_plan(1000, 4352, 65536) == (True, 2)    # last wide tile half outside d
+    assert L.lmh_dh_plan(64, 256, 2048) == (False, 1)       # one tile either way
+    assert L.lmh_dh_plan(300, 320, 70000) == (False, 2)
+    for bad in ((0, 64, 100), (10, 96, 100), (10, 64, 0), (10, 64, 1 << 31)):
+        with pytest.raises(L.LmhError):
+            L.lmh_dh_plan(*bad)
+    # the plan's split partials are what a fused chunk's workspace adds for dH
+    for rows, d, V in ((1000, 4096, 65536), (2048, 5120, 151936), (4096, 2048, 32000)):
+        wide, sp = L.lmh_dh_plan(rows, d, V)
+        extra = ws(rows, d, V, chunk=rows, flags=L.F_FUSED_BWD) - ws(rows, d, V, chunk=rows)
+        assert extra == pytest.approx(rows * ((V + 7) // 8 * 8) * 2 +
+                                      (sp * rows * d * 4 if sp > 1 else 0), abs=512)
 
 
 def test_budgeted_workload_fits_two_gigabytes():

@@ -434,6 +434,28 @@ def test_dh_split_over_vocabulary(N, d, V, ign, splits):
     check_grad(ch["dH"], out["dH"], "dH chunked vs split")
 
 
+@pytest.mark.parametrize("N,d,V,ign", [
+    (1000, 4096, 65536, 17),   # 4 x 8 wide tiles, the vocabulary in 2 ranges, ragged rows
+    (1000, 4352, 65536, 0),    # the last wide tile's second half lies past d
+])
+def test_wide_dh_tiles(N, d, V, ign):
+    # 256 x 512 pair tiles for dH (two MMAs per K step share the staged G), summed over two
+    # vocabulary ranges in a fixed order
+    assert L.lmh_dh_plan(N, d, V) == (True, 2)
+    x, xc = device_inputs(_wl(N, d, V, ign))
+    res = {}
+
+    def run():
+        res["o"] = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    names = _kernels_launched(run)
+    assert names.count("split_sum") == 1 and names.count("gemm_dH") == 1
+    out = res["o"]
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    check_ce_fused(out, O.ce_fused(xc["H"], xc["W"], xc["labels"]))
+    again = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    assert torch.equal(again["dH"], out["dH"]) and torch.equal(again["dW"], out["dW"])
+
+
 def test_no_split_when_vocabulary_is_small():
     # V = 32000: the fp32 partials would cost more than the fuller waves give back
     x, _ = device_inputs(_wl(256, 256, 32000, 0))
