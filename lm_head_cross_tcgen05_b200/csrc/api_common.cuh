@@ -369,6 +369,8 @@ constexpr GemmOrder kOrderDHWide{2, kL2Normal, kL2Normal};
 // dW: one 256-word vocabulary tile across all hidden tiles (each G tile is read once while
 // its 16 hidden tiles run side by side; keeping H at evict-last priority measured worse)
 constexpr GemmOrder kOrderDW{1, kL2Normal, kL2Normal};
+// dW's bf16 output of one chunk in 256 x 512 tiles from this many rows (64 K blocks) up
+constexpr int kDwWideRows = 8192;
 
 #define LMH_TRY(x)                      \
   do {                                  \
@@ -576,7 +578,11 @@ lmh_status run_backward_gemms(const Plan& P, int dev, int sms, const lmh_bf16* H
     } else {
       acc_mode = chunk_idx == 0 ? 1 : (last ? 3 : 2);
     }
-    LMH_TRY(run_dw<EpiDW>(P, dev, sms, G, H, r0, rows, acc_mode, acc, dW, dw_scatter, ws, st));
+    if (acc_mode == 0 && rows >= kDwWideRows)
+      LMH_TRY(run_dw<EpiDWWide>(P, dev, sms, G, H, r0, rows, acc_mode, acc, dW, dw_scatter, ws,
+                                st));
+    else
+      LMH_TRY(run_dw<EpiDW>(P, dev, sms, G, H, r0, rows, acc_mode, acc, dW, dw_scatter, ws, st));
     if (dW_acc && dW && last && acc_mode != 5) LMH_TRY(cast_dw(P, acc, dW, st));
   }
   return LMH_OK;

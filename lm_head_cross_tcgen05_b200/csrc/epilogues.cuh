@@ -430,10 +430,14 @@ using EpiDHWide = EpiDHT<2, 128, 2>;
 // kBK_, kStages_, kEpiBufs_: the pipeline shape (Pipe). Trading ring depth for more staging
 // buffers (more reduce-adds in flight per warp) made the accumulate modes slower, not faster
 // (96 x 3 stages with 5 buffers, 64 x 5 with 4, 64 x 4 with 6: 2.94 -> 3.27 ms per 2048-row
-// chunk at 16384 x 5120 x 151936), so every mode runs the default shape.
-template <int kBK_, int kStages_, int kEpiBufs_>
+// chunk at 16384 x 5120 x 151936), so every mode runs the default shape. kWide_ = 2: 256 x 512
+// pair tiles (2 stages of 128-deep K), used for the bf16 output of a single chunk of at least
+// 8192 rows (64 K blocks): a quarter less operand traffic outweighs the exposed epilogue there
+// (8192 x 128256 x 4096: the step 2 % faster), while the fp32 accumulate modes, whose epilogue
+// is several times heavier, keep 256 x 256. No tile width changes dW's bits.
+template <int kBK_, int kStages_, int kEpiBufs_, int kWide_ = 1>
 struct EpiDWT {
-  static constexpr int kBK = kBK_, kStages = kStages_, kEpiBufs = kEpiBufs_, kWide = 1;
+  static constexpr int kBK = kBK_, kStages = kStages_, kEpiBufs = kEpiBufs_, kWide = kWide_;
   static constexpr int kId = 6;        // gemm_dW
   static constexpr int kAMajorMN = 1;  // G^T: G chunk [rows, V] read as [K = rows, M = V]
   static constexpr int kBMajorMN = 1;  // H chunk [rows, d] read as [K = rows, N = d]
@@ -538,5 +542,6 @@ struct EpiDWT {
   }
 };
 using EpiDW = EpiDWT<PipeDefault::kBK, PipeDefault::kStages, PipeDefault::kEpiBufs>;
+using EpiDWWide = EpiDWT<128, 2, 2, 2>;
 
 }  // namespace lmh

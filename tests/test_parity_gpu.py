@@ -456,6 +456,18 @@ def test_wide_dh_tiles(N, d, V, ign):
     assert torch.equal(again["dH"], out["dH"]) and torch.equal(again["dW"], out["dW"])
 
 
+def test_unsplit_wide_dh_has_the_narrow_bits():
+    # one 4096-row chunk runs dH in 64 wide tiles, 1024-row chunks in 32 narrow ones, neither
+    # split: the tensor core adds the same K steps in the same order, so dH has the same bits
+    N, d, V = 4096, 2048, 32000
+    assert L.lmh_dh_plan(N, d, V) == (True, 1) and L.lmh_dh_plan(1024, d, V) == (False, 1)
+    x, _ = device_inputs(_wl(N, d, V, 40))
+    wide = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    narrow = L.loss_fwd(x["H"], x["W"], x["labels"], chunk_rows=1024, grads=True)
+    assert torch.equal(wide["lse"], narrow["lse"])
+    assert torch.equal(wide["dH"], narrow["dH"])
+
+
 def test_no_split_when_vocabulary_is_small():
     # V = 32000: the fp32 partials would cost more than the fuller waves give back
     x, _ = device_inputs(_wl(256, 256, 32000, 0))
