@@ -53,10 +53,11 @@ constexpr int kMaxDynSmem = 232448;          // 227 KiB per CTA on sm_100
 // stage, i.e. 8 MMAs per barrier round trip: each round trip (wait for the stage, commit its
 // release) costs the tensor pipe a roughly fixed bubble, so the deeper stage runs about 18 %
 // more MMAs per clock than a 64-deep one; 3 stages of 64 KiB per CTA, two 4 KiB staging buffers
-// per epilogue warp. Every epilogue uses this shape: the alternatives measured (64-deep stages,
-// ring depth traded for staging in the dW accumulation) were slower. kWide = 2 makes the pair
-// tile 256 x 512: two MMAs per K step share the A stage, the one accumulator takes all 512 TMEM
-// columns, so the epilogue no longer overlaps the next tile's main loop (see dH's wide tile).
+// per epilogue warp. Every 256 x 256 epilogue uses this shape: the alternatives measured
+// (64-deep stages, 2 stages of 192, ring depth traded for staging in the dW accumulation) were
+// slower. kWide = 2 makes the pair tile 256 x 512: two MMAs per K step share the A stage, the one
+// accumulator takes all 512 TMEM columns, so the epilogue no longer overlaps the next tile's
+// main loop; the wide dH and dW epilogues run 2 stages of 96 KiB (16 MMAs per round trip).
 struct PipeDefault {
   static constexpr int kBK = 128, kStages = 3, kEpiBufs = 2, kWide = 1;
 };
