@@ -69,7 +69,8 @@ struct DhPlan {
 constexpr int kPlanPairs = 74;
 DhPlan dh_plan(int64_t rows, int64_t d, int64_t V) {
   const int sn = dh_splits(rows, d, V);
-  const double narrow = static_cast<double>(cdiv(cdiv(rows, PM) * cdiv(d, BN) * sn, kPlanPairs)) / sn;
+  const int64_t tn = cdiv(rows, PM) * cdiv(d, BN);
+  const double narrow = static_cast<double>(cdiv(tn * sn, kPlanPairs)) / sn;
   const int64_t tw = cdiv(rows, PM) * cdiv(d, 2 * BN);
   int64_t max_sp = V / 32768;
   if (max_sp > 8) max_sp = 8;
@@ -143,8 +144,9 @@ Plan make_plan(const lmh_shape* s, int entry, bool fused, bool dw_without_acc) {
   const bool vp = vp_bwd || entry == LMH_ENTRY_VP_PARTIALS || vp_sup;  // dH in fp32, unsplit
   if (p.gbuf && p.nchunks > 0 && !vp) {  // the largest split-K partial of any chunk
     const int64_t last = p.N - (p.nchunks - 1) * p.c;
-    const int64_t a = dh_plan(p.c, p.d, p.V).splits > 1 ? dh_plan(p.c, p.d, p.V).splits * p.c : 0;
-    const int64_t b = dh_plan(last, p.d, p.V).splits > 1 ? dh_plan(last, p.d, p.V).splits * last : 0;
+    const int sa = dh_plan(p.c, p.d, p.V).splits, sb = dh_plan(last, p.d, p.V).splits;
+    const int64_t a = sa > 1 ? sa * p.c : 0;
+    const int64_t b = sb > 1 ? sb * last : 0;
     const int64_t r = a > b ? a : b;
     p.o_dhpart = r ? take(static_cast<size_t>(r) * p.d * 4) : 0;
   }

@@ -355,8 +355,8 @@ struct RowScatter {
 // kWide_ = 2: 256 x 512 pair tiles. dH's K loop runs over the whole vocabulary (about 1000
 // K blocks per tile at V = 128256), so an epilogue that no longer overlaps the next tile costs
 // under 1 %, while reading each staged block of G for two MMAs cuts a quarter of the operand
-// bytes moved from L2 into shared memory (at 8192 x 128256 x 4096 the step ran 7 % faster:
-// less power, higher clock). K per stage is 128 in 2 stages of 96 KiB: 16 MMAs per barrier
+// bytes moved from L2 into shared memory (at 8192 x 128256 x 4096 the step ran 3-7 % faster
+// on two boxes: less power, higher clock). K per stage is 128 in 2 stages of 96 KiB: 16 MMAs per barrier
 // round trip (4 stages of 64 measured 3 % slower). The tensor core adds the same K steps in
 // the same order either way, so an unsplit wide tile gives the narrow tile's bits.
 struct DhParams {
