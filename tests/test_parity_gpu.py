@@ -468,6 +468,24 @@ def test_unsplit_wide_dh_has_the_narrow_bits():
     assert torch.equal(wide["dH"], narrow["dH"])
 
 
+def test_wide_dw_tiles_and_bits():
+    # one chunk of 8192 rows: dW's bf16 output in 256 x 512 pair tiles (and dH's too), with a
+    # ragged vocabulary (12 row tiles of dW, the last partial) and d = 8.5 wide tiles
+    N, d, V = 8192, 4352, 3000
+    assert L.lmh_dh_plan(N, d, V) == (True, 1)
+    x, xc = device_inputs(_wl(N, d, V, 61))
+    out = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True)
+    assert L.lmh_read_errors(out["workspace"]) == 0
+    check_ce_fused(out, O.ce_fused(xc["H"], xc["W"], xc["labels"]))
+    # a caller accumulator makes the same chunk's dW run 256 x 256 tiles (load, add to the
+    # zeros, store the sum, cast): 0 + s is s, so the bits agree up to the sign of zero
+    acc = torch.zeros(V, d, dtype=torch.float32, device="cuda")
+    narrow = L.loss_fwd(x["H"], x["W"], x["labels"], grads=True, dW_acc=acc)
+    assert torch.equal(out["dW"].float() + 0.0, narrow["dW"].float() + 0.0)
+    assert torch.equal(narrow["dW"], acc.to(torch.bfloat16))
+    assert torch.equal(out["dH"], narrow["dH"])
+
+
 def test_no_split_when_vocabulary_is_small():
     # V = 32000: the fp32 partials would cost more than the fuller waves give back
     x, _ = device_inputs(_wl(256, 256, 32000, 0))
