@@ -616,6 +616,10 @@ def main():
             cfg["workspace_bytes"] = int(ws.numel())
             cfg["dW_accumulator"] = ("caller-owned fp32 [V, d], stored by the first chunk"
                                      if dW_acc is not None else "none (one chunk: bf16 dW)")
+        if not vp_entry:  # the first chunk's dH tiling, which decides dH's summation order
+            wide, splits = L.lmh_dh_plan(min(chunk, wl.N), d, V)
+            cfg["dH_tiles"] = (f"{'256x512' if wide else '256x256'} CTA-pair tiles, "
+                               f"{splits} vocabulary range{'s' if splits > 1 else ''}")
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "strong" if vp_entry else "weak",
