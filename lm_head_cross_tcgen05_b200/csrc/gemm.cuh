@@ -79,6 +79,7 @@ struct Pipe {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + 1024;  // + align
   static_assert(BK % 16 == 0 && STAGES >= 2 && EPI_BUFS >= 2 && EPI_BUFS <= 8, "pipeline shape");
   static_assert(WIDE == 1 || WIDE == 2, "a pair tile is 256 or 512 columns wide");
+  static_assert(NACC * BN * WIDE == 512, "the accumulators fill the 512 TMEM columns");
   static_assert((Epi::kAMajorMN && Epi::kBMajorMN) || BK % 64 == 0,
                 "a K-major operand is staged in 64-wide K boxes");
   static_assert(SMEM_BYTES + 256 <= kMaxDynSmem, "shared memory per CTA");
