@@ -54,6 +54,7 @@ def test_dh_tile_plan():
     assert L.lmh_dh_plan(1000, 4352, 65536) == (True, 2)    # last wide tile half outside d
     assert L.lmh_dh_plan(64, 256, 2048) == (False, 1)       # one tile either way
     assert L.lmh_dh_plan(300, 320, 70000) == (False, 2)
+    assert L.lmh_dh_plan(600, 1024, 262144) == (True, 8)      # 6 wide tiles: one round in 8
     for bad in ((0, 64, 100), (10, 96, 100), (10, 64, 0), (10, 64, 1 << 31)):
         with pytest.raises(L.LmhError):
             L.lmh_dh_plan(*bad)

@@ -434,14 +434,15 @@ def test_dh_split_over_vocabulary(N, d, V, ign, splits):
     check_grad(ch["dH"], out["dH"], "dH chunked vs split")
 
 
-@pytest.mark.parametrize("N,d,V,ign", [
-    (1000, 4096, 65536, 17),   # 4 x 8 wide tiles, the vocabulary in 2 ranges, ragged rows
-    (1000, 4352, 65536, 0),    # the last wide tile's second half lies past d
+@pytest.mark.parametrize("N,d,V,ign,splits", [
+    (1000, 4096, 65536, 17, 2),  # 4 x 8 wide tiles, the vocabulary in 2 ranges, ragged rows
+    (1000, 4352, 65536, 0, 2),   # the last wide tile's second half lies past d
+    (600, 1024, 262144, 9, 8),   # 6 wide tiles, 8 ranges of 32768 words
 ])
-def test_wide_dh_tiles(N, d, V, ign):
-    # 256 x 512 pair tiles for dH (two MMAs per K step share the staged G), summed over two
+def test_wide_dh_tiles(N, d, V, ign, splits):
+    # 256 x 512 pair tiles for dH (two MMAs per K step share the staged G), summed over the
     # vocabulary ranges in a fixed order
-    assert L.lmh_dh_plan(N, d, V) == (True, 2)
+    assert L.lmh_dh_plan(N, d, V) == (True, splits)
     x, xc = device_inputs(_wl(N, d, V, ign))
     res = {}
 
