@@ -136,7 +136,8 @@ LMH_API size_t lmh_workspace_size(const lmh_shape* shape, int entry);
 
 /*
  * lmh_dh_plan — how the dH = G W contraction of one chunk of `rows` rows is tiled (host,
- * pure; no CUDA call). *wide (host) receives 1 for 256 x 512 CTA-pair tiles, whose two MMAs
+ * pure; no CUDA call). Not an operation of the method: it makes inspectable a part of what
+ * FlashInfer PR #8059's determinism contract (description) calls the chunk plan. *wide (host) receives 1 for 256 x 512 CTA-pair tiles, whose two MMAs
  * per K step share one staged block of G, or 0 for 256 x 256 tiles; *splits (host) the
  * number of vocabulary ranges whose fp32 partial products are summed in ascending order
  * (1: no split). The plan reads (rows, d, V) only, never the device, so dH's bits do not
